@@ -1,0 +1,236 @@
+/*
+ * kda_oracle.c -- fp64 token-by-token oracle for Kimi Delta Attention (KDA).
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, obviously correct
+ * CPU definition that the CUDA path is checked against. Only the test suite,
+ * the smoke check and the CPU-baseline leg of the benchmark may load it. It
+ * shares no code, header, table or helper with the CUDA library, and the CUDA
+ * library never calls it.
+ *
+ * What it computes, per (sequence, head), token by token, in double precision:
+ *
+ *   g'   = max(g_t, lb)                       per key channel i
+ *   S    = Diag(exp g') S                     row i of S decays by exp(g'_i)
+ *   w    = S^T k_t                            what the decayed state recalls for k_t
+ *   S    = S + beta_t * k_t (v_t - w)^T       delta-rule erase-then-write
+ *   o_t  = scale * S^T q_t                    read-out from the UPDATED state
+ *
+ * i.e. S_t = (I - beta_t k_t k_t^T) Diag(exp g'_t) S_{t-1} + beta_t k_t v_t^T.
+ * S is d_k x d_v (rows indexed by key channels).
+ *
+ * Sources (web pages about the Kimi K3 report):
+ *  - "Kimi K3 深度拆解" (chenxutan.com), section 4.2 "线性注意力与 Delta Rule":
+ *    the delta-rule update S_t = S_{t-1}(I - b k k^T) + b k v^T, the fixed-size
+ *    [d, d_v] state, the per-token write strength beta in (0,1), and the toy
+ *    single-head loop (erase, then write, then read from the new state).
+ *    The printed formula only type-checks with S as d_v x d_k; with S stored
+ *    d_k x d_v (as the toy does) the same map is the left-multiplied form above.
+ *  - "Kimi K3 技術報告：三個架構改動" (akiraxclaw.com), section "長度":
+ *    KDA extends Gated DeltaNet with channel-wise gating (each key channel
+ *    forgets at its own rate), so the decay is Diag(exp g_t) with g_t in R^{d_k}.
+ *  - "3 分钟看懂 Kimi K3" (landx.limxdynamics.com), "第一条主线" and Figure 3:
+ *    the log decay is bounded below; here that is the clamp g' = max(g, lb).
+ *  Reading taken where the pages are silent: the decay acts on the state before
+ *  the erase/write (gated delta rule), and o_t uses 1/sqrt(d_k) by default
+ *  (the caller passes `scale`).
+ *
+ * Inputs are read as float32 or as bfloat16 bit patterns and widened exactly
+ * to double per token, so a 1M-token run never materialises fp64 copies.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define KDA_ORACLE_F32 0
+#define KDA_ORACLE_BF16 1
+
+/* Exact widening of one input element to double. */
+static double load_elem(const void *base, int dtype, int64_t idx)
+{
+    if (dtype == KDA_ORACLE_F32) {
+        return (double)((const float *)base)[idx];
+    }
+    /* bfloat16: the upper 16 bits of an IEEE float32. */
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    int64_t T;
+    int H, dk, dv, n_seqs;
+    const int64_t *cu_seqlens;
+    int dtype;
+    const void *q, *k, *v, *g, *beta;
+    const double *initial_state;
+    double lb, scale;
+    double *out;
+    const int64_t *out_rows;
+    int64_t n_out_rows;
+    double *final_state;
+    int64_t next_item; /* shared work counter over (seq, head) */
+    pthread_mutex_t lock;
+} job_t;
+
+/* First index in the sorted list `rows` whose value is >= t. */
+static int64_t lower_bound_rows(const int64_t *rows, int64_t n, int64_t t)
+{
+    int64_t lo = 0, hi = n;
+    while (lo < hi) {
+        int64_t mid = lo + (hi - lo) / 2;
+        if (rows[mid] < t) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+/* One (sequence, head) pair, token by token. */
+static void run_one(const job_t *J, int seq, int h, double *S, double *kt,
+                    double *qt, double *vt, double *decay, double *w)
+{
+    const int dk = J->dk, dv = J->dv, H = J->H;
+    const int64_t t0 = J->cu_seqlens[seq], t1 = J->cu_seqlens[seq + 1];
+    const int64_t state_off = ((int64_t)seq * H + h) * dk * dv;
+
+    if (J->initial_state) {
+        memcpy(S, J->initial_state + state_off, sizeof(double) * dk * dv);
+    } else {
+        memset(S, 0, sizeof(double) * dk * dv);
+    }
+
+    int64_t next_out = J->out_rows ? lower_bound_rows(J->out_rows, J->n_out_rows, t0) : 0;
+
+    for (int64_t t = t0; t < t1; ++t) {
+        const int64_t tok_k = (t * H + h) * dk;
+        const int64_t tok_v = (t * H + h) * dv;
+        for (int i = 0; i < dk; ++i) {
+            kt[i] = load_elem(J->k, J->dtype, tok_k + i);
+            qt[i] = load_elem(J->q, J->dtype, tok_k + i);
+            double gi = load_elem(J->g, J->dtype, tok_k + i);
+            if (gi < J->lb) gi = J->lb;              /* lower bound on the log decay */
+            decay[i] = exp(gi);
+        }
+        for (int j = 0; j < dv; ++j) vt[j] = load_elem(J->v, J->dtype, tok_v + j);
+        const double b = load_elem(J->beta, J->dtype, t * H + h);
+
+        /* S <- Diag(exp g') S */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) S[i * dv + j] *= decay[i];
+
+        /* w = S^T k */
+        for (int j = 0; j < dv; ++j) w[j] = 0.0;
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) w[j] += kt[i] * S[i * dv + j];
+
+        /* S <- S + beta k (v - w)^T */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) S[i * dv + j] += b * kt[i] * (vt[j] - w[j]);
+
+        /* o = scale * S^T q, written only where an output row is wanted */
+        int64_t out_row = -1;
+        if (J->out) {
+            if (!J->out_rows) {
+                out_row = t;
+            } else if (next_out < J->n_out_rows && J->out_rows[next_out] == t) {
+                out_row = next_out++;
+            }
+        }
+        if (out_row >= 0) {
+            double *o = J->out + (out_row * H + h) * dv;
+            for (int j = 0; j < dv; ++j) o[j] = 0.0;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) o[j] += qt[i] * S[i * dv + j];
+            for (int j = 0; j < dv; ++j) o[j] *= J->scale;
+        }
+    }
+
+    if (J->final_state) memcpy(J->final_state + state_off, S, sizeof(double) * dk * dv);
+}
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const int dk = J->dk, dv = J->dv;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(3 * dk + 2 * dv));
+    if (!S || !buf) {
+        free(S);
+        free(buf);
+        return (void *)1;
+    }
+    double *kt = buf, *qt = buf + dk, *decay = buf + 2 * dk, *vt = buf + 3 * dk, *w = vt + dv;
+    const int64_t n_items = (int64_t)J->n_seqs * J->H;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t item = J->next_item++;
+        pthread_mutex_unlock(&J->lock);
+        if (item >= n_items) break;
+        run_one(J, (int)(item / J->H), (int)(item % J->H), S, kt, qt, vt, decay, w);
+    }
+    free(S);
+    free(buf);
+    return NULL;
+}
+
+/*
+ * Token-by-token fp64 recurrence over packed sequences.
+ *
+ *  q, k, g : [T, H, dk]   v : [T, H, dv]   beta : [T, H]   (dtype f32 or bf16 bits)
+ *  cu_seqlens : [n_seqs + 1], cu_seqlens[0] = 0, non-decreasing, last = T
+ *  initial_state / final_state : [n_seqs, H, dk, dv] fp64 (initial NULL = zeros)
+ *  out : [T, H, dv] fp64, or [n_out_rows, H, dv] when out_rows (sorted token
+ *        indices) is given; NULL skips the read-out.
+ *  Returns 0 on success, -1 on a bad argument, -2 when a thread failed.
+ */
+int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
+                         const int64_t *cu_seqlens, int dtype,
+                         const void *q, const void *k, const void *v,
+                         const void *g, const void *beta,
+                         const double *initial_state, double lb, double scale,
+                         double *out, const int64_t *out_rows, int64_t n_out_rows,
+                         double *final_state, int n_threads)
+{
+    if (T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs <= 0 || !cu_seqlens) return -1;
+    if (dtype != KDA_ORACLE_F32 && dtype != KDA_ORACLE_BF16) return -1;
+    if (cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return -1;
+    for (int s = 0; s < n_seqs; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    if (T > 0 && (!q || !k || !v || !g || !beta)) return -1;
+
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.n_seqs = n_seqs;
+    J.cu_seqlens = cu_seqlens; J.dtype = dtype;
+    J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta;
+    J.initial_state = initial_state; J.lb = lb; J.scale = scale;
+    J.out = out; J.out_rows = out_rows; J.n_out_rows = n_out_rows;
+    J.final_state = final_state;
+    pthread_mutex_init(&J.lock, NULL);
+
+    const int64_t n_items = (int64_t)n_seqs * H;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > n_items) n_threads = (int)n_items;
+
+    int rc = 0;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    if (!th) {
+        pthread_mutex_destroy(&J.lock);
+        return -2;
+    }
+    int started = 0;
+    for (int i = 0; i < n_threads; ++i) {
+        if (pthread_create(&th[i], NULL, worker, &J) != 0) break;
+        ++started;
+    }
+    if (started == 0) rc = -2;
+    for (int i = 0; i < started; ++i) {
+        void *ret = NULL;
+        pthread_join(th[i], &ret);
+        if (ret != NULL) rc = -2;
+    }
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return rc;
+}

@@ -1,0 +1,88 @@
+"""CPU tests: the fp64 oracle against its pins, and the pins against planted mistakes."""
+from __future__ import annotations
+
+import multiprocessing as mp
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from oracle import kda_oracle as ko
+from tests import oracle_pins as pins
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(oracle, pin):
+    pin(oracle.load())
+
+
+def test_chunked_oracle_hand_example():
+    """The chunked form on its own reproduces the two-token hand example."""
+    import numpy as np
+    import torch
+    q = torch.tensor([[[1.0]], [[1.0]]])
+    k = torch.tensor([[[1.0]], [[-1.0]]])
+    v = torch.tensor([[[4.0]], [[0.0]]])
+    g = torch.full((2, 1, 1), float(np.log(0.5)))
+    b = torch.tensor([[0.5], [0.5]])
+    o, s = ko.chunked(q, k, v, g, b, chunk=2, initial_state=np.array([[[[2.0]]]]), scale=1.0)
+    assert np.allclose(o[:, 0, 0], [2.5, 0.625], rtol=1e-6)
+    assert np.allclose(s[0, 0], [[0.625]], rtol=1e-6)
+
+
+# Plausible slips, each planted in a copy of the oracle source. Every one must
+# be caught by at least one pin, or the pins are too weak to trust the oracle.
+MUTANTS = {
+    "drop_decay": ("S[i * dv + j] *= decay[i];", ";"),
+    "decay_sign": ("decay[i] = exp(gi);", "decay[i] = exp(-gi);"),
+    "no_clamp": ("if (gi < J->lb) gi = J->lb;", ";"),
+    "erase_sign": ("(vt[j] - w[j])", "(vt[j] + w[j])"),
+    "drop_erase": ("(vt[j] - w[j])", "(vt[j])"),
+    "drop_beta": ("+= b * kt[i] * (vt[j] - w[j])", "+= kt[i] * (vt[j] - w[j])"),
+    "recall_with_query": ("w[j] += kt[i] * S[i * dv + j];", "w[j] += qt[i] * S[i * dv + j];"),
+    "no_scale": ("o[j] *= J->scale;", ";"),
+    "read_before_write": (
+        "        /* S <- S + beta k (v - w)^T */\n"
+        "        for (int i = 0; i < dk; ++i)\n"
+        "            for (int j = 0; j < dv; ++j) S[i * dv + j] += b * kt[i] * (vt[j] - w[j]);\n",
+        ""),
+    "transposed_readout": (
+        "for (int j = 0; j < dv; ++j) o[j] += qt[i] * S[i * dv + j];",
+        "for (int j = 0; j < dv && i < dv && j < dk; ++j) o[i] += qt[j] * S[i * dv + j];"),
+    "decay_on_columns": ("S[i * dv + j] *= decay[i];", "S[i * dv + j] *= decay[j % dk];"),
+}
+
+
+def _mutant_worker(path, q):
+    q.put(pins.failing_pins(path))
+
+
+def _run_isolated(path: str) -> list[str]:
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_mutant_worker, args=(path, q))
+    p.start()
+    p.join(600)
+    if p.exitcode != 0:
+        return ["<crashed>"]
+    return q.get()
+
+
+def test_pins_catch_planted_mistakes(tmp_path):
+    with open(ko._SRC) as f:
+        src = f.read()
+    clean = tmp_path / "clean.so"
+    ko.build(ko._SRC, str(clean))
+    assert _run_isolated(str(clean)) == []
+    survivors = []
+    for name, (old, new) in MUTANTS.items():
+        assert old in src, f"mutant {name}: pattern not found in oracle source"
+        msrc = tmp_path / f"{name}.c"
+        msrc.write_text(src.replace(old, new, 1))
+        so = tmp_path / f"{name}.so"
+        ko.build(str(msrc), str(so))
+        caught = _run_isolated(str(so))
+        if not caught:
+            survivors.append(name)
+    assert not survivors, f"pins missed planted mistakes: {survivors}"
