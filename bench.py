@@ -1,0 +1,355 @@
+#!/usr/bin/env python
+"""KDA benchmark: chunked prefill (tokens/s, TFLOP/s vs the bf16 tensor-core
+peak) and serving decode (state GB/s vs HBM), one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one prefill of the 8K-token, 32-head, d=128 bf16 workload (fp32
+state, chunk 64), inputs resident in HBM. The decode leg runs the 256-sequence
+x 32-head serving workload for 1000 one-token steps. With N > 1 (torchrun) every
+rank runs its own replica (the work is independent per sequence and head, so
+there is no collective on the data path); `value` is the job total.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "bf16_h32_t8192_d128"
+DECODE = "decode_n256_h32_d128"
+C = 64
+
+
+def prefill_flops_per_token_head(dk: int, dv: int, chunk: int = C) -> float:
+    """Algorithmic FLOPs of the chunked form per (token, head):
+    2C(3dk + 2dv) + 6 dk dv + C^2/3 (Gram products, WY apply, state pass, inverse)."""
+    return 2 * chunk * (3 * dk + 2 * dv) + 6 * dk * dv + chunk * chunk / 3
+
+
+def prefill_bytes_per_token_head(dk: int, dv: int, elem: int = 2) -> int:
+    """Compulsory HBM bytes per (token, head): read q, k, g, v, beta; write out."""
+    return elem * (3 * dk + dv + 1) + elem * dv
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_region(fn, steps: int, stream) -> tuple[float, list[float]]:
+    """Total and per-step device time (ms) of `steps` calls, CUDA events on `stream`."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[-1]), per
+
+
+def bench_ours(args, world, rank, local):
+    from kimi_delta_attention_19_b200 import kda
+    from kimi_delta_attention_19_b200.inputs import (WORKLOADS, decode_state, decode_tokens,
+                                                      workload_inputs)
+    peaks = load_peaks()
+    dev = f"cuda:{local}"
+    stream = torch.cuda.current_stream()
+    w = WORKLOADS[PREFILL]
+    x = workload_inputs(w, seed=rank, device=dev)
+    T, H, dk, dv = w.T, w.H, w.dk, w.dv
+    shape = kda.make_shape(T, H, dk, dv, w.dtype)
+    ws = kda.alloc_workspace(shape, dev)
+    out = torch.empty(T, H, dv, dtype=w.dtype, device=dev)
+    fin = torch.empty(1, H, dk, dv, dtype=torch.float32, device=dev)
+
+    def step():
+        kda.chunk_fwd(x.q, x.k, x.v, x.g, x.beta, initial_state=x.initial_state, out=out,
+                      final_state=fin, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    total_ms, per = time_region(step, args.steps, stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    tokens_per_step = T * world
+    value = tokens_per_step / (ms_step / 1e3)
+    flops = prefill_flops_per_token_head(dk, dv) * T * H
+    kernel_ms = statistics.mean(per)
+    launches_per_step = kda_launches_per_step(kda, shape)
+
+    tc_tflops = flops / (kernel_ms / 1e3) / 1e12
+    algo_bytes = prefill_bytes_per_token_head(dk, dv) * T * H + 2 * 4 * H * dk * dv
+    gbs = algo_bytes / (kernel_ms / 1e3) / 1e9
+    roofline = {"bound": "tensor", "achieved": round(tc_tflops, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
+                "traffic": None, "peak_source": peaks["source"],
+                "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": algo_bytes},
+                "kernel_ms": round(kernel_ms, 4)}
+
+    # ---- end to end through the public API with host buffers
+    pin = {n: getattr(x, n).cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    s0_host = x.initial_state.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    fin_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    dbuf = {n: torch.empty_like(getattr(x, n)) for n in pin}
+    s0_dev = torch.empty_like(x.initial_state)
+
+    def e2e_step():
+        for n in pin:
+            dbuf[n].copy_(pin[n], non_blocking=True)
+        s0_dev.copy_(s0_host, non_blocking=True)
+        kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                      initial_state=s0_dev, out=out, final_state=fin, workspace=ws,
+                      stream=stream)
+        out_host.copy_(out, non_blocking=True)
+        fin_host.copy_(fin, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms, _ = time_region(e2e_step, max(2, args.steps // 4), stream)
+    e2e_ms = max_over_ranks(e2e_ms, world) / max(2, args.steps // 4)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values()) + s0_host.numel() * 4
+    d2h = out_host.numel() * out_host.element_size() + fin_host.numel() * 4
+    e2e = {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
+    del pin, dbuf
+
+    # ---- decode leg
+    wd = WORKLOADS[DECODE]
+    N, Hd, d = wd.B, wd.H, wd.dk
+    dsteps = wd.extra["steps"]
+    state = decode_state(N, Hd, d, d, seed=rank, device=dev)
+    tok = decode_tokens(dsteps, N, Hd, d, d, seed=1000 + rank, device=dev)
+    dout = torch.empty(N, Hd, d, dtype=torch.bfloat16, device=dev)
+
+    def dstep(t):
+        kda.decode_step(tok.q[t], tok.k[t], tok.v[t], tok.g[t], tok.beta[t], state, out=dout,
+                        stream=stream)
+
+    for t in range(3):
+        dstep(t)
+    torch.cuda.synchronize()
+    barrier(world)
+    it = iter(range(dsteps))
+    d_total, d_per = time_region(lambda: dstep(next(it)), dsteps, stream)
+    d_total = max_over_ranks(d_total, world)
+    d_ms = d_total / dsteps
+    state_bytes = 2 * N * Hd * d * d * 4
+    tok_bytes = N * Hd * (3 * d + d + 1) * 2 + N * Hd * d * 2
+    d_gbs = (state_bytes + tok_bytes) / (d_ms / 1e3) / 1e9
+    decode = {"workload": DECODE, "steps": dsteps, "ms_per_step": round(d_ms, 5),
+              "state_gbs": round(d_gbs * world, 1), "unit": "GB/s",
+              "tokens_per_s": round(N * world / (d_ms / 1e3), 1),
+              "roofline": {"bound": "hbm", "achieved": round(d_gbs, 1), "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": round(d_gbs / peaks["hbm_gbs"], 4),
+                           "frac_of_8tbs": round(d_gbs / 8000.0, 4),
+                           "bytes_per_step": state_bytes + tok_bytes, "traffic": None},
+              "gpu_launches": dsteps}
+    return {
+        "value": round(value, 1), "ms_per_step": round(ms_step, 4), "clocks": clk,
+        "roofline": roofline, "e2e": e2e, "decode": decode,
+        "gpu_launches": launches_per_step * args.steps,
+        "tflops": round(tc_tflops * world, 2),
+    }
+
+
+def kda_launches_per_step(kda, shape) -> int:
+    """Kernels this library enqueues per kda_chunk_fwd for `shape` (memset excluded)."""
+    return 1
+
+
+def cpu_oracle_rate(tokens: int, seed: int = 0) -> dict:
+    """Time the fp64 oracle on the first `tokens` tokens of the prefill workload."""
+    from kimi_delta_attention_19_b200.inputs import WORKLOADS, workload_inputs
+    from oracle import kda_oracle as ko
+    w = WORKLOADS[PREFILL]
+    x = workload_inputs(w, seed=seed, device="cpu")
+    sl = slice(0, tokens)
+    threads = min(os.cpu_count() or 1, w.H)
+    ko.load()
+    t0 = time.perf_counter()
+    ko.recurrent(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl],
+                 initial_state=x.initial_state, n_threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": round(tokens / dt, 2), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {tokens} of {w.T} tokens of {PREFILL} (all {w.H} heads), "
+                      f"fp64 token-by-token recurrence, {threads} threads"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = {"workload": PREFILL, "model": "KDA layer (synthetic, no weights)", "global_batch": 1,
+           "seq_len": 8192, "heads": 32, "dk": 128, "dv": 128, "chunk": C,
+           "state": "fp32", "l2": "inputs_exceed_l2 (q,k,v,g 256 MiB > 126 MB L2)"}
+    metric = "KDA prefill tokens/s + % bf16 TC peak; decode state GB/s vs HBM peak"
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        cfg["parallelism"] = f"oracle on host cores (N={world} requested; rank 0 only)"
+        rates = []
+        for _ in range(args.warmup // 3):
+            cpu_oracle_rate(args.cpu_tokens // 4)
+        for _ in range(args.steps):
+            rates.append(cpu_oracle_rate(args.cpu_tokens))
+        v = statistics.median(r["value"] for r in rates)
+        cb = dict(rates[-1])
+        cb["value"] = v
+        print(json.dumps({
+            "metric": metric, "value": v, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * args.cpu_tokens / v, 3) if v else None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg, "impl": "reference", "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    cfg["parallelism"] = f"replicas{world}" if world > 1 else "single_gpu"
+    r = bench_ours(args, world, rank, local)
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_oracle_rate(args.cpu_tokens)
+    if rank == 0:
+        line = {
+            "metric": metric, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; no weights, no dataset)",
+            "config": cfg, "impl": "ours", "tflops": r["tflops"], "roofline": r["roofline"],
+            "cpu_baseline": cpu, "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
+            "clocks": r["clocks"], "decode": r["decode"],
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

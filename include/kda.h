@@ -1,0 +1,143 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library.
+ *
+ * Kimi Delta Attention (KDA) is a gated delta-rule linear attention with a
+ * fixed-size state per head. Sources (web pages about the Kimi K3 report):
+ *   - "Kimi K3 深度拆解" (chenxutan.com), section 4.2 "线性注意力与 Delta Rule":
+ *     the delta-rule state update, the fixed [d_k, d_v] state, the per-token
+ *     write strength beta in (0,1), q/k assumed L2-normalised, read-out from
+ *     the updated state, and the chunk-parallel / inter-chunk-recurrent form.
+ *   - "Kimi K3 技術報告：三個架構改動" (akiraxclaw.com), section "長度":
+ *     channel-wise gating (each key channel has its own forget rate).
+ *   - "3 分钟看懂 Kimi K3" (landx.limxdynamics.com), "第一条主线", Figure 3:
+ *     the log decay is bounded below so every causal chunk is a dense matmul.
+ *
+ * Per head, with S in R^{d_k x d_v} (rows = key channels), each token t does
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp max(g_t, lb)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t
+ * where g_t in R^{d_k} is the per-channel log decay and lb = g_lower_bound.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *     never frees or retains them and never allocates device memory per call
+ *     (scratch is the caller's `workspace`).
+ *   - Layouts are token-major and contiguous: q, k, g [tokens, H, d_k];
+ *     v, out [tokens, H, d_v]; beta [tokens, H]; states [n, H, d_k, d_v] fp32
+ *     row-major. Every tensor pointer must be 16-byte aligned.
+ *   - q, k, v, g, beta and out share `dtype`; states are always fp32.
+ *   - Work is enqueued on `stream`; no call synchronises the stream.
+ *   - Argument errors are reported before anything is launched. A launch
+ *     failure returns KDA_ERR_CUDA; the library does not clear sticky errors.
+ *   - Malformed cu_seqlens contents (only visible on the device) are not
+ *     trapped: the kernels skip the bad sequences and record KDA_ERR_DEVICE in
+ *     the workspace, readable with kda_workspace_status().
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, workspace too small */
+    KDA_ERR_UNSUPPORTED = 2, /* valid but not implemented: head dims, chunk, lb*chunk range */
+    KDA_ERR_CUDA = 3,        /* a CUDA launch or query failed */
+    KDA_ERR_DEVICE = 4       /* a device-side check failed (see kda_workspace_status) */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+typedef struct {
+    int64_t T;          /* tokens per sequence when cu_seqlens == NULL (then B sequences
+                           of T tokens each); total packed tokens when cu_seqlens != NULL */
+    int32_t B;          /* batch; must be 1 when cu_seqlens != NULL */
+    int32_t H;          /* heads */
+    int32_t dk, dv;     /* head dims: each 64 or 128 */
+    int32_t n_seqs;     /* with cu_seqlens: number of sequences (len(cu_seqlens) - 1);
+                           without: ignored (the library uses B) */
+    int64_t max_seqlen; /* with cu_seqlens: an upper bound on one sequence's length
+                           (0 = unknown, taken as T); used only for scheduling */
+    kda_dtype dtype;    /* dtype of q, k, v, g, beta and out */
+    float scale;        /* read-out scale; 0 selects 1/sqrt(dk) */
+    float g_lower_bound;/* lb: g is clamped to >= lb inside the library. Must satisfy
+                           lb < 0 and lb * chunk >= -80 so exp(-cumsum) stays finite */
+    int32_t chunk;      /* chunk length; 64 is the supported value */
+} kda_shape;
+
+/*
+ * Bytes of device scratch kda_chunk_fwd needs for this shape (a pure function
+ * of the shape fields). Returns 0 for an invalid shape.
+ */
+size_t kda_chunk_fwd_workspace_size(const kda_shape *shape);
+
+/*
+ * Chunked prefill ("Kimi K3 深度拆解", section 4.2: chunk-parallel with an
+ * inter-chunk recurrence; "3 分钟看懂 Kimi K3", Figure 3: bounded log decay).
+ *
+ *  q, k, g      [B*T, H, dk] (or [T, H, dk] packed)     dtype
+ *  v            [B*T, H, dv]                            dtype
+ *  beta         [B*T, H]                                dtype
+ *  initial_state[n, H, dk, dv] fp32, or NULL for zeros (n = B, or n_seqs)
+ *  cu_seqlens   int32 [n_seqs + 1] or NULL: 0 = c_0 <= c_1 <= ... <= c_n = T.
+ *               Sequences may be empty (their final state is their initial state).
+ *  out          [B*T, H, dv] dtype (written)
+ *  final_state  [n, H, dk, dv] fp32, or NULL to skip. May alias initial_state
+ *               (resume in place).
+ *  workspace    device scratch of >= kda_chunk_fwd_workspace_size(shape) bytes,
+ *               256-byte aligned, used only for the duration of the enqueued work.
+ *               Calls that share a workspace must be ordered on one stream.
+ */
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
+                         const void *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, void *out, float *final_state,
+                         const kda_shape *shape, void *workspace, size_t workspace_bytes,
+                         kda_stream_t stream);
+
+/*
+ * One decode step for N = shape->B sequences (one token each), updating the
+ * fp32 state in place ("Kimi K3 深度拆解", section 4.2: constant cost per token,
+ * O(d_k d_v) read-out independent of the position).
+ *
+ *  q, k, g     [N, H, dk] dtype      v [N, H, dv] dtype      beta [N, H] dtype
+ *  state       fp32 [n_slots, H, dk, dv], updated in place
+ *  state_slots int32 [N] indices into state (serving), or NULL for slot = n.
+ *              Slots must be distinct within one call and < n_slots; the
+ *              library does not check distinctness (duplicate slots race).
+ *  n_slots     number of state slots (>= N when state_slots is NULL)
+ *  out         [N, H, dv] dtype (written)
+ *  shape       B = N, T = 1; n_seqs, max_seqlen and chunk are ignored.
+ * Allocates nothing; safe to capture in a CUDA graph.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *g,
+                           const void *beta, float *state, const int32_t *state_slots,
+                           int64_t n_slots, void *out, const kda_shape *shape,
+                           kda_stream_t stream);
+
+/*
+ * Synchronises `stream` and reads the device-side status word a previous
+ * kda_chunk_fwd left in `workspace`: KDA_OK, or KDA_ERR_DEVICE when a
+ * malformed cu_seqlens (or an expired bounded wait) was detected. The word is
+ * cleared by the next kda_chunk_fwd on that workspace. Diagnostic only: the
+ * compute path never calls it.
+ */
+kda_status kda_workspace_status(const void *workspace, size_t workspace_bytes,
+                                kda_stream_t stream, int32_t *device_code);
+
+/* Static description of a status code. Never NULL. */
+const char *kda_status_string(kda_status status);
+
+/* Library version, e.g. "0.1.0". */
+const char *kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

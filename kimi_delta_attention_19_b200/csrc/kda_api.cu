@@ -1,0 +1,155 @@
+// kda_api.cu -- the C ABI (include/kda.h): argument validation, workspace
+// layout and dispatch to the kernels. Nothing here allocates device memory or
+// synchronises a stream (except kda_workspace_status, a diagnostic).
+#include <math.h>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dims_supported(int d) { return d == 64 || d == 128; }
+
+// Common shape checks; fills the resolved fields used by the kernels.
+kda_status check_shape(const kda_shape* s, bool prefill) {
+  if (s == nullptr) return KDA_ERR_INVALID_ARG;
+  if (s->dtype != KDA_F32 && s->dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (s->H <= 0 || s->B <= 0 || s->T < 0 || s->dk <= 0 || s->dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (!(s->scale >= 0.f) || !isfinite(s->scale)) return KDA_ERR_INVALID_ARG;
+  if (!isfinite(s->g_lower_bound) || !(s->g_lower_bound < 0.f)) return KDA_ERR_INVALID_ARG;
+  if (!dims_supported(s->dk) || !dims_supported(s->dv)) return KDA_ERR_UNSUPPORTED;
+  if (prefill) {
+    if (s->chunk != kChunk) return KDA_ERR_UNSUPPORTED;
+    // exp(-cumsum) over a chunk must stay finite in fp32 and bf16.
+    if ((double)s->g_lower_bound * kChunk < -80.0) return KDA_ERR_UNSUPPORTED;
+  }
+  return KDA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(const kda_shape* shape) {
+  if (check_shape(shape, true) != KDA_OK) return 0;
+  return align_up(kWorkspaceHeader, 256);
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, void* out, float* final_state,
+                         const kda_shape* shape, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream) {
+  kda_status st = check_shape(shape, true);
+  if (st != KDA_OK) return st;
+  const kda_shape& s = *shape;
+  int n_seqs;
+  int64_t T_total;
+  if (cu_seqlens != nullptr) {
+    if (s.B != 1 || s.n_seqs <= 0) return KDA_ERR_INVALID_ARG;
+    n_seqs = s.n_seqs;
+    T_total = s.T;
+  } else {
+    n_seqs = s.B;
+    T_total = s.T * (int64_t)s.B;
+  }
+  if (s.max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+  const void* tensors[] = {q, k, v, g, beta, out};
+  for (const void* p : tensors) {
+    if (T_total > 0 && p == nullptr) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(initial_state) || !aligned16(final_state) || !aligned16(cu_seqlens))
+    return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return KDA_ERR_INVALID_ARG;
+  const size_t need = kda_chunk_fwd_workspace_size(shape);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return KDA_ERR_INVALID_ARG;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kWorkspaceHeader, cs) != cudaSuccess) return KDA_ERR_CUDA;
+
+  PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+  a.s0 = initial_state;
+  a.cu = cu_seqlens;
+  a.out = out;
+  a.sT = final_state;
+  a.status = static_cast<int32_t*>(workspace);
+  a.ws = static_cast<unsigned char*>(workspace);
+  a.ws_bytes = workspace_bytes;
+  a.T = s.T;
+  a.T_total = T_total;
+  a.max_len = (cu_seqlens && s.max_seqlen > 0) ? s.max_seqlen : s.T;
+  a.n_seqs = n_seqs;
+  a.H = s.H; a.dk = s.dk; a.dv = s.dv;
+  a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
+  a.lb = s.g_lower_bound;
+
+  cudaError_t e = launch_prefill_simt(a, s.dtype, cs);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* g,
+                           const void* beta, float* state, const int32_t* state_slots,
+                           int64_t n_slots, void* out, const kda_shape* shape,
+                           kda_stream_t stream) {
+  kda_status st = check_shape(shape, false);
+  if (st != KDA_OK) return st;
+  const kda_shape& s = *shape;
+  if (s.T != 1) return KDA_ERR_INVALID_ARG;
+  if (n_slots <= 0 || (state_slots == nullptr && n_slots < s.B)) return KDA_ERR_INVALID_ARG;
+  const void* tensors[] = {q, k, v, g, beta, out, state};
+  for (const void* p : tensors)
+    if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if (state_slots != nullptr && (reinterpret_cast<uintptr_t>(state_slots) & 3u))
+    return KDA_ERR_INVALID_ARG;
+
+  DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+  a.state = state;
+  a.slots = state_slots;
+  a.n_slots = n_slots;
+  a.out = out;
+  a.N = s.B; a.H = s.H; a.dk = s.dk; a.dv = s.dv;
+  a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
+  a.lb = s.g_lower_bound;
+  cudaError_t e = launch_decode(a, s.dtype, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
+                                kda_stream_t stream, int32_t* device_code) {
+  if (workspace == nullptr || workspace_bytes < sizeof(int32_t)) return KDA_ERR_INVALID_ARG;
+  int32_t code = 0;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&code, workspace, sizeof code, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return KDA_ERR_CUDA;
+  if (device_code) *device_code = code;
+  return code == kDevOk ? KDA_OK : KDA_ERR_DEVICE;
+}
+
+const char* kda_status_string(kda_status status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported shape or parameter";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA launch or query failed";
+    case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: device-side check failed";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+const char* kda_version(void) { return "0.1.0"; }
+
+}  // extern "C"

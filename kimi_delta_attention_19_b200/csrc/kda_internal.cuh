@@ -1,0 +1,102 @@
+// kda_internal.cuh -- declarations shared by the library's translation units.
+// Not part of the public ABI (that is include/kda.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+constexpr int kChunk = 64;          // chunk length C of the chunked form
+constexpr int kWorkspaceHeader = 256;  // bytes: status word + scheduler counters
+
+// Device status word values (first int32 of the workspace).
+constexpr int32_t kDevOk = 0;
+constexpr int32_t kDevBadSeqlens = 1;   // cu_seqlens not monotone / out of [0, T]
+constexpr int32_t kDevWaitTimeout = 2;  // a bounded wait on another CTA gave up
+
+// Everything a prefill launch needs, resolved on the host.
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* beta;
+  const float* s0;          // [n, H, dk, dv] or null
+  const int32_t* cu;        // [n+1] or null (then sequences are [b*T, (b+1)*T))
+  void* out;                // [T_total, H, dv]
+  float* sT;                // [n, H, dk, dv] or null
+  int32_t* status;          // device status word (workspace header)
+  unsigned char* ws;        // workspace base
+  size_t ws_bytes;
+  int64_t T;                // tokens per sequence (no cu) or total tokens (cu)
+  int64_t T_total;          // total packed tokens
+  int64_t max_len;          // bound on one sequence's length
+  int n_seqs;
+  int H, dk, dv;
+  float scale;
+  float lb;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* beta;
+  float* state;
+  const int32_t* slots;
+  int64_t n_slots;
+  void* out;
+  int N, H, dk, dv;
+  float scale;
+  float lb;
+};
+
+// Sequence bounds [t0, t1) of sequence s; false (and status set) when the
+// device-visible cu_seqlens entry is malformed.
+__device__ __forceinline__ bool seq_bounds(const PrefillArgs& a, int s, int64_t& t0,
+                                           int64_t& t1) {
+  if (a.cu == nullptr) {
+    t0 = (int64_t)s * a.T;
+    t1 = t0 + a.T;
+    return true;
+  }
+  const int64_t c0 = a.cu[s], c1 = a.cu[s + 1];
+  const bool ok = (c0 >= 0) && (c1 >= c0) && (c1 <= a.T_total) &&
+                  (s != 0 || c0 == 0) && (s + 1 != a.n_seqs || c1 == a.T_total);
+  if (!ok) {
+    atomicExch(a.status, kDevBadSeqlens);
+    return false;
+  }
+  t0 = c0;
+  t1 = c1;
+  return true;
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_in(const T* p);
+template <>
+__device__ __forceinline__ float ld_in<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld_in<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
+}
+
+template <typename T>
+__device__ __forceinline__ void st_out(T* p, float x);
+template <>
+__device__ __forceinline__ void st_out<float>(float* p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16* p, float x) {
+  *p = __float2bfloat16_rn(x);
+}
+
+// Launchers (return the cudaGetLastError() of their launches).
+cudaError_t launch_prefill_simt(const PrefillArgs& a, kda_dtype dtype, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t st);
+
+}  // namespace kda

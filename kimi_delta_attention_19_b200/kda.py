@@ -1,0 +1,173 @@
+"""Thin Python binding of the KDA C ABI (include/kda.h).
+
+Argument marshalling only: every step of the computation runs in libkda.so's
+CUDA kernels. PyTorch supplies device memory and the current stream. There is
+no CPU or PyTorch fallback: if libkda.so is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE = range(5)
+KDA_F32, KDA_BF16 = 0, 1
+CHUNK = 64
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.kda_status_string(status).decode()}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("B", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("n_seqs", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int64), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float), ("g_lower_bound", ctypes.c_float),
+                ("chunk", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m kimi_delta_attention_19_b200.build` (no fallback exists)")
+    L = ctypes.CDLL(LIB_PATH)
+    p, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    L.kda_chunk_fwd_workspace_size.restype = sz
+    L.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
+    L.kda_chunk_fwd.restype = st
+    L.kda_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p, sz, p]
+    L.kda_decode_step.restype = st
+    L.kda_decode_step.argtypes = [p, p, p, p, p, p, p, ctypes.c_int64, p,
+                                  ctypes.POINTER(Shape), p]
+    L.kda_workspace_status.restype = st
+    L.kda_workspace_status.argtypes = [p, sz, p, ctypes.POINTER(ctypes.c_int32)]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_status_string.argtypes = [st]
+    L.kda_version.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    return L
+
+
+lib = _load()
+
+EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+            "kda_workspace_status", "kda_status_string", "kda_version")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; KDA takes float32 or bfloat16")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_shape(T: int, H: int, dk: int, dv: int, dtype: torch.dtype, *, B: int = 1,
+               n_seqs: int = 0, max_seqlen: int = 0, scale: float | None = None,
+               lb: float = -1.0, chunk: int = CHUNK) -> Shape:
+    code = KDA_F32 if dtype == torch.float32 else KDA_BF16
+    return Shape(T=T, B=B, H=H, dk=dk, dv=dv, n_seqs=n_seqs, max_seqlen=max_seqlen, dtype=code,
+                 scale=0.0 if scale is None else float(scale), g_lower_bound=float(lb),
+                 chunk=chunk)
+
+
+def workspace_size(shape: Shape) -> int:
+    return int(lib.kda_chunk_fwd_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: Shape, device) -> torch.Tensor:
+    n = workspace_size(shape)
+    if n == 0:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_workspace_size")
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+              beta: torch.Tensor, *, initial_state: torch.Tensor | None = None,
+              cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+              scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
+              final_state: torch.Tensor | None = None, output_final_state: bool = True,
+              workspace: torch.Tensor | None = None, stream=None):
+    """Chunked prefill. q, k, g: [T, H, dk] (or [B, T, H, dk]); v: [..., dv]; beta: [..., H].
+
+    Returns (out, final_state). final_state is fp32 [n, H, dk, dv] (None if not requested).
+    """
+    batched = q.dim() == 4
+    if batched:
+        B, T, H, dk = q.shape
+    else:
+        B = 1
+        T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        assert not batched, "cu_seqlens takes packed [T, H, d] inputs"
+        n = cu_seqlens.numel() - 1
+    else:
+        n = B
+    shape = make_shape(T, H, dk, dv, q.dtype, B=B, n_seqs=n if cu_seqlens is not None else 0,
+                       max_seqlen=max_seqlen, scale=scale, lb=lb)
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(n, H, dk, dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                           _ptr(cu_seqlens), _ptr(out), _ptr(final_state), ctypes.byref(shape),
+                           _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return out, final_state
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                beta: torch.Tensor, state: torch.Tensor, *, state_slots: torch.Tensor | None = None,
+                scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """One token per sequence: q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H].
+
+    Updates fp32 `state` [n_slots, H, dk, dv] in place; returns out [N, H, dv].
+    """
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    shape = make_shape(1, H, dk, dv, q.dtype, B=N, scale=scale, lb=lb)
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                             _ptr(state_slots), state.shape[0], _ptr(out), ctypes.byref(shape),
+                             _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step")
+    return out
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:
+    """(status, device code) left in `workspace` by the last kda_chunk_fwd (synchronises)."""
+    code = ctypes.c_int32(0)
+    rc = lib.kda_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream),
+                                  ctypes.byref(code))
+    return rc, code.value
+
+
+def default_scale(dk: int) -> float:
+    return 1.0 / math.sqrt(dk)

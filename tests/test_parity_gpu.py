@@ -1,0 +1,256 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element, at small sizes spanning several chunks
+and a ragged tail, and at the full workload sizes on sampled rows plus the full
+final states."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from kimi_delta_attention_19_b200.inputs import (WORKLOADS, decode_state, decode_tokens,
+                                                  make_inputs, workload_inputs)
+from oracle import kda_oracle as ko
+from tests.parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def kda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from kimi_delta_attention_19_b200 import kda as k
+    return k
+
+
+def _to(x, dev=DEV):
+    return None if x is None else x.to(dev)
+
+
+def _run_gpu(kda, x, **kw):
+    out, fin = kda.chunk_fwd(_to(x.q), _to(x.k), _to(x.v), _to(x.g), _to(x.beta),
+                             initial_state=_to(x.initial_state), cu_seqlens=_to(x.cu_seqlens),
+                             **kw)
+    torch.cuda.synchronize()
+    return out, fin
+
+
+def _run_oracle(x, out_rows=None, lb=-1.0):
+    cu = None if x.cu_seqlens is None else x.cu_seqlens.cpu().tolist()
+    return ko.recurrent(x.q.cpu(), x.k.cpu(), x.v.cpu(), x.g.cpu(), x.beta.cpu(),
+                        cu_seqlens=cu, initial_state=None if x.initial_state is None
+                        else x.initial_state.cpu(), out_rows=out_rows, lb=lb)
+
+
+def _check_full(kda, x, dtype, what, lb=-1.0):
+    out, fin = _run_gpu(kda, x, lb=lb)
+    ro, rs = _run_oracle(x, lb=lb)
+    assert_close(out, ro, dtype, f"{what} out")
+    assert_close(fin, rs, dtype, f"{what} final_state")
+
+
+# ---------------------------------------------------------------- small cases
+def test_fp32_h2_t256_d64(kda):
+    w = WORKLOADS["fp32_h2_t256_d64"]
+    _check_full(kda, workload_inputs(w), torch.float32, w.name)
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_lengths(kda, T, d):
+    x = make_inputs(T, H=3, dk=d, dv=d, dtype=torch.bfloat16, seed=100 + T, state_std=0.02)
+    _check_full(kda, x, torch.bfloat16, f"bf16 T={T} d={d}")
+
+
+@pytest.mark.parametrize("T", [1, 65, 300])
+def test_fp32_lengths(kda, T):
+    x = make_inputs(T, H=2, dk=128, dv=128, dtype=torch.float32, seed=200 + T, state_std=0.02)
+    _check_full(kda, x, torch.float32, f"fp32 T={T}")
+
+
+def test_mixed_head_dims(kda):
+    x = make_inputs(150, H=2, dk=128, dv=64, dtype=torch.bfloat16, seed=7, state_std=0.02)
+    _check_full(kda, x, torch.bfloat16, "dk=128 dv=64")
+    x = make_inputs(150, H=2, dk=64, dv=128, dtype=torch.float32, seed=8, state_std=0.02)
+    _check_full(kda, x, torch.float32, "dk=64 dv=128")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_varlen_ragged_and_empty(kda, dtype):
+    x = make_inputs(None, H=4, dk=128, dv=128, dtype=dtype, seed=9,
+                    lengths=[1, 0, 100, 64, 130, 0, 257], state_std=0.02)
+    _check_full(kda, x, dtype, f"varlen {dtype}")
+
+
+def test_batched_without_cu_seqlens(kda):
+    x = make_inputs(96, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=10, batch=3,
+                    state_std=0.02)
+    q, k, v, g, b = (t.to(DEV).view(3, 96, *t.shape[1:]) for t in (x.q, x.k, x.v, x.g, x.beta))
+    out, fin = kda.chunk_fwd(q, k, v, g, b, initial_state=x.initial_state.to(DEV))
+    torch.cuda.synchronize()
+    ro, rs = _run_oracle(x)
+    assert_close(out.view(-1, 2, 128), ro, torch.bfloat16, "batched out")
+    assert_close(fin, rs, torch.bfloat16, "batched final_state")
+
+
+def test_zero_initial_state_and_no_final(kda):
+    x = make_inputs(130, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=11, state_std=None)
+    out, fin = kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV),
+                             x.beta.to(DEV), output_final_state=False)
+    torch.cuda.synchronize()
+    assert fin is None
+    ro, _ = _run_oracle(x)
+    assert_close(out, ro, torch.bfloat16, "no initial state")
+
+
+def test_decay_clamp_active(kda):
+    """g ~ -3*sigmoid goes below lb = -1; the library clamps exactly as the oracle."""
+    x = make_inputs(200, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=12, g_scale=3.0,
+                    state_std=0.02)
+    assert float(x.g.float().min()) < -1.0
+    _check_full(kda, x, torch.bfloat16, "clamp active")
+
+
+def test_resume_split_and_alias(kda):
+    """Prefill [0,T) == prefill [0,m) then [m,T) from its final state, in place."""
+    x = make_inputs(333, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=13, state_std=0.02)
+    ro, rs = _run_oracle(x)
+    m = 130
+    state = x.initial_state.to(DEV).clone()
+    o1, _ = kda.chunk_fwd(x.q[:m].to(DEV), x.k[:m].to(DEV), x.v[:m].to(DEV), x.g[:m].to(DEV),
+                          x.beta[:m].to(DEV), initial_state=state, final_state=state)
+    o2, _ = kda.chunk_fwd(x.q[m:].to(DEV), x.k[m:].to(DEV), x.v[m:].to(DEV), x.g[m:].to(DEV),
+                          x.beta[m:].to(DEV), initial_state=state, final_state=state)
+    torch.cuda.synchronize()
+    assert_close(torch.cat([o1, o2]), ro, torch.bfloat16, "split out")
+    assert_close(state, rs, torch.bfloat16, "split final_state")
+
+
+def test_bad_cu_seqlens_reports_without_trap(kda):
+    x = make_inputs(200, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=14, state_std=None)
+    cu = torch.tensor([0, 100, 50, 200], dtype=torch.int32, device=DEV)
+    shape = kda.make_shape(200, 2, 128, 128, torch.bfloat16, n_seqs=3)
+    ws = kda.alloc_workspace(shape, DEV)
+    kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV), x.beta.to(DEV),
+                  cu_seqlens=cu, workspace=ws)
+    rc, code = kda.workspace_status(ws)
+    assert rc == kda.KDA_ERR_DEVICE and code != 0
+    # a good call on the same workspace clears the word
+    kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV), x.beta.to(DEV),
+                  workspace=ws)
+    assert kda.workspace_status(ws) == (kda.KDA_OK, 0)
+
+
+# ------------------------------------------------------------------- decode
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_matches_oracle(kda, dtype):
+    N, H, d, steps = 5, 3, 128, 4
+    tok = decode_tokens(steps, N, H, d, d, dtype=dtype, seed=21)
+    S0 = decode_state(N, H, d, d, seed=22)
+    state = S0.to(DEV).clone()
+    outs = []
+    for t in range(steps):
+        outs.append(kda.decode_step(tok.q[t].to(DEV), tok.k[t].to(DEV), tok.v[t].to(DEV),
+                                    tok.g[t].to(DEV), tok.beta[t].to(DEV), state))
+    torch.cuda.synchronize()
+    # oracle: sequence n's tokens are step-major rows n, N+n, ...; pack per sequence
+    perm = [t * N + n for n in range(N) for t in range(steps)]
+
+    def pack(a):
+        return a.reshape(steps * N, *a.shape[2:])[perm]
+    cu = [n * steps for n in range(N + 1)]
+    ro, rs = ko.recurrent(pack(tok.q), pack(tok.k), pack(tok.v), pack(tok.g), pack(tok.beta),
+                          cu_seqlens=cu, initial_state=S0)
+    got = torch.stack(outs).reshape(steps * N, H, d)[perm]
+    assert_close(got, ro, dtype, "decode out")
+    assert_close(state, rs, dtype, "decode state")
+
+
+def test_decode_state_slots(kda):
+    N, H, d = 6, 2, 128
+    tok = decode_tokens(1, N, H, d, d, seed=31)
+    S0 = decode_state(10, H, d, d, seed=32)
+    slots = torch.tensor([7, 0, 3, 9, 2, 5], dtype=torch.int32)
+    state = S0.to(DEV).clone()
+    out = kda.decode_step(tok.q[0].to(DEV), tok.k[0].to(DEV), tok.v[0].to(DEV), tok.g[0].to(DEV),
+                          tok.beta[0].to(DEV), state, state_slots=slots.to(DEV))
+    torch.cuda.synchronize()
+    ro, rs = ko.recurrent(tok.q[0], tok.k[0], tok.v[0], tok.g[0], tok.beta[0],
+                          cu_seqlens=list(range(N + 1)), initial_state=S0[slots.long()])
+    assert_close(out, ro, torch.bfloat16, "slots out")
+    assert_close(state[slots.long()], rs, torch.bfloat16, "slots state")
+    untouched = [i for i in range(10) if i not in slots.tolist()]
+    assert torch.equal(state[untouched].cpu(), S0[untouched])
+
+
+def test_decode_equals_prefill_one_token(kda):
+    x = make_inputs(None, H=4, dk=128, dv=128, dtype=torch.bfloat16, seed=41,
+                    lengths=[1] * 6, state_std=0.02)
+    out_p, fin_p = _run_gpu(kda, x)
+    state = x.initial_state.to(DEV).clone()
+    out_d = kda.decode_step(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV),
+                            x.beta.to(DEV), state)
+    torch.cuda.synchronize()
+    assert_close(out_d, out_p.float(), torch.bfloat16, "decode vs prefill out")
+    assert_close(state, fin_p, torch.bfloat16, "decode vs prefill state")
+
+
+# ------------------------------------------------------ full workload sizes
+def _device_inputs(name, seed=0):
+    return workload_inputs(WORKLOADS[name], seed=seed, device=DEV)
+
+
+def test_full_bf16_h32_t8192_d128(kda):
+    x = _device_inputs("bf16_h32_t8192_d128")
+    _check_full(kda, x, torch.bfloat16, "bf16_h32_t8192_d128")
+
+
+def _sampled_rows(T_total, n=2048, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([rng.choice(T_total, min(n, T_total), replace=False),
+                                     [0, T_total - 1]]))
+    return rows
+
+
+def test_full_varlen8_h32_d128(kda):
+    x = _device_inputs("varlen8_h32_d128")
+    out, fin = _run_gpu(kda, x, max_seqlen=max(x.lengths))
+    rows = _sampled_rows(x.q.shape[0])
+    ro, rs = _run_oracle(x, out_rows=rows)
+    assert_close(out[torch.as_tensor(rows, device=DEV)], ro, torch.bfloat16, "varlen out (sampled)")
+    assert_close(fin, rs, torch.bfloat16, "varlen final_state")
+
+
+@pytest.mark.timeout(3600)
+def test_full_bf16_h16_t1m_d128(kda):
+    x = _device_inputs("bf16_h16_t1m_d128")
+    out, fin = _run_gpu(kda, x)
+    T = x.q.shape[0]
+    rows = np.arange(0, T, 509)  # strided token samples across the whole sequence
+    rows = np.unique(np.concatenate([rows, [T - 1]]))
+    ro, rs = _run_oracle(x, out_rows=rows)
+    assert_close(out[torch.as_tensor(rows, device=DEV)], ro, torch.bfloat16, "1M out (strided)")
+    assert_close(fin, rs, torch.bfloat16, "1M final_state")
+
+
+def test_full_decode_n256_h32_d128(kda):
+    """The served configuration, chained over 64 steps, against the oracle."""
+    N, H, d, steps = 256, 32, 128, 64
+    S0 = decode_state(N, H, d, d, seed=0, device=DEV)
+    tok = decode_tokens(steps, N, H, d, d, seed=1, device=DEV)
+    state = S0.clone()
+    outs = [kda.decode_step(tok.q[t], tok.k[t], tok.v[t], tok.g[t], tok.beta[t], state)
+            for t in range(steps)]
+    torch.cuda.synchronize()
+    perm = torch.tensor([t * N + n for n in range(N) for t in range(steps)])
+
+    def pack(a):
+        return a.reshape(steps * N, *a.shape[2:])[perm.to(a.device)].cpu()
+    ro, rs = ko.recurrent(pack(tok.q), pack(tok.k), pack(tok.v), pack(tok.g), pack(tok.beta),
+                          cu_seqlens=[n * steps for n in range(N + 1)], initial_state=S0.cpu())
+    got = torch.stack(outs).reshape(steps * N, H, d)[perm.to(DEV)]
+    assert_close(got, ro, torch.bfloat16, "decode full out")
+    assert_close(state, rs, torch.bfloat16, "decode full state")
