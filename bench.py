@@ -55,56 +55,55 @@ def load_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle-reason sampling (NVML, read-only) during the timed region."""
 
-    def __init__(self, index: int):
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index: int, period_s: float = 0.002):
         self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:  # noqa: BLE001 -- no NVML: no clock record
+            return
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for name, bit in self.REASONS.items():
+                        if mask & bit:
+                            self.reasons.add(name)
+                except Exception:  # noqa: BLE001
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self) -> dict | None:
-        if self.proc is None:
+        if self._thread is None:
             return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.fh.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = max(mx, float(parts[2]))
-                except ValueError:
-                    continue
-                for nm, val in zip(names, parts[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(nm)
-        if not sm:
+        self._stop.set()
+        self._thread.join()
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def dist_setup(n_gpus: int):
@@ -272,32 +271,40 @@ def kda_launches_per_step(kda, shape) -> int:
     return 1
 
 
-def cpu_oracle_rate(tokens: int, seed: int = 0) -> dict:
-    """Time the fp64 oracle on the first `tokens` tokens of the prefill workload."""
+def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: int = 0) -> dict:
+    """Time the fp64 oracle on the prefill workload's tokens (all heads), repeating
+    whole passes until at least `min_seconds` of CPU work has been timed."""
     from kimi_delta_attention_19_b200.inputs import WORKLOADS, workload_inputs
     from oracle import kda_oracle as ko
     w = WORKLOADS[PREFILL]
     x = workload_inputs(w, seed=seed, device="cpu")
+    tokens = w.T if tokens is None else min(tokens, w.T)
     sl = slice(0, tokens)
     threads = min(os.cpu_count() or 1, w.H)
     ko.load()
-    t0 = time.perf_counter()
-    ko.recurrent(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl],
-                 initial_state=x.initial_state, n_threads=threads)
-    dt = time.perf_counter() - t0
-    return {"value": round(tokens / dt, 2), "unit": "tokens/s", "cores": threads,
+    done, dt = 0, 0.0
+    while dt < min_seconds or done == 0:
+        t0 = time.perf_counter()
+        ko.recurrent(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl],
+                     initial_state=x.initial_state, n_threads=threads)
+        dt += time.perf_counter() - t0
+        done += tokens
+    return {"value": round(done / dt, 2), "unit": "tokens/s", "cores": threads,
             "kind": "oracle", "seconds": round(dt, 3),
-            "sample": f"first {tokens} of {w.T} tokens of {PREFILL} (all {w.H} heads), "
-                      f"fp64 token-by-token recurrence, {threads} threads"}
+            "sample": f"{done // tokens} pass(es) over {tokens} of {w.T} tokens of {PREFILL} "
+                      f"(all {w.H} heads), fp64 token-by-token recurrence, {threads} threads"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--cpu-tokens", type=int, default=2048,
+                    help="tokens per reference-arm step (bounded oracle sample)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="minimum timed oracle work for the cpu_baseline object")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = {"workload": PREFILL, "model": "KDA layer (synthetic, no weights)", "global_batch": 1,
@@ -312,10 +319,9 @@ def main():
             return
         cfg["parallelism"] = f"oracle on host cores (N={world} requested; rank 0 only)"
         rates = []
-        for _ in range(args.warmup // 3):
-            cpu_oracle_rate(args.cpu_tokens // 4)
+        cpu_oracle_rate(min_seconds=0.0, tokens=256)  # warm-up (library load, page-in)
         for _ in range(args.steps):
-            rates.append(cpu_oracle_rate(args.cpu_tokens))
+            rates.append(cpu_oracle_rate(min_seconds=0.0, tokens=args.cpu_tokens))
         v = statistics.median(r["value"] for r in rates)
         cb = dict(rates[-1])
         cb["value"] = v
@@ -334,7 +340,7 @@ def main():
     r = bench_ours(args, world, rank, local)
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_oracle_rate(args.cpu_tokens)
+        cpu = cpu_oracle_rate(min_seconds=args.cpu_seconds)
     if rank == 0:
         line = {
             "metric": metric, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
