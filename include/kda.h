@@ -101,6 +101,34 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                          kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd without a workspace argument, for callers that cannot call
+ * cudaMalloc: code running while a CUDA graph is being captured (allocation is
+ * not capturable), plugin hosts that hand a library no scratch buffer, and
+ * serving loops where an allocation would synchronise the device. The pages
+ * describe no such entry point; it exists only for these callers.
+ *
+ * Arguments and results are those of kda_chunk_fwd; the caller still passes
+ * every input and output. The scratch comes from one fixed device array of
+ * KDA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. It allocates nothing.
+ *  - Returns KDA_ERR_UNSUPPORTED when kda_chunk_fwd_workspace_size(shape)
+ *    exceeds KDA_NOALLOC_SCRATCH_BYTES (use kda_chunk_fwd with a workspace).
+ *  - The first call on a device looks up that device's copy of the array
+ *    (cudaGetSymbolAddress, once per device, for the current device); make
+ *    that first call before any stream capture. The current device must be the
+ *    device of `stream`.
+ *  - All calls on a device share the array and it keeps the previous call's
+ *    contents (the prefill clears what must start at zero). Calls whose work
+ *    overlaps on the GPU, e.g. on unordered streams, race on the array.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
+                                 const void *beta, const float *initial_state,
+                                 const int32_t *cu_seqlens, void *out, float *final_state,
+                                 const kda_shape *shape, kda_stream_t stream);
+
+/*
  * One decode step for N = shape->B sequences (one token each), updating the
  * fp32 state in place ("Kimi K3 深度拆解", section 4.2: constant cost per token,
  * O(d_k d_v) read-out independent of the position).

@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
     L.kda_chunk_fwd.restype = st
     L.kda_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p, sz, p]
+    L.kda_chunk_fwd_noalloc.restype = st
+    L.kda_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p]
     L.kda_decode_step.restype = st
     L.kda_decode_step.argtypes = [p, p, p, p, p, p, p, ctypes.c_int64, p,
                                   ctypes.POINTER(Shape), p]
@@ -59,7 +61,8 @@ def _load() -> ctypes.CDLL:
 
 lib = _load()
 
-EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
+            "kda_decode_step",
             "kda_workspace_status", "kda_status_string", "kda_version")
 
 
@@ -137,6 +140,37 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
                            _ptr(workspace), workspace.numel(), _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
+    return out, final_state
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                      beta: torch.Tensor, *, out: torch.Tensor, final_state: torch.Tensor | None,
+                      initial_state: torch.Tensor | None = None,
+                      cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+                      scale: float | None = None, lb: float = -1.0, stream=None):
+    """kda_chunk_fwd_noalloc: the prefill with the library's fixed scratch array.
+
+    For callers that cannot allocate device memory, so `out` (and `final_state`,
+    if wanted) must be passed in. Same layouts as chunk_fwd.
+    """
+    batched = q.dim() == 4
+    if batched:
+        B, T, H, dk = q.shape
+    else:
+        B = 1
+        T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = cu_seqlens.numel() - 1 if cu_seqlens is not None else 0
+    shape = make_shape(T, H, dk, dv, q.dtype, B=B, n_seqs=n, max_seqlen=max_seqlen,
+                       scale=scale, lb=lb)
+    rc = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                   _ptr(final_state), ctypes.byref(shape), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_noalloc")
     return out, final_state
 
 
