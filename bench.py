@@ -267,8 +267,22 @@ def bench_ours(args, world, rank, local):
 
 
 def kda_launches_per_step(kda, shape) -> int:
-    """Kernels this library enqueues per kda_chunk_fwd for `shape` (memset excluded)."""
-    return 1
+    """Kernels one kda_chunk_fwd enqueues for `shape` (the header memset excluded).
+
+    bf16 with d_k = d_v = 128 takes the tensor-core path: output pass, plus the
+    summary pass and the combine when the longest sequence spans several
+    segments; other shapes run one CUDA-core kernel. The segment rule is the
+    library's (tokens per segment = 64 * next power of two of
+    ceil(H * (ceil(T/64) + n) / 148), at least 8 chunks)."""
+    T_total = shape.T * (1 if shape.n_seqs > 0 else shape.B)
+    n = shape.n_seqs if shape.n_seqs > 0 else shape.B
+    if not (shape.dtype == kda.KDA_BF16 and shape.dk == 128 and shape.dv == 128 and T_total > 0):
+        return 1
+    chunks = -(-T_total // 64) + n
+    per_sm = max(8, -(-shape.H * chunks // 148))
+    seg = 64 * (1 << (per_sm - 1).bit_length())
+    max_len = shape.max_seqlen if (shape.n_seqs > 0 and shape.max_seqlen > 0) else shape.T
+    return 3 if -(-max_len // seg) > 1 else 1
 
 
 def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: int = 0) -> dict:

@@ -60,10 +60,12 @@ typedef struct {
     int32_t B;          /* batch; must be 1 when cu_seqlens != NULL */
     int32_t H;          /* heads */
     int32_t dk, dv;     /* head dims: each 64 or 128 */
-    int32_t n_seqs;     /* with cu_seqlens: number of sequences (len(cu_seqlens) - 1);
-                           without: ignored (the library uses B) */
-    int64_t max_seqlen; /* with cu_seqlens: an upper bound on one sequence's length
-                           (0 = unknown, taken as T); used only for scheduling */
+    int32_t n_seqs;     /* with cu_seqlens: number of sequences (len(cu_seqlens) - 1, >= 1);
+                           without cu_seqlens: must be 0 (the library uses B) */
+    int64_t max_seqlen; /* with cu_seqlens: an upper bound on every sequence's length
+                           (0 = unknown, taken as T). It sizes the workspace and the
+                           schedule; a sequence longer than it is skipped and reported
+                           as KDA_ERR_DEVICE. Ignored without cu_seqlens. */
     kda_dtype dtype;    /* dtype of q, k, v, g, beta and out */
     float scale;        /* read-out scale; 0 selects 1/sqrt(dk) */
     float g_lower_bound;/* lb: g is clamped to >= lb inside the library. Must satisfy

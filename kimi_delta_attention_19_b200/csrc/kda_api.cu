@@ -30,6 +30,19 @@ kda_status check_shape(const kda_shape* s, bool prefill) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Packed-token view of a shape: cu_seqlens mode when n_seqs > 0, batch mode otherwise.
+void resolve(const kda_shape& s, int64_t& T_total, int& n_seqs, int64_t& max_len) {
+  if (s.n_seqs > 0) {
+    T_total = s.T;
+    n_seqs = s.n_seqs;
+    max_len = s.max_seqlen > 0 ? s.max_seqlen : s.T;
+  } else {
+    T_total = s.T * static_cast<int64_t>(s.B);
+    n_seqs = s.B;
+    max_len = s.T;
+  }
+}
+
 }  // namespace
 }  // namespace kda
 
@@ -39,6 +52,12 @@ extern "C" {
 
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape) {
   if (check_shape(shape, true) != KDA_OK) return 0;
+  if (shape->n_seqs < 0 || shape->max_seqlen < 0 || (shape->n_seqs > 0 && shape->B != 1)) return 0;
+  int64_t T_total, max_len;
+  int n_seqs;
+  resolve(*shape, T_total, n_seqs, max_len);
+  if (tc_path_applies(*shape, T_total))
+    return align_up(tc_plan(T_total, n_seqs, shape->H, max_len).ws_bytes, 256);
   return align_up(kWorkspaceHeader, 256);
 }
 
@@ -50,17 +69,13 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   kda_status st = check_shape(shape, true);
   if (st != KDA_OK) return st;
   const kda_shape& s = *shape;
+  // cu_seqlens mode needs B == 1 and n_seqs > 0; batch mode needs n_seqs == 0
+  if ((cu_seqlens != nullptr) != (s.n_seqs > 0)) return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens != nullptr && s.B != 1) return KDA_ERR_INVALID_ARG;
+  if (s.n_seqs < 0 || s.max_seqlen < 0) return KDA_ERR_INVALID_ARG;
   int n_seqs;
-  int64_t T_total;
-  if (cu_seqlens != nullptr) {
-    if (s.B != 1 || s.n_seqs <= 0) return KDA_ERR_INVALID_ARG;
-    n_seqs = s.n_seqs;
-    T_total = s.T;
-  } else {
-    n_seqs = s.B;
-    T_total = s.T * (int64_t)s.B;
-  }
-  if (s.max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+  int64_t T_total, max_len;
+  resolve(s, T_total, n_seqs, max_len);
   const void* tensors[] = {q, k, v, g, beta, out};
   for (const void* p : tensors) {
     if (T_total > 0 && p == nullptr) return KDA_ERR_INVALID_ARG;
@@ -89,13 +104,14 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   a.ws_bytes = workspace_bytes;
   a.T = s.T;
   a.T_total = T_total;
-  a.max_len = (cu_seqlens && s.max_seqlen > 0) ? s.max_seqlen : s.T;
+  a.max_len = max_len;
   a.n_seqs = n_seqs;
   a.H = s.H; a.dk = s.dk; a.dv = s.dv;
   a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
   a.lb = s.g_lower_bound;
 
-  cudaError_t e = launch_prefill_simt(a, s.dtype, cs);
+  cudaError_t e = tc_path_applies(s, T_total) ? launch_prefill_tc(a, cs)
+                                              : launch_prefill_simt(a, s.dtype, cs);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -95,8 +95,19 @@ __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16* p, float x)
   *p = __float2bfloat16_rn(x);
 }
 
+// Segment plan of the tensor-core prefill (a pure function of the shape).
+struct TcPlan {
+  int seg_tokens;   // tokens per segment (a multiple of the chunk length)
+  int max_segs;     // segments of the longest sequence
+  int64_t pairs;    // (sequence, head) pairs
+  size_t ws_bytes;  // workspace it needs, header included
+};
+TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len);
+bool tc_path_applies(const kda_shape& s, int64_t T_total);
+
 // Launchers (return the cudaGetLastError() of their launches).
 cudaError_t launch_prefill_simt(const PrefillArgs& a, kda_dtype dtype, cudaStream_t st);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t st);
 
 }  // namespace kda

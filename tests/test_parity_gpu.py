@@ -144,6 +144,43 @@ def test_bad_cu_seqlens_reports_without_trap(kda):
     assert kda.workspace_status(ws) == (kda.KDA_OK, 0)
 
 
+def test_tensor_core_segments(kda):
+    """Long sequences with few heads split into segments (summary, combine, output passes)."""
+    x = make_inputs(3000, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=15, state_std=0.02)
+    _check_full(kda, x, torch.bfloat16, "segments T=3000")
+    x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=16,
+                    lengths=[5000, 1, 1200, 0, 2500, 64], state_std=0.02)
+    out, fin = _run_gpu(kda, x, max_seqlen=5000)
+    ro, rs = _run_oracle(x)
+    assert_close(out, ro, torch.bfloat16, "varlen segments out")
+    assert_close(fin, rs, torch.bfloat16, "varlen segments final_state")
+
+
+def test_tensor_core_segments_resume_in_place(kda):
+    """final_state aliasing initial_state with several segments per sequence."""
+    x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=17,
+                    lengths=[2600, 700], state_std=0.02)
+    ro, rs = _run_oracle(x)
+    state = x.initial_state.to(DEV).clone()
+    out, _ = kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV), x.beta.to(DEV),
+                           initial_state=state, final_state=state,
+                           cu_seqlens=x.cu_seqlens.to(DEV), max_seqlen=2600)
+    torch.cuda.synchronize()
+    assert_close(out, ro, torch.bfloat16, "alias out")
+    assert_close(state, rs, torch.bfloat16, "alias final_state")
+
+
+def test_max_seqlen_too_small_reports_without_trap(kda):
+    x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=18,
+                    lengths=[4000, 100], state_std=None)
+    shape = kda.make_shape(4100, 2, 128, 128, torch.bfloat16, n_seqs=2, max_seqlen=600)
+    ws = kda.alloc_workspace(shape, DEV)
+    kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV), x.beta.to(DEV),
+                  cu_seqlens=x.cu_seqlens.to(DEV), max_seqlen=600, workspace=ws)
+    rc, code = kda.workspace_status(ws)
+    assert rc == kda.KDA_ERR_DEVICE and code != 0
+
+
 # ------------------------------------------------------------------- decode
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_decode_matches_oracle(kda, dtype):

@@ -65,17 +65,18 @@ def test_noalloc_fp32_inputs(kda):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(kda):
     big = None
-    for T, H in ((1 << 20, 16), (1 << 22, 64), (1 << 24, 128)):
-        sh = kda.make_shape(T, H, 128, 128, torch.bfloat16)
+    # packed sequences without a max_seqlen bound: scratch is sized for the worst case
+    for T, H, n in ((1 << 19, 32, 64), (1 << 20, 16, 1), (1 << 22, 64, 0)):
+        sh = kda.make_shape(T, H, 128, 128, torch.bfloat16, n_seqs=n)
         if kda.workspace_size(sh) > kda.NOALLOC_SCRATCH_BYTES:
-            big = (T, H)
+            big = (T, H, n)
             break
     if big is None:
         pytest.skip("no supported shape needs more scratch than the fixed array")
-    T, H = big
+    T, H, n = big
     x = torch.empty(16, device=DEV)  # never read: the size check comes first
     with pytest.raises(kda.KdaError) as e:
-        lib_shape = kda.make_shape(T, H, 128, 128, torch.bfloat16)
+        lib_shape = kda.make_shape(T, H, 128, 128, torch.bfloat16, n_seqs=n)
         import ctypes
         rc = kda.lib.kda_chunk_fwd_noalloc(*([ctypes.c_void_p(x.data_ptr())] * 5), None, None,
                                            ctypes.c_void_p(x.data_ptr()), None,
