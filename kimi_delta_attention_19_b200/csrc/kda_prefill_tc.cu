@@ -40,7 +40,7 @@ using namespace sm100;
 
 constexpr int C = kChunk;  // 64
 constexpr int D = 128;     // d_k = d_v on this path
-constexpr int NT = 256;
+constexpr int NT = 512;
 constexpr uint32_t K8 = 8192, K16 = 16384, K32 = 32768;
 constexpr int kTmemCols = 512;
 
@@ -81,10 +81,10 @@ struct Sm {
   static constexpr uint32_t SG = SK + K16;
   static constexpr uint32_t SV = SG + K16;
   static constexpr uint32_t GL = SV + K16;             // float[128]
-  static constexpr uint32_t TOT = GL + 512;            // float[4][128]
-  static constexpr uint32_t BET = TOT + 2048;          // float[64]
-  static constexpr uint32_t BT = BET + 256;            // float[3][256]
-  static constexpr uint32_t BARS = BT + 3072;          // 3 mbarriers
+  static constexpr uint32_t TOT = GL + 512;            // float[8][128]
+  static constexpr uint32_t BET = TOT + 4096;          // float[64]
+  static constexpr uint32_t BT = BET + 256;            // inverse scratch, float[32][36]
+  static constexpr uint32_t BARS = BT + 4608;          // 3 mbarriers
   static constexpr uint32_t TPTR = BARS + 64;          // tensor-memory base
   static constexpr uint32_t BYTES = TPTR + 64;
   // fp32 A (strictly lower, beta-scaled) lives in the K^ tile once MMA-g has read it
@@ -100,10 +100,6 @@ struct Sm {
 };
 static_assert(Sm<true>::BYTES + 1024 <= 232448, "output pass shared memory");
 static_assert(Sm<false>::BYTES + 1024 <= 232448, "summary pass shared memory");
-
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
@@ -137,6 +133,23 @@ __device__ __forceinline__ float* f64x64(unsigned char* base, int r, int s) {
   return reinterpret_cast<float*>(base) + r * 64 + (s ^ (r & 31));
 }
 
+// Global load issued where it stands (the asm keeps the compiler from sinking it
+// next to its first use, one chunk later).
+__device__ __forceinline__ uint16_t ldg_u16_early(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                    pack_bf16(f[6], f[7]));
+}
+
+// One CTA of 16 warps per (sequence, head, segment). Warpgroup g = warp / 4 reaches
+// every tensor-memory lane; phases split their columns over the four warpgroups.
 template <bool PC>
 __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcArgs a) {
   using L_ = Sm<PC>;
@@ -192,8 +205,8 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
   tc_fence_after();
   const uint32_t tb = *tptr;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const int row = tid & 127;   // TMEM lane = state column j for the state-side work
-  const int half = tid >> 7;   // which warpgroup
+  const int row = tid & 127;  // tensor-memory lane = state column j on the state side
+  const int wg = tid >> 7;    // warpgroup 0..3
 
   uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
   bool pend_qkg = false, pend_v = false, pend_mma = false;
@@ -220,6 +233,12 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
   }
   pend_qkg = pend_v = (c_begin < c_end);
 
+  // columns of the state this thread handles: output pass, warpgroup g takes
+  // columns [32g, 32g+32); summary pass, block g/2, columns [64(g%2), +64)
+  const int st_b = PC ? 0 : (wg >> 1);
+  const int st_lo = PC ? 32 * wg : 64 * (wg & 1);
+  const int st_hi = st_lo + (PC ? 32 : 64);
+
   // ---- initial state: fp32 into tensor memory, bf16 copy as the MMA operand
   {
     const float* src = nullptr;
@@ -227,42 +246,34 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
       if (nseg > 1) src = a.sstart + ((int64_t)pair * a.max_segs + seg) * D * D;
       else if (a.s0) src = a.s0 + (int64_t)pair * D * D;
     }
-    for (int b = 0; b < NB; ++b) {
-      if (!PC && b != half) continue;
-      for (int c = (PC ? half * 64 : 0); c < (PC ? half * 64 + 64 : D); c += 32) {
-        uint32_t v[32];
+    for (int c = st_lo; c < st_hi; c += 32) {
+      uint32_t v[32];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          float x;
-          if (PC) x = src ? src[(int64_t)(c + t) * D + row] : 0.f;
-          else x = (b == 0 && c + t == row) ? 1.f : 0.f;
-          v[t] = __float_as_uint(x);
-        }
-        tmem_st32(tb + lane_base + L_::st(b) + c, v);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          uint4 pk;
-          pk.x = pack_bf16(__uint_as_float(v[8 * q8 + 0]), __uint_as_float(v[8 * q8 + 1]));
-          pk.y = pack_bf16(__uint_as_float(v[8 * q8 + 2]), __uint_as_float(v[8 * q8 + 3]));
-          pk.z = pack_bf16(__uint_as_float(v[8 * q8 + 4]), __uint_as_float(v[8 * q8 + 5]));
-          pk.w = pack_bf16(__uint_as_float(v[8 * q8 + 6]), __uint_as_float(v[8 * q8 + 7]));
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-              pk;
-        }
+      for (int t = 0; t < 32; ++t) {
+        float x;
+        if (PC) x = src ? src[(int64_t)(c + t) * D + row] : 0.f;
+        else x = (st_b == 0 && c + t == row) ? 1.f : 0.f;
+        v[t] = __float_as_uint(x);
       }
+      tmem_st32(tb + lane_base + L_::st(st_b) + c, v);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8)
+        *reinterpret_cast<uint4*>(sm + L_::S + st_b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
+            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
     }
     tmem_st_wait();
   }
 
-  // beta for the first chunk (threads 0..63 keep the next chunk's value in a register)
-  float bnext = 0.f;
-  if (tid < C && c_begin + tid < c_end) bnext = __bfloat162float(a.beta[(c_begin + tid) * a.H + h]);
+  // beta: threads 0..63 hold the next chunk's value (bf16 bits) in a register
+  uint16_t bnext = 0;
+  if (tid < C && c_begin + tid < c_end)
+    bnext = ldg_u16_early(a.beta + (c_begin + tid) * a.H + h);
 
   tc_fence_before();
   fence_async_smem();
   __syncthreads();
 
-  const int p = tid & 63, qr = tid >> 6;  // elementwise: channel pair, row quarter
+  const int p = tid & 63, e8 = tid >> 6;  // elementwise: channel pair, group of 8 rows
   const int ch = 2 * p, bx = p >> 5, cofs = (p & 31) * 4;
   bool failed = false;
 
@@ -272,10 +283,10 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
 
     // ---------------- [A] decay prefix sums and the decayed operand tiles
     if (tid < C) {
-      bet[tid] = bnext;
-      bnext = 0.f;
+      bet[tid] = bf16_bits_to_float(bnext);
+      bnext = 0;
       if (has_next && c0 + C + tid < c_end)
-        bnext = __bfloat162float(a.beta[(c0 + C + tid) * a.H + h]);
+        bnext = ldg_u16_early(a.beta + (c0 + C + tid) * a.H + h);
     }
     {
       const bool ok = mbar_wait(bar_qkg, ph_qkg) && mbar_wait(bar_v, ph_v);
@@ -284,12 +295,12 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
       ph_v ^= 1;
       pend_qkg = pend_v = false;
     }
-    float G0[16], G1[16];
+    float G0[8], G1[8];
     {
       float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * e8 + i;
         const float2 gg =
             unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + bx * K8 + r * 128 + cofs));
         if (r < L) {
@@ -299,24 +310,27 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
         G0[i] = r0;
         G1[i] = r1;
       }
-      tot[qr * 128 + ch] = r0;
-      tot[qr * 128 + ch + 1] = r1;
+      *reinterpret_cast<float2*>(tot + e8 * 128 + ch) = make_float2(r0, r1);
     }
     __syncthreads();
-    float kh0[16], kh1[16];
     {
-      float o0 = 0.f, o1 = 0.f;
-      for (int q = 0; q < qr; ++q) {
-        o0 += tot[q * 128 + ch];
-        o1 += tot[q * 128 + ch + 1];
-      }
-      if (qr == 3) {
-        gl[ch] = expf(G0[15] + o0);
-        gl[ch + 1] = expf(G1[15] + o1);
-      }
+      float o0 = 0.f, o1 = 0.f, s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
+      for (int q = 0; q < 8; ++q) {
+        const float2 tq = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
+        if (q < e8) {
+          o0 += tq.x;
+          o1 += tq.y;
+        }
+        s0 += tq.x;
+        s1 += tq.y;
+      }
+      // gamma at the last row of the chunk (rows past L add nothing)
+      const float gl0 = expf(s0), gl1 = expf(s1);
+      if (e8 == 7) *reinterpret_cast<float2*>(gl + ch) = make_float2(gl0, gl1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * e8 + i;
         const float g0 = G0[i] + o0, g1 = G1[i] + o1;
         const float e0 = __expf(g0), e1 = __expf(g1);
         const float ei0 = __expf(-g0), ei1 = __expf(-g1);
@@ -324,10 +338,11 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
         if (r >= L) kk = make_float2(0.f, 0.f);
         *reinterpret_cast<uint32_t*>(sm + L_::KQ + sw128_off(r, ch, K16)) =
             pack_bf16(kk.x * e0, kk.y * e1);
-        kh0[i] = kk.x * ei0;
-        kh1[i] = kk.y * ei1;
+        const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
         *reinterpret_cast<uint32_t*>(sm + L_::KH + sw128_off(r, ch, L_::KH_AS)) =
-            pack_bf16(kh0[i], kh1[i]);
+            pack_bf16(kh0, kh1);
+        *reinterpret_cast<uint32_t*>(sm + L_::KB + sw128_off(r, ch, K8)) =
+            pack_bf16(kh0 * gl0, kh1 * gl1);
         if (PC) {
           float2 qq =
               unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SQ + bx * K8 + r * 128 + cofs));
@@ -337,22 +352,12 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
         }
       }
     }
-    __syncthreads();  // gl ready; every read of the q/k/g staging is done
+    fence_async_smem();
+    __syncthreads();  // operand tiles complete; every read of the q/k/g staging is done
     if (tid == 0 && has_next) {
       issue_qkg(c0 + C);
       pend_qkg = true;
     }
-    {
-      const float gl0 = gl[ch], gl1 = gl[ch + 1];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
-        *reinterpret_cast<uint32_t*>(sm + L_::KB + sw128_off(r, ch, K8)) =
-            pack_bf16(kh0[i] * gl0, kh1[i] * gl1);
-      }
-    }
-    fence_async_smem();
-    __syncthreads();
 
     // ---------------- [B] MMA-g: [K~;Q~|K^] K^^T  and  MMA-a: S^T [K~;Q~]^T
     if (tid == 0) {
@@ -385,24 +390,40 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
     }
     tc_fence_after();
 
-    // ---------------- [C] warpgroup 0: T = (I + A)^{-1} Diag(beta), P;  warpgroup 1: (V - X)^T
-    if (half == 0) {
-      if (tid < 64) {
-        const int r = tid;
-        const float br = bet[r];
+    // ---------------- [C] T = (I + A)^{-1} Diag(beta) and P (warps 0-3), (V - X)^T (4-15)
+    // fp32 64x64 tiles A (in the K^ tile, no longer needed) and N = (I + A)^{-1}:
+    // element (r, c) at r*64 + 4*((c/4) ^ (r%16)) + c%4, so 16-byte groups stay whole.
+    auto a_ptr = [&](int r, int c) -> float* {
+      return reinterpret_cast<float*>(sm + L_::as_piece(r >> 5)) + (r & 31) * 64 +
+             ((((c >> 2) ^ (r & 15))) << 2) + (c & 3);
+    };
+    auto n_ptr = [&](int r, int c) -> float* {
+      return reinterpret_cast<float*>(sm + L_::NS) + r * 64 + ((((c >> 2) ^ (r & 15))) << 2) +
+             (c & 3);
+    };
+    if (warp < 2) {
+      // A = Diag(beta) strict_lower(K~ K^^T): thread r owns row r (tensor-memory lanes 0..63)
+      const int r = tid;
+      const float br = bet[r];
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + lane_base + L_::G + cb, v);
-          tmem_ld_wait(v);
-          float* arow = reinterpret_cast<float*>(sm + L_::as_piece(r >> 5)) + (r & 31) * 64;
+      for (int cb = 0; cb < 64; cb += 32) {
+        uint32_t v[32];
+        tmem_ld32(tb + lane_base + L_::G + cb, v);
+        tmem_ld_wait(v);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const int sc = cb + t;
-            arow[sc ^ (r & 31)] = (sc < r) ? br * __uint_as_float(v[t]) : 0.f;
-          }
+        for (int g4 = 0; g4 < 8; ++g4) {
+          float4 f;
+          const int c = cb + 4 * g4;
+          f.x = (c + 0 < r) ? br * __uint_as_float(v[4 * g4 + 0]) : 0.f;
+          f.y = (c + 1 < r) ? br * __uint_as_float(v[4 * g4 + 1]) : 0.f;
+          f.z = (c + 2 < r) ? br * __uint_as_float(v[4 * g4 + 2]) : 0.f;
+          f.w = (c + 3 < r) ? br * __uint_as_float(v[4 * g4 + 3]) : 0.f;
+          *reinterpret_cast<float4*>(a_ptr(r, c)) = f;
         }
-      } else if (PC) {
+      }
+    } else if (warp < 4) {
+      if (PC) {
+        // P = lower_incl(Q~ K^^T): tensor-memory lanes 64..127, bf16 operand tile
         const int r = tid - 64;
 #pragma unroll
         for (int cb = 0; cb < 64; cb += 32) {
@@ -417,108 +438,119 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
               const int sc = cb + 8 * q8 + t;
               f[t] = (sc <= r) ? __uint_as_float(v[8 * q8 + t]) : 0.f;
             }
-            uint4 pk = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]),
-                                  pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
-            *reinterpret_cast<uint4*>(sm + L_::P + sw128_chunk(r, cb / 8 + q8, K8)) = pk;
+            *reinterpret_cast<uint4*>(sm + L_::P + sw128_chunk(r, cb / 8 + q8, K8)) = pack8(f);
           }
-        }
-      }
-      named_bar(1, 128);
-      auto As = [&](int r, int c) -> float {
-        return reinterpret_cast<const float*>(sm + L_::as_piece(r >> 5))[(r & 31) * 64 + (c ^ (r & 31))];
-      };
-      unsigned char* ns = sm + L_::NS;
-      // diagonal 16x16 blocks: lane l of warp w owns column 16w + l
-      if (lane < 16) {
-        const int w = warp;
-        float n[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-          float val = (rr == lane) ? 1.f : 0.f;
-#pragma unroll
-          for (int ss = 0; ss < rr; ++ss) val -= As(16 * w + rr, 16 * w + ss) * n[ss];
-          n[rr] = (rr < lane) ? 0.f : val;
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) *f64x64(ns, 16 * w + rr, 16 * w + lane) = n[rr];
-      }
-      named_bar(1, 128);
-      // off-diagonal blocks, by distance d from the diagonal:
-      //   N_ij = -N_ii * sum_{k=j}^{i-1} A_ik N_kj
-#pragma unroll 1
-      for (int d = 1; d < 4; ++d) {
-        const int nblk = 4 - d;
-        for (int e = tid; e < nblk * 256; e += 128) {
-          const int bj = e >> 8, bi = bj + d, rr = (e >> 4) & 15, cc = e & 15;
-          const int r = 16 * bi + rr, c = 16 * bj + cc;
-          float acc = 0.f;
-          for (int kk = 16 * bj; kk < 16 * bi; ++kk) acc += As(r, kk) * *f64x64(ns, kk, c);
-          bt[e] = acc;
-        }
-        named_bar(1, 128);
-        for (int e = tid; e < nblk * 256; e += 128) {
-          const int bj = e >> 8, bi = bj + d, rr = (e >> 4) & 15, cc = e & 15;
-          float acc = 0.f;
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            acc += *f64x64(ns, 16 * bi + rr, 16 * bi + m) * bt[(bj << 8) + (m << 4) + cc];
-          *f64x64(ns, 16 * bi + rr, 16 * bj + cc) = -acc;
-        }
-        named_bar(1, 128);
-      }
-      // T = N Diag(beta), lower triangle, bf16
-      {
-        const int r = tid >> 1, hf = tid & 1;
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const int c8 = hf * 4 + q8;
-          float f[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int sc = 8 * c8 + t;
-            f[t] = (sc <= r) ? *f64x64(ns, r, sc) * bet[sc] : 0.f;
-          }
-          *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(r, c8, K8)) =
-              make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                         pack_bf16(f[6], f[7]));
         }
       }
     } else {
+      // (V - X)^T in 32-column units (block b, half), dealt to warpgroups 1..3
       const int j = row;
-#pragma unroll 1
-      for (int b = 0; b < NB; ++b) {
+      for (int u = wg - 1; u < 2 * NB; u += 3) {
+        const int b = u >> 1, cb = (u & 1) * 32;
         const bool use_v = PC || b == 1;
+        uint32_t v[32];
+        tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
+        tmem_ld_wait(v);
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
-          tmem_ld_wait(v);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float f[8];
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            float f[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int r = cb + 8 * q8 + t;
-              const float vv =
-                  use_v ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                              sm + L_::SV + (j >> 6) * K8 + r * 128 + (j & 63) * 2))
-                        : 0.f;
-              f[t] = vv - __uint_as_float(v[8 * q8 + t]);
-            }
-            *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(j, cb / 8 + q8, K16)) =
-                make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                           pack_bf16(f[6], f[7]));
+          for (int t = 0; t < 8; ++t) {
+            const int r = cb + 8 * q8 + t;
+            const float vv =
+                use_v ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                            sm + L_::SV + (j >> 6) * K8 + r * 128 + (j & 63) * 2))
+                      : 0.f;
+            f[t] = vv - __uint_as_float(v[8 * q8 + t]);
           }
+          *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(j, cb / 8 + q8, K16)) =
+              pack8(f);
         }
       }
+    }
+    __syncthreads();  // A, P and (V - X)^T written; every read of the v staging is done
+    if (tid == 0 && has_next) {
+      issue_v(c0 + C);
+      pend_v = true;
+    }
+    // diagonal 16x16 blocks of N by right-looking forward substitution:
+    // warp w, half h -> block 2w+h; lane l -> column l of the block
+    if (warp < 2) {
+      const int base = 16 * (2 * warp + (lane >> 4)), l = lane & 15;
+      float acc[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == l) ? 1.f : 0.f;
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        const float nv = acc[rr];
+        *n_ptr(base + rr, base + l) = nv;
+#pragma unroll
+        for (int r2 = rr + 1; r2 < 16; ++r2)
+          acc[r2] = fmaf(-*a_ptr(base + r2, base + rr), nv, acc[r2]);
+      }
+    }
+    __syncthreads();
+    float* bt1 = bt;  // [2][16][16]
+    float* bt2 = bt;  // [32][36]
+    {
+      // level 1: in each 32-block, N10 = -N11 (A10 N00) with 16x16 blocks
+      const int b = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+      const int R0 = 32 * b, R1 = 32 * b + 16;
+      float sacc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sacc = fmaf(*a_ptr(R1 + r, R0 + k), *n_ptr(R0 + k, R0 + c), sacc);
+      bt1[b * 256 + r * 16 + c] = sacc;
+      __syncthreads();
+      float tacc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) tacc = fmaf(*n_ptr(R1 + r, R1 + k), bt1[b * 256 + k * 16 + c], tacc);
+      *n_ptr(R1 + r, R0 + c) = -tacc;
+      *n_ptr(R0 + r, R1 + c) = 0.f;  // upper-right 16x16 block of each 32-block (read by level 2)
+      __syncthreads();
+    }
+    {
+      // level 2: N10 = -N11 (A10 N00) with 32x32 blocks
+      const int r = tid >> 4, c = (tid & 15) * 2;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float av = *a_ptr(32 + r, k);
+        const float2 nn = *reinterpret_cast<const float2*>(n_ptr(k, c));
+        s0 = fmaf(av, nn.x, s0);
+        s1 = fmaf(av, nn.y, s1);
+      }
+      *reinterpret_cast<float2*>(bt2 + r * 36 + c) = make_float2(s0, s1);
+      __syncthreads();
+      float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float nv = *n_ptr(32 + r, 32 + k);
+        const float2 bb = *reinterpret_cast<const float2*>(bt2 + k * 36 + c);
+        u0 = fmaf(nv, bb.x, u0);
+        u1 = fmaf(nv, bb.y, u1);
+      }
+      *reinterpret_cast<float2*>(n_ptr(32 + r, c)) = make_float2(-u0, -u1);
+      __syncthreads();
+    }
+    {
+      // T = N Diag(beta), lower triangle, as the bf16 operand: one 16-byte chunk per thread
+      const int r = tid >> 3, c8 = tid & 7;
+      float f[8];
+#pragma unroll
+      for (int h4 = 0; h4 < 2; ++h4) {
+        const int c = 8 * c8 + 4 * h4;
+        const float4 nn = *reinterpret_cast<const float4*>(n_ptr(r, c));
+        const float4 bb = *reinterpret_cast<const float4*>(bet + c);
+        f[4 * h4 + 0] = (c + 0 <= r) ? nn.x * bb.x : 0.f;
+        f[4 * h4 + 1] = (c + 1 <= r) ? nn.y * bb.y : 0.f;
+        f[4 * h4 + 2] = (c + 2 <= r) ? nn.z * bb.z : 0.f;
+        f[4 * h4 + 3] = (c + 3 <= r) ? nn.w * bb.w : 0.f;
+      }
+      *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(r, c8, K8)) = pack8(f);
     }
     tc_fence_before();
     fence_async_smem();
     __syncthreads();
-    if (tid == 0 && has_next) {  // every read of the v staging is done
-      issue_v(c0 + C);
-      pend_v = true;
-    }
 
     // ---------------- [D] MMA-b: U^T = (V - X)^T T^T
     if (tid == 0) {
@@ -542,21 +574,24 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
     tc_fence_after();
 
     // ---------------- [E] U^T -> bf16 operand
-    {
-      const int b = PC ? 0 : half;
-      const int cb0 = PC ? half * 32 : 0, cb1 = PC ? half * 32 + 32 : 64;
-      for (int cb = cb0; cb < cb1; cb += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
-        tmem_ld_wait(v);
+    if (PC) {
+      const int cb = 16 * wg;
+      uint32_t v[16];
+      tmem_ld16(tb + lane_base + L_::xu(0) + cb, v);
+      tmem_ld_wait(v);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const float* f = reinterpret_cast<const float*>(v) + 8 * q8;
-          *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, cb / 8 + q8, K16)) =
-              make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                         pack_bf16(f[6], f[7]));
-        }
-      }
+      for (int q8 = 0; q8 < 2; ++q8)
+        *reinterpret_cast<uint4*>(sm + L_::Y + sw128_chunk(row, cb / 8 + q8, K16)) =
+            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+    } else {
+      const int b = wg >> 1, cb = 32 * (wg & 1);
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8)
+        *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, cb / 8 + q8, K16)) =
+            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
     }
     tc_fence_before();
     fence_async_smem();
@@ -592,39 +627,37 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
 
     // ---------------- [G] outputs; S <- Diag(gl) S + Z; bf16 S^T for the next chunk
     if (PC) {
-      uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::YO + half * 32, v);
+      const int cb = 16 * wg;
+      uint32_t v[16];
+      tmem_ld16(tb + lane_base + L_::YO + cb, v);
       tmem_ld_wait(v);
-      __nv_bfloat16* o = a.out + (c0 * a.H + h) * D + row;
+      __nv_bfloat16* o = a.out + ((c0 + cb) * a.H + h) * D + row;
+      const int64_t ostride = (int64_t)a.H * D;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const int r = half * 32 + t;
-        if (r < L) o[(int64_t)r * a.H * D] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
-      }
+      for (int t = 0; t < 16; ++t)
+        if (cb + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
     }
-    {
-      const int b = PC ? 0 : half;
-      const int c_lo = PC ? half * 64 : 0, c_hi = PC ? half * 64 + 64 : D;
-      for (int c = c_lo; c < c_hi; c += 32) {
-        uint32_t sv[32], zv[32];
-        tmem_ld32(tb + lane_base + L_::st(b) + c, sv);
-        tmem_ld_wait(sv);
-        tmem_ld32(tb + lane_base + L_::z(b) + c, zv);
-        tmem_ld_wait(zv);
+    for (int c = st_lo; c < st_hi; c += 32) {
+      uint32_t sv[32], zv[32];
+      tmem_ld32(tb + lane_base + L_::st(st_b) + c, sv);
+      tmem_ld32(tb + lane_base + L_::z(st_b) + c, zv);
+      tmem_ld_wait(sv);
+      tmem_ld_wait(zv);
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          sv[t] = __float_as_uint(fmaf(gl[c + t], __uint_as_float(sv[t]), __uint_as_float(zv[t])));
-        tmem_st32(tb + lane_base + L_::st(b) + c, sv);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          const float* f = reinterpret_cast<const float*>(sv) + 8 * q8;
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-              make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                         pack_bf16(f[6], f[7]));
-        }
+      for (int t4 = 0; t4 < 8; ++t4) {
+        const float4 g4 = *reinterpret_cast<const float4*>(gl + c + 4 * t4);
+        sv[4 * t4 + 0] = __float_as_uint(fmaf(g4.x, __uint_as_float(sv[4 * t4 + 0]), __uint_as_float(zv[4 * t4 + 0])));
+        sv[4 * t4 + 1] = __float_as_uint(fmaf(g4.y, __uint_as_float(sv[4 * t4 + 1]), __uint_as_float(zv[4 * t4 + 1])));
+        sv[4 * t4 + 2] = __float_as_uint(fmaf(g4.z, __uint_as_float(sv[4 * t4 + 2]), __uint_as_float(zv[4 * t4 + 2])));
+        sv[4 * t4 + 3] = __float_as_uint(fmaf(g4.w, __uint_as_float(sv[4 * t4 + 3]), __uint_as_float(zv[4 * t4 + 3])));
       }
-      tmem_st_wait();
+      tmem_st32(tb + lane_base + L_::st(st_b) + c, sv);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8)
+        *reinterpret_cast<uint4*>(sm + L_::S + st_b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
+            pack8(reinterpret_cast<const float*>(sv) + 8 * q8);
     }
+    tmem_st_wait();
     tc_fence_before();
     fence_async_smem();
     __syncthreads();
@@ -639,22 +672,18 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
       if (pend_mma) mbar_wait(bar_mma, ph_mma, 400000000LL);
     }
   } else {
-    // ---- write the final / summary state
+    // ---- write the final / summary state (row-major [i][j], fp32)
     float* dst = nullptr;
     if (PC) {
       if (a.sT && seg == nseg - 1) dst = a.sT + (int64_t)pair * D * D;
+    } else {
+      const int64_t u = (int64_t)pair * (a.max_segs - 1) + seg;
+      dst = (st_b == 0 ? a.mbuf : a.lbuf) + u * D * D;
     }
-    for (int b = 0; b < NB; ++b) {
-      if (!PC) {
-        if (b != half) continue;
-        const int64_t u = (int64_t)pair * (a.max_segs - 1) + seg;
-        dst = (b == 0 ? a.mbuf : a.lbuf) + u * D * D;
-      }
-      if (dst == nullptr) continue;
-      const int c_lo = PC ? half * 64 : 0, c_hi = PC ? half * 64 + 64 : D;
-      for (int c = c_lo; c < c_hi; c += 32) {
+    if (dst != nullptr) {
+      for (int c = st_lo; c < st_hi; c += 32) {
         uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::st(b) + c, v);
+        tmem_ld32(tb + lane_base + L_::st(st_b) + c, v);
         tmem_ld_wait(v);
 #pragma unroll
         for (int t = 0; t < 32; ++t) dst[(int64_t)(c + t) * D + row] = __uint_as_float(v[t]);
@@ -670,12 +699,23 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
 }
 
 // Start state of every segment: S_{j+1} = M_j S_j + L_j, fp32, one CTA per
-// (sequence, head, 32-column slice).
+// (sequence, head, 16-column slice). M_{j+1} streams into shared memory
+// (cp.async, double-buffered) while step j is computed.
+constexpr int kCombSlices = 8, kCombCols = D / kCombSlices, kMStride = D + 4;
+constexpr int kCombSmem = (2 * D * kMStride + D * kCombCols) * 4;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ TcArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* Ms = reinterpret_cast<float*>(smem_raw);  // [128][129]
-  float* Ss = Ms + 128 * 129;                      // [128][32]
-  const int pair = blockIdx.x >> 2, j0 = (blockIdx.x & 3) * 32;
+  float* Ms = reinterpret_cast<float*>(smem_raw);  // [2][128][132]
+  float* Ss = Ms + 2 * D * kMStride;               // [128][16]
+  const int pair = blockIdx.x / kCombSlices, j0 = (blockIdx.x % kCombSlices) * kCombCols;
   const int s = pair / a.H;
   int64_t t0, t1;
   if (!tc_seq_bounds(a, s, t0, t1)) return;
@@ -684,43 +724,56 @@ __global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ Tc
   if (nseg <= 1 || nseg > a.max_segs) return;
   const int tid = threadIdx.x;
   float* st0 = a.sstart + (int64_t)pair * a.max_segs * D * D;
-  for (int e = tid; e < D * 32; e += 256) {
-    const int i = e >> 5, c = e & 31;
+  auto load_m = [&](int sg, int buf) {
+    const float* M = a.mbuf + ((int64_t)pair * (a.max_segs - 1) + sg) * D * D;
+    float* dst = Ms + buf * D * kMStride;
+    for (int e = tid; e < D * D / 4; e += 256) {
+      const int r = e >> 5, c = (e & 31) * 4;
+      cp_async16(dst + r * kMStride + c, M + r * D + c);
+    }
+    cp_async_commit();
+  };
+  load_m(0, 0);
+  for (int e = tid; e < D * kCombCols; e += 256) {
+    const int i = e / kCombCols, c = e % kCombCols;
     const float x = a.s0 ? a.s0[(int64_t)pair * D * D + i * D + j0 + c] : 0.f;
-    Ss[i * 32 + c] = x;
+    Ss[i * kCombCols + c] = x;
     st0[i * D + j0 + c] = x;
   }
-  const int i = tid >> 1, cs = (tid & 1) * 16;
+  const int i = tid >> 1, ch = (tid & 1) * 8;
   for (int sg = 0; sg < nseg - 1; ++sg) {
-    const int64_t u = (int64_t)pair * (a.max_segs - 1) + sg;
-    const float* M = a.mbuf + u * D * D;
-    const float* Lm = a.lbuf + u * D * D;
-    __syncthreads();
-    for (int e = tid; e < D * D / 4; e += 256) {
-      const float4 m4 = reinterpret_cast<const float4*>(M)[e];
-      const int r = (e * 4) >> 7, c = (e * 4) & 127;
-      Ms[r * 129 + c] = m4.x;
-      Ms[r * 129 + c + 1] = m4.y;
-      Ms[r * 129 + c + 2] = m4.z;
-      Ms[r * 129 + c + 3] = m4.w;
-    }
-    __syncthreads();
-    float acc[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) acc[c] = Lm[i * D + j0 + cs + c];
+    const int buf = sg & 1;
+    cp_async_wait_all();
+    __syncthreads();  // M_sg landed; S of the previous step is visible; other buffer free
+    if (sg + 1 < nseg - 1) load_m(sg + 1, buf ^ 1);
+    const float* Lm = a.lbuf + ((int64_t)pair * (a.max_segs - 1) + sg) * D * D + i * D + j0 + ch;
+    const float4 l0 = *reinterpret_cast<const float4*>(Lm);
+    const float4 l1 = *reinterpret_cast<const float4*>(Lm + 4);
+    float acc[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    const float* Mrow = Ms + buf * D * kMStride + i * kMStride;
+#pragma unroll 8
     for (int k = 0; k < D; ++k) {
-      const float m = Ms[i * 129 + k];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) acc[c] = fmaf(m, Ss[k * 32 + cs + c], acc[c]);
+      const float m = Mrow[k];
+      const float4 s0 = *reinterpret_cast<const float4*>(Ss + k * kCombCols + ch);
+      const float4 s1 = *reinterpret_cast<const float4*>(Ss + k * kCombCols + ch + 4);
+      acc[0] = fmaf(m, s0.x, acc[0]);
+      acc[1] = fmaf(m, s0.y, acc[1]);
+      acc[2] = fmaf(m, s0.z, acc[2]);
+      acc[3] = fmaf(m, s0.w, acc[3]);
+      acc[4] = fmaf(m, s1.x, acc[4]);
+      acc[5] = fmaf(m, s1.y, acc[5]);
+      acc[6] = fmaf(m, s1.z, acc[6]);
+      acc[7] = fmaf(m, s1.w, acc[7]);
     }
-    __syncthreads();
-    float* dst = st0 + (int64_t)(sg + 1) * D * D;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      Ss[i * 32 + cs + c] = acc[c];
-      dst[i * D + j0 + cs + c] = acc[c];
-    }
+    __syncthreads();  // every read of S done
+    float* dst = st0 + (int64_t)(sg + 1) * D * D + i * D + j0 + ch;
+    *reinterpret_cast<float4*>(Ss + i * kCombCols + ch) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(Ss + i * kCombCols + ch + 4) =
+        make_float4(acc[4], acc[5], acc[6], acc[7]);
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
+  cp_async_wait_all();
 }
 
 // ------------------------------------------------------------------ host side
@@ -819,14 +872,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
                              Sm<false>::BYTES + 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kda_tc_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (128 * 129 + 128 * 32) * 4);
+                             kCombSmem);
   if (e != cudaSuccess) return e;
 
   if (plan.max_segs > 1) {
     kda_tc_pass<false><<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), NT,
                          Sm<false>::BYTES + 1024, st>>>(a);
-    kda_tc_combine<<<static_cast<unsigned>(plan.pairs * 4), 256, (128 * 129 + 128 * 32) * 4,
-                     st>>>(a);
+    kda_tc_combine<<<static_cast<unsigned>(plan.pairs * kCombSlices), 256, kCombSmem, st>>>(a);
   }
   kda_tc_pass<true><<<static_cast<unsigned>(plan.pairs * plan.max_segs), NT,
                       Sm<true>::BYTES + 1024, st>>>(a);
