@@ -43,6 +43,22 @@ def prefill_bytes_per_token_head(dk: int, dv: int, elem: int = 2) -> int:
     return elem * (3 * dk + dv + 1) + elem * dv
 
 
+def measured_traffic(key: str) -> int | None:
+    """DRAM bytes per launch from the committed ncu capture, while the kernel source
+    that was captured is unchanged (sha256 prefix); otherwise None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[key]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+                return None
+        return int(rec.get("bytes_per_call") or rec.get("bytes_per_launch"))
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -127,13 +143,20 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Slowest rank's time: every rank's device time, reduced with MAX."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every replica processes its own tokens each step, and the
+    step takes as long as the slowest rank."""
+    return tokens_per_rank_step * world / (ms_per_step / 1e3)
 
 
 def time_region(fn, steps: int, stream) -> tuple[float, list[float]]:
@@ -181,7 +204,7 @@ def bench_ours(args, world, rank, local):
     total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / args.steps
     tokens_per_step = T * world
-    value = tokens_per_step / (ms_step / 1e3)
+    value = job_tokens_per_s(T, world, ms_step)
     flops = prefill_flops_per_token_head(dk, dv) * T * H
     kernel_ms = statistics.mean(per)
     launches_per_step = kda_launches_per_step(kda, shape)
@@ -192,7 +215,9 @@ def bench_ours(args, world, rank, local):
     roofline = {"bound": "tensor", "achieved": round(tc_tflops, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
-                "traffic": None, "peak_source": peaks["source"],
+                "traffic": measured_traffic("prefill_bf16_h32_t8192_d128"),
+                "traffic_scope": "one kda_chunk_fwd call (summary + combine + output kernels)",
+                "peak_source": peaks["source"],
                 "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": algo_bytes},
                 "kernel_ms": round(kernel_ms, 4)}
@@ -256,7 +281,8 @@ def bench_ours(args, world, rank, local):
               "roofline": {"bound": "hbm", "achieved": round(d_gbs, 1), "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": round(d_gbs / peaks["hbm_gbs"], 4),
                            "frac_of_8tbs": round(d_gbs / 8000.0, 4),
-                           "bytes_per_step": state_bytes + tok_bytes, "traffic": None},
+                           "bytes_per_step": state_bytes + tok_bytes,
+                           "traffic": measured_traffic("decode_n256_h32_d128")},
               "gpu_launches": dsteps}
     return {
         "value": round(value, 1), "ms_per_step": round(ms_step, 4), "clocks": clk,
