@@ -216,7 +216,7 @@ def bench_ours(args, world, rank, local):
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
                 "traffic": measured_traffic("prefill_bf16_h32_t8192_d128"),
-                "traffic_scope": "one kda_chunk_fwd call (summary + combine + output kernels)",
+                "traffic_scope": "one kda_chunk_fwd call (intra-chunk + summary walk + combine + output walk)",
                 "peak_source": peaks["source"],
                 "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": algo_bytes},
@@ -295,10 +295,10 @@ def bench_ours(args, world, rank, local):
 def kda_launches_per_step(kda, shape) -> int:
     """Kernels one kda_chunk_fwd enqueues for `shape` (the header memset excluded).
 
-    bf16 with d_k = d_v = 128 takes the tensor-core path: output pass, plus the
-    summary pass and the combine when the longest sequence spans several
-    segments; other shapes run one CUDA-core kernel. The segment rule is the
-    library's (tokens per segment = 64 * next power of two of
+    bf16 with d_k = d_v = 128 takes the tensor-core path: the intra-chunk kernel
+    and the output walk, plus the summary walk and the combine when the longest
+    sequence spans several segments; other shapes run one CUDA-core kernel. The
+    segment rule is the library's (tokens per segment = 64 * next power of two of
     ceil(H * (ceil(T/64) + n) / 148), at least 8 chunks)."""
     T_total = shape.T * (1 if shape.n_seqs > 0 else shape.B)
     n = shape.n_seqs if shape.n_seqs > 0 else shape.B
@@ -308,7 +308,7 @@ def kda_launches_per_step(kda, shape) -> int:
     per_sm = max(8, -(-shape.H * chunks // 148))
     seg = 64 * (1 << (per_sm - 1).bit_length())
     max_len = shape.max_seqlen if (shape.n_seqs > 0 and shape.max_seqlen > 0) else shape.T
-    return 3 if -(-max_len // seg) > 1 else 1
+    return 4 if -(-max_len // seg) > 1 else 2
 
 
 def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: int = 0) -> dict:

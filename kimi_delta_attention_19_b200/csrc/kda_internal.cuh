@@ -97,10 +97,12 @@ __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16* p, float x)
 
 // Segment plan of the tensor-core prefill (a pure function of the shape).
 struct TcPlan {
-  int seg_tokens;   // tokens per segment (a multiple of the chunk length)
-  int max_segs;     // segments of the longest sequence
-  int64_t pairs;    // (sequence, head) pairs
-  size_t ws_bytes;  // workspace it needs, header included
+  int seg_tokens;    // tokens per segment (a multiple of the chunk length)
+  int max_segs;      // segments of the longest sequence
+  int64_t pairs;     // (sequence, head) pairs
+  int64_t n_slots;   // chunk slots: ceil(T_total / chunk) + n_seqs
+  size_t tiles_off;  // workspace offset of the per-chunk tiles
+  size_t ws_bytes;   // workspace it needs, header included
 };
 TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len);
 bool tc_path_applies(const kda_shape& s, int64_t T_total);

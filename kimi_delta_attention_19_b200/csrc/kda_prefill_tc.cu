@@ -12,19 +12,23 @@
 //   K~ = K*exp(Gamma), K^ = K*exp(-Gamma), Q~ = Q*exp(Gamma), Kb = K^*gl
 //   A  = Diag(beta) strict_lower(K~ K^^T)        P = lower_incl(Q~ K^^T)
 //   T  = (I + A)^{-1} Diag(beta)                 (blocked forward substitution)
-//   U  = T (V - K~ S)                            O = scale (Q~ S + P U)
+//   W  = T K~,  U0 = T V                         (the chunk's WY factors)
+//   U  = U0 - W S                                O = scale (Q~ S + P U)
 //   S <- Diag(gl) S + Kb^T U
-// Everything is computed in the transposed frame so every MMA has M = 128
-// (the d_v index of S): X^T = S^T K~^T, U^T = (V - X)^T T^T, O^T += U^T P^T,
-// Z = U^T Kb. Operands are bf16 tiles in shared memory, accumulators fp32 in
-// tensor memory, and the state S stays fp32 in tensor memory for the whole walk.
+// Everything above the last two lines depends on the chunk alone. An intra-chunk
+// kernel computes it for every (chunk, head) at once and leaves -W, U0, Kb, Q~,
+// P^T and gl in the workspace. The walk over the chunks of a sequence, which
+// carries S, is then four tensor-core products per chunk in the transposed frame
+// (M = 128, the d_v index of S):
+//   U^T = U0^T + S^T (-W)^T,  (Q~ S)^T = S^T Q~^T,  O^T += U^T P^T,  S^T += U^T Kb
+// with S fp32 in tensor memory for the whole walk and a bf16 copy as the operand.
 //
-// Long sequences are split into segments that run in parallel (two passes):
-//   summary pass: per segment, the affine map S_end = M S_start + L, found by
+// Long sequences are split into segments that are walked in parallel:
+//   summary walk: per segment, the affine map S_end = M S_start + L, found by
 //                 walking the segment with the 256-column state [M | L] started
-//                 at [I | 0] (the M half sees V = 0);
+//                 at [I | 0] (the M half sees V = 0, i.e. U0 = 0);
 //   combine:      S_start of every segment, sequentially per (sequence, head), fp32;
-//   output pass:  per segment, the walk from its true S_start, writing outputs.
+//   output walk:  per segment, the walk from its true S_start, writing outputs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -40,67 +44,85 @@ using namespace sm100;
 
 constexpr int C = kChunk;  // 64
 constexpr int D = 128;     // d_k = d_v on this path
-constexpr int NT = 512;
 constexpr uint32_t K8 = 8192, K16 = 16384, K32 = 32768;
-constexpr int kTmemCols = 512;
 
-struct TcArgs {
-  CUtensorMap tm_q, tm_k, tm_g, tm_v;
+// Workspace tiles per (chunk slot, head); rows are the chunk's tokens.
+//   wn, u0, kb, qt: [64][128] bf16  (-W, U0, Kb, Q~)
+//   pt:             [64][64]  bf16  (P^T: row s, column r)
+//   gl:             [128]     fp32
+constexpr size_t kTileBig = size_t(C) * D * 2;
+constexpr size_t kTilePt = size_t(C) * C * 2;
+constexpr size_t kTileGl = size_t(D) * 4;
+constexpr size_t kTileBytes = 4 * kTileBig + kTilePt + kTileGl;
+
+// Sequence boundaries as both kernels see them.
+struct SeqTable {
+  const int32_t* cu;  // [n_seqs + 1] or null (then sequence s is [s T, (s + 1) T))
+  int32_t* status;
+  int64_t T, T_total;
+  int n_seqs;
+};
+
+__device__ __forceinline__ int64_t seq_start(const SeqTable& q, int s) {
+  return q.cu ? static_cast<int64_t>(q.cu[s]) : static_cast<int64_t>(s) * q.T;
+}
+
+__device__ __forceinline__ bool seq_bounds_tc(const SeqTable& q, int s, int64_t& t0, int64_t& t1) {
+  if (q.cu == nullptr) {
+    t0 = (int64_t)s * q.T;
+    t1 = t0 + q.T;
+    return true;
+  }
+  const int64_t c0 = q.cu[s], c1 = q.cu[s + 1];
+  const bool ok = (c0 >= 0) && (c1 >= c0) && (c1 <= q.T_total) && (s != 0 || c0 == 0) &&
+                  (s + 1 != q.n_seqs || c1 == q.T_total);
+  if (!ok) {
+    atomicExch(q.status, kDevBadSeqlens);
+    return false;
+  }
+  t0 = c0;
+  t1 = c1;
+  return true;
+}
+
+// Workspace slot of chunk 0 of the sequence starting at token t0; chunk c uses slot
+// base + c. A sequence of n tokens has ceil(n/64) <= floor(n/64) + 1 chunks, so the
+// slots of consecutive sequences never collide and all stay below
+// ceil(T_total/64) + n_seqs.
+__device__ __forceinline__ int64_t slot_base(int64_t t0, int s) { return t0 / C + s; }
+
+struct IntraArgs {
+  CUtensorMap tm_q, tm_k, tm_g;  // [T_total][H*128] bf16, 64x64 boxes, no swizzle
+  CUtensorMap tm_v;              // the same shape, 128-byte swizzle (an MMA operand as loaded)
+  SeqTable seq;
   const __nv_bfloat16* beta;
+  __nv_bfloat16 *wn, *u0, *kb, *qt, *pt;
+  float* gl;
+  int H;
+  float lb;
+};
+
+struct WalkArgs {
+  CUtensorMap tm_wn, tm_u0, tm_kb, tm_qt;  // [tiles*64][128] bf16, 64x64 boxes, 128-byte swizzle
+  CUtensorMap tm_pt;                       // [tiles*64][64]
+  CUtensorMap tm_o;                        // out [T_total][H*128], 64x64 boxes, no swizzle
+  SeqTable seq;
+  const float* gl;
   __nv_bfloat16* out;
   const float* s0;
   float* sT;
-  const int32_t* cu;
-  int32_t* status;
   float* mbuf;    // [pairs, max_segs-1, D, D]  summary: M (row-major [i][j])
   float* lbuf;    // [pairs, max_segs-1, D, D]  summary: L
   float* sstart;  // [pairs, max_segs, D, D]    start state of every segment
-  int64_t T, T_total;
-  int n_seqs, H;
+  int H;
   int seg_tokens, max_segs;
-  float scale, lb;
+  float scale;
 };
 
-// Shared-memory map (byte offsets from a 1024-aligned base). PC = output pass.
-template <bool PC>
-struct Sm {
-  static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks
-  // KQ region: [K~ atom0 | X atom0 | K~ atom1 | X atom1] (8 KB each), X = Q~ (output
-  // pass) or K^ (summary pass), so rows 0..127 form one M=128 operand.
-  static constexpr uint32_t KQ = 0;
-  static constexpr uint32_t KH = PC ? K32 : K8;        // K^ tile
-  static constexpr uint32_t KH_AS = PC ? K8 : K16;     // its atom stride
-  static constexpr uint32_t KB = PC ? K32 + K16 : K32;  // Kb tile (atom stride 8 KB)
-  static constexpr uint32_t S = KB + K16;              // bf16 S^T blocks, 32 KB each
-  static constexpr uint32_t Y = S + NB * K32;          // (V - X)^T, then U^T; 16 KB each
-  static constexpr uint32_t T = Y + NB * K16;          // T (8 KB)
-  static constexpr uint32_t P = T + K8;                // P (8 KB, output pass)
-  static constexpr uint32_t NS = P + (PC ? K8 : 0);    // fp32 (I + A)^{-1}, 16 KB
-  static constexpr uint32_t SQ = NS + K16;             // TMA staging q (output pass)
-  static constexpr uint32_t SK = SQ + (PC ? K16 : 0);
-  static constexpr uint32_t SG = SK + K16;
-  static constexpr uint32_t SV = SG + K16;
-  static constexpr uint32_t GL = SV + K16;             // float[128]
-  static constexpr uint32_t TOT = GL + 512;            // float[8][128]
-  static constexpr uint32_t BET = TOT + 4096;          // float[64]
-  static constexpr uint32_t BT = BET + 256;            // inverse scratch, float[32][36]
-  static constexpr uint32_t BARS = BT + 4608;          // 3 mbarriers
-  static constexpr uint32_t TPTR = BARS + 64;          // tensor-memory base
-  static constexpr uint32_t BYTES = TPTR + 64;
-  // fp32 A (strictly lower, beta-scaled) lives in the K^ tile once MMA-g has read it
-  __device__ static constexpr uint32_t as_piece(int p) {
-    return PC ? KH + p * K8 : KQ + K8 + p * K16;
-  }
-  // tensor-memory columns
-  __device__ static constexpr uint32_t st(int b) { return PC ? 320 : 128 * b; }      // fp32 S^T
-  __device__ static constexpr uint32_t xu(int b) { return PC ? 0 : 256 + 64 * b; }   // X^T, U^T
-  static constexpr uint32_t YO = 64;                                                  // O^T
-  static constexpr uint32_t G = PC ? 128 : 384;                                       // K~K^^T|Q~K^^T
-  __device__ static constexpr uint32_t z(int b) { return PC ? 192 : 256 + 128 * b; }  // Kb^T U
-};
-static_assert(Sm<true>::BYTES + 1024 <= 232448, "output pass shared memory");
-static_assert(Sm<false>::BYTES + 1024 <= 232448, "summary pass shared memory");
-
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                          ~static_cast<uintptr_t>(1023));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -109,584 +131,708 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(t);
 }
-
-__device__ __forceinline__ bool tc_seq_bounds(const TcArgs& a, int s, int64_t& t0, int64_t& t1) {
-  if (a.cu == nullptr) {
-    t0 = (int64_t)s * a.T;
-    t1 = t0 + a.T;
-    return true;
-  }
-  const int64_t c0 = a.cu[s], c1 = a.cu[s + 1];
-  const bool ok = (c0 >= 0) && (c1 >= c0) && (c1 <= a.T_total) && (s != 0 || c0 == 0) &&
-                  (s + 1 != a.n_seqs || c1 == a.T_total);
-  if (!ok) {
-    atomicExch(a.status, kDevBadSeqlens);
-    return false;
-  }
-  t0 = c0;
-  t1 = c1;
-  return true;
-}
-
-// fp32 64x64 tile with a per-row XOR swizzle (conflict-free row and column access).
-__device__ __forceinline__ float* f64x64(unsigned char* base, int r, int s) {
-  return reinterpret_cast<float*>(base) + r * 64 + (s ^ (r & 31));
-}
-
-// Global load issued where it stands (the asm keeps the compiler from sinking it
-// next to its first use, one chunk later).
-__device__ __forceinline__ uint16_t ldg_u16_early(const void* p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
 __device__ __forceinline__ uint4 pack8(const float* f) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
 }
+// Uniform decision after a bounded wait: true when any thread of the CTA timed out.
+__device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity);
+  return __syncthreads_or(!ok) != 0;
+}
 
-// One CTA of 16 warps per (sequence, head, segment). Warpgroup g = warp / 4 reaches
-// every tensor-memory lane; phases split their columns over the four warpgroups.
-template <bool PC>
-__global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcArgs a) {
-  using L_ = Sm<PC>;
-  constexpr int NB = L_::NB;
+// ------------------------------------------------------------------ intra-chunk kernel
+// One CTA of 8 warps per (chunk slot, head); two CTAs per SM. Everything of a chunk
+// that does not depend on the state: decay tiles, the Gram products on the tensor
+// cores, T = (I + A)^{-1} Diag(beta) by blocked forward substitution in fp32, and
+// the WY factors W = T K~, U0 = T V on the tensor cores.
+constexpr int kIntraThreads = 256;
+struct IntraSm {
+  // raw inputs as loaded by TMA; each region is reused once its contents are read
+  static constexpr uint32_t SV = 0;        // V, swizzled: [64 s][64 j] boxes (U0's A operand)
+  static constexpr uint32_t KQ = K16;      // [K~ a0 | Q~ a0 | K~ a1 | Q~ a1], 8 KB each
+  static constexpr uint32_t SK = 3 * K16;  // raw k, then fp32 A
+  static constexpr uint32_t SG = 4 * K16;  // raw g, then fp32 N = (I + A)^{-1}
+  static constexpr uint32_t SQ = 5 * K16;  // raw q, then K^, then merge scratch and T
+  static constexpr uint32_t A = SK, NS = SG, KH = SQ, BT = SQ, T = SQ + K8;
+  static constexpr uint32_t TOT = 6 * K16;     // float[4][128] partial decay sums
+  static constexpr uint32_t BET = TOT + 2048;  // float[64]
+  static constexpr uint32_t BARS = BET + 256;
+  static constexpr uint32_t TPTR = BARS + 64;
+  static constexpr uint32_t BYTES = TPTR + 16;
+  // tensor-memory columns: [K~;Q~] K^^T, W^T, U0^T
+  static constexpr uint32_t G = 0, W = 64, U = 128, COLS = 256;
+};
+static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTAs per SM");
+
+__global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_constant__ IntraArgs a) {
+  using L_ = IntraSm;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t u = blockIdx.x / a.H;
+  const int h = static_cast<int>(blockIdx.x % a.H);
 
-  // ---- which (sequence, head, segment) this CTA owns
-  const int per = PC ? a.max_segs : a.max_segs - 1;
-  const int seg = blockIdx.x % per;
-  const int pair = blockIdx.x / per;
-  const int s = pair / a.H, h = pair % a.H;
-  int64_t t0, t1;
-  if (!tc_seq_bounds(a, s, t0, t1)) return;
-  const int64_t len = t1 - t0;
-  const int nseg = len > 0 ? (int)((len + a.seg_tokens - 1) / a.seg_tokens) : 1;
-  if (nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
-    if (seg == 0 && tid == 0) atomicExch(a.status, kDevBadSeqlens);
-    return;
+  // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
+  int lo = 0, hi = a.seq.n_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (slot_base(seq_start(a.seq, mid), mid) <= u) lo = mid;
+    else hi = mid - 1;
   }
-  if (PC ? (seg >= nseg) : (seg >= nseg - 1)) return;
-  const int64_t c_begin = t0 + (int64_t)seg * a.seg_tokens;
-  const int64_t c_end = (c_begin + a.seg_tokens < t1) ? c_begin + a.seg_tokens : t1;
+  const int s = lo;
+  int64_t t0, t1;
+  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
+  const int64_t c = u - slot_base(t0, s);
+  if (c < 0 || c * C >= t1 - t0) return;  // a slot between two sequences
+  const int64_t r0 = t0 + c * C;
+  const int L = (t1 - r0) < C ? static_cast<int>(t1 - r0) : C;
+  const int64_t tile = u * a.H + h;
 
-  float* gl = reinterpret_cast<float*>(sm + L_::GL);
   float* tot = reinterpret_cast<float*>(sm + L_::TOT);
   float* bet = reinterpret_cast<float*>(sm + L_::BET);
   float* bt = reinterpret_cast<float*>(sm + L_::BT);
-  uint64_t* bar_qkg = reinterpret_cast<uint64_t*>(sm + L_::BARS);
-  uint64_t* bar_v = bar_qkg + 1;
-  uint64_t* bar_mma = bar_qkg + 2;
+  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);
+  uint64_t* bar_mma = bar_in + 1;
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
 
   if (warp == 0) {
-    tmem_alloc(tptr, kTmemCols);
+    tmem_alloc(tptr, L_::COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar_qkg, 1);
-    mbar_init(bar_v, 1);
+    mbar_init(bar_in, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
-    tma_prefetch_desc(&a.tm_k);
-    tma_prefetch_desc(&a.tm_g);
-    tma_prefetch_desc(&a.tm_v);
-    if (PC) tma_prefetch_desc(&a.tm_q);
+    mbar_arrive_expect_tx(bar_in, 4 * K16);
+    for (int bx = 0; bx < 2; ++bx) {
+      const int x = h * D + 64 * bx;
+      tma_load_2d(sm + L_::SK + bx * K8, &a.tm_k, bar_in, x, static_cast<int>(r0));
+      tma_load_2d(sm + L_::SG + bx * K8, &a.tm_g, bar_in, x, static_cast<int>(r0));
+      tma_load_2d(sm + L_::SQ + bx * K8, &a.tm_q, bar_in, x, static_cast<int>(r0));
+      tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_in, x, static_cast<int>(r0));
+    }
   }
+  if (tid < C) bet[tid] = tid < L ? __bfloat162float(a.beta[(r0 + tid) * a.H + h]) : 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = *tptr;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const int row = tid & 127;  // tensor-memory lane = state column j on the state side
-  const int wg = tid >> 7;    // warpgroup 0..3
+  int mma_issued = 0, mma_done = 0;
+  bool in_done = false, failed = false;
 
-  uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
-  bool pend_qkg = false, pend_v = false, pend_mma = false;
-  constexpr uint32_t qkg_bytes = (PC ? 3 : 2) * K16;
-
-  auto issue_qkg = [&](int64_t cs) {
-    mbar_arrive_expect_tx(bar_qkg, qkg_bytes);
-    for (int bx = 0; bx < 2; ++bx) {
-      const int x = h * D + 64 * bx;
-      tma_load_2d(sm + L_::SK + bx * K8, &a.tm_k, bar_qkg, x, (int)cs);
-      tma_load_2d(sm + L_::SG + bx * K8, &a.tm_g, bar_qkg, x, (int)cs);
-      if (PC) tma_load_2d(sm + L_::SQ + bx * K8, &a.tm_q, bar_qkg, x, (int)cs);
-    }
+  auto a_ptr = [&](int r, int cc) -> float* {
+    return reinterpret_cast<float*>(sm + L_::A) + r * 64 + ((((cc >> 2) ^ (r & 15))) << 2) +
+           (cc & 3);
   };
-  auto issue_v = [&](int64_t cs) {
-    mbar_arrive_expect_tx(bar_v, K16);
-    for (int bx = 0; bx < 2; ++bx)
-      tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_v, h * D + 64 * bx, (int)cs);
+  auto n_ptr = [&](int r, int cc) -> float* {
+    return reinterpret_cast<float*>(sm + L_::NS) + r * 64 + ((((cc >> 2) ^ (r & 15))) << 2) +
+           (cc & 3);
+  };
+  auto a4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(a_ptr(r, cc)); };
+  auto n4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(n_ptr(r, cc)); };
+  auto fma4 = [](float sv, const float4& v, float4& acc) {
+    acc.x = fmaf(sv, v.x, acc.x);
+    acc.y = fmaf(sv, v.y, acc.y);
+    acc.z = fmaf(sv, v.z, acc.z);
+    acc.w = fmaf(sv, v.w, acc.w);
   };
 
-  if (tid == 0 && c_begin < c_end) {
-    issue_qkg(c_begin);
-    issue_v(c_begin);
-  }
-  pend_qkg = pend_v = (c_begin < c_end);
-
-  // columns of the state this thread handles: output pass, warpgroup g takes
-  // columns [32g, 32g+32); summary pass, block g/2, columns [64(g%2), +64)
-  const int st_b = PC ? 0 : (wg >> 1);
-  const int st_lo = PC ? 32 * wg : 64 * (wg & 1);
-  const int st_hi = st_lo + (PC ? 32 : 64);
-
-  // ---- initial state: fp32 into tensor memory, bf16 copy as the MMA operand
-  {
-    const float* src = nullptr;
-    if (PC) {
-      if (nseg > 1) src = a.sstart + ((int64_t)pair * a.max_segs + seg) * D * D;
-      else if (a.s0) src = a.s0 + (int64_t)pair * D * D;
-    }
-    for (int c = st_lo; c < st_hi; c += 32) {
-      uint32_t v[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        float x;
-        if (PC) x = src ? src[(int64_t)(c + t) * D + row] : 0.f;
-        else x = (st_b == 0 && c + t == row) ? 1.f : 0.f;
-        v[t] = __float_as_uint(x);
-      }
-      tmem_st32(tb + lane_base + L_::st(st_b) + c, v);
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8)
-        *reinterpret_cast<uint4*>(sm + L_::S + st_b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
-    }
-    tmem_st_wait();
-  }
-
-  // beta: threads 0..63 hold the next chunk's value (bf16 bits) in a register
-  uint16_t bnext = 0;
-  if (tid < C && c_begin + tid < c_end)
-    bnext = ldg_u16_early(a.beta + (c_begin + tid) * a.H + h);
-
-  tc_fence_before();
-  fence_async_smem();
-  __syncthreads();
-
-  const int p = tid & 63, e8 = tid >> 6;  // elementwise: channel pair, group of 8 rows
-  const int ch = 2 * p, bx = p >> 5, cofs = (p & 31) * 4;
-  bool failed = false;
-
-  for (int64_t c0 = c_begin; c0 < c_end && !failed; c0 += C) {
-    const int L = (c_end - c0) < C ? (int)(c_end - c0) : C;
-    const bool has_next = c0 + C < c_end;
-
-    // ---------------- [A] decay prefix sums and the decayed operand tiles
-    if (tid < C) {
-      bet[tid] = bf16_bits_to_float(bnext);
-      bnext = 0;
-      if (has_next && c0 + C + tid < c_end)
-        bnext = ldg_u16_early(a.beta + (c0 + C + tid) * a.H + h);
-    }
+  do {
+    if (cta_wait_failed(bar_in, 0)) { failed = true; break; }
+    in_done = true;
+    // ---- 1. raw k, q into registers; prefix sums of the clamped log decay.
+    //         Thread = (channel pair p, quarter qr of 16 rows).
+    const int p = tid & 63, qr = tid >> 6;
+    const int ch = 2 * p, bx = p >> 5, cofs = (p & 31) * 4;
+    uint32_t kraw[16], qraw[16];
+    float G0[16], G1[16];
     {
-      const bool ok = mbar_wait(bar_qkg, ph_qkg) && mbar_wait(bar_v, ph_v);
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      ph_qkg ^= 1;
-      ph_v ^= 1;
-      pend_qkg = pend_v = false;
-    }
-    float G0[8], G1[8];
-    {
-      float r0 = 0.f, r1 = 0.f;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * e8 + i;
-        const float2 gg =
-            unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + bx * K8 + r * 128 + cofs));
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * qr + i;
+        const uint32_t off = bx * K8 + r * 128 + cofs;
+        kraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SK + off);
+        qraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SQ + off);
+        const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + off));
         if (r < L) {
-          r0 += fmaxf(gg.x, a.lb);
-          r1 += fmaxf(gg.y, a.lb);
+          acc0 += fmaxf(gg.x, a.lb);
+          acc1 += fmaxf(gg.y, a.lb);
         }
-        G0[i] = r0;
-        G1[i] = r1;
+        G0[i] = acc0;
+        G1[i] = acc1;
       }
-      *reinterpret_cast<float2*>(tot + e8 * 128 + ch) = make_float2(r0, r1);
+      *reinterpret_cast<float2*>(tot + qr * 128 + ch) = make_float2(acc0, acc1);
     }
-    __syncthreads();
+    __syncthreads();  // every raw read is done: SK, SG and SQ may be overwritten
+    // ---- 2. decay tiles: K~, Q~ (MMA operands), K^ (MMA operand); Kb, Q~, gl to the workspace
     {
       float o0 = 0.f, o1 = 0.f, s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         const float2 tq = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
-        if (q < e8) {
+        if (q < qr) {
           o0 += tq.x;
           o1 += tq.y;
         }
         s0 += tq.x;
         s1 += tq.y;
       }
-      // gamma at the last row of the chunk (rows past L add nothing)
       const float gl0 = expf(s0), gl1 = expf(s1);
-      if (e8 == 7) *reinterpret_cast<float2*>(gl + ch) = make_float2(gl0, gl1);
+      if (qr == 3) *reinterpret_cast<float2*>(a.gl + tile * D + ch) = make_float2(gl0, gl1);
+      uint32_t* kbo = reinterpret_cast<uint32_t*>(a.kb + tile * C * D + ch);
+      uint32_t* qto = reinterpret_cast<uint32_t*>(a.qt + tile * C * D + ch);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * e8 + i;
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * qr + i;
         const float g0 = G0[i] + o0, g1 = G1[i] + o1;
         const float e0 = __expf(g0), e1 = __expf(g1);
         const float ei0 = __expf(-g0), ei1 = __expf(-g1);
-        float2 kk = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SK + bx * K8 + r * 128 + cofs));
-        if (r >= L) kk = make_float2(0.f, 0.f);
-        *reinterpret_cast<uint32_t*>(sm + L_::KQ + sw128_off(r, ch, K16)) =
-            pack_bf16(kk.x * e0, kk.y * e1);
-        const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
-        *reinterpret_cast<uint32_t*>(sm + L_::KH + sw128_off(r, ch, L_::KH_AS)) =
-            pack_bf16(kh0, kh1);
-        *reinterpret_cast<uint32_t*>(sm + L_::KB + sw128_off(r, ch, K8)) =
-            pack_bf16(kh0 * gl0, kh1 * gl1);
-        if (PC) {
-          float2 qq =
-              unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SQ + bx * K8 + r * 128 + cofs));
-          if (r >= L) qq = make_float2(0.f, 0.f);
-          *reinterpret_cast<uint32_t*>(sm + L_::KQ + K8 + sw128_off(r, ch, K16)) =
-              pack_bf16(qq.x * e0, qq.y * e1);
+        float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
+        if (r >= L) {
+          kk = make_float2(0.f, 0.f);
+          qq = make_float2(0.f, 0.f);
         }
+        const uint32_t kt = pack_bf16(kk.x * e0, kk.y * e1);
+        const uint32_t qt = pack_bf16(qq.x * e0, qq.y * e1);
+        const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
+        *reinterpret_cast<uint32_t*>(sm + L_::KQ + sw128_off(r, ch, K16)) = kt;
+        *reinterpret_cast<uint32_t*>(sm + L_::KQ + K8 + sw128_off(r, ch, K16)) = qt;
+        *reinterpret_cast<uint32_t*>(sm + L_::KH + sw128_off(r, ch, K8)) = pack_bf16(kh0, kh1);
+        kbo[r * (D / 2)] = pack_bf16(kh0 * gl0, kh1 * gl1);
+        qto[r * (D / 2)] = qt;
       }
     }
     fence_async_smem();
-    __syncthreads();  // operand tiles complete; every read of the q/k/g staging is done
-    if (tid == 0 && has_next) {
-      issue_qkg(c0 + C);
-      pend_qkg = true;
-    }
-
-    // ---------------- [B] MMA-g: [K~;Q~|K^] K^^T  and  MMA-a: S^T [K~;Q~]^T
+    __syncthreads();
+    // ---- 3. MMA-g: [K~; Q~] K^^T, M = 128 (64 rows of K~, then 64 of Q~), N = 64
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ig = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;
-        const uint32_t kho = (k >> 2) * L_::KH_AS + (k & 3) * 32;
+        const uint32_t kho = (k >> 2) * K8 + (k & 3) * 32;
         umma_bf16(tb + L_::G, sdesc_sw128(sb + L_::KQ + ko, 16, 1024),
                   sdesc_sw128(sb + L_::KH + kho, 16, 1024), ig, k > 0);
       }
-      const uint32_t ia = idesc_bf16(128, PC ? 128 : 64, 0, 0);
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;
-          umma_bf16(tb + L_::xu(b), sdesc_sw128(sb + L_::S + b * K32 + ko, 16, 1024),
-                    sdesc_sw128(sb + L_::KQ + ko, 16, 1024), ia, k > 0);
-        }
       umma_commit(bar_mma);
     }
-    pend_mma = true;
-    {
-      const bool ok = mbar_wait(bar_mma, ph_mma);
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      ph_mma ^= 1;
-      pend_mma = false;
-    }
+    mma_issued = 1;
+    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
+    mma_done = 1;
     tc_fence_after();
-
-    // ---------------- [C] T = (I + A)^{-1} Diag(beta) and P (warps 0-3), (V - X)^T (4-15)
-    // fp32 64x64 tiles A (in the K^ tile, no longer needed) and N = (I + A)^{-1}:
-    // element (r, c) at r*64 + 4*((c/4) ^ (r%16)) + c%4, so 16-byte groups stay whole.
-    auto a_ptr = [&](int r, int c) -> float* {
-      return reinterpret_cast<float*>(sm + L_::as_piece(r >> 5)) + (r & 31) * 64 +
-             ((((c >> 2) ^ (r & 15))) << 2) + (c & 3);
-    };
-    auto n_ptr = [&](int r, int c) -> float* {
-      return reinterpret_cast<float*>(sm + L_::NS) + r * 64 + ((((c >> 2) ^ (r & 15))) << 2) +
-             (c & 3);
-    };
-    if (warp < 2) {
-      // A = Diag(beta) strict_lower(K~ K^^T): thread r owns row r (tensor-memory lanes 0..63)
-      const int r = tid;
-      const float br = bet[r];
-#pragma unroll
-      for (int cb = 0; cb < 64; cb += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::G + cb, v);
-        tmem_ld_wait(v);
+    // ---- 4. A (fp32, beta-scaled strict lower) to shared memory; P^T to the workspace
+    {
+      const int wq = warp & 3, cb = (warp >> 2) * 32;
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::G + cb, v);
+      tmem_ld_wait(v);
+      if (wq < 2) {
+        const int r = wq * 32 + lane;
+        const float br = bet[r];
 #pragma unroll
         for (int g4 = 0; g4 < 8; ++g4) {
           float4 f;
-          const int c = cb + 4 * g4;
-          f.x = (c + 0 < r) ? br * __uint_as_float(v[4 * g4 + 0]) : 0.f;
-          f.y = (c + 1 < r) ? br * __uint_as_float(v[4 * g4 + 1]) : 0.f;
-          f.z = (c + 2 < r) ? br * __uint_as_float(v[4 * g4 + 2]) : 0.f;
-          f.w = (c + 3 < r) ? br * __uint_as_float(v[4 * g4 + 3]) : 0.f;
-          *reinterpret_cast<float4*>(a_ptr(r, c)) = f;
+          const int cc = cb + 4 * g4;
+          f.x = (cc + 0 < r) ? br * __uint_as_float(v[4 * g4 + 0]) : 0.f;
+          f.y = (cc + 1 < r) ? br * __uint_as_float(v[4 * g4 + 1]) : 0.f;
+          f.z = (cc + 2 < r) ? br * __uint_as_float(v[4 * g4 + 2]) : 0.f;
+          f.w = (cc + 3 < r) ? br * __uint_as_float(v[4 * g4 + 3]) : 0.f;
+          *reinterpret_cast<float4*>(a_ptr(r, cc)) = f;
         }
-      }
-    } else if (warp < 4) {
-      if (PC) {
-        // P = lower_incl(Q~ K^^T): tensor-memory lanes 64..127, bf16 operand tile
-        const int r = tid - 64;
+      } else {
+        const int r = (wq - 2) * 32 + lane;
+        __nv_bfloat16* po = a.pt + (tile * C + cb) * C + r;
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + lane_base + L_::G + cb, v);
-          tmem_ld_wait(v);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            float f[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int sc = cb + 8 * q8 + t;
-              f[t] = (sc <= r) ? __uint_as_float(v[8 * q8 + t]) : 0.f;
-            }
-            *reinterpret_cast<uint4*>(sm + L_::P + sw128_chunk(r, cb / 8 + q8, K8)) = pack8(f);
-          }
-        }
-      }
-    } else {
-      // (V - X)^T in 32-column units (block b, half), dealt to warpgroups 1..3
-      const int j = row;
-      for (int u = wg - 1; u < 2 * NB; u += 3) {
-        const int b = u >> 1, cb = (u & 1) * 32;
-        const bool use_v = PC || b == 1;
-        uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
-        tmem_ld_wait(v);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          float f[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int r = cb + 8 * q8 + t;
-            const float vv =
-                use_v ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                            sm + L_::SV + (j >> 6) * K8 + r * 128 + (j & 63) * 2))
-                      : 0.f;
-            f[t] = vv - __uint_as_float(v[8 * q8 + t]);
-          }
-          *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(j, cb / 8 + q8, K16)) =
-              pack8(f);
-        }
+        for (int t = 0; t < 32; ++t)
+          po[t * C] = __float2bfloat16_rn(cb + t <= r ? __uint_as_float(v[t]) : 0.f);
       }
     }
-    __syncthreads();  // A, P and (V - X)^T written; every read of the v staging is done
-    if (tid == 0 && has_next) {
-      issue_v(c0 + C);
-      pend_v = true;
-    }
-    // diagonal 16x16 blocks of N by right-looking forward substitution:
-    // warp w, half h -> block 2w+h; lane l -> column l of the block
-    if (warp < 2) {
-      const int base = 16 * (2 * warp + (lane >> 4)), l = lane & 15;
-      float acc[16];
-#pragma unroll
-      for (int rr = 0; rr < 16; ++rr) acc[rr] = (rr == l) ? 1.f : 0.f;
+    tc_fence_before();
+    __syncthreads();
+    // ---- 5. N = (I + A)^{-1}: 16x16 diagonal blocks, then 16->32 and 32->64 merges
+    if (warp < 4 && lane < 16) {
+      const int base = 16 * warp, l = lane;
+      float nv[16];
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr) {
-        const float nv = acc[rr];
-        *n_ptr(base + rr, base + l) = nv;
+        float arow[16];
 #pragma unroll
-        for (int r2 = rr + 1; r2 < 16; ++r2)
-          acc[r2] = fmaf(-*a_ptr(base + r2, base + rr), nv, acc[r2]);
+        for (int g4 = 0; g4 < (rr + 3) / 4; ++g4) {
+          const float4 v4 = a4(base + rr, base + 4 * g4);
+          arow[4 * g4 + 0] = v4.x;
+          arow[4 * g4 + 1] = v4.y;
+          arow[4 * g4 + 2] = v4.z;
+          arow[4 * g4 + 3] = v4.w;
+        }
+        float e0 = (rr == l) ? 1.f : 0.f, e1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < rr; kk += 2) {
+          e0 = fmaf(-arow[kk], nv[kk], e0);
+          if (kk + 1 < rr) e1 = fmaf(-arow[kk + 1], nv[kk + 1], e1);
+        }
+        nv[rr] = (rr < l) ? 0.f : e0 + e1;
+        *n_ptr(base + rr, base + l) = nv[rr];
       }
     }
     __syncthreads();
     float* bt1 = bt;  // [2][16][16]
     float* bt2 = bt;  // [32][36]
-    {
-      // level 1: in each 32-block, N10 = -N11 (A10 N00) with 16x16 blocks
-      const int b = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
-      const int R0 = 32 * b, R1 = 32 * b + 16;
-      float sacc = 0.f;
+    if (tid < 128) {
+      const int b = tid >> 6, r = (tid >> 2) & 15, cg = tid & 3;
+      const int R0 = 32 * b, R1 = R0 + 16;
+      float av[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) sacc = fmaf(*a_ptr(R1 + r, R0 + k), *n_ptr(R0 + k, R0 + c), sacc);
-      bt1[b * 256 + r * 16 + c] = sacc;
-      __syncthreads();
-      float tacc = 0.f;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) tacc = fmaf(*n_ptr(R1 + r, R1 + k), bt1[b * 256 + k * 16 + c], tacc);
-      *n_ptr(R1 + r, R0 + c) = -tacc;
-      *n_ptr(R0 + r, R1 + c) = 0.f;  // upper-right 16x16 block of each 32-block (read by level 2)
-      __syncthreads();
-    }
-    {
-      // level 2: N10 = -N11 (A10 N00) with 32x32 blocks
-      const int r = tid >> 4, c = (tid & 15) * 2;
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float av = *a_ptr(32 + r, k);
-        const float2 nn = *reinterpret_cast<const float2*>(n_ptr(k, c));
-        s0 = fmaf(av, nn.x, s0);
-        s1 = fmaf(av, nn.y, s1);
+      for (int g4 = 0; g4 < 4; ++g4) {
+        const float4 v4 = a4(R1 + r, R0 + 4 * g4);
+        av[4 * g4 + 0] = v4.x;
+        av[4 * g4 + 1] = v4.y;
+        av[4 * g4 + 2] = v4.z;
+        av[4 * g4 + 3] = v4.w;
       }
-      *reinterpret_cast<float2*>(bt2 + r * 36 + c) = make_float2(s0, s1);
-      __syncthreads();
-      float u0 = 0.f, u1 = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float nv = *n_ptr(32 + r, 32 + k);
-        const float2 bb = *reinterpret_cast<const float2*>(bt2 + k * 36 + c);
-        u0 = fmaf(nv, bb.x, u0);
-        u1 = fmaf(nv, bb.y, u1);
-      }
-      *reinterpret_cast<float2*>(n_ptr(32 + r, c)) = make_float2(-u0, -u1);
-      __syncthreads();
+      for (int k = 0; k < 16; ++k) fma4(av[k], n4(R0 + k, R0 + 4 * cg), acc);
+      *reinterpret_cast<float4*>(bt1 + b * 256 + r * 16 + 4 * cg) = acc;
     }
+    __syncthreads();
+    if (tid < 128) {
+      const int b = tid >> 6, r = (tid >> 2) & 15, cg = tid & 3;
+      const int R0 = 32 * b, R1 = R0 + 16;
+      float nr[16];
+#pragma unroll
+      for (int g4 = 0; g4 < 4; ++g4) {
+        const float4 v4 = n4(R1 + r, R1 + 4 * g4);
+        nr[4 * g4 + 0] = v4.x;
+        nr[4 * g4 + 1] = v4.y;
+        nr[4 * g4 + 2] = v4.z;
+        nr[4 * g4 + 3] = v4.w;
+      }
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        fma4(nr[k], *reinterpret_cast<const float4*>(bt1 + b * 256 + k * 16 + 4 * cg), acc);
+      *reinterpret_cast<float4*>(n_ptr(R1 + r, R0 + 4 * cg)) =
+          make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+      *reinterpret_cast<float4*>(n_ptr(R0 + r, R1 + 4 * cg)) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
     {
-      // T = N Diag(beta), lower triangle, as the bf16 operand: one 16-byte chunk per thread
-      const int r = tid >> 3, c8 = tid & 7;
-      float f[8];
+      const int r = tid >> 3, cg = tid & 7;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int h4 = 0; h4 < 2; ++h4) {
-        const int c = 8 * c8 + 4 * h4;
-        const float4 nn = *reinterpret_cast<const float4*>(n_ptr(r, c));
-        const float4 bb = *reinterpret_cast<const float4*>(bet + c);
-        f[4 * h4 + 0] = (c + 0 <= r) ? nn.x * bb.x : 0.f;
-        f[4 * h4 + 1] = (c + 1 <= r) ? nn.y * bb.y : 0.f;
-        f[4 * h4 + 2] = (c + 2 <= r) ? nn.z * bb.z : 0.f;
-        f[4 * h4 + 3] = (c + 3 <= r) ? nn.w * bb.w : 0.f;
+      for (int g4 = 0; g4 < 8; ++g4) {
+        const float4 v4 = a4(32 + r, 4 * g4);
+        fma4(v4.x, n4(4 * g4 + 0, 4 * cg), acc);
+        fma4(v4.y, n4(4 * g4 + 1, 4 * cg), acc);
+        fma4(v4.z, n4(4 * g4 + 2, 4 * cg), acc);
+        fma4(v4.w, n4(4 * g4 + 3, 4 * cg), acc);
       }
-      *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(r, c8, K8)) = pack8(f);
+      *reinterpret_cast<float4*>(bt2 + r * 36 + 4 * cg) = acc;
     }
-    tc_fence_before();
+    __syncthreads();
+    {
+      const int r = tid >> 3, cg = tid & 7;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int g4 = 0; g4 < 8; ++g4) {
+        const float4 v4 = n4(32 + r, 32 + 4 * g4);
+        fma4(v4.x, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 0) * 36 + 4 * cg), acc);
+        fma4(v4.y, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 1) * 36 + 4 * cg), acc);
+        fma4(v4.z, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 2) * 36 + 4 * cg), acc);
+        fma4(v4.w, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 3) * 36 + 4 * cg), acc);
+      }
+      *reinterpret_cast<float4*>(n_ptr(32 + r, 4 * cg)) =
+          make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+    // ---- 6. T = N Diag(beta), lower triangle, bf16 operand: two 16-byte chunks per thread
+    {
+      const int r = tid >> 2;
+#pragma unroll
+      for (int q8 = 0; q8 < 2; ++q8) {
+        const int c8 = (tid & 3) * 2 + q8;
+        float f[8];
+#pragma unroll
+        for (int h4 = 0; h4 < 2; ++h4) {
+          const int cc = 8 * c8 + 4 * h4;
+          const float4 nn = n4(r, cc);
+          const float4 bb = *reinterpret_cast<const float4*>(bet + cc);
+          f[4 * h4 + 0] = (cc + 0 <= r) ? nn.x * bb.x : 0.f;
+          f[4 * h4 + 1] = (cc + 1 <= r) ? nn.y * bb.y : 0.f;
+          f[4 * h4 + 2] = (cc + 2 <= r) ? nn.z * bb.z : 0.f;
+          f[4 * h4 + 3] = (cc + 3 <= r) ? nn.w * bb.w : 0.f;
+        }
+        *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(r, c8, K8)) = pack8(f);
+      }
+    }
     fence_async_smem();
     __syncthreads();
-
-    // ---------------- [D] MMA-b: U^T = (V - X)^T T^T
+    // ---- 7. W^T = K~^T T^T and U0^T = V^T T^T. K~ (in the Gram operand) and V (as
+    //         loaded) serve as MN-major A operands: 64-element column groups LBO apart,
+    //         8-row groups 1024 bytes apart, 16 rows of K per instruction.
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ib = idesc_bf16(128, 64, 0, 0);
+      const uint32_t iw = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(tb + L_::xu(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
-                    sdesc_sw128(sb + L_::T + k * 32, 16, 1024), ib, k > 0);
+      for (int k = 0; k < C / 16; ++k) {
+        const uint64_t tdesc = sdesc_sw128(sb + L_::T + k * 32, 16, 1024);
+        umma_bf16(tb + L_::W, sdesc_sw128(sb + L_::KQ + k * 2048, K16, 1024), tdesc, iw, k > 0);
+        umma_bf16(tb + L_::U, sdesc_sw128(sb + L_::SV + k * 2048, K8, 1024), tdesc, iw, k > 0);
+      }
       umma_commit(bar_mma);
     }
-    pend_mma = true;
-    {
-      const bool ok = mbar_wait(bar_mma, ph_mma);
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      ph_mma ^= 1;
-      pend_mma = false;
-    }
+    mma_issued = 2;
+    if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
+    mma_done = 2;
     tc_fence_after();
-
-    // ---------------- [E] U^T -> bf16 operand
-    if (PC) {
-      const int cb = 16 * wg;
-      uint32_t v[16];
-      tmem_ld16(tb + lane_base + L_::xu(0) + cb, v);
-      tmem_ld_wait(v);
-#pragma unroll
-      for (int q8 = 0; q8 < 2; ++q8)
-        *reinterpret_cast<uint4*>(sm + L_::Y + sw128_chunk(row, cb / 8 + q8, K16)) =
-            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
-    } else {
-      const int b = wg >> 1, cb = 32 * (wg & 1);
+    // ---- 8. -W and U0 to the workspace: tensor-memory lane i holds column i of both
+    {
+      const int i = (warp & 3) * 32 + lane, cb = (warp >> 2) * 32;
       uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::xu(b) + cb, v);
+      tmem_ld32(tb + lane_base + L_::W + cb, v);
+      tmem_ld_wait(v);
+      __nv_bfloat16* wo = a.wn + (tile * C + cb) * D + i;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) wo[t * D] = __float2bfloat16_rn(-__uint_as_float(v[t]));
+      tmem_ld32(tb + lane_base + L_::U + cb, v);
+      tmem_ld_wait(v);
+      __nv_bfloat16* uo = a.u0 + (tile * C + cb) * D + i;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) uo[t * D] = __float2bfloat16_rn(__uint_as_float(v[t]));
+    }
+  } while (0);
+  if (failed && tid == 0) {
+    atomicExch(a.seq.status, kDevWaitTimeout);
+    // copies and products in flight finish before the CTA releases its memory
+    if (!in_done) mbar_wait(bar_in, 0, 400000000LL);
+    for (int m = mma_done; m < mma_issued; ++m) mbar_wait(bar_mma, m & 1, 400000000LL);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, L_::COLS);
+  }
+}
+
+// ------------------------------------------------------------------ walk over chunks
+// One CTA of 8 warps per (sequence, head, segment). Warps w and w + 4 share the
+// tensor-memory lanes 32 (w % 4) .. + 31 (state columns j) and split the columns.
+// Thread 0 streams the next chunk's workspace tiles (two stages) and issues the MMAs.
+constexpr int kWalkThreads = 256;
+template <bool PC>
+struct WalkSm {
+  static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks: [S] or [M | L]
+  // one input stage: -W | U0 | Kb | (Q~ | P^T); two 64-column boxes per [64][128] tile
+  static constexpr uint32_t WN = 0, U0 = K16, KB = 2 * K16, QT = 3 * K16, PT = 4 * K16;
+  static constexpr uint32_t STAGE = PC ? 4 * K16 + K8 : 3 * K16;
+  static constexpr uint32_t STAGE_TX = STAGE + 512;  // + gl
+  static constexpr uint32_t S = 2 * STAGE;             // bf16 S^T, [128 j][128 i], 32 KB/block
+  static constexpr uint32_t Y = S + NB * K32;          // bf16 U^T, [128 j][64 r], 16 KB/block
+  static constexpr uint32_t OS = Y + NB * K16;         // output staging: two [64 r][64 j] boxes
+  static constexpr uint32_t ID = OS + (PC ? K16 : 0);  // bf16 64x64 identity
+  static constexpr uint32_t GL = ID + K8;              // float[2][128]
+  static constexpr uint32_t BARS = GL + 1024;
+  static constexpr uint32_t TPTR = BARS + 64;
+  static constexpr uint32_t BYTES = TPTR + 16;
+  // tensor-memory columns: fp32 S^T per block, U^T per block, O^T
+  __device__ static constexpr uint32_t st(int b) { return 128 * b; }
+  __device__ static constexpr uint32_t uc(int b) { return PC ? 128 : 256 + 64 * b; }
+  static constexpr uint32_t YO = 192;
+  static constexpr uint32_t COLS = PC ? 256 : 512;
+};
+static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
+static_assert(WalkSm<false>::BYTES + 1024 <= 232448, "summary walk shared memory");
+
+template <bool PC>
+__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_constant__ WalkArgs a) {
+  using L_ = WalkSm<PC>;
+  constexpr int NB = L_::NB;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = align1024(smem_raw);
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int per = PC ? a.max_segs : a.max_segs - 1;
+  const int seg = blockIdx.x % per;
+  const int pair = blockIdx.x / per;
+  const int s = pair / a.H, h = pair % a.H;
+  int64_t t0, t1;
+  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
+  const int64_t len = t1 - t0;
+  const int nseg = len > 0 ? static_cast<int>((len + a.seg_tokens - 1) / a.seg_tokens) : 1;
+  if (nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
+    if (seg == 0 && tid == 0) atomicExch(a.seq.status, kDevBadSeqlens);
+    return;
+  }
+  if (PC ? (seg >= nseg) : (seg >= nseg - 1)) return;
+  const int64_t c_begin = t0 + static_cast<int64_t>(seg) * a.seg_tokens;
+  const int64_t c_end = (c_begin + a.seg_tokens < t1) ? c_begin + a.seg_tokens : t1;
+  const int n_chunks = static_cast<int>((c_end - c_begin + C - 1) / C);
+  // workspace tile of chunk n of this segment: tile0 + n H
+  const int64_t tile0 =
+      (slot_base(t0, s) + static_cast<int64_t>(seg) * (a.seg_tokens / C)) * a.H + h;
+
+  float* gls = reinterpret_cast<float*>(sm + L_::GL);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_::BARS);
+  uint64_t* bar_full = bars;  // two stages
+  uint64_t* bar_m1 = bars + 2;
+  uint64_t* bar_m2 = bars + 3;
+  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
+
+  auto issue_stage = [&](int n) {  // thread 0
+    const int st = n & 1;
+    unsigned char* dst = sm + st * L_::STAGE;
+    const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
+    const int y = static_cast<int>(tile * C);
+    mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
+    for (int bx = 0; bx < 2; ++bx) {
+      tma_load_2d(dst + L_::WN + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
+      tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 64 * bx, y);
+      tma_load_2d(dst + L_::KB + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
+      if (PC) tma_load_2d(dst + L_::QT + bx * K8, &a.tm_qt, bar_full + st, 64 * bx, y);
+    }
+    if (PC) tma_load_2d(dst + L_::PT, &a.tm_pt, bar_full + st, 0, y);
+    bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
+  };
+
+  if (warp == 0) {
+    tmem_alloc(tptr, L_::COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+    if (n_chunks > 0) {
+      tma_prefetch_desc(&a.tm_wn);
+      tma_prefetch_desc(&a.tm_u0);
+      tma_prefetch_desc(&a.tm_kb);
+      if (PC) {
+        tma_prefetch_desc(&a.tm_qt);
+        tma_prefetch_desc(&a.tm_pt);
+      }
+      issue_stage(0);
+    }
+  }
+  // identity operand: zeros, then the diagonal
+  for (int e = tid; e < static_cast<int>(K8 / 16); e += kWalkThreads)
+    *reinterpret_cast<uint4*>(sm + L_::ID + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid < C) *reinterpret_cast<uint16_t*>(sm + L_::ID + sw128_off(tid, tid, K8)) = 0x3F80u;
+  const uint32_t tb = *tptr;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
+  const int hc = warp >> 2;                // column half this thread converts
+
+  // initial state: fp32 into tensor memory, bf16 copy as the MMA operand
+  {
+    const float* src = nullptr;
+    if (PC) {
+      if (nseg > 1) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
+      else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
+    }
+    for (int b = 0; b < NB; ++b)
+      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+        uint32_t v[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          float x;
+          if (PC) x = src ? src[static_cast<int64_t>(c + t) * D + row] : 0.f;
+          else x = (b == 0 && c + t == row) ? 1.f : 0.f;
+          v[t] = __float_as_uint(x);
+        }
+        tmem_st32(tb + lane_base + L_::st(b) + c, v);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
+              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+      }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  fence_async_smem();
+  __syncthreads();
+  tc_fence_after();
+
+  int full_issued = n_chunks > 0 ? 1 : 0, full_done = 0;
+  int m1_issued = 0, m2_issued = 0, m1_done = 0, m2_done = 0;
+  bool failed = false;
+  for (int n = 0; n < n_chunks; ++n) {
+    const int st = n & 1;
+    const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
+    const int L = (c_end - c0) < C ? static_cast<int>(c_end - c0) : C;
+    const uint32_t stg = sb + st * L_::STAGE;
+    if (cta_wait_failed(bar_full + st, (n >> 1) & 1)) { failed = true; break; }
+    ++full_done;
+    // ---- MMA-1: U^T = U0^T I + S^T (-W)^T per block; (Q~ S)^T = S^T Q~^T
+    if (tid == 0) {
+      if (n + 1 < n_chunks) issue_stage(n + 1);
+      tc_fence_after();
+      const uint32_t i_k = idesc_bf16(128, 64, 0, 0), i_mn = idesc_bf16(128, 64, 1, 0);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
+        if (with_u0) {
+#pragma unroll
+          for (int k = 0; k < C / 16; ++k)
+            umma_bf16(tb + L_::uc(b), sdesc_sw128(stg + L_::U0 + k * 2048, K8, 1024),
+                      sdesc_sw128(sb + L_::ID + k * 32, 16, 1024), i_mn, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32, ko_w = (k >> 2) * K8 + (k & 3) * 32;
+          umma_bf16(tb + L_::uc(b), sdesc_sw128(sb + L_::S + b * K32 + ko_s, 16, 1024),
+                    sdesc_sw128(stg + L_::WN + ko_w, 16, 1024), i_k, (with_u0 || k > 0) ? 1u : 0u);
+        }
+      }
+      if (PC) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32, ko_w = (k >> 2) * K8 + (k & 3) * 32;
+          umma_bf16(tb + L_::YO, sdesc_sw128(sb + L_::S + ko_s, 16, 1024),
+                    sdesc_sw128(stg + L_::QT + ko_w, 16, 1024), i_k, k > 0);
+        }
+      }
+      umma_commit(bar_m1);
+    }
+    ++m1_issued;
+    if (n + 1 < n_chunks) ++full_issued;
+    // ---- while MMA-1 runs: S <- Diag(gl) S in tensor memory (MMA-1 reads the bf16 copy)
+    {
+      const float* gl = gls + st * D;
+#pragma unroll 1
+      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+        float gv[32];
+#pragma unroll
+        for (int t4 = 0; t4 < 8; ++t4)
+          *reinterpret_cast<float4*>(gv + 4 * t4) = *reinterpret_cast<const float4*>(gl + c + 4 * t4);
+#pragma unroll 1
+        for (int b = 0; b < NB; ++b) {
+          uint32_t sv[32];
+          tmem_ld32(tb + lane_base + L_::st(b) + c, sv);
+          tmem_ld_wait(sv);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) sv[t] = __float_as_uint(gv[t] * __uint_as_float(sv[t]));
+          tmem_st32(tb + lane_base + L_::st(b) + c, sv);
+        }
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    if (cta_wait_failed(bar_m1, n & 1)) { failed = true; break; }
+    ++m1_done;
+    tc_fence_after();
+    // ---- U^T -> bf16 operand (this thread's 32 columns of each block)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::uc(b) + 32 * hc, v);
       tmem_ld_wait(v);
 #pragma unroll
       for (int q8 = 0; q8 < 4; ++q8)
-        *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, cb / 8 + q8, K16)) =
+        *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, 4 * hc + q8, K16)) =
             pack8(reinterpret_cast<const float*>(v) + 8 * q8);
     }
+    if (PC && tid == 0) bulk_wait_read();  // the previous output store has read OS
     tc_fence_before();
     fence_async_smem();
     __syncthreads();
-
-    // ---------------- [F] MMA-c: O^T += U^T P^T (output pass);  MMA-d: Z = U^T Kb
+    // ---- MMA-2: O^T += U^T P^T (output walk); S^T += U^T Kb (B operands MN-major)
     if (tid == 0) {
       tc_fence_after();
       if (PC) {
-        const uint32_t ic = idesc_bf16(128, 64, 0, 0);
+        const uint32_t ic = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
         for (int k = 0; k < C / 16; ++k)
           umma_bf16(tb + L_::YO, sdesc_sw128(sb + L_::Y + k * 32, 16, 1024),
-                    sdesc_sw128(sb + L_::P + k * 32, 16, 1024), ic, 1);
+                    sdesc_sw128(stg + L_::PT + k * 2048, K8, 1024), ic, 1);
       }
       const uint32_t id = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
       for (int b = 0; b < NB; ++b)
 #pragma unroll
         for (int k = 0; k < C / 16; ++k)
-          umma_bf16(tb + L_::z(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
-                    sdesc_sw128(sb + L_::KB + k * 2048, K8, 1024), id, k > 0);
-      umma_commit(bar_mma);
+          umma_bf16(tb + L_::st(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
+                    sdesc_sw128(stg + L_::KB + k * 2048, K8, 1024), id, 1);
+      umma_commit(bar_m2);
     }
-    pend_mma = true;
-    {
-      const bool ok = mbar_wait(bar_mma, ph_mma);
-      if (__syncthreads_or(!ok)) { failed = true; break; }
-      ph_mma ^= 1;
-      pend_mma = false;
-    }
+    ++m2_issued;
+    if (cta_wait_failed(bar_m2, n & 1)) { failed = true; break; }
+    ++m2_done;
     tc_fence_after();
-
-    // ---------------- [G] outputs; S <- Diag(gl) S + Z; bf16 S^T for the next chunk
+    // ---- outputs; bf16 S^T for the next chunk
     if (PC) {
-      const int cb = 16 * wg;
-      uint32_t v[16];
-      tmem_ld16(tb + lane_base + L_::YO + cb, v);
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::YO + 32 * hc, v);
       tmem_ld_wait(v);
-      __nv_bfloat16* o = a.out + ((c0 + cb) * a.H + h) * D + row;
-      const int64_t ostride = (int64_t)a.H * D;
+      if (L == C) {
+        // O[r][j] into two 64x64 row-major boxes; one TMA store each below
+        __nv_bfloat16* ob =
+            reinterpret_cast<__nv_bfloat16*>(sm + L_::OS + (row >> 6) * K8) + 32 * hc * 64 + (row & 63);
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        if (cb + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
-    }
-    for (int c = st_lo; c < st_hi; c += 32) {
-      uint32_t sv[32], zv[32];
-      tmem_ld32(tb + lane_base + L_::st(st_b) + c, sv);
-      tmem_ld32(tb + lane_base + L_::z(st_b) + c, zv);
-      tmem_ld_wait(sv);
-      tmem_ld_wait(zv);
+        for (int t = 0; t < 32; ++t) ob[t * 64] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
+      } else {
+        // a sequence's ragged last chunk: rows past L belong to the next sequence
+        __nv_bfloat16* o = a.out + ((c0 + 32 * hc) * a.H + h) * D + row;
+        const int64_t ostride = static_cast<int64_t>(a.H) * D;
 #pragma unroll
-      for (int t4 = 0; t4 < 8; ++t4) {
-        const float4 g4 = *reinterpret_cast<const float4*>(gl + c + 4 * t4);
-        sv[4 * t4 + 0] = __float_as_uint(fmaf(g4.x, __uint_as_float(sv[4 * t4 + 0]), __uint_as_float(zv[4 * t4 + 0])));
-        sv[4 * t4 + 1] = __float_as_uint(fmaf(g4.y, __uint_as_float(sv[4 * t4 + 1]), __uint_as_float(zv[4 * t4 + 1])));
-        sv[4 * t4 + 2] = __float_as_uint(fmaf(g4.z, __uint_as_float(sv[4 * t4 + 2]), __uint_as_float(zv[4 * t4 + 2])));
-        sv[4 * t4 + 3] = __float_as_uint(fmaf(g4.w, __uint_as_float(sv[4 * t4 + 3]), __uint_as_float(zv[4 * t4 + 3])));
+        for (int t = 0; t < 32; ++t)
+          if (32 * hc + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
       }
-      tmem_st32(tb + lane_base + L_::st(st_b) + c, sv);
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8)
-        *reinterpret_cast<uint4*>(sm + L_::S + st_b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-            pack8(reinterpret_cast<const float*>(sv) + 8 * q8);
     }
-    tmem_st_wait();
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tb + lane_base + L_::st(b) + c, v);
+        tmem_ld_wait(v);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
+              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+      }
     tc_fence_before();
     fence_async_smem();
     __syncthreads();
+    if (PC && L == C && tid == 0) {
+      tma_store_2d(&a.tm_o, sm + L_::OS, h * D, static_cast<int>(c0));
+      tma_store_2d(&a.tm_o, sm + L_::OS + K8, h * D + 64, static_cast<int>(c0));
+      bulk_commit();
+    }
   }
-
+  if (PC && tid == 0) bulk_wait_all();  // outputs written before the kernel ends
   if (failed) {
     if (tid == 0) {
-      atomicExch(a.status, kDevWaitTimeout);
-      // let copies and MMAs that were issued finish before tensor memory is released
-      if (pend_qkg) mbar_wait(bar_qkg, ph_qkg, 400000000LL);
-      if (pend_v) mbar_wait(bar_v, ph_v, 400000000LL);
-      if (pend_mma) mbar_wait(bar_mma, ph_mma, 400000000LL);
+      atomicExch(a.seq.status, kDevWaitTimeout);
+      // copies and products in flight finish before the CTA releases its memory
+      for (int f = full_done; f < full_issued; ++f) mbar_wait(bar_full + (f & 1), (f >> 1) & 1, 400000000LL);
+      for (int m = m1_done; m < m1_issued; ++m) mbar_wait(bar_m1, m & 1, 400000000LL);
+      for (int m = m2_done; m < m2_issued; ++m) mbar_wait(bar_m2, m & 1, 400000000LL);
     }
   } else {
-    // ---- write the final / summary state (row-major [i][j], fp32)
-    float* dst = nullptr;
-    if (PC) {
-      if (a.sT && seg == nseg - 1) dst = a.sT + (int64_t)pair * D * D;
-    } else {
-      const int64_t u = (int64_t)pair * (a.max_segs - 1) + seg;
-      dst = (st_b == 0 ? a.mbuf : a.lbuf) + u * D * D;
-    }
-    if (dst != nullptr) {
-      for (int c = st_lo; c < st_hi; c += 32) {
+    // ---- final / summary state (row-major [i][j], fp32)
+    for (int b = 0; b < NB; ++b) {
+      float* dst = nullptr;
+      if (PC) {
+        if (a.sT && seg == nseg - 1) dst = a.sT + static_cast<int64_t>(pair) * D * D;
+      } else {
+        const int64_t un = static_cast<int64_t>(pair) * (a.max_segs - 1) + seg;
+        dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
+      }
+      if (dst == nullptr) continue;
+      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
         uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::st(st_b) + c, v);
+        tmem_ld32(tb + lane_base + L_::st(b) + c, v);
         tmem_ld_wait(v);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) dst[(int64_t)(c + t) * D + row] = __uint_as_float(v[t]);
+        for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(c + t) * D + row] = __uint_as_float(v[t]);
       }
     }
   }
@@ -694,10 +840,11 @@ __global__ void __launch_bounds__(NT, 1) kda_tc_pass(const __grid_constant__ TcA
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tb, kTmemCols);
+    tmem_dealloc(tb, L_::COLS);
   }
 }
 
+// ------------------------------------------------------------------ combine
 // Start state of every segment: S_{j+1} = M_j S_j + L_j, fp32, one CTA per
 // (sequence, head, 16-column slice). M_{j+1} streams into shared memory
 // (cp.async, double-buffered) while step j is computed.
@@ -711,14 +858,14 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ WalkArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* Ms = reinterpret_cast<float*>(smem_raw);  // [2][128][132]
   float* Ss = Ms + 2 * D * kMStride;               // [128][16]
   const int pair = blockIdx.x / kCombSlices, j0 = (blockIdx.x % kCombSlices) * kCombCols;
   const int s = pair / a.H;
   int64_t t0, t1;
-  if (!tc_seq_bounds(a, s, t0, t1)) return;
+  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t len = t1 - t0;
   const int nseg = len > 0 ? (int)((len + a.seg_tokens - 1) / a.seg_tokens) : 1;
   if (nseg <= 1 || nseg > a.max_segs) return;
@@ -791,15 +938,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int H) {
+// 2-D bf16 tensor map over `rows` rows of `cols` elements, `pitch` bytes apart,
+// moved in 64x64 boxes; with `swizzle` a box lands in the 128-byte-swizzled
+// operand layout.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t pitch,
+              bool swizzle) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * D, static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * D * 2};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch)};
   cuuint32_t box[2] = {64, 64};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -809,6 +961,8 @@ int64_t pow2_ceil(int64_t x) {
   return p;
 }
 
+size_t align_to(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
 }  // namespace
 
 bool tc_path_applies(const kda_shape& s, int64_t T_total) {
@@ -817,8 +971,8 @@ bool tc_path_applies(const kda_shape& s, int64_t T_total) {
 
 TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   TcPlan p{};
-  const int64_t chunks = (T_total + C - 1) / C + n_seqs;
-  int64_t per_sm = (static_cast<int64_t>(H) * chunks + 147) / 148;
+  p.n_slots = (T_total + C - 1) / C + n_seqs;
+  int64_t per_sm = (static_cast<int64_t>(H) * p.n_slots + 147) / 148;
   if (per_sm < 8) per_sm = 8;
   const int64_t seg_chunks = pow2_ceil(per_sm);
   p.seg_tokens = static_cast<int>(seg_chunks * C > (int64_t(1) << 30) ? (int64_t(1) << 30)
@@ -828,60 +982,94 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   if (p.max_segs < 1) p.max_segs = 1;
   p.pairs = static_cast<int64_t>(n_seqs) * H;
   const size_t state = sizeof(float) * D * D;
-  p.ws_bytes = kWorkspaceHeader;
+  size_t off = kWorkspaceHeader;
   if (p.max_segs > 1)
-    p.ws_bytes += state * static_cast<size_t>(p.pairs) *
-                  (2 * static_cast<size_t>(p.max_segs - 1) + static_cast<size_t>(p.max_segs));
+    off += state * static_cast<size_t>(p.pairs) *
+           (2 * static_cast<size_t>(p.max_segs - 1) + static_cast<size_t>(p.max_segs));
+  p.tiles_off = align_to(off, 1024);
+  p.ws_bytes = p.tiles_off + kTileBytes * static_cast<size_t>(p.n_slots) * static_cast<size_t>(H);
   return p;
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   const TcPlan plan = tc_plan(pa.T_total, pa.n_seqs, pa.H, pa.max_len);
   if (pa.ws_bytes < plan.ws_bytes) return cudaErrorInvalidValue;
-  TcArgs a;
-  memset(&a, 0, sizeof a);
-  if (!make_map(&a.tm_q, pa.q, pa.T_total, pa.H) || !make_map(&a.tm_k, pa.k, pa.T_total, pa.H) ||
-      !make_map(&a.tm_g, pa.g, pa.T_total, pa.H) || !make_map(&a.tm_v, pa.v, pa.T_total, pa.H))
+  const int64_t tiles = plan.n_slots * pa.H;
+  const SeqTable seq{pa.cu, pa.status, pa.T, pa.T_total, pa.n_seqs};
+  // workspace: header | M, L, S_start (segmented walks only) | per-chunk tiles
+  unsigned char* tp = pa.ws + plan.tiles_off;
+  auto* wn = reinterpret_cast<__nv_bfloat16*>(tp);
+  __nv_bfloat16* u0 = wn + tiles * C * D;
+  __nv_bfloat16* kb = u0 + tiles * C * D;
+  __nv_bfloat16* qt = kb + tiles * C * D;
+  __nv_bfloat16* pt = qt + tiles * C * D;
+  auto* gl = reinterpret_cast<float*>(pt + tiles * C * C);
+  const uint64_t in_cols = static_cast<uint64_t>(pa.H) * D, in_pitch = in_cols * 2;
+  const uint64_t rows_t = static_cast<uint64_t>(tiles) * C;
+
+  IntraArgs ia;
+  memset(&ia, 0, sizeof ia);
+  WalkArgs wa;
+  memset(&wa, 0, sizeof wa);
+  if (!make_map(&ia.tm_q, pa.q, in_cols, pa.T_total, in_pitch, false) ||
+      !make_map(&ia.tm_k, pa.k, in_cols, pa.T_total, in_pitch, false) ||
+      !make_map(&ia.tm_g, pa.g, in_cols, pa.T_total, in_pitch, false) ||
+      !make_map(&ia.tm_v, pa.v, in_cols, pa.T_total, in_pitch, true) ||
+      !make_map(&wa.tm_wn, wn, D, rows_t, D * 2, true) ||
+      !make_map(&wa.tm_u0, u0, D, rows_t, D * 2, true) ||
+      !make_map(&wa.tm_kb, kb, D, rows_t, D * 2, true) ||
+      !make_map(&wa.tm_qt, qt, D, rows_t, D * 2, true) ||
+      !make_map(&wa.tm_pt, pt, C, rows_t, C * 2, true) ||
+      !make_map(&wa.tm_o, pa.out, in_cols, pa.T_total, in_pitch, false))
     return cudaErrorInvalidValue;
-  a.beta = static_cast<const __nv_bfloat16*>(pa.beta);
-  a.out = static_cast<__nv_bfloat16*>(pa.out);
-  a.s0 = pa.s0;
-  a.sT = pa.sT;
-  a.cu = pa.cu;
-  a.status = pa.status;
+  ia.seq = seq;
+  ia.beta = static_cast<const __nv_bfloat16*>(pa.beta);
+  ia.wn = wn;
+  ia.u0 = u0;
+  ia.kb = kb;
+  ia.qt = qt;
+  ia.pt = pt;
+  ia.gl = gl;
+  ia.H = pa.H;
+  ia.lb = pa.lb;
+
+  wa.seq = seq;
+  wa.gl = gl;
+  wa.out = static_cast<__nv_bfloat16*>(pa.out);
+  wa.s0 = pa.s0;
+  wa.sT = pa.sT;
   const size_t state = static_cast<size_t>(D) * D;
   float* base = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
-  a.mbuf = base;
-  a.lbuf = a.mbuf + state * plan.pairs * (plan.max_segs - 1);
-  a.sstart = a.lbuf + state * plan.pairs * (plan.max_segs - 1);
-  a.T = pa.T;
-  a.T_total = pa.T_total;
-  a.n_seqs = pa.n_seqs;
-  a.H = pa.H;
-  a.seg_tokens = plan.seg_tokens;
-  a.max_segs = plan.max_segs;
-  a.scale = pa.scale;
-  a.lb = pa.lb;
+  wa.mbuf = base;
+  wa.lbuf = wa.mbuf + state * plan.pairs * (plan.max_segs - 1);
+  wa.sstart = wa.lbuf + state * plan.pairs * (plan.max_segs - 1);
+  wa.H = pa.H;
+  wa.seg_tokens = plan.seg_tokens;
+  wa.max_segs = plan.max_segs;
+  wa.scale = pa.scale;
 
   // dynamic shared memory limits are per function and per device: set them every call
-  cudaError_t e = cudaFuncSetAttribute(kda_tc_pass<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Sm<true>::BYTES + 1024);
+  cudaError_t e = cudaFuncSetAttribute(kda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       IntraSm::BYTES + 1024);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Sm<false>::BYTES + 1024);
+    e = cudaFuncSetAttribute(kda_tc_walk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WalkSm<true>::BYTES + 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kda_tc_walk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WalkSm<false>::BYTES + 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kda_tc_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kCombSmem);
   if (e != cudaSuccess) return e;
 
+  kda_tc_intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
   if (plan.max_segs > 1) {
-    kda_tc_pass<false><<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), NT,
-                         Sm<false>::BYTES + 1024, st>>>(a);
-    kda_tc_combine<<<static_cast<unsigned>(plan.pairs * kCombSlices), 256, kCombSmem, st>>>(a);
+    kda_tc_walk<false><<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), kWalkThreads,
+                         WalkSm<false>::BYTES + 1024, st>>>(wa);
+    kda_tc_combine<<<static_cast<unsigned>(plan.pairs * kCombSlices), 256, kCombSmem, st>>>(wa);
   }
-  kda_tc_pass<true><<<static_cast<unsigned>(plan.pairs * plan.max_segs), NT,
-                      Sm<true>::BYTES + 1024, st>>>(a);
+  kda_tc_walk<true><<<static_cast<unsigned>(plan.pairs * plan.max_segs), kWalkThreads,
+                      WalkSm<true>::BYTES + 1024, st>>>(wa);
   return cudaGetLastError();
 }
 
