@@ -94,9 +94,10 @@ __device__ __forceinline__ int64_t slot_base(int64_t t0, int s) { return t0 / C 
 struct IntraArgs {
   CUtensorMap tm_q, tm_k, tm_g;  // [T_total][H*128] bf16, 64x64 boxes, no swizzle
   CUtensorMap tm_v;              // the same shape, 128-byte swizzle (an MMA operand as loaded)
+  CUtensorMap tm_qt, tm_kb;      // workspace Q~ and Kb, [tiles*64][128], 128-byte swizzle
   SeqTable seq;
   const __nv_bfloat16* beta;
-  __nv_bfloat16 *wn, *u0, *kb, *qt, *pt;
+  __nv_bfloat16 *wn, *u0, *pt;
   float* gl;
   int H;
   float lb;
@@ -131,15 +132,26 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(t);
 }
+// 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error ~2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint4 pack8(const float* f) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
 }
-// Uniform decision after a bounded wait: true when any thread of the CTA timed out.
+// Bounded wait by thread 0 alone (the others sleep in the barrier instead of polling),
+// then a uniform decision: true when it timed out. The other threads then observe the
+// completed phase themselves, which orders the data it guards before their reads.
 __device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity) {
-  const bool ok = mbar_wait(bar, parity);
-  return __syncthreads_or(!ok) != 0;
+  const bool ok = threadIdx.x != 0 || mbar_wait(bar, parity);
+  if (__syncthreads_or(!ok)) return true;
+  if (threadIdx.x != 0) mbar_try_wait(bar, parity);
+  return false;
 }
+
 
 // ------------------------------------------------------------------ intra-chunk kernel
 // One CTA of 8 warps per (chunk slot, head); two CTAs per SM. Everything of a chunk
@@ -148,15 +160,21 @@ __device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity) 
 // the WY factors W = T K~, U0 = T V on the tensor cores.
 constexpr int kIntraThreads = 256;
 struct IntraSm {
-  // raw inputs as loaded by TMA; each region is reused once its contents are read
+  // Raw inputs as loaded by TMA; each region is reused once its contents are read.
+  // fp32 64x64 matrices (A, N) use a padded row of 68 floats: conflict-free row and
+  // column access with plain addressing.
+  static constexpr int FP = 68;
+  static constexpr uint32_t FP_BYTES = 64 * FP * 4;  // 17 KB
   static constexpr uint32_t SV = 0;        // V, swizzled: [64 s][64 j] boxes (U0's A operand)
   static constexpr uint32_t KQ = K16;      // [K~ a0 | Q~ a0 | K~ a1 | Q~ a1], 8 KB each
-  static constexpr uint32_t SK = 3 * K16;  // raw k, then fp32 A
-  static constexpr uint32_t SG = 4 * K16;  // raw g, then fp32 N = (I + A)^{-1}
-  static constexpr uint32_t SQ = 5 * K16;  // raw q, then K^, then merge scratch and T
-  static constexpr uint32_t A = SK, NS = SG, KH = SQ, BT = SQ, T = SQ + K8;
-  static constexpr uint32_t TOT = 6 * K16;     // float[4][128] partial decay sums
-  static constexpr uint32_t BET = TOT + 2048;  // float[64]
+  static constexpr uint32_t SK = 3 * K16;  // raw k, then K^, then T and the merge scratch
+  static constexpr uint32_t SG = 4 * K16;  // raw g, then Kb (store staging), then N
+  static constexpr uint32_t SQ = 5 * K16;  // raw q, then A
+  static constexpr uint32_t KH = SK, T = SK, BT = SK + K8;
+  static constexpr uint32_t NS = SG - 1024;  // N spans [63 KB, 80 KB)
+  static constexpr uint32_t A = SQ;          // A spans [80 KB, 97 KB)
+  static constexpr uint32_t TOT = SQ + FP_BYTES;  // float[4][128] partial decay sums
+  static constexpr uint32_t BET = TOT + 2048;     // float[64]
   static constexpr uint32_t BARS = BET + 256;
   static constexpr uint32_t TPTR = BARS + 64;
   static constexpr uint32_t BYTES = TPTR + 16;
@@ -164,6 +182,8 @@ struct IntraSm {
   static constexpr uint32_t G = 0, W = 64, U = 128, COLS = 256;
 };
 static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTAs per SM");
+static_assert(IntraSm::BT + 4096 <= IntraSm::NS && IntraSm::NS + IntraSm::FP_BYTES == IntraSm::SQ,
+              "intra-chunk shared-memory regions overlap");
 
 __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_constant__ IntraArgs a) {
   using L_ = IntraSm;
@@ -193,8 +213,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   float* tot = reinterpret_cast<float*>(sm + L_::TOT);
   float* bet = reinterpret_cast<float*>(sm + L_::BET);
   float* bt = reinterpret_cast<float*>(sm + L_::BT);
-  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);
-  uint64_t* bar_mma = bar_in + 1;
+  uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);  // g, k, q
+  uint64_t* bar_v = bar_in + 1;
+  uint64_t* bar_mma = bar_in + 2;
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
 
   if (warp == 0) {
@@ -203,16 +224,20 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   }
   if (tid == 0) {
     mbar_init(bar_in, 1);
+    mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_in, 4 * K16);
+    // v is needed last (by the WY products): its own barrier
+    mbar_arrive_expect_tx(bar_in, 3 * K16);
+    mbar_arrive_expect_tx(bar_v, K16);
     for (int bx = 0; bx < 2; ++bx) {
       const int x = h * D + 64 * bx;
-      tma_load_2d(sm + L_::SK + bx * K8, &a.tm_k, bar_in, x, static_cast<int>(r0));
       tma_load_2d(sm + L_::SG + bx * K8, &a.tm_g, bar_in, x, static_cast<int>(r0));
+      tma_load_2d(sm + L_::SK + bx * K8, &a.tm_k, bar_in, x, static_cast<int>(r0));
       tma_load_2d(sm + L_::SQ + bx * K8, &a.tm_q, bar_in, x, static_cast<int>(r0));
-      tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_in, x, static_cast<int>(r0));
     }
+    for (int bx = 0; bx < 2; ++bx)
+      tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_v, h * D + 64 * bx, static_cast<int>(r0));
   }
   if (tid < C) bet[tid] = tid < L ? __bfloat162float(a.beta[(r0 + tid) * a.H + h]) : 0.f;
   tc_fence_before();
@@ -221,16 +246,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   const uint32_t tb = *tptr;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   int mma_issued = 0, mma_done = 0;
-  bool in_done = false, failed = false;
+  bool in_done = false, v_done = false, failed = false;
 
-  auto a_ptr = [&](int r, int cc) -> float* {
-    return reinterpret_cast<float*>(sm + L_::A) + r * 64 + ((((cc >> 2) ^ (r & 15))) << 2) +
-           (cc & 3);
-  };
-  auto n_ptr = [&](int r, int cc) -> float* {
-    return reinterpret_cast<float*>(sm + L_::NS) + r * 64 + ((((cc >> 2) ^ (r & 15))) << 2) +
-           (cc & 3);
-  };
+  float* const Am = reinterpret_cast<float*>(sm + L_::A);
+  float* const Nm = reinterpret_cast<float*>(sm + L_::NS);
+  auto a_ptr = [&](int r, int cc) -> float* { return Am + r * L_::FP + cc; };
+  auto n_ptr = [&](int r, int cc) -> float* { return Nm + r * L_::FP + cc; };
   auto a4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(a_ptr(r, cc)); };
   auto n4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(n_ptr(r, cc)); };
   auto fma4 = [](float sv, const float4& v, float4& acc) {
@@ -243,32 +264,50 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   do {
     if (cta_wait_failed(bar_in, 0)) { failed = true; break; }
     in_done = true;
-    // ---- 1. raw k, q into registers; prefix sums of the clamped log decay.
+    if (L < C) {
+      // a sequence's ragged last chunk: rows past L (the next sequence's tokens, or the
+      // zero fill past the end) become k = q = 0 and g = 0, so no later step masks rows
+      for (int e = tid; e < (C - L) * 32; e += kIntraThreads) {
+        const int r = L + (e >> 5), w = e & 31;  // 16-byte words per row: two boxes x 8
+        const uint32_t off = (w >> 3 & 1) * K8 + r * 128 + (w & 7) * 16;
+        const int which = w >> 4;  // 0: k and g, 1: q
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if (which == 0) {
+          *reinterpret_cast<uint4*>(sm + L_::SK + off) = z;
+          *reinterpret_cast<uint4*>(sm + L_::SG + off) = z;
+        } else {
+          *reinterpret_cast<uint4*>(sm + L_::SQ + off) = z;
+        }
+      }
+      __syncthreads();
+    }
+    // ---- 1. raw k, q into registers; prefix sums of the clamped log decay in log2 units.
     //         Thread = (channel pair p, quarter qr of 16 rows).
     const int p = tid & 63, qr = tid >> 6;
     const int ch = 2 * p, bx = p >> 5, cofs = (p & 31) * 4;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const float lb2 = a.lb * kLog2e;
     uint32_t kraw[16], qraw[16];
     float G0[16], G1[16];
     {
       float acc0 = 0.f, acc1 = 0.f;
+      const uint32_t off0 = bx * K8 + 16 * qr * 128 + cofs;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
-        const uint32_t off = bx * K8 + r * 128 + cofs;
+        const uint32_t off = off0 + i * 128;
         kraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SK + off);
         qraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SQ + off);
         const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + off));
-        if (r < L) {
-          acc0 += fmaxf(gg.x, a.lb);
-          acc1 += fmaxf(gg.y, a.lb);
-        }
+        acc0 += fmaxf(gg.x * kLog2e, lb2);
+        acc1 += fmaxf(gg.y * kLog2e, lb2);
         G0[i] = acc0;
         G1[i] = acc1;
       }
       *reinterpret_cast<float2*>(tot + qr * 128 + ch) = make_float2(acc0, acc1);
     }
     __syncthreads();  // every raw read is done: SK, SG and SQ may be overwritten
-    // ---- 2. decay tiles: K~, Q~ (MMA operands), K^ (MMA operand); Kb, Q~, gl to the workspace
+    // ---- 2. decay tiles: K~, Q~, K^ (MMA operands), Kb (store staging); gl to the workspace.
+    //         Rows 16 qr + i: the swizzle term depends on i % 8 only.
     {
       float o0 = 0.f, o1 = 0.f, s0 = 0.f, s1 = 0.f;
 #pragma unroll
@@ -281,34 +320,30 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
         s0 += tq.x;
         s1 += tq.y;
       }
-      const float gl0 = expf(s0), gl1 = expf(s1);
+      const float gl0 = ex2_approx(s0), gl1 = ex2_approx(s1);
       if (qr == 3) *reinterpret_cast<float2*>(a.gl + tile * D + ch) = make_float2(gl0, gl1);
-      uint32_t* kbo = reinterpret_cast<uint32_t*>(a.kb + tile * C * D + ch);
-      uint32_t* qto = reinterpret_cast<uint32_t*>(a.qt + tile * C * D + ch);
+      const int c3 = (ch & 63) >> 3;
+      const uint32_t row0 = 2 * qr * 1024 + (ch & 7) * 2;
+      const uint32_t kq0 = L_::KQ + bx * K16 + row0, kh0b = L_::KH + bx * K8 + row0,
+                     kb0b = L_::SG + bx * K8 + row0;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int r = 16 * qr + i;
+        const uint32_t ro = (i >> 3) * 1024 + (i & 7) * 128 + ((c3 ^ (i & 7)) << 4);
         const float g0 = G0[i] + o0, g1 = G1[i] + o1;
-        const float e0 = __expf(g0), e1 = __expf(g1);
-        const float ei0 = __expf(-g0), ei1 = __expf(-g1);
-        float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
-        if (r >= L) {
-          kk = make_float2(0.f, 0.f);
-          qq = make_float2(0.f, 0.f);
-        }
-        const uint32_t kt = pack_bf16(kk.x * e0, kk.y * e1);
-        const uint32_t qt = pack_bf16(qq.x * e0, qq.y * e1);
+        const float e0 = ex2_approx(g0), e1 = ex2_approx(g1);
+        const float ei0 = ex2_approx(-g0), ei1 = ex2_approx(-g1);
+        const float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
         const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
-        *reinterpret_cast<uint32_t*>(sm + L_::KQ + sw128_off(r, ch, K16)) = kt;
-        *reinterpret_cast<uint32_t*>(sm + L_::KQ + K8 + sw128_off(r, ch, K16)) = qt;
-        *reinterpret_cast<uint32_t*>(sm + L_::KH + sw128_off(r, ch, K8)) = pack_bf16(kh0, kh1);
-        kbo[r * (D / 2)] = pack_bf16(kh0 * gl0, kh1 * gl1);
-        qto[r * (D / 2)] = qt;
+        *reinterpret_cast<uint32_t*>(sm + kq0 + ro) = pack_bf16(kk.x * e0, kk.y * e1);
+        *reinterpret_cast<uint32_t*>(sm + kq0 + K8 + ro) = pack_bf16(qq.x * e0, qq.y * e1);
+        *reinterpret_cast<uint32_t*>(sm + kh0b + ro) = pack_bf16(kh0, kh1);
+        *reinterpret_cast<uint32_t*>(sm + kb0b + ro) = pack_bf16(kh0 * gl0, kh1 * gl1);
       }
     }
     fence_async_smem();
     __syncthreads();
-    // ---- 3. MMA-g: [K~; Q~] K^^T, M = 128 (64 rows of K~, then 64 of Q~), N = 64
+    // ---- 3. Q~ (its two boxes inside the Gram operand) and Kb to the workspace by TMA;
+    //         MMA-g: [K~; Q~] K^^T, M = 128 (64 rows of K~, then 64 of Q~), N = 64
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ig = idesc_bf16(128, 64, 0, 0);
@@ -320,6 +355,13 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
                   sdesc_sw128(sb + L_::KH + kho, 16, 1024), ig, k > 0);
       }
       umma_commit(bar_mma);
+    } else if (tid == 32) {
+      const int y = static_cast<int>(tile * C);
+      tma_store_2d(&a.tm_qt, sm + L_::KQ + K8, 0, y);
+      tma_store_2d(&a.tm_qt, sm + L_::KQ + K8 + K16, 64, y);
+      tma_store_2d(&a.tm_kb, sm + L_::SG, 0, y);
+      tma_store_2d(&a.tm_kb, sm + L_::SG + K8, 64, y);
+      bulk_commit();
     }
     mma_issued = 1;
     if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
@@ -352,6 +394,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
           po[t * C] = __float2bfloat16_rn(cb + t <= r ? __uint_as_float(v[t]) : 0.f);
       }
     }
+    if (tid == 32) bulk_wait_read();  // Kb staging is read before N overwrites it
     tc_fence_before();
     __syncthreads();
     // ---- 5. N = (I + A)^{-1}: 16x16 diagonal blocks, then 16->32 and 32->64 merges
@@ -380,74 +423,71 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
     }
     __syncthreads();
-    float* bt1 = bt;  // [2][16][16]
-    float* bt2 = bt;  // [32][36]
-    if (tid < 128) {
-      const int b = tid >> 6, r = (tid >> 2) & 15, cg = tid & 3;
-      const int R0 = 32 * b, R1 = R0 + 16;
-      float av[16];
-#pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
-        const float4 v4 = a4(R1 + r, R0 + 4 * g4);
-        av[4 * g4 + 0] = v4.x;
-        av[4 * g4 + 1] = v4.y;
-        av[4 * g4 + 2] = v4.z;
-        av[4 * g4 + 3] = v4.w;
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) fma4(av[k], n4(R0 + k, R0 + 4 * cg), acc);
-      *reinterpret_cast<float4*>(bt1 + b * 256 + r * 16 + 4 * cg) = acc;
-    }
-    __syncthreads();
-    if (tid < 128) {
-      const int b = tid >> 6, r = (tid >> 2) & 15, cg = tid & 3;
-      const int R0 = 32 * b, R1 = R0 + 16;
-      float nr[16];
-#pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
-        const float4 v4 = n4(R1 + r, R1 + 4 * g4);
-        nr[4 * g4 + 0] = v4.x;
-        nr[4 * g4 + 1] = v4.y;
-        nr[4 * g4 + 2] = v4.z;
-        nr[4 * g4 + 3] = v4.w;
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-        fma4(nr[k], *reinterpret_cast<const float4*>(bt1 + b * 256 + k * 16 + 4 * cg), acc);
-      *reinterpret_cast<float4*>(n_ptr(R1 + r, R0 + 4 * cg)) =
-          make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-      *reinterpret_cast<float4*>(n_ptr(R0 + r, R1 + 4 * cg)) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
+    // Merges. Column c of an off-diagonal block N21 = -N22 (A21 N11) needs only column
+    // c of N11, so each warp owns a few columns: it forms P = A21 N11 for them, hands P
+    // round through its own scratch (a warp barrier), then writes -N22 P.
     {
-      const int r = tid >> 3, cg = tid & 7;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float* pw = bt + warp * 128;  // per-warp scratch, 512 bytes
+      // 16 -> 32: blocks b = warp / 4 (rows and columns 32b..32b+31), four columns per warp
+      {
+        const int b = warp >> 2, R0 = 32 * b, R1 = R0 + 16;
+        const int r = lane & 15, c0 = 4 * (warp & 3) + 2 * (lane >> 4);
+        float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        const float4 v4 = a4(32 + r, 4 * g4);
-        fma4(v4.x, n4(4 * g4 + 0, 4 * cg), acc);
-        fma4(v4.y, n4(4 * g4 + 1, 4 * cg), acc);
-        fma4(v4.z, n4(4 * g4 + 2, 4 * cg), acc);
-        fma4(v4.w, n4(4 * g4 + 3, 4 * cg), acc);
-      }
-      *reinterpret_cast<float4*>(bt2 + r * 36 + 4 * cg) = acc;
-    }
-    __syncthreads();
-    {
-      const int r = tid >> 3, cg = tid & 7;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const float4 av = a4(R1 + r, R0 + 4 * g4);
+          const float af[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        const float4 v4 = n4(32 + r, 32 + 4 * g4);
-        fma4(v4.x, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 0) * 36 + 4 * cg), acc);
-        fma4(v4.y, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 1) * 36 + 4 * cg), acc);
-        fma4(v4.z, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 2) * 36 + 4 * cg), acc);
-        fma4(v4.w, *reinterpret_cast<const float4*>(bt2 + (4 * g4 + 3) * 36 + 4 * cg), acc);
+          for (int e = 0; e < 4; ++e) {
+            const float2 nn = *reinterpret_cast<const float2*>(n_ptr(R0 + 4 * g4 + e, R0 + c0));
+            p0 = fmaf(af[e], nn.x, p0);
+            p1 = fmaf(af[e], nn.y, p1);
+          }
+        }
+        *reinterpret_cast<float2*>(pw + r * 4 + (c0 & 3)) = make_float2(p0, p1);
+        __syncwarp();
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const float4 nv4 = n4(R1 + r, R1 + 4 * g4);
+          const float nf[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 pp = *reinterpret_cast<const float2*>(pw + (4 * g4 + e) * 4 + (c0 & 3));
+            o0 = fmaf(nf[e], pp.x, o0);
+            o1 = fmaf(nf[e], pp.y, o1);
+          }
+        }
+        *reinterpret_cast<float2*>(n_ptr(R1 + r, R0 + c0)) = make_float2(-o0, -o1);
+        *reinterpret_cast<float2*>(n_ptr(R0 + r, R1 + c0)) = make_float2(0.f, 0.f);
       }
-      *reinterpret_cast<float4*>(n_ptr(32 + r, 4 * cg)) =
-          make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+      __syncthreads();
+      // 32 -> 64: rows 32..63, columns 0..31, four columns per warp, lane = row
+      {
+        const int r = lane, cc = 4 * warp;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4) {
+          const float4 av = a4(32 + r, 4 * g4);
+          fma4(av.x, n4(4 * g4 + 0, cc), acc);
+          fma4(av.y, n4(4 * g4 + 1, cc), acc);
+          fma4(av.z, n4(4 * g4 + 2, cc), acc);
+          fma4(av.w, n4(4 * g4 + 3, cc), acc);
+        }
+        __syncwarp();  // the 16 -> 32 scratch of this warp is no longer read
+        *reinterpret_cast<float4*>(pw + r * 4) = acc;
+        __syncwarp();
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4) {
+          const float4 nv4 = n4(32 + r, 32 + 4 * g4);
+          fma4(nv4.x, *reinterpret_cast<const float4*>(pw + (4 * g4 + 0) * 4), o);
+          fma4(nv4.y, *reinterpret_cast<const float4*>(pw + (4 * g4 + 1) * 4), o);
+          fma4(nv4.z, *reinterpret_cast<const float4*>(pw + (4 * g4 + 2) * 4), o);
+          fma4(nv4.w, *reinterpret_cast<const float4*>(pw + (4 * g4 + 3) * 4), o);
+        }
+        *reinterpret_cast<float4*>(n_ptr(32 + r, cc)) = make_float4(-o.x, -o.y, -o.z, -o.w);
+      }
     }
     __syncthreads();
     // ---- 6. T = N Diag(beta), lower triangle, bf16 operand: two 16-byte chunks per thread
@@ -471,7 +511,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
     }
     fence_async_smem();
-    __syncthreads();
+    if (cta_wait_failed(bar_v, 0)) { failed = true; break; }  // also the barrier for T
+    v_done = true;
     // ---- 7. W^T = K~^T T^T and U0^T = V^T T^T. K~ (in the Gram operand) and V (as
     //         loaded) serve as MN-major A operands: 64-element column groups LBO apart,
     //         8-row groups 1024 bytes apart, 16 rows of K per instruction.
@@ -506,10 +547,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       for (int t = 0; t < 32; ++t) uo[t * D] = __float2bfloat16_rn(__uint_as_float(v[t]));
     }
   } while (0);
+  if (tid == 32) bulk_wait_all();  // workspace stores complete
   if (failed && tid == 0) {
     atomicExch(a.seq.status, kDevWaitTimeout);
     // copies and products in flight finish before the CTA releases its memory
     if (!in_done) mbar_wait(bar_in, 0, 400000000LL);
+    if (!v_done) mbar_wait(bar_v, 0, 400000000LL);
     for (int m = mma_done; m < mma_issued; ++m) mbar_wait(bar_mma, m & 1, 400000000LL);
   }
   tc_fence_before();
@@ -521,16 +564,27 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 }
 
 // ------------------------------------------------------------------ walk over chunks
-// One CTA of 8 warps per (sequence, head, segment). Warps w and w + 4 share the
-// tensor-memory lanes 32 (w % 4) .. + 31 (state columns j) and split the columns.
-// Thread 0 streams the next chunk's workspace tiles (two stages) and issues the MMAs.
-constexpr int kWalkThreads = 256;
+// One CTA per (sequence, head, segment), warp-specialized:
+//   warps 0..7  conversion: warps w and w + 4 share the tensor-memory lanes 32 (w % 4)..+31
+//               (state columns j) and split the columns; they rescale the fp32 state,
+//               turn U^T and S^T into bf16 operands and write the outputs;
+//   warp 8      issues the MMAs (one thread);
+//   warp 9      streams each chunk's workspace tiles into two stages by TMA (one thread).
+// Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and
+// s_ready/y_ready (the bf16 S^T and U^T operands are in shared memory).
+constexpr int kWalkConvThreads = 256, kWalkThreads = 320;
+constexpr int kWalkMmaWarp = 8, kWalkLoadWarp = 9;
+constexpr int kConvBar = 1;  // named barrier of the conversion warps
 template <bool PC>
 struct WalkSm {
   static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks: [S] or [M | L]
-  // one input stage: -W | U0 | Kb | (Q~ | P^T); two 64-column boxes per [64][128] tile
-  static constexpr uint32_t WN = 0, U0 = K16, KB = 2 * K16, QT = 3 * K16, PT = 4 * K16;
-  static constexpr uint32_t STAGE = PC ? 4 * K16 + K8 : 3 * K16;
+  // One input stage. Output walk: [-W a0 | Q~ a0 | -W a1 | Q~ a1] (one N = 128 operand),
+  // U0, Kb, P^T; summary walk: -W, U0, Kb. Each [64][128] tile is two 64-column boxes.
+  static constexpr uint32_t WN = 0;
+  static constexpr uint32_t U0 = PC ? K32 : K16;
+  static constexpr uint32_t KB = U0 + K16;
+  static constexpr uint32_t PT = KB + K16;
+  static constexpr uint32_t STAGE = PT + (PC ? K8 : 0);
   static constexpr uint32_t STAGE_TX = STAGE + 512;  // + gl
   static constexpr uint32_t S = 2 * STAGE;             // bf16 S^T, [128 j][128 i], 32 KB/block
   static constexpr uint32_t Y = S + NB * K32;          // bf16 U^T, [128 j][64 r], 16 KB/block
@@ -538,13 +592,14 @@ struct WalkSm {
   static constexpr uint32_t ID = OS + (PC ? K16 : 0);  // bf16 64x64 identity
   static constexpr uint32_t GL = ID + K8;              // float[2][128]
   static constexpr uint32_t BARS = GL + 1024;
-  static constexpr uint32_t TPTR = BARS + 64;
+  static constexpr uint32_t TPTR = BARS + 128;
   static constexpr uint32_t BYTES = TPTR + 16;
-  // tensor-memory columns: fp32 S^T per block, U^T per block, O^T
+  // tensor-memory columns: fp32 S^T per block; output walk: [U^T | O^T] in two buffers,
+  // summary walk: U^T per block
   __device__ static constexpr uint32_t st(int b) { return 128 * b; }
-  __device__ static constexpr uint32_t uc(int b) { return PC ? 128 : 256 + 64 * b; }
-  static constexpr uint32_t YO = 192;
-  static constexpr uint32_t COLS = PC ? 256 : 512;
+  __device__ static constexpr uint32_t uc(int b, int p) { return PC ? 128 + 128 * p : 256 + 64 * b; }
+  __device__ static constexpr uint32_t yo(int p) { return 192 + 128 * p; }
+  static constexpr uint32_t COLS = 512;
 };
 static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
 static_assert(WalkSm<false>::BYTES + 1024 <= 232448, "summary walk shared memory");
@@ -579,35 +634,35 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
 
   float* gls = reinterpret_cast<float*>(sm + L_::GL);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_::BARS);
-  uint64_t* bar_full = bars;  // two stages
-  uint64_t* bar_m1 = bars + 2;
-  uint64_t* bar_m2 = bars + 3;
+  uint64_t* bar_full = bars;       // two stages
+  uint64_t* bar_empty = bars + 2;  // two stages
+  uint64_t* bar_m1 = bars + 4;
+  uint64_t* bar_m2 = bars + 5;
+  uint64_t* bar_sready = bars + 6;
+  uint64_t* bar_yready = bars + 7;
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
-
-  auto issue_stage = [&](int n) {  // thread 0
-    const int st = n & 1;
-    unsigned char* dst = sm + st * L_::STAGE;
-    const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
-    const int y = static_cast<int>(tile * C);
-    mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
-    for (int bx = 0; bx < 2; ++bx) {
-      tma_load_2d(dst + L_::WN + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
-      tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 64 * bx, y);
-      tma_load_2d(dst + L_::KB + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
-      if (PC) tma_load_2d(dst + L_::QT + bx * K8, &a.tm_qt, bar_full + st, 64 * bx, y);
-    }
-    if (PC) tma_load_2d(dst + L_::PT, &a.tm_pt, bar_full + st, 0, y);
-    bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
-  };
 
   if (warp == 0) {
     tmem_alloc(tptr, L_::COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
-    if (n_chunks > 0) {
+  }
+  // identity operand: zeros, then the diagonal
+  for (int e = tid; e < static_cast<int>(K8 / 16); e += kWalkThreads)
+    *reinterpret_cast<uint4*>(sm + L_::ID + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid < C) *reinterpret_cast<uint16_t*>(sm + L_::ID + sw128_off(tid, tid, K8)) = 0x3F80u;
+  const uint32_t tb = *tptr;
+
+  if (warp == kWalkLoadWarp) {
+    // ============================================================ stage loads
+    if (lane == 0 && n_chunks > 0) {
       tma_prefetch_desc(&a.tm_wn);
       tma_prefetch_desc(&a.tm_u0);
       tma_prefetch_desc(&a.tm_kb);
@@ -615,166 +670,142 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
         tma_prefetch_desc(&a.tm_qt);
         tma_prefetch_desc(&a.tm_pt);
       }
-      issue_stage(0);
-    }
-  }
-  // identity operand: zeros, then the diagonal
-  for (int e = tid; e < static_cast<int>(K8 / 16); e += kWalkThreads)
-    *reinterpret_cast<uint4*>(sm + L_::ID + e * 16) = make_uint4(0u, 0u, 0u, 0u);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (tid < C) *reinterpret_cast<uint16_t*>(sm + L_::ID + sw128_off(tid, tid, K8)) = 0x3F80u;
-  const uint32_t tb = *tptr;
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
-  const int hc = warp >> 2;                // column half this thread converts
-
-  // initial state: fp32 into tensor memory, bf16 copy as the MMA operand
-  {
-    const float* src = nullptr;
-    if (PC) {
-      if (nseg > 1) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
-      else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
-    }
-    for (int b = 0; b < NB; ++b)
-      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
-        uint32_t v[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          float x;
-          if (PC) x = src ? src[static_cast<int64_t>(c + t) * D + row] : 0.f;
-          else x = (b == 0 && c + t == row) ? 1.f : 0.f;
-          v[t] = __float_as_uint(x);
+      int issued = 0;
+      bool ok = true;
+      for (int n = 0; n < n_chunks; ++n) {
+        const int st = n & 1;
+        if (n >= 2 && !(ok = mbar_wait(bar_empty + st, ((n - 2) >> 1) & 1))) break;
+        unsigned char* dst = sm + st * L_::STAGE;
+        const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
+        const int y = static_cast<int>(tile * C);
+        mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
+        for (int bx = 0; bx < 2; ++bx) {
+          if (PC) {
+            tma_load_2d(dst + L_::WN + bx * K16, &a.tm_wn, bar_full + st, 64 * bx, y);
+            tma_load_2d(dst + L_::WN + K8 + bx * K16, &a.tm_qt, bar_full + st, 64 * bx, y);
+          } else {
+            tma_load_2d(dst + L_::WN + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
+          }
+          tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 64 * bx, y);
+          tma_load_2d(dst + L_::KB + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
         }
-        tmem_st32(tb + lane_base + L_::st(b) + c, v);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+        if (PC) tma_load_2d(dst + L_::PT, &a.tm_pt, bar_full + st, 0, y);
+        bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
+        ++issued;
       }
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  fence_async_smem();
-  __syncthreads();
-  tc_fence_after();
-
-  int full_issued = n_chunks > 0 ? 1 : 0, full_done = 0;
-  int m1_issued = 0, m2_issued = 0, m1_done = 0, m2_done = 0;
-  bool failed = false;
-  for (int n = 0; n < n_chunks; ++n) {
-    const int st = n & 1;
-    const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
-    const int L = (c_end - c0) < C ? static_cast<int>(c_end - c0) : C;
-    const uint32_t stg = sb + st * L_::STAGE;
-    if (cta_wait_failed(bar_full + st, (n >> 1) & 1)) { failed = true; break; }
-    ++full_done;
-    // ---- MMA-1: U^T = U0^T I + S^T (-W)^T per block; (Q~ S)^T = S^T Q~^T
-    if (tid == 0) {
-      if (n + 1 < n_chunks) issue_stage(n + 1);
-      tc_fence_after();
-      const uint32_t i_k = idesc_bf16(128, 64, 0, 0), i_mn = idesc_bf16(128, 64, 1, 0);
+      if (!ok) atomicExch(a.seq.status, kDevWaitTimeout);
+      // the copies in flight land before the CTA can exit
+      for (int n = issued >= 2 ? issued - 2 : 0; n < issued; ++n)
+        mbar_wait(bar_full + (n & 1), (n >> 1) & 1, 400000000LL);
+    }
+  } else if (warp == kWalkMmaWarp) {
+    // ============================================================ MMA issue
+    if (lane == 0) {
+      int m_issued = 0;
+      bool ok = true;
+      for (int n = 0; n < n_chunks && ok; ++n) {
+        const int st = n & 1;
+        const uint32_t stg = sb + st * L_::STAGE;
+        if (!(ok = mbar_wait(bar_full + st, (n >> 1) & 1))) break;
+        if (!(ok = mbar_wait(bar_sready, n & 1))) break;
+        tc_fence_after();
+        // MMA-1: [U^T | (Q~ S)^T] = S^T [-W; Q~]^T (+ U0^T I on the U^T half)
+        const uint32_t i_mn = idesc_bf16(128, 64, 1, 0);
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
-        if (with_u0) {
+        for (int b = 0; b < NB; ++b) {
+          const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 0);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32;
+            const uint32_t ko_w = (k >> 2) * (PC ? K16 : K8) + (k & 3) * 32;
+            umma_bf16(tb + L_::uc(b, st), sdesc_sw128(sb + L_::S + b * K32 + ko_s, 16, 1024),
+                      sdesc_sw128(stg + L_::WN + ko_w, 16, 1024), i_k, k > 0);
+          }
+          if (PC || b == 1) {  // the M block of the summary walk has V = 0
+#pragma unroll
+            for (int k = 0; k < C / 16; ++k)
+              umma_bf16(tb + L_::uc(b, st), sdesc_sw128(stg + L_::U0 + k * 2048, K8, 1024),
+                        sdesc_sw128(sb + L_::ID + k * 32, 16, 1024), i_mn, 1);
+          }
+        }
+        umma_commit(bar_m1);
+        ++m_issued;
+        if (!(ok = mbar_wait(bar_yready, n & 1))) break;
+        tc_fence_after();
+        // MMA-2: O^T += U^T P^T (output walk); S^T += U^T Kb (B operands MN-major)
+        if (PC) {
+          const uint32_t ic = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
           for (int k = 0; k < C / 16; ++k)
-            umma_bf16(tb + L_::uc(b), sdesc_sw128(stg + L_::U0 + k * 2048, K8, 1024),
-                      sdesc_sw128(sb + L_::ID + k * 32, 16, 1024), i_mn, k > 0);
+            umma_bf16(tb + L_::yo(st), sdesc_sw128(sb + L_::Y + k * 32, 16, 1024),
+                      sdesc_sw128(stg + L_::PT + k * 2048, K8, 1024), ic, 1);
         }
+        const uint32_t id = idesc_bf16(128, 128, 0, 1);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32, ko_w = (k >> 2) * K8 + (k & 3) * 32;
-          umma_bf16(tb + L_::uc(b), sdesc_sw128(sb + L_::S + b * K32 + ko_s, 16, 1024),
-                    sdesc_sw128(stg + L_::WN + ko_w, 16, 1024), i_k, (with_u0 || k > 0) ? 1u : 0u);
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int k = 0; k < C / 16; ++k)
+            umma_bf16(tb + L_::st(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
+                      sdesc_sw128(stg + L_::KB + k * 2048, K8, 1024), id, 1);
+        umma_commit(bar_m2);
+        umma_commit(bar_empty + st);
+        ++m_issued;
+      }
+      if (!ok) {
+        atomicExch(a.seq.status, kDevWaitTimeout);
+        // the products issued so far finish before tensor memory is released
+        if (m_issued > 0) {
+          const int last = m_issued - 1;
+          mbar_wait((last & 1) ? bar_m2 : bar_m1, (last >> 1) & 1, 400000000LL);
         }
       }
-      if (PC) {
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32, ko_w = (k >> 2) * K8 + (k & 3) * 32;
-          umma_bf16(tb + L_::YO, sdesc_sw128(sb + L_::S + ko_s, 16, 1024),
-                    sdesc_sw128(stg + L_::QT + ko_w, 16, 1024), i_k, k > 0);
-        }
-      }
-      umma_commit(bar_m1);
     }
-    ++m1_issued;
-    if (n + 1 < n_chunks) ++full_issued;
-    // ---- while MMA-1 runs: S <- Diag(gl) S in tensor memory (MMA-1 reads the bf16 copy)
+  } else {
+    // ============================================================ conversion warps
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
+    const int hc = warp >> 2;                // column half this thread converts
+    // initial state: fp32 into tensor memory, bf16 copy as the MMA operand
     {
-      const float* gl = gls + st * D;
-#pragma unroll 1
-      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
-        float gv[32];
-#pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4)
-          *reinterpret_cast<float4*>(gv + 4 * t4) = *reinterpret_cast<const float4*>(gl + c + 4 * t4);
-#pragma unroll 1
-        for (int b = 0; b < NB; ++b) {
-          uint32_t sv[32];
-          tmem_ld32(tb + lane_base + L_::st(b) + c, sv);
-          tmem_ld_wait(sv);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) sv[t] = __float_as_uint(gv[t] * __uint_as_float(sv[t]));
-          tmem_st32(tb + lane_base + L_::st(b) + c, sv);
-        }
+      const float* src = nullptr;
+      if (PC) {
+        if (nseg > 1) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
+        else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
       }
+      for (int b = 0; b < NB; ++b)
+        for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+          uint32_t v[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            float x;
+            if (PC) x = src ? src[static_cast<int64_t>(c + t) * D + row] : 0.f;
+            else x = (b == 0 && c + t == row) ? 1.f : 0.f;
+            v[t] = __float_as_uint(x);
+          }
+          tmem_st32(tb + lane_base + L_::st(b) + c, v);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8)
+            *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
+                pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+        }
       tmem_st_wait();
     }
     tc_fence_before();
-    if (cta_wait_failed(bar_m1, n & 1)) { failed = true; break; }
-    ++m1_done;
-    tc_fence_after();
-    // ---- U^T -> bf16 operand (this thread's 32 columns of each block)
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::uc(b) + 32 * hc, v);
-      tmem_ld_wait(v);
-#pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8)
-        *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, 4 * hc + q8, K16)) =
-            pack8(reinterpret_cast<const float*>(v) + 8 * q8);
-    }
-    if (PC && tid == 0) bulk_wait_read();  // the previous output store has read OS
-    tc_fence_before();
     fence_async_smem();
-    __syncthreads();
-    // ---- MMA-2: O^T += U^T P^T (output walk); S^T += U^T Kb (B operands MN-major)
-    if (tid == 0) {
-      tc_fence_after();
-      if (PC) {
-        const uint32_t ic = idesc_bf16(128, 64, 0, 1);
-#pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(tb + L_::YO, sdesc_sw128(sb + L_::Y + k * 32, 16, 1024),
-                    sdesc_sw128(stg + L_::PT + k * 2048, K8, 1024), ic, 1);
-      }
-      const uint32_t id = idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-      for (int b = 0; b < NB; ++b)
-#pragma unroll
-        for (int k = 0; k < C / 16; ++k)
-          umma_bf16(tb + L_::st(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
-                    sdesc_sw128(stg + L_::KB + k * 2048, K8, 1024), id, 1);
-      umma_commit(bar_m2);
-    }
-    ++m2_issued;
-    if (cta_wait_failed(bar_m2, n & 1)) { failed = true; break; }
-    ++m2_done;
-    tc_fence_after();
-    // ---- outputs; bf16 S^T for the next chunk
-    if (PC) {
+    group_sync(kConvBar, kWalkConvThreads);
+    if (tid == 0 && n_chunks > 0) mbar_arrive(bar_sready);
+
+    // O of chunk n (tensor-memory buffer yo(n & 1)) to global memory: full chunks
+    // through the staging tile and a TMA store, a ragged last chunk directly
+    auto emit_out = [&](int n) {
+      const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
+      const int L = (c_end - c0) < C ? static_cast<int>(c_end - c0) : C;
       uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::YO + 32 * hc, v);
+      tmem_ld32(tb + lane_base + L_::yo(n & 1) + 32 * hc, v);
       tmem_ld_wait(v);
       if (L == C) {
-        // O[r][j] into two 64x64 row-major boxes; one TMA store each below
-        __nv_bfloat16* ob =
-            reinterpret_cast<__nv_bfloat16*>(sm + L_::OS + (row >> 6) * K8) + 32 * hc * 64 + (row & 63);
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sm + L_::OS + (row >> 6) * K8) +
+                            32 * hc * 64 + (row & 63);
 #pragma unroll
         for (int t = 0; t < 32; ++t) ob[t * 64] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
       } else {
@@ -785,54 +816,137 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
         for (int t = 0; t < 32; ++t)
           if (32 * hc + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
       }
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-#pragma unroll
-      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::st(b) + c, v);
-        tmem_ld_wait(v);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
-      }
-    tc_fence_before();
-    fence_async_smem();
-    __syncthreads();
-    if (PC && L == C && tid == 0) {
+      return L == C;
+    };
+    auto store_out = [&](int n) {  // thread 0, once the staging tile is visible
+      const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
       tma_store_2d(&a.tm_o, sm + L_::OS, h * D, static_cast<int>(c0));
       tma_store_2d(&a.tm_o, sm + L_::OS + K8, h * D + 64, static_cast<int>(c0));
       bulk_commit();
-    }
-  }
-  if (PC && tid == 0) bulk_wait_all();  // outputs written before the kernel ends
-  if (failed) {
-    if (tid == 0) {
-      atomicExch(a.seq.status, kDevWaitTimeout);
-      // copies and products in flight finish before the CTA releases its memory
-      for (int f = full_done; f < full_issued; ++f) mbar_wait(bar_full + (f & 1), (f >> 1) & 1, 400000000LL);
-      for (int m = m1_done; m < m1_issued; ++m) mbar_wait(bar_m1, m & 1, 400000000LL);
-      for (int m = m2_done; m < m2_issued; ++m) mbar_wait(bar_m2, m & 1, 400000000LL);
-    }
-  } else {
-    // ---- final / summary state (row-major [i][j], fp32)
-    for (int b = 0; b < NB; ++b) {
-      float* dst = nullptr;
-      if (PC) {
-        if (a.sT && seg == nseg - 1) dst = a.sT + static_cast<int64_t>(pair) * D * D;
-      } else {
-        const int64_t un = static_cast<int64_t>(pair) * (a.max_segs - 1) + seg;
-        dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
+    };
+
+    bool failed = false, pend_store = false;
+    for (int n = 0; n < n_chunks; ++n) {
+      const int st = n & 1;
+      if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + st, (n >> 1) & 1))) {
+        failed = true;
+        break;
       }
-      if (dst == nullptr) continue;
-      for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+      // ---- while MMA-1 runs: S <- Diag(gl) S in tensor memory (MMA-1 reads the bf16
+      //      copy), then the previous chunk's outputs
+      {
+        const float* gl = gls + st * D + 64 * hc;
+#pragma unroll 1
+        for (int b = 0; b < NB; ++b) {
+          uint32_t s0[32], s1[32];
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, s0);
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, s1);
+          tmem_ld_wait(s0);
+          tmem_ld_wait(s1);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) {
+            const float4 g0 = *reinterpret_cast<const float4*>(gl + 4 * t4);
+            const float4 g1 = *reinterpret_cast<const float4*>(gl + 32 + 4 * t4);
+            s0[4 * t4 + 0] = __float_as_uint(g0.x * __uint_as_float(s0[4 * t4 + 0]));
+            s0[4 * t4 + 1] = __float_as_uint(g0.y * __uint_as_float(s0[4 * t4 + 1]));
+            s0[4 * t4 + 2] = __float_as_uint(g0.z * __uint_as_float(s0[4 * t4 + 2]));
+            s0[4 * t4 + 3] = __float_as_uint(g0.w * __uint_as_float(s0[4 * t4 + 3]));
+            s1[4 * t4 + 0] = __float_as_uint(g1.x * __uint_as_float(s1[4 * t4 + 0]));
+            s1[4 * t4 + 1] = __float_as_uint(g1.y * __uint_as_float(s1[4 * t4 + 1]));
+            s1[4 * t4 + 2] = __float_as_uint(g1.z * __uint_as_float(s1[4 * t4 + 2]));
+            s1[4 * t4 + 3] = __float_as_uint(g1.w * __uint_as_float(s1[4 * t4 + 3]));
+          }
+          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, s0);
+          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, s1);
+        }
+        tmem_st_wait();
+      }
+      const bool staged = (PC && n > 0) ? emit_out(n - 1) : false;
+      if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_m1, n & 1))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      // ---- U^T -> bf16 operand (this thread's 32 columns of each block)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
         uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::st(b) + c, v);
+        tmem_ld32(tb + lane_base + L_::uc(b, st) + 32 * hc, v);
         tmem_ld_wait(v);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(c + t) * D + row] = __uint_as_float(v[t]);
+        for (int q8 = 0; q8 < 4; ++q8)
+          *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, 4 * hc + q8, K16)) =
+              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+      }
+      tc_fence_before();
+      fence_async_smem();
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0) {
+        mbar_arrive(bar_yready);
+        if (staged) {
+          store_out(n - 1);
+          pend_store = true;
+        }
+      }
+      if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_m2, n & 1))) {
+        failed = true;
+        break;
+      }
+      tc_fence_after();
+      // ---- bf16 S^T for the next chunk
+#pragma unroll 1
+      for (int b = 0; b < NB; ++b) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, v0);
+        tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+        tmem_ld_wait(v0);
+        tmem_ld_wait(v1);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, 8 * hc + q8, K16)) =
+              pack8(reinterpret_cast<const float*>(v0) + 8 * q8);
+          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, 8 * hc + 4 + q8, K16)) =
+              pack8(reinterpret_cast<const float*>(v1) + 8 * q8);
+        }
+      }
+      if (tid == 0 && pend_store) {
+        bulk_wait_read();  // the staging tile may be rewritten after the barrier below
+        pend_store = false;
+      }
+      tc_fence_before();
+      fence_async_smem();
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready);
+    }
+    if (PC && !failed && n_chunks > 0) {
+      // the last chunk's outputs
+      tc_fence_after();
+      const bool staged = emit_out(n_chunks - 1);
+      fence_async_smem();
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0 && staged) store_out(n_chunks - 1);
+    }
+    if (PC && tid == 0) bulk_wait_all();  // outputs written before the kernel ends
+    if (failed) {
+      if (tid == 0) atomicExch(a.seq.status, kDevWaitTimeout);
+    } else {
+      // ---- final / summary state (row-major [i][j], fp32)
+      for (int b = 0; b < NB; ++b) {
+        float* dst = nullptr;
+        if (PC) {
+          if (a.sT && seg == nseg - 1) dst = a.sT + static_cast<int64_t>(pair) * D * D;
+        } else {
+          const int64_t un = static_cast<int64_t>(pair) * (a.max_segs - 1) + seg;
+          dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
+        }
+        if (dst == nullptr) continue;
+        for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tb + lane_base + L_::st(b) + c, v);
+          tmem_ld_wait(v);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(c + t) * D + row] = __uint_as_float(v[t]);
+        }
       }
     }
   }
@@ -1015,6 +1129,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
       !make_map(&ia.tm_k, pa.k, in_cols, pa.T_total, in_pitch, false) ||
       !make_map(&ia.tm_g, pa.g, in_cols, pa.T_total, in_pitch, false) ||
       !make_map(&ia.tm_v, pa.v, in_cols, pa.T_total, in_pitch, true) ||
+      !make_map(&ia.tm_qt, qt, D, rows_t, D * 2, true) ||
+      !make_map(&ia.tm_kb, kb, D, rows_t, D * 2, true) ||
+
       !make_map(&wa.tm_wn, wn, D, rows_t, D * 2, true) ||
       !make_map(&wa.tm_u0, u0, D, rows_t, D * 2, true) ||
       !make_map(&wa.tm_kb, kb, D, rows_t, D * 2, true) ||
@@ -1026,8 +1143,6 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   ia.beta = static_cast<const __nv_bfloat16*>(pa.beta);
   ia.wn = wn;
   ia.u0 = u0;
-  ia.kb = kb;
-  ia.qt = qt;
   ia.pt = pt;
   ia.gl = gl;
   ia.H = pa.H;
