@@ -46,10 +46,11 @@ constexpr int C = kChunk;  // 64
 constexpr int D = 128;     // d_k = d_v on this path
 constexpr uint32_t K8 = 8192, K16 = 16384, K32 = 32768;
 
-// Workspace tiles per (chunk slot, head); rows are the chunk's tokens.
-//   wn, u0, kb, qt: [64][128] bf16  (-W, U0, Kb, Q~)
-//   pt:             [64][64]  bf16  (P^T: row s, column r)
-//   gl:             [128]     fp32
+// Workspace tiles per (chunk slot, head); rows are the chunk's tokens except for U0.
+//   wn, kb, qt: [64][128] bf16  (-W, Kb, Q~)
+//   u0:         [128][64] bf16  (U0^T: row j, column r)
+//   pt:         [64][64]  bf16  (P^T: row s, column r)
+//   gl:         [128]     fp32
 constexpr size_t kTileBig = size_t(C) * D * 2;
 constexpr size_t kTilePt = size_t(C) * C * 2;
 constexpr size_t kTileGl = size_t(D) * 4;
@@ -542,9 +543,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       for (int t = 0; t < 32; ++t) wo[t * D] = __float2bfloat16_rn(-__uint_as_float(v[t]));
       tmem_ld32(tb + lane_base + L_::U + cb, v);
       tmem_ld_wait(v);
-      __nv_bfloat16* uo = a.u0 + (tile * C + cb) * D + i;
+      // U0 is stored transposed ([j][r] per tile): this lane's 32 values are contiguous
+      uint4* uo = reinterpret_cast<uint4*>(a.u0 + (tile * D + i) * C + cb);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) uo[t * D] = __float2bfloat16_rn(__uint_as_float(v[t]));
+      for (int q = 0; q < 4; ++q)
+        uo[q] = pack8(reinterpret_cast<const float*>(v) + 8 * q);
     }
   } while (0);
   if (tid == 32) bulk_wait_all();  // workspace stores complete
@@ -566,39 +569,46 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 // ------------------------------------------------------------------ walk over chunks
 // One CTA per (sequence, head, segment), warp-specialized:
 //   warps 0..7  conversion: warps w and w + 4 share the tensor-memory lanes 32 (w % 4)..+31
-//               (state columns j) and split the columns; they rescale the fp32 state,
-//               turn U^T and S^T into bf16 operands and write the outputs;
+//               (state columns j); warps 0..3 own the first half of the columns, warps
+//               4..7 the second. They rescale the fp32 state, add U0 and pack U^T and S^T
+//               into bf16 MMA operands kept in tensor memory, and write the outputs;
 //   warp 8      issues the MMAs (one thread);
 //   warp 9      streams each chunk's workspace tiles into two stages by TMA (one thread).
-// Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and
-// s_ready/y_ready (the bf16 S^T and U^T operands are in shared memory).
+// Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and per column
+// half s_ready/y_ready (that half of the bf16 S^T or U^T operand is in tensor memory), so
+// the first half of a product starts while the second half is still being packed.
 constexpr int kWalkConvThreads = 256, kWalkThreads = 320;
 constexpr int kWalkMmaWarp = 8, kWalkLoadWarp = 9;
-constexpr int kConvBar = 1;  // named barrier of the conversion warps
+constexpr int kConvBar = 1;  // named barrier of the conversion warps; 2 + half for a half
 template <bool PC>
 struct WalkSm {
   static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks: [S] or [M | L]
-  // One input stage. Output walk: [-W a0 | Q~ a0 | -W a1 | Q~ a1] (one N = 128 operand),
-  // U0, Kb, P^T; summary walk: -W, U0, Kb. Each [64][128] tile is two 64-column boxes.
-  static constexpr uint32_t WN = 0;
+  // One input stage; every [64][128] tile is two 64-column boxes.
+  //   output walk, even stage: WQ = [-W a0 | Q~ a0 | -W a1 | Q~ a1], PK = [P^T | Kb a0 | Kb a1]
+  //   output walk, odd stage:  WQ = [Q~ a0 | -W a0 | Q~ a1 | -W a1], PK = [Kb a0 | Kb a1 | P^T]
+  //   summary walk: WQ = -W, PK = Kb.
+  // The order follows the tensor-memory order of the accumulators in the two products.
+  static constexpr uint32_t WQ = 0;
   static constexpr uint32_t U0 = PC ? K32 : K16;
-  static constexpr uint32_t KB = U0 + K16;
-  static constexpr uint32_t PT = KB + K16;
-  static constexpr uint32_t STAGE = PT + (PC ? K8 : 0);
+  static constexpr uint32_t PK = U0 + K16;
+  static constexpr uint32_t STAGE = PK + (PC ? K16 + K8 : K16);
   static constexpr uint32_t STAGE_TX = STAGE + 512;  // + gl
-  static constexpr uint32_t S = 2 * STAGE;             // bf16 S^T, [128 j][128 i], 32 KB/block
-  static constexpr uint32_t Y = S + NB * K32;          // bf16 U^T, [128 j][64 r], 16 KB/block
-  static constexpr uint32_t OS = Y + NB * K16;         // output staging: two [64 r][64 j] boxes
-  static constexpr uint32_t ID = OS + (PC ? K16 : 0);  // bf16 64x64 identity
-  static constexpr uint32_t GL = ID + K8;              // float[2][128]
+  static constexpr uint32_t OS = 2 * STAGE;            // output staging: two [64 r][64 j] boxes
+  static constexpr uint32_t GL = OS + (PC ? K16 : 0);  // float[2][128]
   static constexpr uint32_t BARS = GL + 1024;
   static constexpr uint32_t TPTR = BARS + 128;
   static constexpr uint32_t BYTES = TPTR + 16;
-  // tensor-memory columns: fp32 S^T per block; output walk: [U^T | O^T] in two buffers,
-  // summary walk: U^T per block
-  __device__ static constexpr uint32_t st(int b) { return 128 * b; }
-  __device__ static constexpr uint32_t uc(int b, int p) { return PC ? 128 + 128 * p : 256 + 64 * b; }
-  __device__ static constexpr uint32_t yo(int p) { return 192 + 128 * p; }
+  // Tensor-memory columns. Output walk, by chunk parity p: p = 0: [U | O] at 0..127,
+  // S at 128..255 (so MMA-2's accumulator [O | S] is 64..255); p = 1: S at 128..255,
+  // [O | U] at 256..383 (MMA-2's [S | O] is 128..319). Summary walk: S per block at
+  // 128 b, U per block at 256 + 64 b. The bf16 S^T operand (64 columns of pairs) per
+  // block at 384 + 64 b; the bf16 U^T operand is packed in place over U: thread half hc
+  // packs its 32 columns into the first 16, so K step k sits at U + uk(k).
+  __device__ static constexpr uint32_t st(int b) { return PC ? 128 : 128 * b; }
+  __device__ static constexpr uint32_t uc(int b, int p) { return PC ? (p ? 320 : 0) : 256 + 64 * b; }
+  __device__ static constexpr uint32_t yo(int p) { return p ? 256 : 64; }
+  __device__ static constexpr uint32_t sbf(int b) { return 384 + 64 * b; }
+  __device__ static constexpr uint32_t uk(int k) { return (k >> 1) * 32 + (k & 1) * 8; }
   static constexpr uint32_t COLS = 512;
 };
 static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
@@ -638,8 +648,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
   uint64_t* bar_empty = bars + 2;  // two stages
   uint64_t* bar_m1 = bars + 4;
   uint64_t* bar_m2 = bars + 5;
-  uint64_t* bar_sready = bars + 6;
-  uint64_t* bar_yready = bars + 7;
+  uint64_t* bar_sready = bars + 6;  // two column halves
+  uint64_t* bar_yready = bars + 8;  // two column halves
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
 
   if (warp == 0) {
@@ -647,17 +657,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 10; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
   }
-  // identity operand: zeros, then the diagonal
-  for (int e = tid; e < static_cast<int>(K8 / 16); e += kWalkThreads)
-    *reinterpret_cast<uint4*>(sm + L_::ID + e * 16) = make_uint4(0u, 0u, 0u, 0u);
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid < C) *reinterpret_cast<uint16_t*>(sm + L_::ID + sw128_off(tid, tid, K8)) = 0x3F80u;
   const uint32_t tb = *tptr;
 
   if (warp == kWalkLoadWarp) {
@@ -681,15 +686,19 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
         mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
         for (int bx = 0; bx < 2; ++bx) {
           if (PC) {
-            tma_load_2d(dst + L_::WN + bx * K16, &a.tm_wn, bar_full + st, 64 * bx, y);
-            tma_load_2d(dst + L_::WN + K8 + bx * K16, &a.tm_qt, bar_full + st, 64 * bx, y);
+            // even stages: [-W | Q~] rows, odd stages: [Q~ | -W]
+            tma_load_2d(dst + L_::WQ + st * K8 + bx * K16, &a.tm_wn, bar_full + st, 64 * bx, y);
+            tma_load_2d(dst + L_::WQ + (st ^ 1) * K8 + bx * K16, &a.tm_qt, bar_full + st, 64 * bx, y);
+            // even stages: [P^T | Kb], odd stages: [Kb | P^T]
+            tma_load_2d(dst + L_::PK + (st ? 0 : K8) + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
           } else {
-            tma_load_2d(dst + L_::WN + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
+            tma_load_2d(dst + L_::WQ + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
+            tma_load_2d(dst + L_::PK + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
           }
-          tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 64 * bx, y);
-          tma_load_2d(dst + L_::KB + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
+          tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 0,
+                      static_cast<int>(tile * D) + 64 * bx);
         }
-        if (PC) tma_load_2d(dst + L_::PT, &a.tm_pt, bar_full + st, 0, y);
+        if (PC) tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_pt, bar_full + st, 0, y);
         bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
         ++issued;
       }
@@ -707,57 +716,65 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
         const int st = n & 1;
         const uint32_t stg = sb + st * L_::STAGE;
         if (!(ok = mbar_wait(bar_full + st, (n >> 1) & 1))) break;
-        if (!(ok = mbar_wait(bar_sready, n & 1))) break;
-        tc_fence_after();
-        // MMA-1: [U^T | (Q~ S)^T] = S^T [-W; Q~]^T (+ U0^T I on the U^T half)
-        const uint32_t i_mn = idesc_bf16(128, 64, 1, 0);
+        // MMA-1: U^T (output walk: with (Q~ S)^T in the same accumulator) = S^T [-W; Q~]^T,
+        // K = the 128 state rows in two halves, each started once its half of S^T is packed
+        const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 0);
+        const uint32_t d1 = PC ? (st ? L_::yo(1) : L_::uc(0, 0)) : 0;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 0);
+        for (int half = 0; half < 2; ++half) {
+          if (!(ok = mbar_wait(bar_sready + half, n & 1))) break;
+          tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ko_s = (k >> 2) * K16 + (k & 3) * 32;
-            const uint32_t ko_w = (k >> 2) * (PC ? K16 : K8) + (k & 3) * 32;
-            umma_bf16(tb + L_::uc(b, st), sdesc_sw128(sb + L_::S + b * K32 + ko_s, 16, 1024),
-                      sdesc_sw128(stg + L_::WN + ko_w, 16, 1024), i_k, k > 0);
-          }
-          if (PC || b == 1) {  // the M block of the summary walk has V = 0
+          for (int b = 0; b < NB; ++b)
 #pragma unroll
-            for (int k = 0; k < C / 16; ++k)
-              umma_bf16(tb + L_::uc(b, st), sdesc_sw128(stg + L_::U0 + k * 2048, K8, 1024),
-                        sdesc_sw128(sb + L_::ID + k * 32, 16, 1024), i_mn, 1);
-          }
+            for (int kk = 0; kk < 4; ++kk) {
+              const int k = 4 * half + kk;
+              const uint32_t ko_w = half * (PC ? K16 : K8) + kk * 32;
+              umma_bf16_tmem_a(tb + (PC ? d1 : L_::uc(b, 0)), tb + L_::sbf(b) + 8 * k,
+                               sdesc_sw128(stg + L_::WQ + ko_w, 16, 1024), i_k, k > 0);
+            }
         }
+        if (!ok) break;
         umma_commit(bar_m1);
         ++m_issued;
-        if (!(ok = mbar_wait(bar_yready, n & 1))) break;
-        tc_fence_after();
-        // MMA-2: O^T += U^T P^T (output walk); S^T += U^T Kb (B operands MN-major)
-        if (PC) {
-          const uint32_t ic = idesc_bf16(128, 64, 0, 1);
+        // MMA-2: output walk: [O^T | S^T] (or [S^T | O^T]) += U^T [P^T | Kb] in one N = 192
+        // product; summary walk: S^T += U^T Kb per block (B operands MN-major)
 #pragma unroll
-          for (int k = 0; k < C / 16; ++k)
-            umma_bf16(tb + L_::yo(st), sdesc_sw128(sb + L_::Y + k * 32, 16, 1024),
-                      sdesc_sw128(stg + L_::PT + k * 2048, K8, 1024), ic, 1);
+        for (int half = 0; half < 2; ++half) {
+          if (!(ok = mbar_wait(bar_yready + half, n & 1))) break;
+          tc_fence_after();
+          if (PC) {
+            const uint32_t i2 = idesc_bf16(128, 192, 0, 1);
+            const uint32_t d2 = st ? L_::st(0) : L_::yo(0);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int k = 2 * half + kk;
+              umma_bf16_tmem_a(tb + d2, tb + L_::uc(0, st) + L_::uk(k),
+                               sdesc_sw128(stg + L_::PK + k * 2048, K8, 1024), i2, 1);
+            }
+          } else {
+            const uint32_t i2 = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {
+                const int k = 2 * half + kk;
+                umma_bf16_tmem_a(tb + L_::st(b), tb + L_::uc(b, 0) + L_::uk(k),
+                                 sdesc_sw128(stg + L_::PK + k * 2048, K8, 1024), i2, 1);
+              }
+          }
         }
-        const uint32_t id = idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int k = 0; k < C / 16; ++k)
-            umma_bf16(tb + L_::st(b), sdesc_sw128(sb + L_::Y + b * K16 + k * 32, 16, 1024),
-                      sdesc_sw128(stg + L_::KB + k * 2048, K8, 1024), id, 1);
+        if (!ok) break;
         umma_commit(bar_m2);
         umma_commit(bar_empty + st);
         ++m_issued;
       }
       if (!ok) {
         atomicExch(a.seq.status, kDevWaitTimeout);
-        // the products issued so far finish before tensor memory is released
-        if (m_issued > 0) {
-          const int last = m_issued - 1;
-          mbar_wait((last & 1) ? bar_m2 : bar_m1, (last >> 1) & 1, 400000000LL);
-        }
+        // every product issued so far (committed or not) finishes before tensor memory
+        // is released: one more commit on m1, whose phase count is (m_issued + 1) / 2
+        umma_commit(bar_m1);
+        mbar_wait(bar_m1, ((m_issued + 1) / 2) & 1, 400000000LL);
       }
     }
   } else {
@@ -765,35 +782,99 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
     const int hc = warp >> 2;                // column half this thread converts
-    // initial state: fp32 into tensor memory, bf16 copy as the MMA operand
+    const int half_bar = 2 + hc;             // named barrier of this half's 128 threads
+    const bool half_lead = (warp & 3) == 0 && lane == 0;
+    // S <- Diag(gl) S on this thread's 64 fp32 columns of block b (held in v0, v1),
+    // written back to tensor memory: the decay of the chunk about to be walked
+    auto rescale = [&](int b, int st, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+      const float* gl = gls + st * D + 64 * hc;
+#pragma unroll
+      for (int t4 = 0; t4 < 8; ++t4) {
+        const float4 g0 = *reinterpret_cast<const float4*>(gl + 4 * t4);
+        const float4 g1 = *reinterpret_cast<const float4*>(gl + 32 + 4 * t4);
+        v0[4 * t4 + 0] = __float_as_uint(g0.x * __uint_as_float(v0[4 * t4 + 0]));
+        v0[4 * t4 + 1] = __float_as_uint(g0.y * __uint_as_float(v0[4 * t4 + 1]));
+        v0[4 * t4 + 2] = __float_as_uint(g0.z * __uint_as_float(v0[4 * t4 + 2]));
+        v0[4 * t4 + 3] = __float_as_uint(g0.w * __uint_as_float(v0[4 * t4 + 3]));
+        v1[4 * t4 + 0] = __float_as_uint(g1.x * __uint_as_float(v1[4 * t4 + 0]));
+        v1[4 * t4 + 1] = __float_as_uint(g1.y * __uint_as_float(v1[4 * t4 + 1]));
+        v1[4 * t4 + 2] = __float_as_uint(g1.z * __uint_as_float(v1[4 * t4 + 2]));
+        v1[4 * t4 + 3] = __float_as_uint(g1.w * __uint_as_float(v1[4 * t4 + 3]));
+      }
+      tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, v0);
+      tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+    };
+    // The decay of stage st on every block: the output walk's single block is still in
+    // v0, v1; the summary walk's blocks are reloaded from tensor memory.
+    auto rescale_all = [&](int st, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+      if (NB == 1) {
+        rescale(0, st, v0, v1);
+      } else {
+#pragma unroll 1
+        for (int b = 0; b < NB; ++b) {
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, v0);
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+          tmem_ld_wait(v0);
+          tmem_ld_wait(v1);
+          rescale(b, st, v0, v1);
+        }
+      }
+      tmem_st_wait();
+    };
+    // S^T of block b (this thread's 64 columns, in v0, v1) into the bf16 operand
+    auto pack_state = [&](int b, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        pk[t] = pack_bf16(__uint_as_float(v0[2 * t]), __uint_as_float(v0[2 * t + 1]));
+        pk[16 + t] = pack_bf16(__uint_as_float(v1[2 * t]), __uint_as_float(v1[2 * t + 1]));
+      }
+      tmem_st32(tb + lane_base + L_::sbf(b) + 32 * hc, pk);
+    };
+    bool failed = false, pend_store = false;
+    // initial state: fp32 into tensor memory, bf16 copy as the MMA operand; then the
+    // first chunk's decay on the fp32 copy
     {
       const float* src = nullptr;
       if (PC) {
         if (nseg > 1) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
         else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
       }
-      for (int b = 0; b < NB; ++b)
-        for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
-          uint32_t v[32];
+      uint32_t v0[32], v1[32];  // the last block's values (the only one in the output walk)
+#pragma unroll 1
+      for (int b = 0; b < NB; ++b) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            float x;
-            if (PC) x = src ? src[static_cast<int64_t>(c + t) * D + row] : 0.f;
-            else x = (b == 0 && c + t == row) ? 1.f : 0.f;
-            v[t] = __float_as_uint(x);
+        for (int t = 0; t < 32; ++t) {
+          const int c0 = 64 * hc + t, c1 = 64 * hc + 32 + t;
+          float x0, x1;
+          if (PC) {
+            x0 = src ? src[static_cast<int64_t>(c0) * D + row] : 0.f;
+            x1 = src ? src[static_cast<int64_t>(c1) * D + row] : 0.f;
+          } else {
+            x0 = (b == 0 && c0 == row) ? 1.f : 0.f;
+            x1 = (b == 0 && c1 == row) ? 1.f : 0.f;
           }
-          tmem_st32(tb + lane_base + L_::st(b) + c, v);
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8)
-            *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, c / 8 + q8, K16)) =
-                pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+          v0[t] = __float_as_uint(x0);
+          v1[t] = __float_as_uint(x1);
         }
+        pack_state(b, v0, v1);
+        if (NB > 1 || n_chunks == 0) {  // the unscaled fp32 state (reloaded below / final)
+          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, v0);
+          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+        }
+      }
       tmem_st_wait();
+      tc_fence_before();
+      group_sync(half_bar, 128);
+      if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + hc);
+      if (n_chunks > 0) {
+        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0))) {
+          failed = true;
+        } else {
+          rescale_all(0, v0, v1);
+        }
+      }
     }
-    tc_fence_before();
-    fence_async_smem();
-    group_sync(kConvBar, kWalkConvThreads);
-    if (tid == 0 && n_chunks > 0) mbar_arrive(bar_sready);
 
     // O of chunk n (tensor-memory buffer yo(n & 1)) to global memory: full chunks
     // through the staging tile and a TMA store, a ragged last chunk directly
@@ -825,65 +906,61 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
       bulk_commit();
     };
 
-    bool failed = false, pend_store = false;
-    for (int n = 0; n < n_chunks; ++n) {
+    // Per chunk n (stage st = n % 2 has landed): MMA-1(n) runs -> U^T (+ U0^T) packed ->
+    // MMA-2(n) runs while the previous chunk's outputs are written -> S^T packed for
+    // MMA-1(n + 1), then the fp32 state rescaled by the next chunk's decay.
+    for (int n = 0; n < n_chunks && !failed; ++n) {
       const int st = n & 1;
-      if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + st, (n >> 1) & 1))) {
-        failed = true;
-        break;
-      }
-      // ---- while MMA-1 runs: S <- Diag(gl) S in tensor memory (MMA-1 reads the bf16
-      //      copy), then the previous chunk's outputs
+      // U0^T[j][r] for this thread's rows r = 32 hc .. 32 hc + 31 (four 16-byte chunks
+      // of row j of the swizzled [64 j][64 r] box)
+      float u0v[32];
       {
-        const float* gl = gls + st * D + 64 * hc;
-#pragma unroll 1
-        for (int b = 0; b < NB; ++b) {
-          uint32_t s0[32], s1[32];
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, s0);
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, s1);
-          tmem_ld_wait(s0);
-          tmem_ld_wait(s1);
+        const unsigned char* u0r = sm + st * L_::STAGE + L_::U0 + (row >> 6) * K8;
 #pragma unroll
-          for (int t4 = 0; t4 < 8; ++t4) {
-            const float4 g0 = *reinterpret_cast<const float4*>(gl + 4 * t4);
-            const float4 g1 = *reinterpret_cast<const float4*>(gl + 32 + 4 * t4);
-            s0[4 * t4 + 0] = __float_as_uint(g0.x * __uint_as_float(s0[4 * t4 + 0]));
-            s0[4 * t4 + 1] = __float_as_uint(g0.y * __uint_as_float(s0[4 * t4 + 1]));
-            s0[4 * t4 + 2] = __float_as_uint(g0.z * __uint_as_float(s0[4 * t4 + 2]));
-            s0[4 * t4 + 3] = __float_as_uint(g0.w * __uint_as_float(s0[4 * t4 + 3]));
-            s1[4 * t4 + 0] = __float_as_uint(g1.x * __uint_as_float(s1[4 * t4 + 0]));
-            s1[4 * t4 + 1] = __float_as_uint(g1.y * __uint_as_float(s1[4 * t4 + 1]));
-            s1[4 * t4 + 2] = __float_as_uint(g1.z * __uint_as_float(s1[4 * t4 + 2]));
-            s1[4 * t4 + 3] = __float_as_uint(g1.w * __uint_as_float(s1[4 * t4 + 3]));
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row & 63, 4 * hc + q, K8));
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16(w[e]);
+            u0v[8 * q + 2 * e] = f.x;
+            u0v[8 * q + 2 * e + 1] = f.y;
           }
-          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, s0);
-          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, s1);
         }
-        tmem_st_wait();
       }
-      const bool staged = (PC && n > 0) ? emit_out(n - 1) : false;
       if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_m1, n & 1))) {
         failed = true;
         break;
       }
       tc_fence_after();
-      // ---- U^T -> bf16 operand (this thread's 32 columns of each block)
+      // ---- U^T (+ U0^T) -> bf16 operand, packed in place (this thread's 32 columns)
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        uint32_t v[32];
+        uint32_t v[32], pk[16];
         tmem_ld32(tb + lane_base + L_::uc(b, st) + 32 * hc, v);
         tmem_ld_wait(v);
+        const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          *reinterpret_cast<uint4*>(sm + L_::Y + b * K16 + sw128_chunk(row, 4 * hc + q8, K16)) =
-              pack8(reinterpret_cast<const float*>(v) + 8 * q8);
+        for (int t = 0; t < 16; ++t) {
+          float x0 = __uint_as_float(v[2 * t]), x1 = __uint_as_float(v[2 * t + 1]);
+          if (with_u0) {
+            x0 += u0v[2 * t];
+            x1 += u0v[2 * t + 1];
+          }
+          pk[t] = pack_bf16(x0, x1);
+        }
+        tmem_st16(tb + lane_base + L_::uc(b, st) + 32 * hc, pk);
       }
+      tmem_st_wait();
       tc_fence_before();
-      fence_async_smem();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0) {
-        mbar_arrive(bar_yready);
-        if (staged) {
+      group_sync(half_bar, 128);
+      if (half_lead) mbar_arrive(bar_yready + hc);
+      // ---- while MMA-2(n) runs: the previous chunk's outputs
+      if (PC && n > 0) {
+        const bool staged = emit_out(n - 1);
+        fence_async_smem();
+        group_sync(kConvBar, kWalkConvThreads);
+        if (tid == 0 && staged) {
           store_out(n - 1);
           pend_store = true;
         }
@@ -893,30 +970,33 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
         break;
       }
       tc_fence_after();
-      // ---- bf16 S^T for the next chunk
+      // ---- bf16 S^T operand for MMA-1(n + 1), then the next chunk's decay on the fp32 state
+      uint32_t v0[32], v1[32];
 #pragma unroll 1
       for (int b = 0; b < NB; ++b) {
-        uint32_t v0[32], v1[32];
         tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, v0);
         tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
         tmem_ld_wait(v0);
         tmem_ld_wait(v1);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, 8 * hc + q8, K16)) =
-              pack8(reinterpret_cast<const float*>(v0) + 8 * q8);
-          *reinterpret_cast<uint4*>(sm + L_::S + b * K32 + sw128_chunk(row, 8 * hc + 4 + q8, K16)) =
-              pack8(reinterpret_cast<const float*>(v1) + 8 * q8);
+        pack_state(b, v0, v1);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      group_sync(half_bar, 128);
+      if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + hc);
+      if (n + 1 < n_chunks) {
+        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
+          failed = true;
+          break;
         }
+        rescale_all(st ^ 1, v0, v1);
       }
       if (tid == 0 && pend_store) {
         bulk_wait_read();  // the staging tile may be rewritten after the barrier below
         pend_store = false;
       }
       tc_fence_before();
-      fence_async_smem();
       group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready);
     }
     if (PC && !failed && n_chunks > 0) {
       // the last chunk's outputs
@@ -1133,7 +1213,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
       !make_map(&ia.tm_kb, kb, D, rows_t, D * 2, true) ||
 
       !make_map(&wa.tm_wn, wn, D, rows_t, D * 2, true) ||
-      !make_map(&wa.tm_u0, u0, D, rows_t, D * 2, true) ||
+      !make_map(&wa.tm_u0, u0, C, static_cast<uint64_t>(tiles) * D, C * 2, true) ||
       !make_map(&wa.tm_kb, kb, D, rows_t, D * 2, true) ||
       !make_map(&wa.tm_qt, qt, D, rows_t, D * 2, true) ||
       !make_map(&wa.tm_pt, pt, C, rows_t, C * 2, true) ||
