@@ -92,6 +92,16 @@ __device__ __forceinline__ bool seq_bounds_tc(const SeqTable& q, int s, int64_t&
 // ceil(T_total/64) + n_seqs.
 __device__ __forceinline__ int64_t slot_base(int64_t t0, int s) { return t0 / C + s; }
 
+// Segments of a sequence: segment 0 holds first_tokens tokens, every later one
+// seg_tokens (both multiples of the chunk length; the last segment may be shorter).
+__device__ __forceinline__ int seg_count(int64_t len, int first_tokens, int seg_tokens) {
+  if (len <= first_tokens) return 1;
+  return 1 + static_cast<int>((len - first_tokens + seg_tokens - 1) / seg_tokens);
+}
+__device__ __forceinline__ int64_t seg_offset(int seg, int first_tokens, int seg_tokens) {
+  return seg == 0 ? 0 : first_tokens + static_cast<int64_t>(seg - 1) * seg_tokens;
+}
+
 struct IntraArgs {
   CUtensorMap tm_q, tm_k, tm_g;  // [T_total][H*128] bf16, 64x64 boxes, no swizzle
   CUtensorMap tm_v;              // the same shape, 128-byte swizzle (an MMA operand as loaded)
@@ -113,11 +123,13 @@ struct WalkArgs {
   __nv_bfloat16* out;
   const float* s0;
   float* sT;
-  float* mbuf;    // [pairs, max_segs-1, D, D]  summary: M (row-major [i][j])
-  float* lbuf;    // [pairs, max_segs-1, D, D]  summary: L
-  float* sstart;  // [pairs, max_segs, D, D]    start state of every segment
+  float* mbuf;    // [pairs, max_segs, D, D]  summary of segment j: M (row-major [i][j])
+  float* lbuf;    // [pairs, max_segs, D, D]  summary of segment j: L
+  float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 1
   int H;
-  int seg_tokens, max_segs;
+  int first_tokens, seg_tokens;  // segment 0, then every later segment (the last may be short)
+  int max_segs;
+  int64_t max_len;  // the caller's bound on a sequence's length
   float scale;
 };
 
@@ -614,33 +626,36 @@ struct WalkSm {
 static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
 static_assert(WalkSm<false>::BYTES + 1024 <= 232448, "summary walk shared memory");
 
+// One CTA walks segment `seg` of the (sequence, head) pair: the output walk (PC) from
+// the segment's true start state, writing outputs (and the state where a later step
+// needs it), or the summary walk of a middle segment.
 template <bool PC>
-__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_constant__ WalkArgs a) {
+__device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* smem_raw, int pair,
+                                             int seg) {
   using L_ = WalkSm<PC>;
   constexpr int NB = L_::NB;
-  extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int per = PC ? a.max_segs : a.max_segs - 1;
-  const int seg = blockIdx.x % per;
-  const int pair = blockIdx.x / per;
   const int s = pair / a.H, h = pair % a.H;
   int64_t t0, t1;
   if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t len = t1 - t0;
-  const int nseg = len > 0 ? static_cast<int>((len + a.seg_tokens - 1) / a.seg_tokens) : 1;
-  if (nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
+  const int nseg = seg_count(len, a.first_tokens, a.seg_tokens);
+  if (len > a.max_len || nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
     if (seg == 0 && tid == 0) atomicExch(a.seq.status, kDevBadSeqlens);
     return;
   }
-  if (PC ? (seg >= nseg) : (seg >= nseg - 1)) return;
-  const int64_t c_begin = t0 + static_cast<int64_t>(seg) * a.seg_tokens;
-  const int64_t c_end = (c_begin + a.seg_tokens < t1) ? c_begin + a.seg_tokens : t1;
+  // output walks: every segment; summary walks: the middle ones (segment 0's end state
+  // comes from its output walk, the last segment's is never needed)
+  if (PC ? (seg >= nseg) : (seg < 1 || seg > nseg - 2)) return;
+  const int64_t off = seg_offset(seg, a.first_tokens, a.seg_tokens);
+  const int64_t c_begin = t0 + off;
+  const int64_t c_next = t0 + seg_offset(seg + 1, a.first_tokens, a.seg_tokens);
+  const int64_t c_end = c_next < t1 ? c_next : t1;
   const int n_chunks = static_cast<int>((c_end - c_begin + C - 1) / C);
   // workspace tile of chunk n of this segment: tile0 + n H
-  const int64_t tile0 =
-      (slot_base(t0, s) + static_cast<int64_t>(seg) * (a.seg_tokens / C)) * a.H + h;
+  const int64_t tile0 = (slot_base(t0, s) + off / C) * a.H + h;
 
   float* gls = reinterpret_cast<float*>(sm + L_::GL);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_::BARS);
@@ -837,7 +852,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
     {
       const float* src = nullptr;
       if (PC) {
-        if (nseg > 1) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
+        if (seg > 0) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
         else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
       }
       uint32_t v0[32], v1[32];  // the last block's values (the only one in the output walk)
@@ -1014,9 +1029,13 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
       for (int b = 0; b < NB; ++b) {
         float* dst = nullptr;
         if (PC) {
-          if (a.sT && seg == nseg - 1) dst = a.sT + static_cast<int64_t>(pair) * D * D;
+          if (seg == nseg - 1) {
+            if (a.sT) dst = a.sT + static_cast<int64_t>(pair) * D * D;
+          } else if (seg == 0) {  // S at the end of segment 0 starts the combine
+            dst = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + 1) * D * D;
+          }
         } else {
-          const int64_t un = static_cast<int64_t>(pair) * (a.max_segs - 1) + seg;
+          const int64_t un = static_cast<int64_t>(pair) * a.max_segs + seg;
           dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
         }
         if (dst == nullptr) continue;
@@ -1038,10 +1057,28 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
   }
 }
 
+// Phase 1, per (sequence, head): CTA 0 walks segment 0 with outputs (its end state is
+// S_1), CTA r >= 1 is the summary walk of segment r, in parallel.
+constexpr uint32_t kWalkFirstSmem =
+    (WalkSm<true>::BYTES > WalkSm<false>::BYTES ? WalkSm<true>::BYTES : WalkSm<false>::BYTES) + 1024;
+__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_first(const __grid_constant__ WalkArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const int per = a.max_segs > 2 ? a.max_segs - 1 : 1;
+  const int role = blockIdx.x % per, pair = blockIdx.x / per;
+  if (role == 0) walk_segment<true>(a, smem_raw, pair, 0);
+  else walk_segment<false>(a, smem_raw, pair, role);
+}
+// Phase 2 (after the combine): the output walks of segments 1 .. nseg - 1.
+__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid_constant__ WalkArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  const int per = a.max_segs - 1;
+  walk_segment<true>(a, smem_raw, blockIdx.x / per, 1 + blockIdx.x % per);
+}
+
 // ------------------------------------------------------------------ combine
-// Start state of every segment: S_{j+1} = M_j S_j + L_j, fp32, one CTA per
-// (sequence, head, 16-column slice). M_{j+1} streams into shared memory
-// (cp.async, double-buffered) while step j is computed.
+// Start state of every segment j >= 2: S_{j+1} = M_j S_j + L_j from S_1 (written by the
+// output walk of segment 0), fp32, one CTA per (sequence, head, 16-column slice).
+// M_{j+1} streams into shared memory (cp.async, double-buffered) while step j is computed.
 constexpr int kCombSlices = 8, kCombCols = D / kCombSlices, kMStride = D + 4;
 constexpr int kCombSmem = (2 * D * kMStride + D * kCombCols) * 4;
 
@@ -1061,12 +1098,12 @@ __global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ Wa
   int64_t t0, t1;
   if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t len = t1 - t0;
-  const int nseg = len > 0 ? (int)((len + a.seg_tokens - 1) / a.seg_tokens) : 1;
-  if (nseg <= 1 || nseg > a.max_segs) return;
+  const int nseg = seg_count(len, a.first_tokens, a.seg_tokens);
+  if (len > a.max_len || nseg <= 2 || nseg > a.max_segs) return;
   const int tid = threadIdx.x;
   float* st0 = a.sstart + (int64_t)pair * a.max_segs * D * D;
   auto load_m = [&](int sg, int buf) {
-    const float* M = a.mbuf + ((int64_t)pair * (a.max_segs - 1) + sg) * D * D;
+    const float* M = a.mbuf + ((int64_t)pair * a.max_segs + sg) * D * D;
     float* dst = Ms + buf * D * kMStride;
     for (int e = tid; e < D * D / 4; e += 256) {
       const int r = e >> 5, c = (e & 31) * 4;
@@ -1074,20 +1111,18 @@ __global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ Wa
     }
     cp_async_commit();
   };
-  load_m(0, 0);
+  load_m(1, 1);
   for (int e = tid; e < D * kCombCols; e += 256) {
     const int i = e / kCombCols, c = e % kCombCols;
-    const float x = a.s0 ? a.s0[(int64_t)pair * D * D + i * D + j0 + c] : 0.f;
-    Ss[i * kCombCols + c] = x;
-    st0[i * D + j0 + c] = x;
+    Ss[i * kCombCols + c] = st0[static_cast<int64_t>(D) * D + i * D + j0 + c];  // S_1
   }
   const int i = tid >> 1, ch = (tid & 1) * 8;
-  for (int sg = 0; sg < nseg - 1; ++sg) {
+  for (int sg = 1; sg < nseg - 1; ++sg) {
     const int buf = sg & 1;
     cp_async_wait_all();
     __syncthreads();  // M_sg landed; S of the previous step is visible; other buffer free
     if (sg + 1 < nseg - 1) load_m(sg + 1, buf ^ 1);
-    const float* Lm = a.lbuf + ((int64_t)pair * (a.max_segs - 1) + sg) * D * D + i * D + j0 + ch;
+    const float* Lm = a.lbuf + ((int64_t)pair * a.max_segs + sg) * D * D + i * D + j0 + ch;
     const float4 l0 = *reinterpret_cast<const float4*>(Lm);
     const float4 l1 = *reinterpret_cast<const float4*>(Lm + 4);
     float acc[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
@@ -1149,12 +1184,6 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int64_t pow2_ceil(int64_t x) {
-  int64_t p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
 size_t align_to(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
@@ -1166,20 +1195,33 @@ bool tc_path_applies(const kda_shape& s, int64_t T_total) {
 TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   TcPlan p{};
   p.n_slots = (T_total + C - 1) / C + n_seqs;
-  int64_t per_sm = (static_cast<int64_t>(H) * p.n_slots + 147) / 148;
-  if (per_sm < 8) per_sm = 8;
-  const int64_t seg_chunks = pow2_ceil(per_sm);
-  p.seg_tokens = static_cast<int>(seg_chunks * C > (int64_t(1) << 30) ? (int64_t(1) << 30)
-                                                                       : seg_chunks * C);
-  if (max_len < 1) max_len = 1;
-  p.max_segs = static_cast<int>((max_len + p.seg_tokens - 1) / p.seg_tokens);
-  if (p.max_segs < 1) p.max_segs = 1;
   p.pairs = static_cast<int64_t>(n_seqs) * H;
+  if (max_len < 1) max_len = 1;
+  // Segments: the walks run one CTA per SM, and a chunk costs about the same in every
+  // CTA, so a sequence of Lc chunks is cut into segment 0 plus m later segments with
+  // m = SMs / pairs: phase 1 = segment 0's output walk beside the summary walks of
+  // segments 1 .. m - 1, phase 2 = the output walks of segments 1 .. m. Segment 0 is
+  // 1.125 x longer, matching the summary walk's slower chunk step.
+  const int64_t Lc = (max_len + C - 1) / C;
+  const int64_t m = p.pairs > 0 ? 148 / p.pairs : 1;
+  if (m < 2 || Lc < 16) {
+    p.first_tokens = p.seg_tokens = 1 << 30;  // one segment per sequence
+    p.max_segs = 1;
+  } else {
+    int64_t n = (8 * Lc + 8 * m + 9 - 1) / (8 * m + 9);  // ceil(Lc / (m + 1.125))
+    if (n < 4) n = 4;
+    const int64_t n0 = (9 * n + 7) / 8;  // ceil(1.125 n)
+    p.first_tokens = static_cast<int>(n0 * C);
+    p.seg_tokens = static_cast<int>(n * C);
+    p.max_segs = max_len <= p.first_tokens
+                     ? 1
+                     : 1 + static_cast<int>((max_len - p.first_tokens + p.seg_tokens - 1) /
+                                            p.seg_tokens);
+  }
   const size_t state = sizeof(float) * D * D;
   size_t off = kWorkspaceHeader;
-  if (p.max_segs > 1)
-    off += state * static_cast<size_t>(p.pairs) *
-           (2 * static_cast<size_t>(p.max_segs - 1) + static_cast<size_t>(p.max_segs));
+  if (p.max_segs > 1)  // M, L and the start state of every segment
+    off += state * static_cast<size_t>(p.pairs) * 3 * static_cast<size_t>(p.max_segs);
   p.tiles_off = align_to(off, 1024);
   p.ws_bytes = p.tiles_off + kTileBytes * static_cast<size_t>(p.n_slots) * static_cast<size_t>(H);
   return p;
@@ -1236,9 +1278,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   const size_t state = static_cast<size_t>(D) * D;
   float* base = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
   wa.mbuf = base;
-  wa.lbuf = wa.mbuf + state * plan.pairs * (plan.max_segs - 1);
-  wa.sstart = wa.lbuf + state * plan.pairs * (plan.max_segs - 1);
+  wa.lbuf = wa.mbuf + state * plan.pairs * plan.max_segs;
+  wa.sstart = wa.lbuf + state * plan.pairs * plan.max_segs;
   wa.H = pa.H;
+  wa.first_tokens = plan.first_tokens;
+  wa.max_len = pa.max_len;
   wa.seg_tokens = plan.seg_tokens;
   wa.max_segs = plan.max_segs;
   wa.scale = pa.scale;
@@ -1247,24 +1291,25 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        IntraSm::BYTES + 1024);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_walk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             WalkSm<true>::BYTES + 1024);
+    e = cudaFuncSetAttribute(kda_tc_walk_first, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kWalkFirstSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_walk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             WalkSm<false>::BYTES + 1024);
+    e = cudaFuncSetAttribute(kda_tc_walk_rest, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             WalkSm<true>::BYTES + 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kda_tc_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kCombSmem);
   if (e != cudaSuccess) return e;
 
   kda_tc_intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
-  if (plan.max_segs > 1) {
-    kda_tc_walk<false><<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), kWalkThreads,
-                         WalkSm<false>::BYTES + 1024, st>>>(wa);
+  const int64_t per_first = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
+  kda_tc_walk_first<<<static_cast<unsigned>(plan.pairs * per_first), kWalkThreads, kWalkFirstSmem,
+                      st>>>(wa);
+  if (plan.max_segs > 2)
     kda_tc_combine<<<static_cast<unsigned>(plan.pairs * kCombSlices), 256, kCombSmem, st>>>(wa);
-  }
-  kda_tc_walk<true><<<static_cast<unsigned>(plan.pairs * plan.max_segs), kWalkThreads,
-                      WalkSm<true>::BYTES + 1024, st>>>(wa);
+  if (plan.max_segs > 1)
+    kda_tc_walk_rest<<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), kWalkThreads,
+                       WalkSm<true>::BYTES + 1024, st>>>(wa);
   return cudaGetLastError();
 }
 
