@@ -1076,80 +1076,173 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid
 }
 
 // ------------------------------------------------------------------ combine
-// Start state of every segment j >= 2: S_{j+1} = M_j S_j + L_j from S_1 (written by the
-// output walk of segment 0), fp32, one CTA per (sequence, head, 16-column slice).
-// M_{j+1} streams into shared memory (cp.async, double-buffered) while step j is computed.
-constexpr int kCombSlices = 8, kCombCols = D / kCombSlices, kMStride = D + 4;
-constexpr int kCombSmem = (2 * D * kMStride + D * kCombCols) * 4;
+// Start state of every segment j >= 2 from S_1 (written by segment 0's output walk):
+// S_{j+1} = M_j S_j + L_j for j = 1 .. nseg - 2, one CTA per (sequence, head). Each step
+// is one 128x128x128 product on the tensor cores in the transposed frame,
+// S_{j+1}^T = S_j^T M_j^T + L_j^T, at fp32 accuracy through a bf16 split of both factors,
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi):
+//   S^T M^T ~= S_hi^T M_hi^T + S_hi^T M_lo^T + S_lo^T M_hi^T
+// (the dropped lo x lo term is ~2^-16 of the product). S^T, the A operand, lives in tensor
+// memory; M_j, the B operand (row-major = K-major), in shared memory; L_j^T seeds the
+// accumulator.
+constexpr int kCombThreads = 256;
+constexpr uint32_t kCombSmem = 2 * K32 + 1024 + 64;  // M hi and lo tiles, barrier, TMEM base
+struct CombTm {
+  static constexpr uint32_t D = 0, AH = 128, AL = 192, COLS = 256;
+};
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16(x - hf.x, y - hf.y);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(256) kda_tc_combine(const __grid_constant__ WalkArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* Ms = reinterpret_cast<float*>(smem_raw);  // [2][128][132]
-  float* Ss = Ms + 2 * D * kMStride;               // [128][16]
-  const int pair = blockIdx.x / kCombSlices, j0 = (blockIdx.x % kCombSlices) * kCombCols;
+__global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_constant__ WalkArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = align1024(smem_raw);
+  const uint32_t sb = smem_u32(sm);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * K32);
+  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + 2 * K32 + 8);
+  const int pair = blockIdx.x;
   const int s = pair / a.H;
   int64_t t0, t1;
   if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t len = t1 - t0;
   const int nseg = seg_count(len, a.first_tokens, a.seg_tokens);
   if (len > a.max_len || nseg <= 2 || nseg > a.max_segs) return;
-  const int tid = threadIdx.x;
-  float* st0 = a.sstart + (int64_t)pair * a.max_segs * D * D;
-  auto load_m = [&](int sg, int buf) {
-    const float* M = a.mbuf + ((int64_t)pair * a.max_segs + sg) * D * D;
-    float* dst = Ms + buf * D * kMStride;
-    for (int e = tid; e < D * D / 4; e += 256) {
-      const int r = e >> 5, c = (e & 31) * 4;
-      cp_async16(dst + r * kMStride + c, M + r * D + c);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = (warp & 3) * 32 + lane, hc = warp >> 2;  // lane j; this thread's column half
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  float* st0 = a.sstart + static_cast<int64_t>(pair) * a.max_segs * D * D;
+
+  if (warp == 0) {
+    tmem_alloc(tptr, CombTm::COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  } else if (tid == 32) {
+    // every step's M and L into L2 now: the steps read them one after another
+    for (int sg = 1; sg < nseg - 1; ++sg) {
+      const int64_t o = (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D;
+      bulk_prefetch_l2(a.mbuf + o, D * D * 4);
+      bulk_prefetch_l2(a.lbuf + o, D * D * 4);
     }
-    cp_async_commit();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = *tptr;
+
+  // this thread's 64 values of S^T (row j, columns 64 hc ..) -> the split A operand
+  auto put_a = [&](const uint32_t (&v0)[32], const uint32_t (&v1)[32]) {
+    uint32_t h[32], l[32];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      split_bf16(__uint_as_float(v0[2 * t]), __uint_as_float(v0[2 * t + 1]), h[t], l[t]);
+      split_bf16(__uint_as_float(v1[2 * t]), __uint_as_float(v1[2 * t + 1]), h[16 + t], l[16 + t]);
+    }
+    tmem_st32(tb + lane_base + CombTm::AH + 32 * hc, h);
+    tmem_st32(tb + lane_base + CombTm::AL + 32 * hc, l);
   };
-  load_m(1, 1);
-  for (int e = tid; e < D * kCombCols; e += 256) {
-    const int i = e / kCombCols, c = e % kCombCols;
-    Ss[i * kCombCols + c] = st0[static_cast<int64_t>(D) * D + i * D + j0 + c];  // S_1
-  }
-  const int i = tid >> 1, ch = (tid & 1) * 8;
-  for (int sg = 1; sg < nseg - 1; ++sg) {
-    const int buf = sg & 1;
-    cp_async_wait_all();
-    __syncthreads();  // M_sg landed; S of the previous step is visible; other buffer free
-    if (sg + 1 < nseg - 1) load_m(sg + 1, buf ^ 1);
-    const float* Lm = a.lbuf + ((int64_t)pair * a.max_segs + sg) * D * D + i * D + j0 + ch;
-    const float4 l0 = *reinterpret_cast<const float4*>(Lm);
-    const float4 l1 = *reinterpret_cast<const float4*>(Lm + 4);
-    float acc[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-    const float* Mrow = Ms + buf * D * kMStride + i * kMStride;
-#pragma unroll 8
-    for (int k = 0; k < D; ++k) {
-      const float m = Mrow[k];
-      const float4 s0 = *reinterpret_cast<const float4*>(Ss + k * kCombCols + ch);
-      const float4 s1 = *reinterpret_cast<const float4*>(Ss + k * kCombCols + ch + 4);
-      acc[0] = fmaf(m, s0.x, acc[0]);
-      acc[1] = fmaf(m, s0.y, acc[1]);
-      acc[2] = fmaf(m, s0.z, acc[2]);
-      acc[3] = fmaf(m, s0.w, acc[3]);
-      acc[4] = fmaf(m, s1.x, acc[4]);
-      acc[5] = fmaf(m, s1.y, acc[5]);
-      acc[6] = fmaf(m, s1.z, acc[6]);
-      acc[7] = fmaf(m, s1.w, acc[7]);
+  {
+    // S_1^T[j][k] = S_1[k][j]
+    uint32_t v0[32], v1[32];
+    const float* src = st0 + static_cast<int64_t>(D) * D + row;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      v0[t] = __float_as_uint(src[(64 * hc + t) * D]);
+      v1[t] = __float_as_uint(src[(64 * hc + 32 + t) * D]);
     }
-    __syncthreads();  // every read of S done
-    float* dst = st0 + (int64_t)(sg + 1) * D * D + i * D + j0 + ch;
-    *reinterpret_cast<float4*>(Ss + i * kCombCols + ch) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(Ss + i * kCombCols + ch + 4) =
-        make_float4(acc[4], acc[5], acc[6], acc[7]);
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    put_a(v0, v1);
   }
-  cp_async_wait_all();
+  bool failed = false;
+  for (int sg = 1; sg < nseg - 1; ++sg) {
+    // M_sg -> split B operand tiles: thread = (row c, half of its 128 columns)
+    {
+      const int c = tid >> 1, half = tid & 1;
+      const float4* mr = reinterpret_cast<const float4*>(
+          a.mbuf + (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D + c * D + 64 * half);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 x0 = mr[2 * q], x1 = mr[2 * q + 1];
+        uint4 hi, lo;
+        split_bf16(x0.x, x0.y, hi.x, lo.x);
+        split_bf16(x0.z, x0.w, hi.y, lo.y);
+        split_bf16(x1.x, x1.y, hi.z, lo.z);
+        split_bf16(x1.z, x1.w, hi.w, lo.w);
+        const uint32_t off = sw128_chunk(c, 8 * half + q, K16);
+        *reinterpret_cast<uint4*>(sm + off) = hi;
+        *reinterpret_cast<uint4*>(sm + K32 + off) = lo;
+      }
+    }
+    // L_sg^T seeds the accumulator: lane j, columns c = 64 hc ..
+    {
+      const float* lr = a.lbuf + (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D + row;
+      uint32_t v0[32], v1[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        v0[t] = __float_as_uint(lr[(64 * hc + t) * D]);
+        v1[t] = __float_as_uint(lr[(64 * hc + 32 + t) * D]);
+      }
+      tmem_st32(tb + lane_base + CombTm::D + 64 * hc, v0);
+      tmem_st32(tb + lane_base + CombTm::D + 64 * hc + 32, v1);
+    }
+    tmem_st_wait();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;
+        const uint64_t bh = sdesc_sw128(sb + ko, 16, 1024), bl = sdesc_sw128(sb + K32 + ko, 16, 1024);
+        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bh, id, 1);
+        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bl, id, 1);
+        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AL + 8 * k, bh, id, 1);
+      }
+      umma_commit(bar);
+    }
+    if (cta_wait_failed(bar, (sg - 1) & 1)) {
+      failed = true;
+      break;
+    }
+    tc_fence_after();
+    // S_{sg+1}^T: to the workspace (row-major [k][j]) and, for a further step, to A
+    {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tb + lane_base + CombTm::D + 64 * hc, v0);
+      tmem_ld32(tb + lane_base + CombTm::D + 64 * hc + 32, v1);
+      tmem_ld_wait(v0);
+      tmem_ld_wait(v1);
+      float* dst = st0 + static_cast<int64_t>(sg + 1) * D * D + row;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        dst[(64 * hc + t) * D] = __uint_as_float(v0[t]);
+        dst[(64 * hc + 32 + t) * D] = __uint_as_float(v1[t]);
+      }
+      if (sg + 1 < nseg - 1) put_a(v0, v1);
+    }
+    // the next step rewrites the B tiles and the accumulator: every thread is done here
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (failed && tid == 0) {
+    atomicExch(a.seq.status, kDevWaitTimeout);
+    mbar_wait(bar, 0, 400000000LL);  // the products in flight finish before TMEM is freed
+    mbar_wait(bar, 1, 400000000LL);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, CombTm::COLS);
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1306,7 +1399,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   kda_tc_walk_first<<<static_cast<unsigned>(plan.pairs * per_first), kWalkThreads, kWalkFirstSmem,
                       st>>>(wa);
   if (plan.max_segs > 2)
-    kda_tc_combine<<<static_cast<unsigned>(plan.pairs * kCombSlices), 256, kCombSmem, st>>>(wa);
+    kda_tc_combine<<<static_cast<unsigned>(plan.pairs), kCombThreads, kCombSmem, st>>>(wa);
   if (plan.max_segs > 1)
     kda_tc_walk_rest<<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), kWalkThreads,
                        WalkSm<true>::BYTES + 1024, st>>>(wa);
