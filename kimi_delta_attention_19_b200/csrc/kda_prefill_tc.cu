@@ -1084,9 +1084,11 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid
 //   S^T M^T ~= S_hi^T M_hi^T + S_hi^T M_lo^T + S_lo^T M_hi^T
 // (the dropped lo x lo term is ~2^-16 of the product). S^T, the A operand, lives in tensor
 // memory; M_j, the B operand (row-major = K-major), in shared memory; L_j^T seeds the
-// accumulator.
+// accumulator. The next step's M and L (fp32) are copied into shared memory while the
+// current step's products run.
 constexpr int kCombThreads = 256;
-constexpr uint32_t kCombSmem = 2 * K32 + 1024 + 64;  // M hi and lo tiles, barrier, TMEM base
+constexpr uint32_t kCombMS = 2 * K32, kCombLS = kCombMS + 4 * K16, kCombBars = kCombLS + 4 * K16;
+constexpr uint32_t kCombSmem = kCombBars + 64 + 1024;  // M hi/lo tiles, M and L staging, barriers
 struct CombTm {
   static constexpr uint32_t D = 0, AH = 128, AL = 192, COLS = 256;
 };
@@ -1102,8 +1104,11 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * K32);
-  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + 2 * K32 + 8);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kCombBars);  // products done
+  uint64_t* bar_ld = bar + 1;                                     // M, L staged
+  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + kCombBars + 16);
+  const float* Mst = reinterpret_cast<const float*>(sm + kCombMS);
+  const float* Lst = reinterpret_cast<const float*>(sm + kCombLS);
   const int pair = blockIdx.x;
   const int s = pair / a.H;
   int64_t t0, t1;
@@ -1120,9 +1125,20 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     tmem_alloc(tptr, CombTm::COLS);
     tmem_relinquish();
   }
+  // M_sg and L_sg (64 KB each) into the staging buffers, in 16 KB pieces
+  auto stage_ml = [&](int sg) {
+    const int64_t o = (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D;
+    mbar_arrive_expect_tx(bar_ld, 2 * D * D * 4);
+    for (int q = 0; q < 4; ++q) {
+      bulk_load(sm + kCombMS + q * K16, a.mbuf + o + q * (K16 / 4), K16, bar_ld);
+      bulk_load(sm + kCombLS + q * K16, a.lbuf + o + q * (K16 / 4), K16, bar_ld);
+    }
+  };
   if (tid == 0) {
     mbar_init(bar, 1);
+    mbar_init(bar_ld, 1);
     fence_mbar_init();
+    stage_ml(1);
   } else if (tid == 32) {
     // every step's M and L into L2 now: the steps read them one after another
     for (int sg = 1; sg < nseg - 1; ++sg) {
@@ -1158,29 +1174,34 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     }
     put_a(v0, v1);
   }
-  bool failed = false;
+  bool failed = false, ld_pending = true;
   for (int sg = 1; sg < nseg - 1; ++sg) {
-    // M_sg -> split B operand tiles: thread = (row c, half of its 128 columns)
+    if (cta_wait_failed(bar_ld, (sg - 1) & 1)) {
+      failed = true;
+      break;
+    }
+    ld_pending = false;
+    // M_sg -> split B operand tiles. Thread t takes the 16-byte pieces t + 256 q of the
+    // row-major staging copy (consecutive lanes, consecutive addresses: no bank
+    // conflicts): row (t >> 5) + 8 q, columns 4 (t & 31) .. + 3; each becomes an 8-byte
+    // half of a 16-byte chunk of the swizzled tiles.
     {
-      const int c = tid >> 1, half = tid & 1;
-      const float4* mr = reinterpret_cast<const float4*>(
-          a.mbuf + (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D + c * D + 64 * half);
+      const int c4 = 4 * (tid & 31);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 x0 = mr[2 * q], x1 = mr[2 * q + 1];
-        uint4 hi, lo;
-        split_bf16(x0.x, x0.y, hi.x, lo.x);
-        split_bf16(x0.z, x0.w, hi.y, lo.y);
-        split_bf16(x1.x, x1.y, hi.z, lo.z);
-        split_bf16(x1.z, x1.w, hi.w, lo.w);
-        const uint32_t off = sw128_chunk(c, 8 * half + q, K16);
-        *reinterpret_cast<uint4*>(sm + off) = hi;
-        *reinterpret_cast<uint4*>(sm + K32 + off) = lo;
+      for (int q = 0; q < 16; ++q) {
+        const int r = (tid >> 5) + 8 * q;
+        const float4 x = *reinterpret_cast<const float4*>(Mst + r * D + c4);
+        uint2 hi, lo;
+        split_bf16(x.x, x.y, hi.x, lo.x);
+        split_bf16(x.z, x.w, hi.y, lo.y);
+        const uint32_t off = sw128_chunk(r, c4 >> 3, K16) + (c4 & 7) * 2;
+        *reinterpret_cast<uint2*>(sm + off) = hi;
+        *reinterpret_cast<uint2*>(sm + K32 + off) = lo;
       }
     }
     // L_sg^T seeds the accumulator: lane j, columns c = 64 hc ..
     {
-      const float* lr = a.lbuf + (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D + row;
+      const float* lr = Lst + row;
       uint32_t v0[32], v1[32];
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
@@ -1195,6 +1216,10 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
+      if (sg + 1 < nseg - 1) {  // every thread has read the staging buffers
+        stage_ml(sg + 1);
+        ld_pending = true;
+      }
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
@@ -1234,7 +1259,12 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
   }
   if (failed && tid == 0) {
     atomicExch(a.seq.status, kDevWaitTimeout);
-    mbar_wait(bar, 0, 400000000LL);  // the products in flight finish before TMEM is freed
+    // copies and products in flight finish before the CTA releases its memory
+    if (ld_pending) {
+      mbar_wait(bar_ld, 0, 400000000LL);
+      mbar_wait(bar_ld, 1, 400000000LL);
+    }
+    mbar_wait(bar, 0, 400000000LL);
     mbar_wait(bar, 1, 400000000LL);
   }
   tc_fence_before();

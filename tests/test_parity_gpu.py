@@ -156,6 +156,33 @@ def test_tensor_core_segments(kda):
     assert_close(fin, rs, torch.bfloat16, "varlen segments final_state")
 
 
+def _segment_plan(n_seqs, H, max_len):
+    """The library's segment rule (first segment, later segments, in tokens)."""
+    pairs = n_seqs * H
+    lc = -(-max_len // 64)
+    m = 148 // pairs
+    if m < 2 or lc < 16:
+        return None
+    n = max(4, -(-(8 * lc) // (8 * m + 9)))
+    return 64 * (-(-(9 * n) // 8)), 64 * n
+
+
+def test_tensor_core_segment_counts(kda):
+    """Sequences with exactly 1, 2, 3 and many segments in one call: segment 0 alone,
+    S_1 used directly by segment 1 (no combine step), one combine step, a long chain."""
+    lengths = [320, 321, 576, 577, 0, 3000]
+    first, seg = _segment_plan(len(lengths), 2, max(lengths))
+    assert (first, seg) == (320, 256)
+    nseg = [1 if n <= first else 1 + -(-(n - first) // seg) for n in lengths]
+    assert nseg == [1, 2, 2, 3, 1, 12]
+    x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=19,
+                    lengths=lengths, state_std=0.02)
+    out, fin = _run_gpu(kda, x, max_seqlen=max(lengths))
+    ro, rs = _run_oracle(x)
+    assert_close(out, ro, torch.bfloat16, "segment counts out")
+    assert_close(fin, rs, torch.bfloat16, "segment counts final_state")
+
+
 def test_tensor_core_segments_resume_in_place(kda):
     """final_state aliasing initial_state with several segments per sequence."""
     x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=17,
