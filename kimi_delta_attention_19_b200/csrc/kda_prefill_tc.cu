@@ -576,6 +576,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     tc_fence_after();
     tmem_dealloc(tb, L_::COLS);
   }
+  griddep_launch_dependents();
 }
 
 // ------------------------------------------------------------------ walk over chunks
@@ -679,6 +680,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = *tptr;
+  griddep_wait();  // the workspace and start states come from the previous kernels
 
   if (warp == kWalkLoadWarp) {
     // ============================================================ stage loads
@@ -1055,6 +1057,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     tc_fence_after();
     tmem_dealloc(tb, L_::COLS);
   }
+  griddep_launch_dependents();
 }
 
 // Phase 1, per (sequence, head): CTA 0 walks segment 0 with outputs (its end state is
@@ -1111,6 +1114,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
   const float* Lst = reinterpret_cast<const float*>(sm + kCombLS);
   const int pair = blockIdx.x;
   const int s = pair / a.H;
+  griddep_wait();  // M, L and S_1 come from the first walk phase
   int64_t t0, t1;
   if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t len = t1 - t0;
@@ -1273,6 +1277,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     tc_fence_after();
     tmem_dealloc(tb, CombTm::COLS);
   }
+  griddep_launch_dependents();
 }
 
 // ------------------------------------------------------------------ host side
@@ -1425,14 +1430,34 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   if (e != cudaSuccess) return e;
 
   kda_tc_intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
+  // The later kernels are launched with programmatic serialization: their CTAs may be
+  // scheduled while the previous kernel's last CTAs finish; they set up (tensor memory,
+  // barriers) and then wait for it (griddepcontrol.wait) before touching its results.
+  auto launch_dep = [&](const void* fn, int64_t grid, int threads, uint32_t smem) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&wa};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  };
   const int64_t per_first = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
-  kda_tc_walk_first<<<static_cast<unsigned>(plan.pairs * per_first), kWalkThreads, kWalkFirstSmem,
-                      st>>>(wa);
-  if (plan.max_segs > 2)
-    kda_tc_combine<<<static_cast<unsigned>(plan.pairs), kCombThreads, kCombSmem, st>>>(wa);
-  if (plan.max_segs > 1)
-    kda_tc_walk_rest<<<static_cast<unsigned>(plan.pairs * (plan.max_segs - 1)), kWalkThreads,
-                       WalkSm<true>::BYTES + 1024, st>>>(wa);
+  if (e == cudaSuccess)
+    e = launch_dep(reinterpret_cast<const void*>(kda_tc_walk_first), plan.pairs * per_first,
+                   kWalkThreads, kWalkFirstSmem);
+  if (e == cudaSuccess && plan.max_segs > 2)
+    e = launch_dep(reinterpret_cast<const void*>(kda_tc_combine), plan.pairs, kCombThreads,
+                   kCombSmem);
+  if (e == cudaSuccess && plan.max_segs > 1)
+    e = launch_dep(reinterpret_cast<const void*>(kda_tc_walk_rest), plan.pairs * (plan.max_segs - 1),
+                   kWalkThreads, WalkSm<true>::BYTES + 1024);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

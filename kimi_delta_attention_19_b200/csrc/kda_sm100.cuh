@@ -105,6 +105,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Block until the grids this one depends on (launched before it on the stream with
+// programmatic serialization) have completed and their memory is visible.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the dependent grid be scheduled once every CTA of this grid has said so (or exited).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ named barriers
 // Barrier `id` over `n` threads (whole warps).
 __device__ __forceinline__ void group_sync(int id, int n) {
