@@ -243,12 +243,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     // v is needed last (by the WY products): its own barrier
     mbar_arrive_expect_tx(bar_in, 3 * K16);
     mbar_arrive_expect_tx(bar_v, K16);
-    for (int bx = 0; bx < 2; ++bx) {
-      const int x = h * D + 64 * bx;
-      tma_load_2d(sm + L_::SG + bx * K8, &a.tm_g, bar_in, x, static_cast<int>(r0));
-      tma_load_2d(sm + L_::SK + bx * K8, &a.tm_k, bar_in, x, static_cast<int>(r0));
-      tma_load_2d(sm + L_::SQ + bx * K8, &a.tm_q, bar_in, x, static_cast<int>(r0));
-    }
+    // k, g, q: one [64 rows][128] box each (256-byte rows, half the row requests of two
+    // 64-column boxes); v: two swizzled 64-column boxes (the MMA operand layout)
+    tma_load_2d(sm + L_::SG, &a.tm_g, bar_in, h * D, static_cast<int>(r0));
+    tma_load_2d(sm + L_::SK, &a.tm_k, bar_in, h * D, static_cast<int>(r0));
+    tma_load_2d(sm + L_::SQ, &a.tm_q, bar_in, h * D, static_cast<int>(r0));
     for (int bx = 0; bx < 2; ++bx)
       tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_v, h * D + 64 * bx, static_cast<int>(r0));
   }
@@ -281,8 +280,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       // a sequence's ragged last chunk: rows past L (the next sequence's tokens, or the
       // zero fill past the end) become k = q = 0 and g = 0, so no later step masks rows
       for (int e = tid; e < (C - L) * 32; e += kIntraThreads) {
-        const int r = L + (e >> 5), w = e & 31;  // 16-byte words per row: two boxes x 8
-        const uint32_t off = (w >> 3 & 1) * K8 + r * 128 + (w & 7) * 16;
+        const int r = L + (e >> 5), w = e & 31;  // 16 16-byte words per 256-byte row
+        const uint32_t off = r * 256 + (w & 15) * 16;
         const int which = w >> 4;  // 0: k and g, 1: q
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
         if (which == 0) {
@@ -297,17 +296,17 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     // ---- 1. raw k, q into registers; prefix sums of the clamped log decay in log2 units.
     //         Thread = (channel pair p, quarter qr of 16 rows).
     const int p = tid & 63, qr = tid >> 6;
-    const int ch = 2 * p, bx = p >> 5, cofs = (p & 31) * 4;
+    const int ch = 2 * p, bx = p >> 5;
     constexpr float kLog2e = 1.4426950408889634f;
     const float lb2 = a.lb * kLog2e;
     uint32_t kraw[16], qraw[16];
     float G0[16], G1[16];
     {
       float acc0 = 0.f, acc1 = 0.f;
-      const uint32_t off0 = bx * K8 + 16 * qr * 128 + cofs;
+      const uint32_t off0 = 16 * qr * 256 + 4 * p;  // raw rows are 256 bytes
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const uint32_t off = off0 + i * 128;
+        const uint32_t off = off0 + i * 256;
         kraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SK + off);
         qraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SQ + off);
         const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + off));
@@ -1296,15 +1295,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 tensor map over `rows` rows of `cols` elements, `pitch` bytes apart,
-// moved in 64x64 boxes; with `swizzle` a box lands in the 128-byte-swizzled
-// operand layout.
+// moved in boxes of 64 rows x `box_cols`; with `swizzle` (64 columns) a box lands in
+// the 128-byte-swizzled operand layout.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t pitch,
-              bool swizzle) {
+              bool swizzle, uint32_t box_cols = 64) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch)};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {box_cols, 64};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1375,9 +1374,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   memset(&ia, 0, sizeof ia);
   WalkArgs wa;
   memset(&wa, 0, sizeof wa);
-  if (!make_map(&ia.tm_q, pa.q, in_cols, pa.T_total, in_pitch, false) ||
-      !make_map(&ia.tm_k, pa.k, in_cols, pa.T_total, in_pitch, false) ||
-      !make_map(&ia.tm_g, pa.g, in_cols, pa.T_total, in_pitch, false) ||
+  if (!make_map(&ia.tm_q, pa.q, in_cols, pa.T_total, in_pitch, false, D) ||
+      !make_map(&ia.tm_k, pa.k, in_cols, pa.T_total, in_pitch, false, D) ||
+      !make_map(&ia.tm_g, pa.g, in_cols, pa.T_total, in_pitch, false, D) ||
       !make_map(&ia.tm_v, pa.v, in_cols, pa.T_total, in_pitch, true) ||
       !make_map(&ia.tm_qt, qt, D, rows_t, D * 2, true) ||
       !make_map(&ia.tm_kb, kb, D, rows_t, D * 2, true) ||
