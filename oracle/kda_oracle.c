@@ -71,6 +71,9 @@ typedef struct {
     const int64_t *out_rows;
     int64_t n_out_rows;
     double *final_state;
+    int64_t snap_tokens;       /* snapshot interval in tokens (0 = none) */
+    const int64_t *snap_first; /* [n_seqs] index of each sequence's first snapshot */
+    double *snaps;             /* [n_snaps, H, dk, dv] */
     int64_t next_item; /* shared work counter over (seq, head) */
     pthread_mutex_t lock;
 } job_t;
@@ -144,6 +147,12 @@ static void run_one(const job_t *J, int seq, int h, double *S, double *kt,
                 for (int j = 0; j < dv; ++j) o[j] += qt[i] * S[i * dv + j];
             for (int j = 0; j < dv; ++j) o[j] *= J->scale;
         }
+
+        /* the state after the first m * snap_tokens tokens of the sequence */
+        if (J->snaps && (t - t0 + 1) % J->snap_tokens == 0) {
+            const int64_t idx = J->snap_first[seq] + (t - t0 + 1) / J->snap_tokens - 1;
+            memcpy(J->snaps + (idx * H + h) * dk * dv, S, sizeof(double) * dk * dv);
+        }
     }
 
     if (J->final_state) memcpy(J->final_state + state_off, S, sizeof(double) * dk * dv);
@@ -184,13 +193,14 @@ static void *worker(void *arg)
  *        indices) is given; NULL skips the read-out.
  *  Returns 0 on success, -1 on a bad argument, -2 when a thread failed.
  */
-int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
-                         const int64_t *cu_seqlens, int dtype,
-                         const void *q, const void *k, const void *v,
-                         const void *g, const void *beta,
-                         const double *initial_state, double lb, double scale,
-                         double *out, const int64_t *out_rows, int64_t n_out_rows,
-                         double *final_state, int n_threads)
+static int run_all(int64_t T, int H, int dk, int dv, int n_seqs,
+                   const int64_t *cu_seqlens, int dtype,
+                   const void *q, const void *k, const void *v,
+                   const void *g, const void *beta,
+                   const double *initial_state, double lb, double scale,
+                   double *out, const int64_t *out_rows, int64_t n_out_rows,
+                   double *final_state, int64_t snap_tokens, const int64_t *snap_first,
+                   double *snaps, int n_threads)
 {
     if (T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs <= 0 || !cu_seqlens) return -1;
     if (dtype != KDA_ORACLE_F32 && dtype != KDA_ORACLE_BF16) return -1;
@@ -207,6 +217,7 @@ int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
     J.initial_state = initial_state; J.lb = lb; J.scale = scale;
     J.out = out; J.out_rows = out_rows; J.n_out_rows = n_out_rows;
     J.final_state = final_state;
+    J.snap_tokens = snap_tokens; J.snap_first = snap_first; J.snaps = snaps;
     pthread_mutex_init(&J.lock, NULL);
 
     const int64_t n_items = (int64_t)n_seqs * H;
@@ -233,4 +244,39 @@ int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
     free(th);
     pthread_mutex_destroy(&J.lock);
     return rc;
+}
+
+int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
+                         const int64_t *cu_seqlens, int dtype,
+                         const void *q, const void *k, const void *v,
+                         const void *g, const void *beta,
+                         const double *initial_state, double lb, double scale,
+                         double *out, const int64_t *out_rows, int64_t n_out_rows,
+                         double *final_state, int n_threads)
+{
+    return run_all(T, H, dk, dv, n_seqs, cu_seqlens, dtype, q, k, v, g, beta, initial_state,
+                   lb, scale, out, out_rows, n_out_rows, final_state, 0, NULL, NULL, n_threads);
+}
+
+/*
+ * kda_oracle_recurrent that also records the state at regular points of each
+ * sequence: for every m >= 1 with m * snap_tokens <= len(seq), the state after
+ * the sequence's first m * snap_tokens tokens (seeded by its initial state) is
+ * copied to snaps[snap_first[seq] + m - 1] ([.., H, dk, dv] fp64). The caller
+ * sizes snaps and chooses snap_first so that the sequences' ranges do not
+ * overlap. A prefix cache keeps exactly these states ("3 分钟看懂 Kimi K3",
+ * 第一条主线: KDA state and prefix-cache scheduling for long requests).
+ */
+int kda_oracle_recurrent_snapshots(int64_t T, int H, int dk, int dv, int n_seqs,
+                                   const int64_t *cu_seqlens, int dtype,
+                                   const void *q, const void *k, const void *v,
+                                   const void *g, const void *beta,
+                                   const double *initial_state, double lb, double scale,
+                                   double *out, double *final_state, int64_t snap_tokens,
+                                   const int64_t *snap_first, double *snaps, int n_threads)
+{
+    if (snap_tokens <= 0 || !snap_first || !snaps) return -1;
+    return run_all(T, H, dk, dv, n_seqs, cu_seqlens, dtype, q, k, v, g, beta, initial_state,
+                   lb, scale, out, NULL, 0, final_state, snap_tokens, snap_first, snaps,
+                   n_threads);
 }

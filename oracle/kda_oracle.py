@@ -58,6 +58,11 @@ def _bind(path: str):
     f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
                   p, p, ctypes.c_int64, p, ctypes.c_int]
+    f = lib.kda_oracle_recurrent_snapshots
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
+                  p, p, ctypes.c_int64, p, p, ctypes.c_int]
     return lib
 
 
@@ -155,6 +160,60 @@ def recurrent(q, k, v, g, beta, *, cu_seqlens=None, initial_state=None,
     if rc != 0:
         raise ValueError(f"kda_oracle_recurrent failed with code {rc}")
     return out, fin
+
+
+def recurrent_snapshots(q, k, v, g, beta, *, snapshot_tokens: int, cu_seqlens=None,
+                        initial_state=None, lb: float = -1.0, scale: float | None = None,
+                        want_out: bool = False, n_threads: int | None = None, lib=None):
+    """The token-by-token recurrence, also recording the state at regular points.
+
+    For each sequence n and every m >= 1 with m * snapshot_tokens <= len_n, the
+    state after the sequence's first m * snapshot_tokens tokens (seeded by its
+    initial state). A prefix cache keeps such states ("3 分钟看懂 Kimi K3",
+    第一条主线: KDA state and prefix-cache scheduling for long requests).
+
+    Returns (out or None, final_state [n, H, dk, dv], snaps [sum_n count_n, H, dk, dv],
+    first [n]): sequence n's snapshots are snaps[first[n] : first[n] + count_n] in order,
+    count_n = len_n // snapshot_tokens (a compact layout, all fp64).
+    """
+    qa, dt = _as_input(q)
+    ka, _ = _as_input(k)
+    va, _ = _as_input(v)
+    ga, _ = _as_input(g)
+    ba, _ = _as_input(beta)
+    T, H, dk = qa.shape
+    dv = va.shape[2]
+    if snapshot_tokens <= 0:
+        raise ValueError("snapshot_tokens must be positive")
+    cu = (np.array([0, T], dtype=np.int64) if cu_seqlens is None
+          else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)))
+    n = len(cu) - 1
+    counts = np.diff(cu) // snapshot_tokens
+    first = np.ascontiguousarray(np.concatenate([[0], np.cumsum(counts)[:-1]]).astype(np.int64))
+    snaps = np.zeros((max(int(counts.sum()), 1), H, dk, dv), dtype=np.float64)
+    s0 = None
+    if initial_state is not None:
+        s0 = np.ascontiguousarray(np.asarray(_to_numpy(initial_state), dtype=np.float64))
+        assert s0.shape == (n, H, dk, dv), s0.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.zeros((T, H, dv), dtype=np.float64) if want_out else None
+    fin = np.zeros((n, H, dk, dv), dtype=np.float64)
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    lib = lib or load()
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    rc = lib.kda_oracle_recurrent_snapshots(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka),
+                                            ptr(va), ptr(ga), ptr(ba), ptr(s0), float(lb),
+                                            float(scale), ptr(out), ptr(fin),
+                                            int(snapshot_tokens), ptr(first), ptr(snaps),
+                                            int(n_threads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_recurrent_snapshots failed with code {rc}")
+    return out, fin, snaps[:int(counts.sum())], first
 
 
 def _to_numpy(x):

@@ -271,10 +271,35 @@ def pin_sampled_rows(lib):
     assert np.array_equal(s_full[1], x.initial_state[1].double().numpy())  # empty sequence
 
 
+def pin_snapshots_are_prefix_states(lib):
+    """Snapshot m of a sequence is the state after its first m * P tokens: the final state
+    of a separate run over that prefix alone, from the same initial state. Recording the
+    snapshots changes neither the read-out nor the final states."""
+    x = make_inputs(None, H=2, dk=8, dv=4, dtype=torch.float32, seed=71,
+                    lengths=[25, 7, 0, 16, 31], state_std=0.5)
+    cu = x.cu_seqlens.tolist()
+    P = 8
+    out, fin, snaps, first = ko.recurrent_snapshots(
+        x.q, x.k, x.v, x.g, x.beta, snapshot_tokens=P, cu_seqlens=cu,
+        initial_state=x.initial_state, want_out=True, lib=lib)
+    o_ref, s_ref = ko.recurrent(x.q, x.k, x.v, x.g, x.beta, cu_seqlens=cu,
+                                initial_state=x.initial_state, lib=lib)
+    assert np.array_equal(out, o_ref) and np.array_equal(fin, s_ref)
+    counts = [(cu[s + 1] - cu[s]) // P for s in range(len(cu) - 1)]
+    assert counts == [3, 0, 0, 2, 3] and snaps.shape[0] == sum(counts)
+    for s, cnt in enumerate(counts):
+        for m in range(1, cnt + 1):
+            sl = slice(cu[s], cu[s] + m * P)
+            _, st = ko.recurrent(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl],
+                                 initial_state=x.initial_state[s:s + 1], lib=lib)
+            assert np.array_equal(snaps[first[s] + m - 1], st[0]), (s, m)
+    assert np.array_equal(snaps[first[3] + 1], fin[3])  # 16 tokens: the last one is final
+
+
 ALL_PINS = [pin_golden, pin_chunked_agreement, pin_beta_zero_pure_decay, pin_delta_rule_reach,
             pin_general_beta_reach, pin_associative_memory, pin_one_token_expansion,
             pin_linearity, pin_contraction_bound, pin_resume_and_varlen, pin_decay_clamp,
-            pin_sampled_rows]
+            pin_sampled_rows, pin_snapshots_are_prefix_states]
 
 
 def failing_pins(lib_path: str) -> list[str]:

@@ -51,6 +51,9 @@ MUTANTS = {
         "for (int j = 0; j < dv; ++j) o[j] += qt[i] * S[i * dv + j];",
         "for (int j = 0; j < dv && i < dv && j < dk; ++j) o[i] += qt[j] * S[i * dv + j];"),
     "decay_on_columns": ("S[i * dv + j] *= decay[i];", "S[i * dv + j] *= decay[j % dk];"),
+    "snapshot_one_token_late": ("(t - t0 + 1) % J->snap_tokens == 0",
+                                "(t - t0) % J->snap_tokens == 0 && t > t0"),
+    "snapshot_wrong_sequence": ("J->snap_first[seq] +", "J->snap_first[0] +"),
 }
 
 
