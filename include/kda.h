@@ -103,6 +103,45 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                          kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd that also keeps the state at regular chunk boundaries of each
+ * sequence, for a prefix cache: a later request that shares the first m
+ * intervals of a sequence resumes from snapshot m by passing it as
+ * initial_state, instead of recomputing the prefix ("3 分钟看懂 Kimi K3",
+ * 第一条主线: KDA state and prefix-cache scheduling for long requests; the state
+ * after any prefix is the recurrence's own S_t, "Kimi K3 深度拆解", section 4.2).
+ *
+ *  snapshot_chunks  k >= 1: one snapshot every k chunks (k * chunk tokens).
+ *  snapshots        fp32 [n_snapshots, H, dk, dv], device, written. For sequence n,
+ *                   whose first token is c_n in the packed layout (c_n = n * T
+ *                   without cu_seqlens), and for m = 1 .. floor(len_n / (k * chunk)),
+ *                   the state after the sequence's first m * k * chunk tokens (seeded
+ *                   by its initial state) is written at index
+ *                   floor(c_n / (k * chunk)) + m - 1. The sequences' index ranges never
+ *                   overlap; an index no sequence reaches is left as it was. Must not
+ *                   overlap any other argument.
+ *  n_snapshots      capacity of `snapshots`; must be >= kda_snapshot_count(shape, k).
+ *                   `snapshots` may be NULL only when that count is 0.
+ * Every other argument, every result and the workspace size are those of
+ * kda_chunk_fwd; out and final_state hold exactly the values kda_chunk_fwd writes.
+ * Returns KDA_ERR_INVALID_ARG for snapshot_chunks < 1, a short or misaligned
+ * `snapshots`, or any argument kda_chunk_fwd rejects.
+ */
+kda_status kda_chunk_fwd_snapshots(const void *q, const void *k, const void *v, const void *g,
+                                   const void *beta, const float *initial_state,
+                                   const int32_t *cu_seqlens, void *out, float *final_state,
+                                   int32_t snapshot_chunks, float *snapshots,
+                                   int64_t n_snapshots, const kda_shape *shape,
+                                   void *workspace, size_t workspace_bytes,
+                                   kda_stream_t stream);
+
+/*
+ * Snapshot slots kda_chunk_fwd_snapshots needs: floor(T_total / (snapshot_chunks *
+ * chunk)), T_total = B * T without cu_seqlens, T with them. Returns -1 for an
+ * invalid shape or snapshot_chunks < 1.
+ */
+int64_t kda_snapshot_count(const kda_shape *shape, int32_t snapshot_chunks);
+
+/*
  * kda_chunk_fwd without a workspace argument, for callers that cannot call
  * cudaMalloc: code running while a CUDA graph is being captured (allocation is
  * not capturable), plugin hosts that hand a library no scratch buffer, and

@@ -61,11 +61,18 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* shape) {
   return align_up(kWorkspaceHeader, 256);
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
-                         const void* beta, const float* initial_state,
-                         const int32_t* cu_seqlens, void* out, float* final_state,
-                         const kda_shape* shape, void* workspace, size_t workspace_bytes,
-                         kda_stream_t stream) {
+}  // extern "C"
+
+namespace kda {
+namespace {
+
+// kda_chunk_fwd, with chunk-boundary snapshots when snaps != nullptr (snap_every >= 1,
+// checked by the caller).
+kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                     const void* beta, const float* initial_state, const int32_t* cu_seqlens,
+                     void* out, float* final_state, int snap_every, float* snaps,
+                     int64_t n_snaps, const kda_shape* shape, void* workspace,
+                     size_t workspace_bytes, kda_stream_t stream) {
   kda_status st = check_shape(shape, true);
   if (st != KDA_OK) return st;
   const kda_shape& s = *shape;
@@ -85,6 +92,12 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     return KDA_ERR_INVALID_ARG;
   if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
     return KDA_ERR_INVALID_ARG;
+  if (snap_every > 0) {
+    const int64_t need_snaps = T_total / (static_cast<int64_t>(snap_every) * kChunk);
+    if (n_snaps < need_snaps || (need_snaps > 0 && snaps == nullptr) || !aligned16(snaps))
+      return KDA_ERR_INVALID_ARG;
+    if (need_snaps == 0) snaps = nullptr;
+  }
   const size_t need = kda_chunk_fwd_workspace_size(shape);
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -99,6 +112,8 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   a.cu = cu_seqlens;
   a.out = out;
   a.sT = final_state;
+  a.snap = snap_every > 0 ? snaps : nullptr;
+  a.snap_every = snap_every > 0 ? snap_every : 1;
   a.status = static_cast<int32_t*>(workspace);
   a.ws = static_cast<unsigned char*>(workspace);
   a.ws_bytes = workspace_bytes;
@@ -113,6 +128,41 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   cudaError_t e = tc_path_applies(s, T_total) ? launch_prefill_tc(a, cs)
                                               : launch_prefill_simt(a, s.dtype, cs);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, void* out, float* final_state,
+                         const kda_shape* shape, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream) {
+  return chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state, 0, nullptr,
+                   0, shape, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_snapshots(const void* q, const void* k, const void* v, const void* g,
+                                   const void* beta, const float* initial_state,
+                                   const int32_t* cu_seqlens, void* out, float* final_state,
+                                   int32_t snapshot_chunks, float* snapshots,
+                                   int64_t n_snapshots, const kda_shape* shape,
+                                   void* workspace, size_t workspace_bytes,
+                                   kda_stream_t stream) {
+  if (snapshot_chunks < 1) return KDA_ERR_INVALID_ARG;
+  return chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, out, final_state,
+                   snapshot_chunks, snapshots, n_snapshots, shape, workspace, workspace_bytes,
+                   stream);
+}
+
+int64_t kda_snapshot_count(const kda_shape* shape, int32_t snapshot_chunks) {
+  if (snapshot_chunks < 1 || kda_chunk_fwd_workspace_size(shape) == 0) return -1;
+  int64_t T_total, max_len;
+  int n_seqs;
+  resolve(*shape, T_total, n_seqs, max_len);
+  return T_total / (static_cast<int64_t>(snapshot_chunks) * kChunk);
 }
 
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* g,

@@ -29,6 +29,8 @@ struct PrefillArgs {
   const int32_t* cu;        // [n+1] or null (then sequences are [b*T, (b+1)*T))
   void* out;                // [T_total, H, dv]
   float* sT;                // [n, H, dk, dv] or null
+  float* snap;              // [floor(T_total / (snap_every C)), H, dk, dv] or null
+  int snap_every;           // chunks between snapshots (>= 1 when snap is set)
   int32_t* status;          // device status word (workspace header)
   unsigned char* ws;        // workspace base
   size_t ws_bytes;

@@ -16,6 +16,8 @@
 //   U  = T (V - K~ S)
 //   O  = scale (Q~ S + P U)
 //   S  = Diag(exp Gamma_L) S + (K^ * exp Gamma_L)^T U
+// When asked, the state after every snap_every-th full chunk of a sequence is also
+// written out (prefix-cache snapshots).
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -221,6 +223,14 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       __syncthreads();
 #pragma unroll
       for (int c = 0; c < PER; ++c) sm.S[i][cs + c] = acc[c];
+      // the state after a full chunk that closes a snapshot interval of the sequence
+      const int64_t done = (c0 - t0) / C + 1;  // chunks of the sequence walked
+      if (a.snap != nullptr && L == C && done % a.snap_every == 0) {
+        const int64_t idx = t0 / (static_cast<int64_t>(C) * a.snap_every) + done / a.snap_every - 1;
+        float* d = a.snap + (idx * H + h) * DK * DV + j0 + static_cast<int64_t>(i) * DV + cs;
+#pragma unroll
+        for (int c = 0; c < PER; ++c) d[c] = acc[c];
+      }
     }
     __syncthreads();
   }

@@ -126,6 +126,8 @@ struct WalkArgs {
   float* mbuf;    // [pairs, max_segs, D, D]  summary of segment j: M (row-major [i][j])
   float* lbuf;    // [pairs, max_segs, D, D]  summary of segment j: L
   float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 1
+  float* snap;    // [floor(T_total / (snap_every C)), H, D, D] or null: prefix-cache snapshots
+  int snap_every; // chunks between snapshots
   int H;
   int first_tokens, seg_tokens;  // segment 0, then every later segment (the last may be short)
   int max_segs;
@@ -922,6 +924,20 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       bulk_commit();
     };
 
+    // The fp32 state after chunk n (this thread's 64 state rows of column `row`, in v0,
+    // v1) when that chunk is full and closes a snapshot interval of the sequence
+    auto store_snapshot = [&](int n, const uint32_t (&v0)[32], const uint32_t (&v1)[32]) {
+      const int64_t done = off / C + n + 1;  // chunks of the sequence walked so far
+      if (done % a.snap_every != 0 || done * C > len) return;
+      const int64_t idx = t0 / (static_cast<int64_t>(C) * a.snap_every) + done / a.snap_every - 1;
+      float* dst = a.snap + (idx * a.H + h) * D * D + static_cast<int64_t>(64 * hc) * D + row;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        dst[t * D] = __uint_as_float(v0[t]);
+        dst[(32 + t) * D] = __uint_as_float(v1[t]);
+      }
+    };
+
     // Per chunk n (stage st = n % 2 has landed): MMA-1(n) runs -> U^T (+ U0^T) packed ->
     // MMA-2(n) runs while the previous chunk's outputs are written -> S^T packed for
     // MMA-1(n + 1), then the fp32 state rescaled by the next chunk's decay.
@@ -1000,6 +1016,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       tc_fence_before();
       group_sync(half_bar, 128);
       if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + hc);
+      if (PC && a.snap != nullptr) store_snapshot(n, v0, v1);  // while MMA-1(n + 1) runs
       if (n + 1 < n_chunks) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
           failed = true;
@@ -1402,6 +1419,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   wa.out = static_cast<__nv_bfloat16*>(pa.out);
   wa.s0 = pa.s0;
   wa.sT = pa.sT;
+  wa.snap = pa.snap;
+  wa.snap_every = pa.snap_every;
   const size_t state = static_cast<size_t>(D) * D;
   float* base = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
   wa.mbuf = base;

@@ -45,6 +45,11 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
     L.kda_chunk_fwd.restype = st
     L.kda_chunk_fwd.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p, sz, p]
+    L.kda_chunk_fwd_snapshots.restype = st
+    L.kda_chunk_fwd_snapshots.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.c_int32, p,
+                                          ctypes.c_int64, ctypes.POINTER(Shape), p, sz, p]
+    L.kda_snapshot_count.restype = ctypes.c_int64
+    L.kda_snapshot_count.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
     L.kda_chunk_fwd_noalloc.restype = st
     L.kda_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p]
     L.kda_decode_step.restype = st
@@ -62,7 +67,7 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
-            "kda_decode_step",
+            "kda_chunk_fwd_snapshots", "kda_snapshot_count", "kda_decode_step",
             "kda_workspace_status", "kda_status_string", "kda_version")
 
 
@@ -105,16 +110,7 @@ def alloc_workspace(shape: Shape, device) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
-              beta: torch.Tensor, *, initial_state: torch.Tensor | None = None,
-              cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
-              scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
-              final_state: torch.Tensor | None = None, output_final_state: bool = True,
-              workspace: torch.Tensor | None = None, stream=None):
-    """Chunked prefill. q, k, g: [T, H, dk] (or [B, T, H, dk]); v: [..., dv]; beta: [..., H].
-
-    Returns (out, final_state). final_state is fp32 [n, H, dk, dv] (None if not requested).
-    """
+def _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb):
     batched = q.dim() == 4
     if batched:
         B, T, H, dk = q.shape
@@ -129,6 +125,21 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
         n = B
     shape = make_shape(T, H, dk, dv, q.dtype, B=B, n_seqs=n if cu_seqlens is not None else 0,
                        max_seqlen=max_seqlen, scale=scale, lb=lb)
+    return shape, n
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+              beta: torch.Tensor, *, initial_state: torch.Tensor | None = None,
+              cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+              scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
+              final_state: torch.Tensor | None = None, output_final_state: bool = True,
+              workspace: torch.Tensor | None = None, stream=None):
+    """Chunked prefill. q, k, g: [T, H, dk] (or [B, T, H, dk]); v: [..., dv]; beta: [..., H].
+
+    Returns (out, final_state). final_state is fp32 [n, H, dk, dv] (None if not requested).
+    """
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    H, dk, dv = shape.H, shape.dk, shape.dv
     if out is None:
         out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
@@ -141,6 +152,51 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
     return out, final_state
+
+
+def snapshot_count(shape: Shape, snapshot_chunks: int) -> int:
+    """Snapshot slots kda_chunk_fwd_snapshots writes into for this shape (-1: invalid)."""
+    return int(lib.kda_snapshot_count(ctypes.byref(shape), int(snapshot_chunks)))
+
+
+def chunk_fwd_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                        beta: torch.Tensor, *, snapshot_chunks: int,
+                        snapshots: torch.Tensor | None = None,
+                        initial_state: torch.Tensor | None = None,
+                        cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+                        scale: float | None = None, lb: float = -1.0,
+                        out: torch.Tensor | None = None, final_state: torch.Tensor | None = None,
+                        output_final_state: bool = True, workspace: torch.Tensor | None = None,
+                        stream=None):
+    """Prefill that also keeps the state every `snapshot_chunks` chunks (prefix cache).
+
+    Returns (out, final_state, snapshots); snapshots is fp32 [snapshot_count, H, dk, dv].
+    Sequence n (first packed token c_n) stores the state after its first m * snapshot_chunks
+    * 64 tokens at index c_n // (snapshot_chunks * 64) + m - 1, m = 1, 2, ...; indices no
+    sequence reaches keep their previous contents (zeros when this call allocates).
+    """
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    H, dk, dv = shape.H, shape.dk, shape.dv
+    count = snapshot_count(shape, snapshot_chunks)
+    if count < 0:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_snapshot_count")
+    if snapshots is None:
+        snapshots = torch.zeros(count, H, dk, dv, dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(n, H, dk, dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(shape, q.device)
+    rc = lib.kda_chunk_fwd_snapshots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                     _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                     _ptr(final_state), int(snapshot_chunks),
+                                     _ptr(snapshots) if snapshots.numel() else None,
+                                     snapshots.shape[0], ctypes.byref(shape), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_snapshots")
+    return out, final_state, snapshots
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20

@@ -92,6 +92,32 @@ def test_chunk_fwd_argument_errors(kda):
                                  None, 0, None) == kda.KDA_ERR_INVALID_ARG
 
 
+def test_snapshot_count_and_argument_errors(kda):
+    """Snapshot capacity is floor(T_total / (k * 64)); bad snapshot arguments return before
+    any CUDA call (the addresses are never dereferenced)."""
+    P = ctypes.c_void_p
+    sh = kda.make_shape(1000, 2, 64, 64, torch.float32, B=3)
+    assert kda.snapshot_count(sh, 1) == 3000 // 64
+    assert kda.snapshot_count(sh, 4) == 3000 // 256
+    assert kda.snapshot_count(sh, 0) == -1
+    assert kda.snapshot_count(kda.make_shape(1000, 2, 64, 48, torch.float32), 1) == -1
+    packed = kda.make_shape(700, 2, 64, 64, torch.float32, n_seqs=3)
+    assert kda.snapshot_count(packed, 2) == 700 // 128
+
+    def call(k_chunks=1, snaps=8192, n_snaps=46, shape=sh, q=4096):
+        return kda.lib.kda_chunk_fwd_snapshots(
+            P(q), P(4096), P(4096), P(4096), P(4096), None, None, P(4096), None, k_chunks,
+            P(snaps), n_snaps, ctypes.byref(shape), P(256 * 1000), 1 << 20, None)
+
+    assert call(k_chunks=0) == kda.KDA_ERR_INVALID_ARG
+    assert call(n_snaps=45) == kda.KDA_ERR_INVALID_ARG          # one slot short
+    assert call(snaps=None) == kda.KDA_ERR_INVALID_ARG          # snapshots needed
+    assert call(snaps=8200) == kda.KDA_ERR_INVALID_ARG          # misaligned
+    assert call(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(shape=kda.make_shape(1000, 2, 64, 48, torch.float32, B=3)) == \
+        kda.KDA_ERR_UNSUPPORTED
+
+
 def test_decode_argument_errors(kda):
     P = ctypes.c_void_p
     sh = kda.make_shape(1, 4, 128, 128, torch.bfloat16, B=8)
