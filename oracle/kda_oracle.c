@@ -18,6 +18,10 @@
  * i.e. S_t = (I - beta_t k_t k_t^T) Diag(exp g'_t) S_{t-1} + beta_t k_t v_t^T.
  * S is d_k x d_v (rows indexed by key channels).
  *
+ * Optionally (kda_oracle_recurrent_ex) the inputs are raw: q_t, k_t are first divided by
+ * their L2 norms, and/or g_t holds gate pre-activations a with g = lb * sigmoid(a); and
+ * the state after every P tokens of a sequence can be recorded (prefix-cache snapshots).
+ *
  * Sources (web pages about the Kimi K3 report):
  *  - "Kimi K3 深度拆解" (chenxutan.com), section 4.2 "线性注意力与 Delta Rule":
  *    the delta-rule update S_t = S_{t-1}(I - b k k^T) + b k v^T, the fixed-size
@@ -45,6 +49,10 @@
 
 #define KDA_ORACLE_F32 0
 #define KDA_ORACLE_BF16 1
+
+/* Optional input prologue (bit flags). */
+#define KDA_ORACLE_QK_L2NORM 1   /* q_t, k_t <- x / max(||x||_2, 1e-12) per (token, head) */
+#define KDA_ORACLE_GATE_SIGMOID 2 /* g holds pre-activations a: log decay = lb * sigmoid(a) */
 
 /* Exact widening of one input element to double. */
 static double load_elem(const void *base, int dtype, int64_t idx)
@@ -74,6 +82,7 @@ typedef struct {
     int64_t snap_tokens;       /* snapshot interval in tokens (0 = none) */
     const int64_t *snap_first; /* [n_seqs] index of each sequence's first snapshot */
     double *snaps;             /* [n_snaps, H, dk, dv] */
+    int prologue;              /* KDA_ORACLE_* prologue flags */
     int64_t next_item; /* shared work counter over (seq, head) */
     pthread_mutex_t lock;
 } job_t;
@@ -112,8 +121,26 @@ static void run_one(const job_t *J, int seq, int h, double *S, double *kt,
             kt[i] = load_elem(J->k, J->dtype, tok_k + i);
             qt[i] = load_elem(J->q, J->dtype, tok_k + i);
             double gi = load_elem(J->g, J->dtype, tok_k + i);
+            if (J->prologue & KDA_ORACLE_GATE_SIGMOID)
+                gi = J->lb / (1.0 + exp(-gi));       /* lb * sigmoid(a), inside (lb, 0) */
             if (gi < J->lb) gi = J->lb;              /* lower bound on the log decay */
             decay[i] = exp(gi);
+        }
+        if (J->prologue & KDA_ORACLE_QK_L2NORM) {
+            /* unit-length q and k (the delta rule assumes them normalised) */
+            double nk = 0.0, nq = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                nk += kt[i] * kt[i];
+                nq += qt[i] * qt[i];
+            }
+            nk = sqrt(nk);
+            nq = sqrt(nq);
+            if (nk < 1e-12) nk = 1e-12;
+            if (nq < 1e-12) nq = 1e-12;
+            for (int i = 0; i < dk; ++i) {
+                kt[i] /= nk;
+                qt[i] /= nq;
+            }
         }
         for (int j = 0; j < dv; ++j) vt[j] = load_elem(J->v, J->dtype, tok_v + j);
         const double b = load_elem(J->beta, J->dtype, t * H + h);
@@ -200,7 +227,7 @@ static int run_all(int64_t T, int H, int dk, int dv, int n_seqs,
                    const double *initial_state, double lb, double scale,
                    double *out, const int64_t *out_rows, int64_t n_out_rows,
                    double *final_state, int64_t snap_tokens, const int64_t *snap_first,
-                   double *snaps, int n_threads)
+                   double *snaps, int prologue, int n_threads)
 {
     if (T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs <= 0 || !cu_seqlens) return -1;
     if (dtype != KDA_ORACLE_F32 && dtype != KDA_ORACLE_BF16) return -1;
@@ -208,6 +235,9 @@ static int run_all(int64_t T, int H, int dk, int dv, int n_seqs,
     for (int s = 0; s < n_seqs; ++s)
         if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
     if (T > 0 && (!q || !k || !v || !g || !beta)) return -1;
+    if (prologue & ~(KDA_ORACLE_QK_L2NORM | KDA_ORACLE_GATE_SIGMOID)) return -1;
+    if (snap_tokens < 0 || (snap_tokens > 0 && (!snap_first || !snaps))) return -1;
+    if (snap_tokens == 0) snaps = NULL;
 
     job_t J;
     memset(&J, 0, sizeof J);
@@ -218,6 +248,7 @@ static int run_all(int64_t T, int H, int dk, int dv, int n_seqs,
     J.out = out; J.out_rows = out_rows; J.n_out_rows = n_out_rows;
     J.final_state = final_state;
     J.snap_tokens = snap_tokens; J.snap_first = snap_first; J.snaps = snaps;
+    J.prologue = prologue;
     pthread_mutex_init(&J.lock, NULL);
 
     const int64_t n_items = (int64_t)n_seqs * H;
@@ -255,28 +286,38 @@ int kda_oracle_recurrent(int64_t T, int H, int dk, int dv, int n_seqs,
                          double *final_state, int n_threads)
 {
     return run_all(T, H, dk, dv, n_seqs, cu_seqlens, dtype, q, k, v, g, beta, initial_state,
-                   lb, scale, out, out_rows, n_out_rows, final_state, 0, NULL, NULL, n_threads);
+                   lb, scale, out, out_rows, n_out_rows, final_state, 0, NULL, NULL, 0,
+                   n_threads);
 }
 
 /*
- * kda_oracle_recurrent that also records the state at regular points of each
- * sequence: for every m >= 1 with m * snap_tokens <= len(seq), the state after
- * the sequence's first m * snap_tokens tokens (seeded by its initial state) is
- * copied to snaps[snap_first[seq] + m - 1] ([.., H, dk, dv] fp64). The caller
- * sizes snaps and chooses snap_first so that the sequences' ranges do not
- * overlap. A prefix cache keeps exactly these states ("3 分钟看懂 Kimi K3",
- * 第一条主线: KDA state and prefix-cache scheduling for long requests).
+ * The general form: kda_oracle_recurrent with optional snapshots and an optional input
+ * prologue.
+ *  Snapshots (snap_tokens > 0; 0 = none): for every m >= 1 with m * snap_tokens <=
+ *  len(seq), the state after the sequence's first m * snap_tokens tokens (seeded by its
+ *  initial state) is copied to snaps[snap_first[seq] + m - 1] ([.., H, dk, dv] fp64).
+ *  The caller sizes snaps and chooses snap_first so that the sequences' ranges do not
+ *  overlap. A prefix cache keeps exactly these states ("3 分钟看懂 Kimi K3", 第一条主线:
+ *  KDA state and prefix-cache scheduling for long requests).
+ *  Prologue flags:
+ *  KDA_ORACLE_QK_L2NORM    q_t and k_t are divided by max(||.||_2, 1e-12) per (token,
+ *                          head) before use ("Kimi K3 深度拆解", section 4.2: the delta
+ *                          rule takes L2-normalised q and k);
+ *  KDA_ORACLE_GATE_SIGMOID g holds gate pre-activations a and the log decay is
+ *                          lb * sigmoid(a), which lies inside (lb, 0) ("3 分钟看懂 Kimi K3",
+ *                          第一条主线 / Figure 3: the log decay is bounded below).
  */
-int kda_oracle_recurrent_snapshots(int64_t T, int H, int dk, int dv, int n_seqs,
-                                   const int64_t *cu_seqlens, int dtype,
-                                   const void *q, const void *k, const void *v,
-                                   const void *g, const void *beta,
-                                   const double *initial_state, double lb, double scale,
-                                   double *out, double *final_state, int64_t snap_tokens,
-                                   const int64_t *snap_first, double *snaps, int n_threads)
+int kda_oracle_recurrent_ex(int64_t T, int H, int dk, int dv, int n_seqs,
+                            const int64_t *cu_seqlens, int dtype,
+                            const void *q, const void *k, const void *v,
+                            const void *g, const void *beta,
+                            const double *initial_state, double lb, double scale,
+                            double *out, const int64_t *out_rows, int64_t n_out_rows,
+                            double *final_state, int64_t snap_tokens,
+                            const int64_t *snap_first, double *snaps, int prologue,
+                            int n_threads)
 {
-    if (snap_tokens <= 0 || !snap_first || !snaps) return -1;
     return run_all(T, H, dk, dv, n_seqs, cu_seqlens, dtype, q, k, v, g, beta, initial_state,
-                   lb, scale, out, NULL, 0, final_state, snap_tokens, snap_first, snaps,
-                   n_threads);
+                   lb, scale, out, out_rows, n_out_rows, final_state, snap_tokens, snap_first,
+                   snaps, prologue, n_threads);
 }

@@ -13,6 +13,11 @@ Two independent fp64 implementations live here:
   section "長度" (channel-wise gating), "3 分钟看懂 Kimi K3" (landx.limxdynamics.com)
   "第一条主线" / Figure 3 (log decay bounded below).
 
+  Options of the same C loop: ``recurrent_snapshots`` also records the state after
+  every P tokens of each sequence (prefix-cache snapshots), and ``prologue`` takes raw
+  inputs: q, k rows L2-normalised per token (QK_L2NORM) and/or gate pre-activations a
+  with log decay lb * sigmoid(a) (GATE_SIGMOID).
+
 * ``chunked`` -- the closed form of the same recurrence over chunks of C
   tokens, derived independently (numpy, plain matrix products, one chunk at a
   time). Used only to pin ``recurrent``; it is the chunk-parallel form the
@@ -41,6 +46,8 @@ _lib_lock = threading.Lock()
 
 F32 = 0
 BF16 = 1
+QK_L2NORM = 1       # prologue: q, k rows divided by max(||.||_2, 1e-12)
+GATE_SIGMOID = 2    # prologue: g holds pre-activations a, log decay = lb * sigmoid(a)
 
 
 def build(src: str = _SRC, out: str = _LIB_PATH) -> str:
@@ -58,11 +65,11 @@ def _bind(path: str):
     f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
                   p, p, ctypes.c_int64, p, ctypes.c_int]
-    f = lib.kda_oracle_recurrent_snapshots
+    f = lib.kda_oracle_recurrent_ex
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
-                  p, p, ctypes.c_int64, p, p, ctypes.c_int]
+                  p, p, ctypes.c_int64, p, ctypes.c_int64, p, p, ctypes.c_int, ctypes.c_int]
     return lib
 
 
@@ -107,8 +114,11 @@ def _as_input(x):
 
 def recurrent(q, k, v, g, beta, *, cu_seqlens=None, initial_state=None,
               lb: float = -1.0, scale: float | None = None, out_rows=None,
-              want_out: bool = True, n_threads: int | None = None, lib=None):
+              want_out: bool = True, prologue: int = 0, n_threads: int | None = None,
+              lib=None):
     """Token-by-token fp64 recurrence.
+
+    prologue: 0, or QK_L2NORM | GATE_SIGMOID (the raw-input prologue, see kda_oracle.c).
 
     q, k, g: [T, H, dk]; v: [T, H, dv]; beta: [T, H] (all the same dtype, f32 or bf16).
     cu_seqlens: None (one sequence) or int sequence [n+1].
@@ -153,10 +163,17 @@ def recurrent(q, k, v, g, beta, *, cu_seqlens=None, initial_state=None,
     def ptr(a):
         return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
-    rc = lib.kda_oracle_recurrent(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka), ptr(va),
-                                  ptr(ga), ptr(ba), ptr(s0), float(lb), float(scale),
-                                  ptr(out), ptr(rows), 0 if rows is None else len(rows),
-                                  ptr(fin), int(n_threads))
+    if prologue:
+        rc = lib.kda_oracle_recurrent_ex(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka),
+                                         ptr(va), ptr(ga), ptr(ba), ptr(s0), float(lb),
+                                         float(scale), ptr(out), ptr(rows),
+                                         0 if rows is None else len(rows), ptr(fin), 0, None,
+                                         None, int(prologue), int(n_threads))
+    else:
+        rc = lib.kda_oracle_recurrent(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka), ptr(va),
+                                      ptr(ga), ptr(ba), ptr(s0), float(lb), float(scale),
+                                      ptr(out), ptr(rows), 0 if rows is None else len(rows),
+                                      ptr(fin), int(n_threads))
     if rc != 0:
         raise ValueError(f"kda_oracle_recurrent failed with code {rc}")
     return out, fin
@@ -164,7 +181,8 @@ def recurrent(q, k, v, g, beta, *, cu_seqlens=None, initial_state=None,
 
 def recurrent_snapshots(q, k, v, g, beta, *, snapshot_tokens: int, cu_seqlens=None,
                         initial_state=None, lb: float = -1.0, scale: float | None = None,
-                        want_out: bool = False, n_threads: int | None = None, lib=None):
+                        want_out: bool = False, prologue: int = 0,
+                        n_threads: int | None = None, lib=None):
     """The token-by-token recurrence, also recording the state at regular points.
 
     For each sequence n and every m >= 1 with m * snapshot_tokens <= len_n, the
@@ -206,11 +224,11 @@ def recurrent_snapshots(q, k, v, g, beta, *, snapshot_tokens: int, cu_seqlens=No
     def ptr(a):
         return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
-    rc = lib.kda_oracle_recurrent_snapshots(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka),
-                                            ptr(va), ptr(ga), ptr(ba), ptr(s0), float(lb),
-                                            float(scale), ptr(out), ptr(fin),
-                                            int(snapshot_tokens), ptr(first), ptr(snaps),
-                                            int(n_threads))
+    rc = lib.kda_oracle_recurrent_ex(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka),
+                                     ptr(va), ptr(ga), ptr(ba), ptr(s0), float(lb),
+                                     float(scale), ptr(out), None, 0, ptr(fin),
+                                     int(snapshot_tokens), ptr(first), ptr(snaps),
+                                     int(prologue), int(n_threads))
     if rc != 0:
         raise ValueError(f"kda_oracle_recurrent_snapshots failed with code {rc}")
     return out, fin, snaps[:int(counts.sum())], first

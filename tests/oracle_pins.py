@@ -296,10 +296,72 @@ def pin_snapshots_are_prefix_states(lib):
     assert np.array_equal(snaps[first[3] + 1], fin[3])  # 16 tokens: the last one is final
 
 
+def _unit_rows(T, H, d, rng):
+    """Rows with entries +-1/2 (d = 4): unit L2 norm exactly in binary; L1 norm 2."""
+    return rng.choice([-0.5, 0.5], size=(T, H, d)).astype(np.float32)
+
+
+def pin_prologue_l2norm(lib):
+    """The q/k normalisation prologue: unit rows pass through unchanged (exact), and the
+    result does not change when any token's q or k row is scaled by a positive factor
+    (powers of two, so the scaled inputs and their norms are exact)."""
+    rng = np.random.default_rng(81)
+    T, H, d = 24, 2, 4
+    x = make_inputs(T, H=H, dk=d, dv=3, dtype=torch.float32, seed=81, state_std=0.5)
+    q, k = _f32(_unit_rows(T, H, d, rng)), _f32(_unit_rows(T, H, d, rng))
+    o1, s1 = ko.recurrent(q, k, x.v, x.g, x.beta, initial_state=x.initial_state, lib=lib)
+    o2, s2 = ko.recurrent(q, k, x.v, x.g, x.beta, initial_state=x.initial_state,
+                          prologue=ko.QK_L2NORM, lib=lib)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+    # raw rows of any length: scale invariance, and the unit-row result is reproduced
+    cq = torch.tensor(rng.choice([0.25, 2.0, 8.0, 0.5], size=(T, H, 1)), dtype=torch.float32)
+    ck = torch.tensor(rng.choice([4.0, 0.125, 2.0, 16.0], size=(T, H, 1)), dtype=torch.float32)
+    o3, s3 = ko.recurrent(q * cq, k * ck, x.v, x.g, x.beta, initial_state=x.initial_state,
+                          prologue=ko.QK_L2NORM, lib=lib)
+    assert np.array_equal(o3, o1) and np.array_equal(s3, s1)
+    # general rows: normalising twice is normalising once
+    y = make_inputs(T, H=H, dk=8, dv=3, dtype=torch.float32, seed=82, state_std=0.5)
+    qr, kr = y.q * 3.0, y.k * 0.5
+    o4, s4 = ko.recurrent(qr * cq, kr * ck, y.v, y.g, y.beta, initial_state=y.initial_state,
+                          prologue=ko.QK_L2NORM, lib=lib)
+    o5, s5 = ko.recurrent(qr, kr, y.v, y.g, y.beta, initial_state=y.initial_state,
+                          prologue=ko.QK_L2NORM, lib=lib)
+    assert _rel(o4, o5) < 1e-13 and _rel(s4, s5) < 1e-13
+    o6, _ = ko.recurrent(qr, kr, y.v, y.g, y.beta, initial_state=y.initial_state, lib=lib)
+    assert _rel(o6, o5) > 1e-2  # the prologue is active on these inputs
+
+
+def pin_prologue_gate(lib):
+    """The gate prologue log decay = lb * sigmoid(a): a = 0 gives exactly lb / 2; a large
+    positive pre-activation gives the bound lb, a large negative one no decay."""
+    lb = -0.75
+    x = make_inputs(20, H=2, dk=8, dv=4, dtype=torch.float32, seed=83, state_std=0.5)
+    run = dict(initial_state=x.initial_state, lb=lb, lib=lib)
+    zero = torch.zeros_like(x.g)
+    o1, s1 = ko.recurrent(x.q, x.k, x.v, zero, x.beta, prologue=ko.GATE_SIGMOID, **run)
+    o2, s2 = ko.recurrent(x.q, x.k, x.v, torch.full_like(x.g, lb / 2), x.beta, **run)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+    o3, s3 = ko.recurrent(x.q, x.k, x.v, torch.full_like(x.g, 40.0), x.beta,
+                          prologue=ko.GATE_SIGMOID, **run)
+    o4, s4 = ko.recurrent(x.q, x.k, x.v, torch.full_like(x.g, lb), x.beta, **run)
+    assert _rel(o3, o4) < 1e-12 and _rel(s3, s4) < 1e-12
+    o5, s5 = ko.recurrent(x.q, x.k, x.v, torch.full_like(x.g, -40.0), x.beta,
+                          prologue=ko.GATE_SIGMOID, **run)
+    o6, s6 = ko.recurrent(x.q, x.k, x.v, zero, x.beta, **run)
+    assert _rel(o5, o6) < 1e-12 and _rel(s5, s6) < 1e-12
+    # both prologues together: each acts on its own inputs
+    both = ko.QK_L2NORM | ko.GATE_SIGMOID
+    o7, s7 = ko.recurrent(x.q * 4.0, x.k * 0.5, x.v, zero, x.beta, prologue=both, **run)
+    o8, s8 = ko.recurrent(x.q, x.k, x.v, zero, x.beta, prologue=both, **run)
+    assert np.array_equal(o7, o8) and np.array_equal(s7, s8)
+    assert _rel(o8, o1) < 1e-5 and _rel(s8, s1) < 1e-5  # q, k are unit rows up to fp32
+
+
 ALL_PINS = [pin_golden, pin_chunked_agreement, pin_beta_zero_pure_decay, pin_delta_rule_reach,
             pin_general_beta_reach, pin_associative_memory, pin_one_token_expansion,
             pin_linearity, pin_contraction_bound, pin_resume_and_varlen, pin_decay_clamp,
-            pin_sampled_rows, pin_snapshots_are_prefix_states]
+            pin_sampled_rows, pin_snapshots_are_prefix_states, pin_prologue_l2norm,
+            pin_prologue_gate]
 
 
 def failing_pins(lib_path: str) -> list[str]:

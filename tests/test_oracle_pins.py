@@ -54,6 +54,10 @@ MUTANTS = {
     "snapshot_one_token_late": ("(t - t0 + 1) % J->snap_tokens == 0",
                                 "(t - t0) % J->snap_tokens == 0 && t > t0"),
     "snapshot_wrong_sequence": ("J->snap_first[seq] +", "J->snap_first[0] +"),
+    "l2norm_by_squared_norm": ("nk = sqrt(nk);", ";"),
+    "l2norm_keys_only": ("qt[i] /= nq;", ";"),
+    "gate_sign": ("gi = J->lb / (1.0 + exp(-gi));", "gi = J->lb / (1.0 + exp(gi));"),
+    "gate_without_bound": ("gi = J->lb / (1.0 + exp(-gi));", "gi = -1.0 / (1.0 + exp(-gi));"),
 }
 
 
