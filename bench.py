@@ -342,6 +342,34 @@ def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: 
                       f"(all {w.H} heads), fp64 token-by-token recurrence, {threads} threads"}
 
 
+def kernels_only(args):
+    """Profiler driver: `warmup + steps` calls of one path on its benchmark workload on
+    cuda:0 (prefill: kda_chunk_fwd on the 8K x 32-head inputs with one workspace; decode:
+    chained decode steps on the 256 x 32-head state), no timing and no CPU leg. ncu
+    captures select launches with -s/-c on this run."""
+    from kimi_delta_attention_19_b200 import kda
+    from kimi_delta_attention_19_b200.inputs import (WORKLOADS, decode_state, decode_tokens,
+                                                      workload_inputs)
+    dev = "cuda:0"
+    n = args.warmup + args.steps
+    if args.kernels_only == "prefill":
+        w = WORKLOADS[PREFILL]
+        x = workload_inputs(w, device=dev)
+        shape = kda.make_shape(w.T, w.H, w.dk, w.dv, w.dtype)
+        ws = kda.alloc_workspace(shape, dev)
+        for _ in range(n):
+            kda.chunk_fwd(x.q, x.k, x.v, x.g, x.beta, initial_state=x.initial_state,
+                          workspace=ws)
+    else:
+        wd = WORKLOADS[DECODE]
+        state = decode_state(wd.B, wd.H, wd.dk, wd.dv, device=dev)
+        tok = decode_tokens(n, wd.B, wd.H, wd.dk, wd.dv, seed=1000, device=dev)
+        for t in range(n):
+            kda.decode_step(tok.q[t], tok.k[t], tok.v[t], tok.g[t], tok.beta[t], state)
+    torch.cuda.synchronize()
+    print(f"kernels-only {args.kernels_only}: {n} calls done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -352,7 +380,13 @@ def main():
                     help="tokens per reference-arm step (bounded oracle sample)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum timed oracle work for the cpu_baseline object")
+    ap.add_argument("--kernels-only", choices=["prefill", "decode"], default=None,
+                    help="profiler driver: run warmup + steps calls of one path, print no "
+                         "measurement (for ncu -s/-c captures)")
     args = ap.parse_args()
+    if args.kernels_only:
+        kernels_only(args)
+        return
     args.warmup = max(args.warmup, 3)
     cfg = {"workload": PREFILL, "model": "KDA layer (synthetic, no weights)", "global_batch": 1,
            "seq_len": 8192, "heads": 32, "dk": 128, "dv": 128, "chunk": C,

@@ -5,8 +5,9 @@
  * fixed-size state per head. Sources (web pages about the Kimi K3 report):
  *   - "Kimi K3 深度拆解" (chenxutan.com), section 4.2 "线性注意力与 Delta Rule":
  *     the delta-rule state update, the fixed [d_k, d_v] state, the per-token
- *     write strength beta in (0,1), q/k assumed L2-normalised, read-out from
- *     the updated state, and the chunk-parallel / inter-chunk-recurrent form.
+ *     write strength beta in (0,1), q/k L2-normalised (by the caller, or by the
+ *     optional prologue below), read-out from the updated state, and the
+ *     chunk-parallel / inter-chunk-recurrent form.
  *   - "Kimi K3 技術報告：三個架構改動" (akiraxclaw.com), section "長度":
  *     channel-wise gating (each key channel has its own forget rate).
  *   - "3 分钟看懂 Kimi K3" (landx.limxdynamics.com), "第一条主线", Figure 3:
@@ -71,7 +72,24 @@ typedef struct {
     float g_lower_bound;/* lb: g is clamped to >= lb inside the library. Must satisfy
                            lb < 0 and lb * chunk >= -80 so exp(-cumsum) stays finite */
     int32_t chunk;      /* chunk length; 64 is the supported value */
+    int32_t prologue;   /* 0, or KDA_PROLOGUE_* flags: inputs are raw and the library
+                           applies the prologue inside its kernels (see below) */
 } kda_shape;
+
+/*
+ * Optional input prologue, fused into every entry point's kernels (prefill, snapshots,
+ * no-alloc prefill, decode). With 0 the inputs are used as given.
+ *  KDA_PROLOGUE_QK_L2NORM   q and k are raw: each (token, head) row is divided by
+ *                           max(||row||_2, 1e-12) in fp32 before use ("Kimi K3 深度拆解",
+ *                           section 4.2: the delta rule takes L2-normalised q and k).
+ *  KDA_PROLOGUE_GATE_SIGMOID g holds gate pre-activations a; the log decay is
+ *                           lb * sigmoid(a), inside (lb, 0), so the lower bound holds by
+ *                           construction ("3 分钟看懂 Kimi K3", 第一条主线 / Figure 3: the
+ *                           log decay is bounded below). The clamp max(., lb) still applies.
+ * Other bits are rejected with KDA_ERR_INVALID_ARG.
+ */
+#define KDA_PROLOGUE_QK_L2NORM 1
+#define KDA_PROLOGUE_GATE_SIGMOID 2
 
 /*
  * Bytes of device scratch kda_chunk_fwd needs for this shape (a pure function

@@ -19,6 +19,8 @@ kda_status check_shape(const kda_shape* s, bool prefill) {
   if (s->H <= 0 || s->B <= 0 || s->T < 0 || s->dk <= 0 || s->dv <= 0) return KDA_ERR_INVALID_ARG;
   if (!(s->scale >= 0.f) || !isfinite(s->scale)) return KDA_ERR_INVALID_ARG;
   if (!isfinite(s->g_lower_bound) || !(s->g_lower_bound < 0.f)) return KDA_ERR_INVALID_ARG;
+  if (s->prologue & ~(KDA_PROLOGUE_QK_L2NORM | KDA_PROLOGUE_GATE_SIGMOID))
+    return KDA_ERR_INVALID_ARG;
   if (!dims_supported(s->dk) || !dims_supported(s->dv)) return KDA_ERR_UNSUPPORTED;
   if (prefill) {
     if (s->chunk != kChunk) return KDA_ERR_UNSUPPORTED;
@@ -124,6 +126,7 @@ kda_status chunk_fwd(const void* q, const void* k, const void* v, const void* g,
   a.H = s.H; a.dk = s.dk; a.dv = s.dv;
   a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
   a.lb = s.g_lower_bound;
+  a.prologue = s.prologue;
 
   cudaError_t e = tc_path_applies(s, T_total) ? launch_prefill_tc(a, cs)
                                               : launch_prefill_simt(a, s.dtype, cs);
@@ -189,6 +192,7 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
   a.N = s.B; a.H = s.H; a.dk = s.dk; a.dv = s.dv;
   a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
   a.lb = s.g_lower_bound;
+  a.prologue = s.prologue;
   cudaError_t e = launch_decode(a, s.dtype, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

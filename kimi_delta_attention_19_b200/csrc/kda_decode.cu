@@ -13,6 +13,8 @@
 // 8 warps owns one (sequence, head); warp w holds rows w, w+8, ...; lane l
 // holds columns [l*V, l*V+V) with V = d_v/32 (a 128-bit access for d_v = 128).
 // No tensor cores: 8 bytes of state traffic per ~7 flops is HBM-bound.
+// The optional raw-input prologue (q/k L2 normalisation, log decay lb * sigmoid(a))
+// is applied to the token's inputs on the fly.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -67,14 +69,34 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   const Tin* k = static_cast<const Tin*>(a.k) + tok * DK;
   const Tin* g = static_cast<const Tin*>(a.g) + tok * DK;
   const Tin* v = static_cast<const Tin*>(a.v) + tok * DV;
+  const bool gsig = (a.prologue & KDA_PROLOGUE_GATE_SIGMOID) != 0;
   for (int i = threadIdx.x; i < DK; i += NW * 32) {
     sk[i] = ld_in(k + i);
     sq[i] = ld_in(q + i);
-    sdec[i] = expf(fmaxf(ld_in(g + i), a.lb));
+    float gi = ld_in(g + i);
+    if (gsig) gi = gate_from_preact(gi, a.lb);
+    sdec[i] = expf(fmaxf(gi, a.lb));
   }
   for (int j = threadIdx.x; j < DV; j += NW * 32) sv[j] = ld_in(v + j);
   const float b = ld_in(static_cast<const Tin*>(a.beta) + tok);
   __syncthreads();
+  // prologue: raw q and k rows are used divided by their L2 norms (every warp forms
+  // the two norms itself, from shared memory)
+  float rk = 1.f, rq = 1.f;
+  if (a.prologue & KDA_PROLOGUE_QK_L2NORM) {
+    float ssk = 0.f, ssq = 0.f;
+    for (int i = lane; i < DK; i += 32) {
+      ssk = fmaf(sk[i], sk[i], ssk);
+      ssq = fmaf(sq[i], sq[i], ssq);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+      ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+    }
+    rk = inv_l2(ssk);
+    rq = inv_l2(ssq);
+  }
 
   float pw[V], py[V];
 #pragma unroll
@@ -82,7 +104,7 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
 #pragma unroll
   for (int rr = 0; rr < R; ++rr) {
     const int i = warp + NW * rr;
-    const float d = sdec[i], ki = sk[i], qi = sq[i];
+    const float d = sdec[i], ki = sk[i] * rk, qi = sq[i] * rq;
 #pragma unroll
     for (int c = 0; c < V; ++c) {
       x[rr][c] *= d;
@@ -107,7 +129,7 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   }
 #pragma unroll
   for (int rr = 0; rr < R; ++rr) {
-    const float ki = sk[warp + NW * rr];
+    const float ki = sk[warp + NW * rr] * rk;
 #pragma unroll
     for (int c = 0; c < V; ++c) x[rr][c] = fmaf(ki, u[c], x[rr][c]);
     Vec<V>::st(S + (int64_t)(warp + NW * rr) * DV + lane * V, x[rr]);
@@ -118,6 +140,7 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
     for (int i = lane; i < DK; i += 32) kq = fmaf(sk[i], sq[i], kq);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    kq *= rk * rq;
     Tin* o = static_cast<Tin*>(a.out) + tok * DV + lane * V;
 #pragma unroll
     for (int c = 0; c < V; ++c) {

@@ -41,6 +41,7 @@ struct PrefillArgs {
   int H, dk, dv;
   float scale;
   float lb;
+  int prologue;             // KDA_PROLOGUE_* flags
 };
 
 struct DecodeArgs {
@@ -56,6 +57,7 @@ struct DecodeArgs {
   int N, H, dk, dv;
   float scale;
   float lb;
+  int prologue;             // KDA_PROLOGUE_* flags
 };
 
 // Sequence bounds [t0, t1) of sequence s; false (and status set) when the
@@ -87,6 +89,16 @@ template <>
 __device__ __forceinline__ float ld_in<__nv_bfloat16>(const __nv_bfloat16* p) {
   return __bfloat162float(__ldg(p));
 }
+
+// The raw-input prologue (KDA_PROLOGUE_*): log decay from a gate pre-activation,
+// lb * sigmoid(a), evaluated without overflow for any a.
+__device__ __forceinline__ float gate_from_preact(float a_pre, float lb) {
+  const float e = __expf(-fabsf(a_pre));     // in (0, 1]
+  const float s = 1.f / (1.f + e);           // sigmoid(|a|)
+  return lb * (a_pre >= 0.f ? s : e * s);    // sigmoid(a) = 1 - sigmoid(-a)
+}
+// 1 / max(||row||, 1e-12) from the row's sum of squares
+__device__ __forceinline__ float inv_l2(float sumsq) { return 1.f / fmaxf(sqrtf(sumsq), 1e-12f); }
 
 template <typename T>
 __device__ __forceinline__ void st_out(T* p, float x);

@@ -17,7 +17,8 @@
 //   O  = scale (Q~ S + P U)
 //   S  = Diag(exp Gamma_L) S + (K^ * exp Gamma_L)^T U
 // When asked, the state after every snap_every-th full chunk of a sequence is also
-// written out (prefix-cache snapshots).
+// written out (prefix-cache snapshots), and raw inputs go through the prologue
+// (q/k rows L2-normalised, log decay lb * sigmoid(a) from gate pre-activations).
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -40,6 +41,7 @@ struct SimtSmem {
   float U[C][DVS];
   float gl[DK];         // exp(Gamma_L) per channel
   float bet[C];
+  float rk[C], rq[C];   // prologue: 1 / |k row|, 1 / |q row|
 };
 
 template <typename Tin, int DK>
@@ -74,6 +76,29 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
   for (int64_t c0 = t0; c0 < t1; c0 += C) {
     const int L = (t1 - c0) < C ? (int)(t1 - c0) : C;
 
+    const bool l2n = (a.prologue & KDA_PROLOGUE_QK_L2NORM) != 0;
+    const bool gsig = (a.prologue & KDA_PROLOGUE_GATE_SIGMOID) != 0;
+    if (l2n) {
+      // prologue: inverse L2 norms of the chunk's raw k and q rows, one warp per row
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int rr = warp; rr < 2 * C; rr += NT / 32) {
+        const int r = rr % C;
+        const bool isq = rr >= C;
+        float ss = 0.f;
+        if (r < L) {
+          const Tin* src = (isq ? q : k) + ((c0 + r) * H + h) * DK;
+          for (int i = lane; i < DK; i += 32) {
+            const float x = ld_in(src + i);
+            ss = fmaf(x, x, ss);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) (isq ? sm.rq : sm.rk)[r] = inv_l2(ss);
+      }
+      __syncthreads();
+    }
+
     // 1. Prefix sums of the clamped log decay and the decayed operands.
     if (tid < DK) {
       const int i = tid;
@@ -82,12 +107,14 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
         float kt = 0.f, kh = 0.f, qt = 0.f;
         if (r < L) {
           const int64_t off = ((c0 + r) * H + h) * DK + i;
-          G += fmaxf(ld_in(g + off), a.lb);
+          float gr = ld_in(g + off);
+          if (gsig) gr = gate_from_preact(gr, a.lb);
+          G += fmaxf(gr, a.lb);
           const float e = expf(G), ei = expf(-G);
-          const float kv = ld_in(k + off);
+          const float kv = ld_in(k + off) * (l2n ? sm.rk[r] : 1.f);
           kt = kv * e;
           kh = kv * ei;
-          qt = ld_in(q + off) * e;
+          qt = ld_in(q + off) * (l2n ? sm.rq[r] : 1.f) * e;
         }
         sm.Kt[r][i] = kt;
         sm.Kh[r][i] = kh;

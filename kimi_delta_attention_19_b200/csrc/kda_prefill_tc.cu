@@ -190,7 +190,8 @@ struct IntraSm {
   static constexpr uint32_t A = SQ;          // A spans [80 KB, 97 KB)
   static constexpr uint32_t TOT = SQ + FP_BYTES;  // float[4][128] partial decay sums
   static constexpr uint32_t BET = TOT + 2048;     // float[64]
-  static constexpr uint32_t BARS = BET + 256;
+  static constexpr uint32_t RN = BET + 256;       // float[2][64]: 1/|k row|, 1/|q row| (prologue)
+  static constexpr uint32_t BARS = RN + 512;
   static constexpr uint32_t TPTR = BARS + 64;
   static constexpr uint32_t BYTES = TPTR + 16;
   // tensor-memory columns: [K~;Q~] K^^T, W^T, U0^T
@@ -200,6 +201,9 @@ static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTA
 static_assert(IntraSm::BT + 4096 <= IntraSm::NS && IntraSm::NS + IntraSm::FP_BYTES == IntraSm::SQ,
               "intra-chunk shared-memory regions overlap");
 
+// PRO: the raw-input prologue flags (KDA_PROLOGUE_*), a template parameter so the plain
+// instance carries no trace of it.
+template <int PRO>
 __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_constant__ IntraArgs a) {
   using L_ = IntraSm;
   extern __shared__ unsigned char smem_raw[];
@@ -228,6 +232,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   float* tot = reinterpret_cast<float*>(sm + L_::TOT);
   float* bet = reinterpret_cast<float*>(sm + L_::BET);
   float* bt = reinterpret_cast<float*>(sm + L_::BT);
+  float* rn = reinterpret_cast<float*>(sm + L_::RN);
   uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);  // g, k, q
   uint64_t* bar_v = bar_in + 1;
   uint64_t* bar_mma = bar_in + 2;
@@ -295,6 +300,27 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       __syncthreads();
     }
+    if (PRO & KDA_PROLOGUE_QK_L2NORM) {
+      // raw k and q rows -> 1 / max(|row|, 1e-12): two threads per row, 64 columns each,
+      // the 16-byte words visited in a lane-rotated order (conflict-free)
+      const int which = tid >> 7, r = (tid & 127) >> 1, hf = tid & 1;
+      const unsigned char* src = sm + (which ? L_::SQ : L_::SK) + r * 256 + hf * 128;
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const uint4 x4 = *reinterpret_cast<const uint4*>(src + 16 * ((w + lane) & 7));
+        const uint32_t xs[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16(xs[e]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
+        }
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      if (hf == 0) rn[which * 64 + r] = inv_l2(ss);
+      __syncthreads();
+    }
     // ---- 1. raw k, q into registers; prefix sums of the clamped log decay in log2 units.
     //         Thread = (channel pair p, quarter qr of 16 rows).
     const int p = tid & 63, qr = tid >> 6;
@@ -311,7 +337,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
         const uint32_t off = off0 + i * 256;
         kraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SK + off);
         qraw[i] = *reinterpret_cast<const uint32_t*>(sm + L_::SQ + off);
-        const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + off));
+        float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + L_::SG + off));
+        if (PRO & KDA_PROLOGUE_GATE_SIGMOID) {
+          // rows past a ragged chunk's end hold a zero fill, which is a log decay of 0 as
+          // given but not as a pre-activation: they must stay decay-free
+          const bool live = 16 * qr + i < L;
+          gg.x = live ? gate_from_preact(gg.x, a.lb) : 0.f;
+          gg.y = live ? gate_from_preact(gg.y, a.lb) : 0.f;
+        }
         acc0 += fmaxf(gg.x * kLog2e, lb2);
         acc1 += fmaxf(gg.y * kLog2e, lb2);
         G0[i] = acc0;
@@ -346,7 +379,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
         const float g0 = G0[i] + o0, g1 = G1[i] + o1;
         const float e0 = ex2_approx(g0), e1 = ex2_approx(g1);
         const float ei0 = ex2_approx(-g0), ei1 = ex2_approx(-g1);
-        const float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
+        float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
+        if (PRO & KDA_PROLOGUE_QK_L2NORM) {
+          const float rk = rn[16 * qr + i], rq = rn[64 + 16 * qr + i];
+          kk.x *= rk;
+          kk.y *= rk;
+          qq.x *= rq;
+          qq.y *= rq;
+        }
         const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
         *reinterpret_cast<uint32_t*>(sm + kq0 + ro) = pack_bf16(kk.x * e0, kk.y * e1);
         *reinterpret_cast<uint32_t*>(sm + kq0 + K8 + ro) = pack_bf16(qq.x * e0, qq.y * e1);
@@ -1433,8 +1473,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   wa.max_segs = plan.max_segs;
   wa.scale = pa.scale;
 
+  void (*intra)(IntraArgs) = pa.prologue == 0 ? kda_tc_intra<0>
+                            : pa.prologue == 1 ? kda_tc_intra<1>
+                            : pa.prologue == 2 ? kda_tc_intra<2>
+                                               : kda_tc_intra<3>;
   // dynamic shared memory limits are per function and per device: set them every call
-  cudaError_t e = cudaFuncSetAttribute(kda_tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        IntraSm::BYTES + 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kda_tc_walk_first, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1447,7 +1491,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
                              kCombSmem);
   if (e != cudaSuccess) return e;
 
-  kda_tc_intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
+  intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
   // The later kernels are launched with programmatic serialization: their CTAs may be
   // scheduled while the previous kernel's last CTAs finish; they set up (tensor memory,
   // barriers) and then wait for it (griddepcontrol.wait) before touching its results.

@@ -11,7 +11,9 @@ Recipe (one torch generator, seeded, drawn in this fixed order):
   g     = -g_scale * sigmoid(N(0, 1))            (per-channel log decay in [-g_scale, 0))
   S0    ~ state_std * N(0, 1), fp32              (or absent -> zeros)
 Everything is drawn in fp32 and cast once to the input dtype, before any
-consumer sees it.
+consumer sees it. With raw=True (inputs for the library's prologue) the same
+draws are returned untransformed: q, k ~ N(0, 1) not normalised, and g holds
+the gate pre-activation g_scale * N(0, 1).
 """
 from __future__ import annotations
 
@@ -83,7 +85,7 @@ def make_inputs(T: int | None = None, H: int = 2, dk: int = 64, dv: int = 64, *,
                 dtype: torch.dtype = torch.float32, seed: int = 0, device: str = "cpu",
                 lengths: list[int] | None = None, n_varlen: int = 0, len_lo: int = 0,
                 len_hi: int = 0, g_scale: float = 1.0, state_std: float | None = 0.02,
-                batch: int | None = None) -> Inputs:
+                batch: int | None = None, raw: bool = False) -> Inputs:
     """Draw one workload's inputs.
 
     Token-major packed layout: q, k, g [T, H, dk]; v [T, H, dv]; beta [T, H].
@@ -107,10 +109,12 @@ def make_inputs(T: int | None = None, H: int = 2, dk: int = 64, dv: int = 64, *,
     def randn(*shape):
         return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
 
-    q = _l2n(randn(T_total, H, dk)).to(dtype)
-    k = _l2n(randn(T_total, H, dk)).to(dtype)
+    unit = (lambda x: x) if raw else _l2n
+    q = unit(randn(T_total, H, dk)).to(dtype)
+    k = unit(randn(T_total, H, dk)).to(dtype)
     v = randn(T_total, H, dv).to(dtype)
-    g = (-g_scale * torch.sigmoid(randn(T_total, H, dk))).to(dtype)
+    g_raw = randn(T_total, H, dk)
+    g = (g_scale * g_raw if raw else -g_scale * torch.sigmoid(g_raw)).to(dtype)
     beta = torch.sigmoid(randn(T_total, H)).to(dtype)
     n = len(lengths)
     s0 = None
@@ -146,17 +150,21 @@ def decode_state(N: int, H: int, dk: int, dv: int, *, seed: int = 0, device: str
 
 
 def decode_tokens(steps: int, N: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
-                  seed: int = 1, device: str = "cpu", g_scale: float = 1.0) -> Inputs:
-    """`steps` tokens for each of N sequences, step-major: q, k, g [steps, N, H, dk] etc."""
+                  seed: int = 1, device: str = "cpu", g_scale: float = 1.0,
+                  raw: bool = False) -> Inputs:
+    """`steps` tokens for each of N sequences, step-major: q, k, g [steps, N, H, dk] etc.
+    raw=True: untransformed draws, as in make_inputs."""
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
 
     def randn(*shape):
         return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32)
 
-    q = _l2n(randn(steps, N, H, dk)).to(dtype)
-    k = _l2n(randn(steps, N, H, dk)).to(dtype)
+    unit = (lambda x: x) if raw else _l2n
+    q = unit(randn(steps, N, H, dk)).to(dtype)
+    k = unit(randn(steps, N, H, dk)).to(dtype)
     v = randn(steps, N, H, dv).to(dtype)
-    g = (-g_scale * torch.sigmoid(randn(steps, N, H, dk))).to(dtype)
+    g_raw = randn(steps, N, H, dk)
+    g = (g_scale * g_raw if raw else -g_scale * torch.sigmoid(g_raw)).to(dtype)
     beta = torch.sigmoid(randn(steps, N, H)).to(dtype)
     return Inputs(q, k, v, g, beta, None, None, [steps] * N)

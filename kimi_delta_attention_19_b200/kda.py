@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE = range(5)
 KDA_F32, KDA_BF16 = 0, 1
 CHUNK = 64
+PROLOGUE_QK_L2NORM = 1     # raw q, k: rows divided by max(||row||_2, 1e-12) in the kernels
+PROLOGUE_GATE_SIGMOID = 2  # g holds gate pre-activations a: log decay = lb * sigmoid(a)
 
 
 class KdaError(RuntimeError):
@@ -32,7 +34,7 @@ class Shape(ctypes.Structure):
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("n_seqs", ctypes.c_int32),
                 ("max_seqlen", ctypes.c_int64), ("dtype", ctypes.c_int),
                 ("scale", ctypes.c_float), ("g_lower_bound", ctypes.c_float),
-                ("chunk", ctypes.c_int32)]
+                ("chunk", ctypes.c_int32), ("prologue", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -91,11 +93,11 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def make_shape(T: int, H: int, dk: int, dv: int, dtype: torch.dtype, *, B: int = 1,
                n_seqs: int = 0, max_seqlen: int = 0, scale: float | None = None,
-               lb: float = -1.0, chunk: int = CHUNK) -> Shape:
+               lb: float = -1.0, chunk: int = CHUNK, prologue: int = 0) -> Shape:
     code = KDA_F32 if dtype == torch.float32 else KDA_BF16
     return Shape(T=T, B=B, H=H, dk=dk, dv=dv, n_seqs=n_seqs, max_seqlen=max_seqlen, dtype=code,
                  scale=0.0 if scale is None else float(scale), g_lower_bound=float(lb),
-                 chunk=chunk)
+                 chunk=chunk, prologue=int(prologue))
 
 
 def workspace_size(shape: Shape) -> int:
@@ -110,7 +112,7 @@ def alloc_workspace(shape: Shape, device) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb):
+def _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb, prologue=0):
     batched = q.dim() == 4
     if batched:
         B, T, H, dk = q.shape
@@ -124,7 +126,7 @@ def _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb):
     else:
         n = B
     shape = make_shape(T, H, dk, dv, q.dtype, B=B, n_seqs=n if cu_seqlens is not None else 0,
-                       max_seqlen=max_seqlen, scale=scale, lb=lb)
+                       max_seqlen=max_seqlen, scale=scale, lb=lb, prologue=prologue)
     return shape, n
 
 
@@ -133,12 +135,13 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
               cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
               scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
               final_state: torch.Tensor | None = None, output_final_state: bool = True,
-              workspace: torch.Tensor | None = None, stream=None):
+              workspace: torch.Tensor | None = None, prologue: int = 0, stream=None):
     """Chunked prefill. q, k, g: [T, H, dk] (or [B, T, H, dk]); v: [..., dv]; beta: [..., H].
 
+    prologue: 0 or PROLOGUE_* flags (raw q/k and/or gate pre-activations in g).
     Returns (out, final_state). final_state is fp32 [n, H, dk, dv] (None if not requested).
     """
-    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb, prologue)
     H, dk, dv = shape.H, shape.dk, shape.dv
     if out is None:
         out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
@@ -167,7 +170,7 @@ def chunk_fwd_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: to
                         scale: float | None = None, lb: float = -1.0,
                         out: torch.Tensor | None = None, final_state: torch.Tensor | None = None,
                         output_final_state: bool = True, workspace: torch.Tensor | None = None,
-                        stream=None):
+                        prologue: int = 0, stream=None):
     """Prefill that also keeps the state every `snapshot_chunks` chunks (prefix cache).
 
     Returns (out, final_state, snapshots); snapshots is fp32 [snapshot_count, H, dk, dv].
@@ -175,7 +178,7 @@ def chunk_fwd_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: to
     * 64 tokens at index c_n // (snapshot_chunks * 64) + m - 1, m = 1, 2, ...; indices no
     sequence reaches keep their previous contents (zeros when this call allocates).
     """
-    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb, prologue)
     H, dk, dv = shape.H, shape.dk, shape.dv
     count = snapshot_count(shape, snapshot_chunks)
     if count < 0:
@@ -206,7 +209,8 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
                       beta: torch.Tensor, *, out: torch.Tensor, final_state: torch.Tensor | None,
                       initial_state: torch.Tensor | None = None,
                       cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
-                      scale: float | None = None, lb: float = -1.0, stream=None):
+                      scale: float | None = None, lb: float = -1.0, prologue: int = 0,
+                      stream=None):
     """kda_chunk_fwd_noalloc: the prefill with the library's fixed scratch array.
 
     For callers that cannot allocate device memory, so `out` (and `final_state`,
@@ -221,7 +225,7 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     dv = v.shape[-1]
     n = cu_seqlens.numel() - 1 if cu_seqlens is not None else 0
     shape = make_shape(T, H, dk, dv, q.dtype, B=B, n_seqs=n, max_seqlen=max_seqlen,
-                       scale=scale, lb=lb)
+                       scale=scale, lb=lb, prologue=prologue)
     rc = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                    _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
                                    _ptr(final_state), ctypes.byref(shape), _stream(stream))
@@ -233,14 +237,14 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, state: torch.Tensor, *, state_slots: torch.Tensor | None = None,
                 scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
-                stream=None) -> torch.Tensor:
+                prologue: int = 0, stream=None) -> torch.Tensor:
     """One token per sequence: q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H].
 
     Updates fp32 `state` [n_slots, H, dk, dv] in place; returns out [N, H, dv].
     """
     N, H, dk = q.shape
     dv = v.shape[-1]
-    shape = make_shape(1, H, dk, dv, q.dtype, B=N, scale=scale, lb=lb)
+    shape = make_shape(1, H, dk, dv, q.dtype, B=N, scale=scale, lb=lb, prologue=prologue)
     if out is None:
         out = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
     rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),

@@ -86,6 +86,10 @@ def test_chunk_fwd_argument_errors(kda):
         kda.KDA_ERR_INVALID_ARG
     bad_b = kda.make_shape(128, 2, 64, 64, torch.float32, B=2, n_seqs=1)
     assert _fwd(kda, bad_b, {"cu": 4096}) == kda.KDA_ERR_INVALID_ARG    # cu_seqlens needs B=1
+    assert _fwd(kda, kda.make_shape(128, 2, 64, 64, torch.float32, prologue=4)) == \
+        kda.KDA_ERR_INVALID_ARG                                          # unknown prologue bit
+    assert kda.workspace_size(kda.make_shape(128, 2, 64, 64, torch.float32, prologue=8)) == 0
+    assert kda.workspace_size(kda.make_shape(128, 2, 64, 64, torch.float32, prologue=3)) > 0
     no_n = kda.make_shape(128, 2, 64, 64, torch.float32, n_seqs=0)
     assert _fwd(kda, no_n, {"cu": 4096}) == kda.KDA_ERR_INVALID_ARG
     assert kda.lib.kda_chunk_fwd(None, None, None, None, None, None, None, None, None, None,
@@ -134,6 +138,8 @@ def test_decode_argument_errors(kda):
         kda.KDA_ERR_INVALID_ARG                                 # decode is one token
     assert call(shape=kda.make_shape(1, 4, 128, 80, torch.bfloat16, B=8)) == \
         kda.KDA_ERR_UNSUPPORTED
+    assert call(shape=kda.make_shape(1, 4, 128, 128, torch.bfloat16, B=8, prologue=-1)) == \
+        kda.KDA_ERR_INVALID_ARG
 
 
 def test_binding_refuses_without_library(tmp_path, monkeypatch):
