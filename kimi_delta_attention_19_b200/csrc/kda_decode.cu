@@ -46,7 +46,9 @@ struct Vec<2> {
   }
 };
 
-template <typename Tin, int DK, int DV>
+// PRO: the raw-input prologue flags (KDA_PROLOGUE_*), a template parameter so the plain
+// instance carries no trace of it.
+template <typename Tin, int DK, int DV, int PRO>
 __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   constexpr int V = DV / 32;    // columns per lane
   constexpr int R = DK / NW;    // rows per warp
@@ -69,12 +71,11 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   const Tin* k = static_cast<const Tin*>(a.k) + tok * DK;
   const Tin* g = static_cast<const Tin*>(a.g) + tok * DK;
   const Tin* v = static_cast<const Tin*>(a.v) + tok * DV;
-  const bool gsig = (a.prologue & KDA_PROLOGUE_GATE_SIGMOID) != 0;
   for (int i = threadIdx.x; i < DK; i += NW * 32) {
     sk[i] = ld_in(k + i);
     sq[i] = ld_in(q + i);
     float gi = ld_in(g + i);
-    if (gsig) gi = gate_from_preact(gi, a.lb);
+    if (PRO & KDA_PROLOGUE_GATE_SIGMOID) gi = gate_from_preact(gi, a.lb);
     sdec[i] = expf(fmaxf(gi, a.lb));
   }
   for (int j = threadIdx.x; j < DV; j += NW * 32) sv[j] = ld_in(v + j);
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   // prologue: raw q and k rows are used divided by their L2 norms (every warp forms
   // the two norms itself, from shared memory)
   float rk = 1.f, rq = 1.f;
-  if (a.prologue & KDA_PROLOGUE_QK_L2NORM) {
+  if (PRO & KDA_PROLOGUE_QK_L2NORM) {
     float ssk = 0.f, ssq = 0.f;
     for (int i = lane; i < DK; i += 32) {
       ssk = fmaf(sk[i], sk[i], ssk);
@@ -152,15 +153,25 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   }
 }
 
+template <typename Tin, int PRO>
+void launch_dims(const DecodeArgs& a, dim3 grid, dim3 block, cudaStream_t st) {
+  if (a.dk == 128 && a.dv == 128) decode_kernel<Tin, 128, 128, PRO><<<grid, block, 0, st>>>(a);
+  else if (a.dk == 128 && a.dv == 64) decode_kernel<Tin, 128, 64, PRO><<<grid, block, 0, st>>>(a);
+  else if (a.dk == 64 && a.dv == 128) decode_kernel<Tin, 64, 128, PRO><<<grid, block, 0, st>>>(a);
+  else decode_kernel<Tin, 64, 64, PRO><<<grid, block, 0, st>>>(a);
+}
+
 template <typename Tin>
 cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t st) {
   const int64_t blocks = (int64_t)a.N * a.H;
   if (blocks == 0) return cudaSuccess;
   const dim3 grid((unsigned)blocks), block(NW * 32);
-  if (a.dk == 128 && a.dv == 128) decode_kernel<Tin, 128, 128><<<grid, block, 0, st>>>(a);
-  else if (a.dk == 128 && a.dv == 64) decode_kernel<Tin, 128, 64><<<grid, block, 0, st>>>(a);
-  else if (a.dk == 64 && a.dv == 128) decode_kernel<Tin, 64, 128><<<grid, block, 0, st>>>(a);
-  else decode_kernel<Tin, 64, 64><<<grid, block, 0, st>>>(a);
+  switch (a.prologue) {
+    case 0: launch_dims<Tin, 0>(a, grid, block, st); break;
+    case 1: launch_dims<Tin, 1>(a, grid, block, st); break;
+    case 2: launch_dims<Tin, 2>(a, grid, block, st); break;
+    default: launch_dims<Tin, 3>(a, grid, block, st); break;
+  }
   return cudaGetLastError();
 }
 

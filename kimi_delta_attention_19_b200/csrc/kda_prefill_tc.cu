@@ -190,8 +190,10 @@ struct IntraSm {
   static constexpr uint32_t A = SQ;          // A spans [80 KB, 97 KB)
   static constexpr uint32_t TOT = SQ + FP_BYTES;  // float[4][128] partial decay sums
   static constexpr uint32_t BET = TOT + 2048;     // float[64]
-  static constexpr uint32_t RN = BET + 256;       // float[2][64]: 1/|k row|, 1/|q row| (prologue)
-  static constexpr uint32_t BARS = RN + 512;
+  static constexpr uint32_t BARS = BET + 256;
+  // float[2][64]: 1/|k row|, 1/|q row| (prologue), in the gap after raw q that A only
+  // reaches in phase 4, after the last use of RN
+  static constexpr uint32_t RN = SQ + K16;
   static constexpr uint32_t TPTR = BARS + 64;
   static constexpr uint32_t BYTES = TPTR + 16;
   // tensor-memory columns: [K~;Q~] K^^T, W^T, U0^T
@@ -200,6 +202,7 @@ struct IntraSm {
 static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTAs per SM");
 static_assert(IntraSm::BT + 4096 <= IntraSm::NS && IntraSm::NS + IntraSm::FP_BYTES == IntraSm::SQ,
               "intra-chunk shared-memory regions overlap");
+static_assert(IntraSm::RN + 512 <= IntraSm::TOT, "prologue norms overlap the decay sums");
 
 // PRO: the raw-input prologue flags (KDA_PROLOGUE_*), a template parameter so the plain
 // instance carries no trace of it.
@@ -671,7 +674,7 @@ static_assert(WalkSm<false>::BYTES + 1024 <= 232448, "summary walk shared memory
 // One CTA walks segment `seg` of the (sequence, head) pair: the output walk (PC) from
 // the segment's true start state, writing outputs (and the state where a later step
 // needs it), or the summary walk of a middle segment.
-template <bool PC>
+template <bool PC, bool SNAP>
 __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* smem_raw, int pair,
                                              int seg) {
   using L_ = WalkSm<PC>;
@@ -1056,7 +1059,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       tc_fence_before();
       group_sync(half_bar, 128);
       if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + hc);
-      if (PC && a.snap != nullptr) store_snapshot(n, v0, v1);  // while MMA-1(n + 1) runs
+      if (PC && SNAP) store_snapshot(n, v0, v1);  // while MMA-1(n + 1) runs
       if (n + 1 < n_chunks) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
           failed = true;
@@ -1120,18 +1123,22 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 // S_1), CTA r >= 1 is the summary walk of segment r, in parallel.
 constexpr uint32_t kWalkFirstSmem =
     (WalkSm<true>::BYTES > WalkSm<false>::BYTES ? WalkSm<true>::BYTES : WalkSm<false>::BYTES) + 1024;
+// SNAP: the output walks also write chunk-boundary snapshots (a separate instance, so
+// the plain walk carries no trace of them).
+template <bool SNAP>
 __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_first(const __grid_constant__ WalkArgs a) {
   extern __shared__ unsigned char smem_raw[];
   const int per = a.max_segs > 2 ? a.max_segs - 1 : 1;
   const int role = blockIdx.x % per, pair = blockIdx.x / per;
-  if (role == 0) walk_segment<true>(a, smem_raw, pair, 0);
-  else walk_segment<false>(a, smem_raw, pair, role);
+  if (role == 0) walk_segment<true, SNAP>(a, smem_raw, pair, 0);
+  else walk_segment<false, false>(a, smem_raw, pair, role);
 }
 // Phase 2 (after the combine): the output walks of segments 1 .. nseg - 1.
+template <bool SNAP>
 __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid_constant__ WalkArgs a) {
   extern __shared__ unsigned char smem_raw[];
   const int per = a.max_segs - 1;
-  walk_segment<true>(a, smem_raw, blockIdx.x / per, 1 + blockIdx.x % per);
+  walk_segment<true, SNAP>(a, smem_raw, blockIdx.x / per, 1 + blockIdx.x % per);
 }
 
 // ------------------------------------------------------------------ combine
@@ -1480,11 +1487,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   // dynamic shared memory limits are per function and per device: set them every call
   cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        IntraSm::BYTES + 1024);
+  const bool snap = pa.snap != nullptr;
+  void (*walk_first)(WalkArgs) = snap ? kda_tc_walk_first<true> : kda_tc_walk_first<false>;
+  void (*walk_rest)(WalkArgs) = snap ? kda_tc_walk_rest<true> : kda_tc_walk_rest<false>;
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_walk_first, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(walk_first, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kWalkFirstSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_walk_rest, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(walk_rest, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              WalkSm<true>::BYTES + 1024);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kda_tc_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1511,13 +1521,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   };
   const int64_t per_first = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
   if (e == cudaSuccess)
-    e = launch_dep(reinterpret_cast<const void*>(kda_tc_walk_first), plan.pairs * per_first,
+    e = launch_dep(reinterpret_cast<const void*>(walk_first), plan.pairs * per_first,
                    kWalkThreads, kWalkFirstSmem);
   if (e == cudaSuccess && plan.max_segs > 2)
     e = launch_dep(reinterpret_cast<const void*>(kda_tc_combine), plan.pairs, kCombThreads,
                    kCombSmem);
   if (e == cudaSuccess && plan.max_segs > 1)
-    e = launch_dep(reinterpret_cast<const void*>(kda_tc_walk_rest), plan.pairs * (plan.max_segs - 1),
+    e = launch_dep(reinterpret_cast<const void*>(walk_rest), plan.pairs * (plan.max_segs - 1),
                    kWalkThreads, WalkSm<true>::BYTES + 1024);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
