@@ -321,3 +321,246 @@ int kda_oracle_recurrent_ex(int64_t T, int H, int dk, int dv, int n_seqs,
                    lb, scale, out, out_rows, n_out_rows, final_state, snap_tokens, snap_first,
                    snaps, prologue, n_threads);
 }
+
+/* ======================================================================== backward
+ * Reverse-mode gradient of the token recurrence above (no prologue), in fp64.
+ * Given upstream gradients dO = dL/do_t [T, H, dv] and dS_T = dL/dS_final [n, H, dk, dv]
+ * (NULL = 0) of some scalar L, returns dL/dq, dL/dk, dL/dg, dL/dbeta, dL/dv and
+ * dL/dS0. It differentiates, step by step in reverse, exactly the forward loop:
+ *
+ *   Sb = Diag(exp g') S_prev     w = Sb^T k     u = beta (v - w)
+ *   S  = Sb + k u^T              o = scale S^T q
+ *
+ * so, with dS the gradient of S_t accumulated from later tokens:
+ *   dS += scale q do^T;  dq = scale S do;  dk = dS u;  du = dS^T k;
+ *   dbeta = du . (v - w);  dv = beta du;  dw = -beta du;
+ *   dSb = dS + k dw^T;  dk += Sb dw;  dg'_i = sum_j Sb_ij dSb_ij;
+ *   dg_i = dg'_i where g_i >= lb (the clamp passes the gradient), else 0;
+ *   dS_prev = Diag(exp g') dSb.
+ * The states S_{t-1} are recomputed per block of 64 tokens from checkpoints taken in
+ * a forward sweep. Training needs this gradient ("Kimi K3 深度拆解", section 4.2
+ * describes the chunk-parallel kernels the model is trained with).
+ */
+typedef struct {
+    int64_t T;
+    int H, dk, dv, n_seqs;
+    const int64_t *cu_seqlens;
+    int dtype;
+    const void *q, *k, *v, *g, *beta;
+    const double *initial_state, *d_out, *d_final;
+    double lb, scale;
+    double *dq, *dkk, *dvv, *dg, *dbeta, *ds0;
+    int64_t next_item;
+    pthread_mutex_t lock;
+} bjob_t;
+
+#define KDA_ORACLE_BWD_BLOCK 64
+
+/* Inputs of token t (head h): k, q, v, beta, the clamped decay and the raw log decay. */
+static void load_token(const bjob_t *J, int64_t t, int h, double *kt, double *qt, double *vt,
+                       double *decay, double *graw, double *b)
+{
+    const int dk = J->dk, dv = J->dv, H = J->H;
+    const int64_t tok_k = (t * H + h) * dk, tok_v = (t * H + h) * dv;
+    for (int i = 0; i < dk; ++i) {
+        kt[i] = load_elem(J->k, J->dtype, tok_k + i);
+        qt[i] = load_elem(J->q, J->dtype, tok_k + i);
+        graw[i] = load_elem(J->g, J->dtype, tok_k + i);
+        decay[i] = exp(graw[i] < J->lb ? J->lb : graw[i]);
+    }
+    for (int j = 0; j < dv; ++j) vt[j] = load_elem(J->v, J->dtype, tok_v + j);
+    *b = load_elem(J->beta, J->dtype, t * H + h);
+}
+
+/* One forward token step in place: S <- (I - b k k^T) Diag(decay) S + b k v^T. */
+static void step_state(double *S, int dk, int dv, const double *kt, const double *vt,
+                       const double *decay, double b, double *w)
+{
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) S[i * dv + j] *= decay[i];
+    for (int j = 0; j < dv; ++j) w[j] = 0.0;
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) w[j] += kt[i] * S[i * dv + j];
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) S[i * dv + j] += b * kt[i] * (vt[j] - w[j]);
+}
+
+static int bwd_one(const bjob_t *J, int seq, int h)
+{
+    const int dk = J->dk, dv = J->dv, H = J->H, B = KDA_ORACLE_BWD_BLOCK;
+    const int64_t t0 = J->cu_seqlens[seq], t1 = J->cu_seqlens[seq + 1];
+    const int64_t nb = (t1 - t0 + B - 1) / B;
+    const size_t st = (size_t)dk * dv;
+    const int64_t state_off = ((int64_t)seq * H + h) * dk * dv;
+    double *ckpt = (double *)malloc(sizeof(double) * st * (size_t)(nb > 0 ? nb : 1));
+    double *pre = (double *)malloc(sizeof(double) * st * (size_t)B); /* S_{t-1} per token */
+    double *S = (double *)malloc(sizeof(double) * st);
+    double *Sb = (double *)malloc(sizeof(double) * st);
+    double *dS = (double *)malloc(sizeof(double) * st);
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(5 * dk + 6 * dv));
+    if (!ckpt || !pre || !S || !Sb || !dS || !buf) {
+        free(ckpt); free(pre); free(S); free(Sb); free(dS); free(buf);
+        return 1;
+    }
+    double *kt = buf, *qt = kt + dk, *decay = qt + dk, *graw = decay + dk, *dgp = graw + dk;
+    double *vt = dgp + dk, *w = vt + dv, *u = w + dv, *du = u + dv, *dw = du + dv, *dov = dw + dv;
+    double b;
+
+    /* forward sweep: the state at the start of every block */
+    if (J->initial_state) memcpy(S, J->initial_state + state_off, sizeof(double) * st);
+    else memset(S, 0, sizeof(double) * st);
+    for (int64_t blk = 0; blk < nb; ++blk) {
+        memcpy(ckpt + (size_t)blk * st, S, sizeof(double) * st);
+        const int64_t e = t0 + (blk + 1) * B < t1 ? t0 + (blk + 1) * B : t1;
+        for (int64_t t = t0 + blk * B; t < e; ++t) {
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            step_state(S, dk, dv, kt, vt, decay, b, w);
+        }
+    }
+
+    if (J->d_final) memcpy(dS, J->d_final + state_off, sizeof(double) * st);
+    else memset(dS, 0, sizeof(double) * st);
+    for (int64_t blk = nb - 1; blk >= 0; --blk) {
+        const int64_t s = t0 + blk * B, e = s + B < t1 ? s + B : t1;
+        memcpy(S, ckpt + (size_t)blk * st, sizeof(double) * st);
+        for (int64_t t = s; t < e; ++t) {
+            memcpy(pre + (size_t)(t - s) * st, S, sizeof(double) * st);
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            step_state(S, dk, dv, kt, vt, decay, b, w);
+        }
+        for (int64_t t = e - 1; t >= s; --t) {
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            const double *Sp = pre + (size_t)(t - s) * st;
+            /* recompute the step: Sb, w, u and S_t (in S) */
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) Sb[i * dv + j] = decay[i] * Sp[i * dv + j];
+            for (int j = 0; j < dv; ++j) w[j] = 0.0;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) w[j] += kt[i] * Sb[i * dv + j];
+            for (int j = 0; j < dv; ++j) u[j] = b * (vt[j] - w[j]);
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) S[i * dv + j] = Sb[i * dv + j] + kt[i] * u[j];
+
+            const int64_t tk = (t * H + h) * dk, tv = (t * H + h) * dv;
+            for (int j = 0; j < dv; ++j) dov[j] = J->d_out ? J->d_out[tv + j] : 0.0;
+            /* o = scale S^T q */
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) dS[i * dv + j] += J->scale * qt[i] * dov[j];
+            for (int i = 0; i < dk; ++i) {
+                double a = 0.0;
+                for (int j = 0; j < dv; ++j) a += S[i * dv + j] * dov[j];
+                J->dq[tk + i] = J->scale * a;
+            }
+            /* S = Sb + k u^T */
+            for (int j = 0; j < dv; ++j) du[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double a = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    a += dS[i * dv + j] * u[j];
+                    du[j] += dS[i * dv + j] * kt[i];
+                }
+                J->dkk[tk + i] = a;
+            }
+            /* u = beta (v - w) */
+            double db = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                db += du[j] * (vt[j] - w[j]);
+                J->dvv[tv + j] = b * du[j];
+                dw[j] = -b * du[j];
+            }
+            J->dbeta[t * H + h] = db;
+            /* w = Sb^T k: dSb = dS + k dw^T, dk += Sb dw */
+            for (int i = 0; i < dk; ++i) {
+                double a = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    dS[i * dv + j] += kt[i] * dw[j];
+                    a += Sb[i * dv + j] * dw[j];
+                }
+                J->dkk[tk + i] += a;
+            }
+            /* Sb = Diag(exp g') S_prev */
+            for (int i = 0; i < dk; ++i) {
+                double a = 0.0;
+                for (int j = 0; j < dv; ++j) a += Sb[i * dv + j] * dS[i * dv + j];
+                dgp[i] = a;
+                J->dg[tk + i] = graw[i] >= J->lb ? dgp[i] : 0.0;
+                for (int j = 0; j < dv; ++j) dS[i * dv + j] *= decay[i];
+            }
+        }
+    }
+    if (J->ds0) memcpy(J->ds0 + state_off, dS, sizeof(double) * st);
+    free(ckpt); free(pre); free(S); free(Sb); free(dS); free(buf);
+    return 0;
+}
+
+static void *bwd_worker(void *arg)
+{
+    bjob_t *J = (bjob_t *)arg;
+    const int64_t n_items = (int64_t)J->n_seqs * J->H;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t item = J->next_item++;
+        pthread_mutex_unlock(&J->lock);
+        if (item >= n_items) break;
+        if (bwd_one(J, (int)(item / J->H), (int)(item % J->H)) != 0) return (void *)1;
+    }
+    return NULL;
+}
+
+/*
+ * Gradients of the recurrence (see the block comment above). Layouts as in the forward;
+ * d_out [T, H, dv] fp64 (NULL = 0), d_final [n_seqs, H, dk, dv] fp64 (NULL = 0); outputs
+ * dq, dk, dg [T, H, dk], dv [T, H, dv], dbeta [T, H], ds0 [n_seqs, H, dk, dv] (NULL to
+ * skip), all fp64. Returns 0, -1 on a bad argument, -2 when a thread failed.
+ */
+int kda_oracle_backward(int64_t T, int H, int dk, int dv, int n_seqs,
+                        const int64_t *cu_seqlens, int dtype,
+                        const void *q, const void *k, const void *v,
+                        const void *g, const void *beta,
+                        const double *initial_state, double lb, double scale,
+                        const double *d_out, const double *d_final,
+                        double *dq, double *dkk, double *dvv, double *dg, double *dbeta,
+                        double *ds0, int n_threads)
+{
+    if (T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs <= 0 || !cu_seqlens) return -1;
+    if (dtype != KDA_ORACLE_F32 && dtype != KDA_ORACLE_BF16) return -1;
+    if (cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return -1;
+    for (int s = 0; s < n_seqs; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !dq || !dkk || !dvv || !dg || !dbeta))
+        return -1;
+
+    bjob_t J;
+    memset(&J, 0, sizeof J);
+    J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.n_seqs = n_seqs;
+    J.cu_seqlens = cu_seqlens; J.dtype = dtype;
+    J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta;
+    J.initial_state = initial_state; J.d_out = d_out; J.d_final = d_final;
+    J.lb = lb; J.scale = scale;
+    J.dq = dq; J.dkk = dkk; J.dvv = dvv; J.dg = dg; J.dbeta = dbeta; J.ds0 = ds0;
+    pthread_mutex_init(&J.lock, NULL);
+
+    const int64_t n_items = (int64_t)n_seqs * H;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > n_items) n_threads = (int)n_items;
+    int rc = 0;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    if (!th) {
+        pthread_mutex_destroy(&J.lock);
+        return -2;
+    }
+    int started = 0;
+    for (int i = 0; i < n_threads; ++i) {
+        if (pthread_create(&th[i], NULL, bwd_worker, &J) != 0) break;
+        ++started;
+    }
+    if (started == 0) rc = -2;
+    for (int i = 0; i < started; ++i) {
+        void *ret = NULL;
+        pthread_join(th[i], &ret);
+        if (ret != NULL) rc = -2;
+    }
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return rc;
+}

@@ -13,6 +13,9 @@ Two independent fp64 implementations live here:
   section "長度" (channel-wise gating), "3 分钟看懂 Kimi K3" (landx.limxdynamics.com)
   "第一条主线" / Figure 3 (log decay bounded below).
 
+  ``backward`` is the reverse-mode gradient of that loop (C), differentiating each
+  step of it in reverse order with recomputed states.
+
   Options of the same C loop: ``recurrent_snapshots`` also records the state after
   every P tokens of each sequence (prefix-cache snapshots), and ``prologue`` takes raw
   inputs: q, k rows L2-normalised per token (QK_L2NORM) and/or gate pre-activations a
@@ -70,6 +73,11 @@ def _bind(path: str):
     f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
                   p, p, ctypes.c_int64, p, ctypes.c_int64, p, p, ctypes.c_int, ctypes.c_int]
+    f = lib.kda_oracle_backward
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
+                  p, p, p, p, p, p, p, p, ctypes.c_int]
     return lib
 
 
@@ -234,6 +242,57 @@ def recurrent_snapshots(q, k, v, g, beta, *, snapshot_tokens: int, cu_seqlens=No
     return out, fin, snaps[:int(counts.sum())], first
 
 
+def backward(q, k, v, g, beta, *, d_out=None, d_final=None, cu_seqlens=None,
+             initial_state=None, lb: float = -1.0, scale: float | None = None,
+             n_threads: int | None = None, lib=None) -> dict:
+    """fp64 reverse-mode gradients of the token recurrence (kda_oracle.c, "backward").
+
+    d_out: dL/do [T, H, dv] (None = 0); d_final: dL/dS_final [n, H, dk, dv] (None = 0).
+    Returns dict dq, dk, dg [T, H, dk], dv [T, H, dv], dbeta [T, H], ds0 [n, H, dk, dv],
+    all fp64 numpy.
+    """
+    qa, dt = _as_input(q)
+    ka, _ = _as_input(k)
+    va, _ = _as_input(v)
+    ga, _ = _as_input(g)
+    ba, _ = _as_input(beta)
+    T, H, dk = qa.shape
+    dv = va.shape[2]
+    cu = (np.array([0, T], dtype=np.int64) if cu_seqlens is None
+          else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)))
+    n = len(cu) - 1
+
+    def f64(x, shape):
+        if x is None:
+            return None
+        a = np.ascontiguousarray(np.asarray(_to_numpy(x), dtype=np.float64))
+        assert a.shape == shape, (a.shape, shape)
+        return a
+    s0 = f64(initial_state, (n, H, dk, dv))
+    do = f64(d_out, (T, H, dv))
+    dS = f64(d_final, (n, H, dk, dv))
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    res = {"dq": np.zeros((T, H, dk)), "dk": np.zeros((T, H, dk)), "dv": np.zeros((T, H, dv)),
+           "dg": np.zeros((T, H, dk)), "dbeta": np.zeros((T, H)),
+           "ds0": np.zeros((n, H, dk, dv))}
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    lib = lib or load()
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    rc = lib.kda_oracle_backward(T, H, dk, dv, n, ptr(cu), dt, ptr(qa), ptr(ka), ptr(va),
+                                 ptr(ga), ptr(ba), ptr(s0), float(lb), float(scale), ptr(do),
+                                 ptr(dS), ptr(res["dq"]), ptr(res["dk"]), ptr(res["dv"]),
+                                 ptr(res["dg"]), ptr(res["dbeta"]), ptr(res["ds0"]),
+                                 int(n_threads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_backward failed with code {rc}")
+    return res
+
+
 def _to_numpy(x):
     try:
         import torch
@@ -245,7 +304,9 @@ def _to_numpy(x):
 
 
 def _widen(x) -> np.ndarray:
-    """Exact widening of an f32 / bf16 input to fp64 numpy."""
+    """Exact widening of an f32 / bf16 input to fp64 numpy (fp64 inputs pass through)."""
+    if isinstance(x, np.ndarray) and x.dtype == np.float64:
+        return x
     a, dt = _as_input(x)
     if dt == BF16:
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -357,11 +357,78 @@ def pin_prologue_gate(lib):
     assert _rel(o8, o1) < 1e-5 and _rel(s8, s1) < 1e-5  # q, k are unit rows up to fp32
 
 
+def pin_backward_finite_differences(lib):
+    """The reverse-mode gradients equal central finite differences of the independently
+    derived chunked fp64 form, element by element for q, k, v, g, beta and S0, with
+    L = sum(d_out * o) + sum(d_final * S_final); varlen with an empty sequence, and the
+    clamp active on some gates (their gradient is zero)."""
+    rng = np.random.default_rng(91)
+    lb = -1.2
+    x = make_inputs(None, H=2, dk=3, dv=2, dtype=torch.float32, seed=91, lengths=[4, 0, 5],
+                    state_std=0.5, g_scale=2.0)
+    cu = x.cu_seqlens.tolist()
+    T = cu[-1]
+    do = rng.standard_normal((T, 2, 2))
+    dS = rng.standard_normal((3, 2, 3, 2))
+    got = ko.backward(x.q, x.k, x.v, x.g, x.beta, d_out=do, d_final=dS, cu_seqlens=cu,
+                      initial_state=x.initial_state, lb=lb, lib=lib)
+    vals = {n: ko._widen(getattr(x, n)).copy() for n in ("q", "k", "v", "g", "beta")}
+    vals["s0"] = x.initial_state.double().numpy().copy()
+    assert (vals["g"] < lb - 1e-3).any() and (vals["g"] > lb + 1e-3).any()
+
+    def loss():
+        o, s = ko.chunked(vals["q"], vals["k"], vals["v"], vals["g"], vals["beta"], chunk=3,
+                          cu_seqlens=cu, initial_state=vals["s0"], lb=lb)
+        return float(np.sum(do * o) + np.sum(dS * s))
+    h = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"),
+                      ("s0", "ds0")):
+        arr = vals[name]
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            if name == "g" and abs(arr[idx] - lb) < 1e-3:
+                fd[idx] = got[key][idx]  # the kink of the clamp: no finite difference
+                continue
+            x0 = arr[idx]
+            arr[idx] = x0 + h
+            lp = loss()
+            arr[idx] = x0 - h
+            lm = loss()
+            arr[idx] = x0
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - got[key]))
+        assert err <= 1e-6 * max(1.0, np.max(np.abs(fd))), (name, err)
+    assert np.all(got["dg"][ko._widen(x.g) < lb] == 0.0)
+
+
+def pin_backward_beta_zero(lib):
+    """beta = 0 leaves only the decay: S_t = Diag(gamma_t) S0 with gamma_t the product of
+    the clamped decays, so dq_t = scale gamma_t * (S0 do_t), dS0 = sum_t scale (gamma_t * q_t)
+    do_t^T + Diag(gamma_T) dS_final, and dk = dv = 0."""
+    rng = np.random.default_rng(93)
+    x = make_inputs(11, H=2, dk=4, dv=3, dtype=torch.float32, seed=93, state_std=0.5)
+    beta = torch.zeros_like(x.beta)
+    do = rng.standard_normal((11, 2, 3))
+    dS = rng.standard_normal((1, 2, 4, 3))
+    sc = 0.7
+    got = ko.backward(x.q, x.k, x.v, x.g, beta, d_out=do, d_final=dS,
+                      initial_state=x.initial_state, scale=sc, lib=lib)
+    G = np.exp(np.cumsum(np.maximum(ko._widen(x.g), -1.0), axis=0))  # [T, H, dk]
+    Q = ko._widen(x.q)
+    S0 = x.initial_state.double().numpy()[0]
+    for h in range(2):
+        dq = sc * G[:, h, :] * (do[:, h, :] @ S0[h].T)
+        ds0 = sc * (G[:, h, :] * Q[:, h, :]).T @ do[:, h, :] + G[-1, h, :, None] * dS[0, h]
+        assert np.allclose(got["dq"][:, h], dq, rtol=1e-12, atol=1e-14)
+        assert np.allclose(got["ds0"][0, h], ds0, rtol=1e-12, atol=1e-14)
+    assert np.all(got["dk"] == 0.0) and np.all(got["dv"] == 0.0)
+
+
 ALL_PINS = [pin_golden, pin_chunked_agreement, pin_beta_zero_pure_decay, pin_delta_rule_reach,
             pin_general_beta_reach, pin_associative_memory, pin_one_token_expansion,
             pin_linearity, pin_contraction_bound, pin_resume_and_varlen, pin_decay_clamp,
             pin_sampled_rows, pin_snapshots_are_prefix_states, pin_prologue_l2norm,
-            pin_prologue_gate]
+            pin_prologue_gate, pin_backward_finite_differences, pin_backward_beta_zero]
 
 
 def failing_pins(lib_path: str) -> list[str]:

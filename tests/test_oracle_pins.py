@@ -58,6 +58,14 @@ MUTANTS = {
     "l2norm_keys_only": ("qt[i] /= nq;", ";"),
     "gate_sign": ("gi = J->lb / (1.0 + exp(-gi));", "gi = J->lb / (1.0 + exp(gi));"),
     "gate_without_bound": ("gi = J->lb / (1.0 + exp(-gi));", "gi = -1.0 / (1.0 + exp(-gi));"),
+    "bwd_clamp_mask_dropped": ("J->dg[tk + i] = graw[i] >= J->lb ? dgp[i] : 0.0;",
+                               "J->dg[tk + i] = dgp[i];"),
+    "bwd_dw_sign": ("dw[j] = -b * du[j];", "dw[j] = b * du[j];"),
+    "bwd_state_grad_not_decayed": ("for (int j = 0; j < dv; ++j) dS[i * dv + j] *= decay[i];",
+                                   ";"),
+    "bwd_dq_from_decayed_prev_state": ("a += S[i * dv + j] * dov[j];",
+                                       "a += Sb[i * dv + j] * dov[j];"),
+    "bwd_dbeta_without_recall": ("db += du[j] * (vt[j] - w[j]);", "db += du[j] * vt[j];"),
 }
 
 
