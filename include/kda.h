@@ -160,6 +160,40 @@ kda_status kda_chunk_fwd_snapshots(const void *q, const void *k, const void *v, 
 int64_t kda_snapshot_count(const kda_shape *shape, int32_t snapshot_chunks);
 
 /*
+ * Bytes of device scratch kda_chunk_bwd needs for this shape (a pure function of the
+ * shape fields). Returns 0 for an invalid shape or a shape the backward does not
+ * support (a nonzero prologue).
+ */
+size_t kda_chunk_bwd_workspace_size(const kda_shape *shape);
+
+/*
+ * Gradients of kda_chunk_fwd for training: given dL/dout and dL/dfinal_state of a scalar
+ * loss L, writes dL/dq, dL/dk, dL/dv, dL/dg, dL/dbeta and dL/dinitial_state. It is the
+ * reverse of the chunk-parallel form with its inter-chunk recurrence ("Kimi K3 深度拆解",
+ * section 4.2), walked from the last chunk back; the state at every chunk start comes
+ * from a forward pass with per-chunk snapshots that this call runs first.
+ *
+ *  q, k, v, g, beta, initial_state, cu_seqlens, shape: as in kda_chunk_fwd (the same
+ *               forward inputs). shape->prologue must be 0 (KDA_ERR_UNSUPPORTED).
+ *  d_out        [B*T, H, dv] dtype, or NULL for zeros
+ *  d_final_state[n, H, dk, dv] fp32, or NULL for zeros
+ *  dq, dk, dg   [B*T, H, dk] dtype (written)     dv [B*T, H, dv] dtype (written)
+ *  dbeta        [B*T, H] dtype (written)
+ *  d_initial_state [n, H, dk, dv] fp32 (written), or NULL to skip
+ *  workspace    >= kda_chunk_bwd_workspace_size(shape) bytes, 256-byte aligned.
+ * g enters through max(g, lb): where g < lb its gradient is 0 (at g == lb it passes).
+ * Computed in fp32 on CUDA cores (one CTA per sequence, head and 32-column slice of dv);
+ * dq, dk, dg and dbeta sum the slices' contributions with fp32 atomics, so their last
+ * bits may differ between runs. Errors as in kda_chunk_fwd.
+ */
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
+                         const void *beta, const float *initial_state,
+                         const int32_t *cu_seqlens, const void *d_out,
+                         const float *d_final_state, void *dq, void *dk, void *dv, void *dg,
+                         void *dbeta, float *d_initial_state, const kda_shape *shape,
+                         void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd without a workspace argument, for callers that cannot call
  * cudaMalloc: code running while a CUDA graph is being captured (allocation is
  * not capturable), plugin hosts that hand a library no scratch buffer, and

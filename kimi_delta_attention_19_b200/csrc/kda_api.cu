@@ -160,6 +160,117 @@ kda_status kda_chunk_fwd_snapshots(const void* q, const void* k, const void* v, 
                    stream);
 }
 
+}  // extern "C"
+
+namespace kda {
+namespace {
+
+// Backward workspace: [forward workspace (status word first) | per-chunk snapshots |
+// forward output scratch | fp32 accumulators dq, dk, dg, dbeta], each 256-byte aligned.
+struct BwdPlan {
+  size_t fwd, snaps, out, acc_q, acc_k, acc_g, acc_b, total;
+  int64_t n_snaps;
+};
+
+bool bwd_plan(const kda_shape* shape, BwdPlan& p) {
+  if (check_shape(shape, true) != KDA_OK || shape->prologue != 0) return false;
+  const size_t fwd = kda_chunk_fwd_workspace_size(shape);
+  if (fwd == 0) return false;
+  int64_t T_total, max_len;
+  int n_seqs;
+  resolve(*shape, T_total, n_seqs, max_len);
+  const size_t elem = shape->dtype == KDA_F32 ? 4 : 2;
+  const size_t th = static_cast<size_t>(T_total) * shape->H;
+  p.n_snaps = T_total / kChunk;
+  p.fwd = 0;
+  p.snaps = align_up(fwd, 256);
+  p.out = align_up(p.snaps + static_cast<size_t>(p.n_snaps) * shape->H * shape->dk * shape->dv * 4, 256);
+  p.acc_q = align_up(p.out + th * shape->dv * elem, 256);
+  p.acc_k = p.acc_q + align_up(th * shape->dk * 4, 256);
+  p.acc_g = p.acc_k + align_up(th * shape->dk * 4, 256);
+  p.acc_b = p.acc_g + align_up(th * shape->dk * 4, 256);
+  p.total = p.acc_b + align_up(th * 4, 256);
+  return true;
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" {
+
+size_t kda_chunk_bwd_workspace_size(const kda_shape* shape) {
+  BwdPlan p;
+  return bwd_plan(shape, p) ? p.total : 0;
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* initial_state,
+                         const int32_t* cu_seqlens, const void* d_out,
+                         const float* d_final_state, void* dq, void* dk, void* dv, void* dg,
+                         void* dbeta, float* d_initial_state, const kda_shape* shape,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_shape(shape, true);
+  if (st != KDA_OK) return st;
+  if (shape->prologue != 0) return KDA_ERR_UNSUPPORTED;
+  const kda_shape& s = *shape;
+  if ((cu_seqlens != nullptr) != (s.n_seqs > 0)) return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens != nullptr && s.B != 1) return KDA_ERR_INVALID_ARG;
+  if (s.n_seqs < 0 || s.max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+  int n_seqs;
+  int64_t T_total, max_len;
+  resolve(s, T_total, n_seqs, max_len);
+  const void* tensors[] = {q, k, v, g, beta, dq, dk, dv, dg, dbeta};
+  for (const void* p : tensors) {
+    if (T_total > 0 && p == nullptr) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(initial_state) || !aligned16(d_out) || !aligned16(d_final_state) ||
+      !aligned16(d_initial_state) || !aligned16(cu_seqlens))
+    return KDA_ERR_INVALID_ARG;
+  BwdPlan p;
+  if (!bwd_plan(shape, p)) return KDA_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < p.total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return KDA_ERR_INVALID_ARG;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  // forward pass keeping the state after every chunk (its outputs go to scratch)
+  float* snaps = reinterpret_cast<float*>(ws + p.snaps);
+  st = chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, ws + p.out, nullptr, 1, snaps,
+                 p.n_snaps, shape, ws, p.snaps, stream);
+  if (st != KDA_OK) return st;
+  if (cudaMemsetAsync(ws + p.acc_q, 0, p.total - p.acc_q, cs) != cudaSuccess) return KDA_ERR_CUDA;
+
+  BackwardArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+  a.dout = d_out;
+  a.s0 = initial_state;
+  a.dsT = d_final_state;
+  a.snap = snaps;
+  a.cu = cu_seqlens;
+  a.acc_q = reinterpret_cast<float*>(ws + p.acc_q);
+  a.acc_k = reinterpret_cast<float*>(ws + p.acc_k);
+  a.acc_g = reinterpret_cast<float*>(ws + p.acc_g);
+  a.acc_b = reinterpret_cast<float*>(ws + p.acc_b);
+  a.dv_out = dv;
+  a.ds0 = d_initial_state;
+  a.status = static_cast<int32_t*>(workspace);
+  a.T = s.T;
+  a.T_total = T_total;
+  a.n_seqs = n_seqs;
+  a.H = s.H; a.dk = s.dk; a.dv = s.dv;
+  a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
+  a.lb = s.g_lower_bound;
+  cudaError_t e = launch_backward(a, s.dtype, cs);
+  const int64_t nk = T_total * s.H * s.dk, nb = T_total * s.H;
+  if (e == cudaSuccess) e = launch_backward_convert(a.acc_q, dq, nk, s.dtype, cs);
+  if (e == cudaSuccess) e = launch_backward_convert(a.acc_k, dk, nk, s.dtype, cs);
+  if (e == cudaSuccess) e = launch_backward_convert(a.acc_g, dg, nk, s.dtype, cs);
+  if (e == cudaSuccess) e = launch_backward_convert(a.acc_b, dbeta, nb, s.dtype, cs);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int64_t kda_snapshot_count(const kda_shape* shape, int32_t snapshot_chunks) {
   if (snapshot_chunks < 1 || kda_chunk_fwd_workspace_size(shape) == 0) return -1;
   int64_t T_total, max_len;

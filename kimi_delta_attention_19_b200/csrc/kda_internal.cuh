@@ -60,10 +60,37 @@ struct DecodeArgs {
   int prologue;             // KDA_PROLOGUE_* flags
 };
 
+// Everything the backward launch needs, resolved on the host.
+struct BackwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* beta;
+  const void* dout;         // dL/dout [T_total, H, dv] or null (zeros)
+  const float* s0;          // [n, H, dk, dv] or null
+  const float* dsT;         // dL/dS_final [n, H, dk, dv] or null (zeros)
+  const float* snap;        // state after every full chunk: [floor(T_total / C), H, dk, dv]
+  const int32_t* cu;        // [n+1] or null
+  float* acc_q;             // fp32 accumulators of the d_v slices' contributions:
+  float* acc_k;             //   dq, dk, dg [T_total, H, dk]
+  float* acc_g;
+  float* acc_b;             //   dbeta [T_total, H]
+  void* dv_out;             // dL/dv [T_total, H, dv] (dtype)
+  float* ds0;               // dL/dS0 [n, H, dk, dv] or null
+  int32_t* status;          // device status word
+  int64_t T;
+  int64_t T_total;
+  int n_seqs;
+  int H, dk, dv;
+  float scale;
+  float lb;
+};
+
 // Sequence bounds [t0, t1) of sequence s; false (and status set) when the
 // device-visible cu_seqlens entry is malformed.
-__device__ __forceinline__ bool seq_bounds(const PrefillArgs& a, int s, int64_t& t0,
-                                           int64_t& t1) {
+template <typename Args>
+__device__ __forceinline__ bool seq_bounds(const Args& a, int s, int64_t& t0, int64_t& t1) {
   if (a.cu == nullptr) {
     t0 = (int64_t)s * a.T;
     t1 = t0 + a.T;
@@ -126,5 +153,8 @@ bool tc_path_applies(const kda_shape& s, int64_t T_total);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, kda_dtype dtype, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t st);
+cudaError_t launch_backward(const BackwardArgs& a, kda_dtype dtype, cudaStream_t st);
+cudaError_t launch_backward_convert(const float* acc, void* out, int64_t n, kda_dtype dtype,
+                                    cudaStream_t st);
 
 }  // namespace kda

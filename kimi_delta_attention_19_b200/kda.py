@@ -50,6 +50,11 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd_snapshots.restype = st
     L.kda_chunk_fwd_snapshots.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.c_int32, p,
                                           ctypes.c_int64, ctypes.POINTER(Shape), p, sz, p]
+    L.kda_chunk_bwd_workspace_size.restype = sz
+    L.kda_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
+    L.kda_chunk_bwd.restype = st
+    L.kda_chunk_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, p, p, p, p, p,
+                                ctypes.POINTER(Shape), p, sz, p]
     L.kda_snapshot_count.restype = ctypes.c_int64
     L.kda_snapshot_count.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32]
     L.kda_chunk_fwd_noalloc.restype = st
@@ -69,7 +74,8 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
-            "kda_chunk_fwd_snapshots", "kda_snapshot_count", "kda_decode_step",
+            "kda_chunk_fwd_snapshots", "kda_snapshot_count", "kda_chunk_bwd_workspace_size",
+            "kda_chunk_bwd", "kda_decode_step",
             "kda_workspace_status", "kda_status_string", "kda_version")
 
 
@@ -200,6 +206,40 @@ def chunk_fwd_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: to
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd_snapshots")
     return out, final_state, snapshots
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+              beta: torch.Tensor, d_out: torch.Tensor | None, *,
+              d_final_state: torch.Tensor | None = None,
+              initial_state: torch.Tensor | None = None,
+              cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+              scale: float | None = None, lb: float = -1.0, want_d_initial: bool = True,
+              workspace: torch.Tensor | None = None, stream=None):
+    """Gradients of chunk_fwd: (dq, dk, dv, dg, dbeta, d_initial_state).
+
+    Same layouts as chunk_fwd; d_out like out, d_final_state like final_state (fp32).
+    d_initial_state is fp32 [n, H, dk, dv] (None unless want_d_initial).
+    """
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    H, dk, dv_ = shape.H, shape.dk, shape.dv
+    dq, dkk, dg = (torch.empty_like(q) for _ in range(3))
+    dvv = torch.empty_like(v)
+    dbeta = torch.empty_like(beta)
+    ds0 = (torch.empty(n, H, dk, dv_, dtype=torch.float32, device=q.device)
+           if want_d_initial else None)
+    if workspace is None:
+        nbytes = int(lib.kda_chunk_bwd_workspace_size(ctypes.byref(shape)))
+        if nbytes == 0:
+            raise KdaError(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    rc = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                           _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_out),
+                           _ptr(d_final_state), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg),
+                           _ptr(dbeta), _ptr(ds0), ctypes.byref(shape), _ptr(workspace),
+                           workspace.numel(), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_bwd")
+    return dq, dkk, dvv, dg, dbeta, ds0
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
