@@ -48,17 +48,37 @@ struct BwdSmem {
   float dO[C][DVS + 1];
   float dU[C][DVS + 1];
   float gl[DK];
+  float sdS[DK];         // sum_j S[i][j] dS'[i][j]: the decay of S's part of dgl
   float bet[C];
   float dbet[C];
-  float part[NT / DK][DK];  // per row group: dgl parts, then suffix totals of dGamma
 };
+static_assert(2 * 16 * 128 <= C * (C + 1), "row-group scans fit in the N buffer");
+
+// A 16-byte vector of inputs as floats
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint4& u, float (&f)[16 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void unpack_vec<float>(const uint4& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+template <>
+__device__ __forceinline__ void unpack_vec<__nv_bfloat16>(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
 
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem<DK>& sm = *reinterpret_cast<BwdSmem<DK>*>(smem_raw);
-  constexpr int RG = NT / DK;   // row groups in the per-element pass
-  constexpr int RPT = C / RG;   // rows per thread there
+  constexpr int CT = DK / 16;   // channels per thread in the per-element pass
   const int n_slices = a.dv / DVS;
   const int slice = blockIdx.x % n_slices;
   const int h = (blockIdx.x / n_slices) % a.H;
@@ -87,50 +107,110 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 
   const int64_t n_chunks = (t1 - t0 + C - 1) / C;
   const int64_t snap0 = t0 / C;  // snapshot index of this sequence's first chunk end
-  const int r4 = tid / 4, cb = (tid % 4) * 8;  // (row, 8-column group) of C x DVS tiles
-  const int tx = tid % 16, ty = tid / 16;      // 4x4 blocks of C x C tiles
+  const int rcr = 2 * (tid >> 3), rcc = tid & 7;  // C x DVS tiles: rows rcr, rcr + 1;
+                                                  // columns rcc + 8 x
+  const int tx = tid % 16, ty = tid / 16;         // 4x4 blocks of C x C tiles
 
   for (int64_t cc = n_chunks - 1; cc >= 0; --cc) {
     const int64_t c0 = t0 + cc * C;
     const int L = (t1 - c0) < C ? (int)(t1 - c0) : C;
     __syncthreads();  // the previous chunk's reads are done
 
-    // ---- 0. decay tiles (threads < DK, one channel each); the slice's S, V, dO and beta
-    if (tid < DK) {
-      const int i = tid;
-      float G = 0.f;
-      for (int r = 0; r < C; ++r) {
-        float kt = 0.f, kh = 0.f, qt = 0.f;
-        if (r < L) {
-          const int64_t off = ((c0 + r) * H + h) * DK + i;
-          G += fmaxf(ld_in(g + off), lb);
-          const float e = expf(G), ei = expf(-G);
-          const float kv = ld_in(k + off);
-          kt = kv * e;
-          kh = kv * ei;
-          qt = ld_in(q + off) * e;
-        }
-        sm.Kt[r][i] = kt;
-        sm.Kh[r][i] = kh;
-        sm.Qt[r][i] = qt;
+    // ---- 0. stage the chunk's raw k, q and clamped g (all threads, coalesced; rows past L
+    //         are zero: no key, no decay) and the slice's S, V, dO and beta; then the decay
+    //         tiles in place, one channel per thread
+    {
+      // k, q, g rows: 16-byte vectors, all of a thread's loads issued before any store
+      constexpr int EV = 16 / sizeof(Tin);        // elements per vector
+      constexpr int VR = DK / EV;                 // vectors per row
+      constexpr int NV = C * VR / NT;             // vectors per thread per tensor
+      uint4 kq[NV], qq[NV], gq[NV];
+#pragma unroll
+      for (int m = 0; m < NV; ++m) {
+        const int e = tid + NT * m, r = e / VR, vi = e % VR;
+        const int64_t off = ((c0 + r) * H + h) * DK + vi * EV;
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        kq[m] = r < L ? *reinterpret_cast<const uint4*>(k + off) : z;
+        qq[m] = r < L ? *reinterpret_cast<const uint4*>(q + off) : z;
+        gq[m] = r < L ? *reinterpret_cast<const uint4*>(g + off) : z;
       }
-      sm.gl[i] = expf(G);
-    } else {
+      // the slice's S (fp32 rows of DVS), V and dO rows (DVS elements), beta
+      constexpr int SV = DVS / 4, NS = DK * SV / NT;          // S: float4 vectors
+      constexpr int OV = DVS / EV, NO = (C * OV + NT - 1) / NT; // V, dO vectors
       const float* src = nullptr;
       if (cc > 0) src = a.snap + ((snap0 + cc - 1) * H + h) * (int64_t)DK * DV + j0;
       else if (a.s0) src = a.s0 + state_base;
-      for (int e = tid - DK; e < DK * DVS; e += NT - DK) {
-        const int i = e / DVS, c = e % DVS;
-        sm.S[i][c] = src ? src[(int64_t)i * DV + c] : 0.f;
+      float4 sq[NS];
+#pragma unroll
+      for (int m = 0; m < NS; ++m) {
+        const int e = tid + NT * m, i = e / SV, vj = e % SV;
+        sq[m] = src ? *reinterpret_cast<const float4*>(src + (int64_t)i * DV + 4 * vj)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      for (int e = tid - DK; e < C * DVS; e += NT - DK) {
-        const int r = e / DVS, c = e % DVS;
-        const int64_t off = ((c0 + r) * H + h) * DV + j0 + c;
-        sm.Y[r][c] = r < L ? ld_in(v + off) : 0.f;
-        sm.dO[r][c] = (r < L && dout) ? ld_in(dout + off) : 0.f;
+      uint4 vq[NO], oq[NO];
+#pragma unroll
+      for (int m = 0; m < NO; ++m) {
+        const int e = tid + NT * m, r = e / OV, vj = e % OV;
+        const int64_t off = ((c0 + r) * H + h) * DV + j0 + vj * EV;
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const bool in = e < C * OV && r < L;
+        vq[m] = in ? *reinterpret_cast<const uint4*>(v + off) : z;
+        oq[m] = (in && dout) ? *reinterpret_cast<const uint4*>(dout + off) : z;
       }
-      for (int r = tid - DK; r < C; r += NT - DK)
-        sm.bet[r] = r < L ? ld_in(beta + (c0 + r) * H + h) : 0.f;
+      if (tid < C) sm.bet[tid] = tid < L ? ld_in(beta + (c0 + tid) * H + h) : 0.f;
+      // unpack into shared memory (raw k -> Kt, raw q -> Qt, clamped g -> Kh; rows past
+      // L are zero: no key, no decay)
+#pragma unroll
+      for (int m = 0; m < NV; ++m) {
+        const int e = tid + NT * m, r = e / VR, i0 = (e % VR) * EV;
+        float kf[EV], qf[EV], gf[EV];
+        unpack_vec<Tin>(kq[m], kf);
+        unpack_vec<Tin>(qq[m], qf);
+        unpack_vec<Tin>(gq[m], gf);
+#pragma unroll
+        for (int x = 0; x < EV; ++x) {
+          sm.Kt[r][i0 + x] = kf[x];
+          sm.Qt[r][i0 + x] = qf[x];
+          sm.Kh[r][i0 + x] = r < L ? fmaxf(gf[x], lb) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NS; ++m) {
+        const int e = tid + NT * m, i = e / SV, j = 4 * (e % SV);
+        sm.S[i][j] = sq[m].x;
+        sm.S[i][j + 1] = sq[m].y;
+        sm.S[i][j + 2] = sq[m].z;
+        sm.S[i][j + 3] = sq[m].w;
+      }
+#pragma unroll
+      for (int m = 0; m < NO; ++m) {
+        const int e = tid + NT * m, r = e / OV, j = (e % OV) * EV;
+        if (e < C * OV) {
+          float vf[EV], of[EV];
+          unpack_vec<Tin>(vq[m], vf);
+          unpack_vec<Tin>(oq[m], of);
+#pragma unroll
+          for (int x = 0; x < EV; ++x) {
+            sm.Y[r][j + x] = vf[x];
+            sm.dO[r][j + x] = of[x];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < DK) {
+      const int i = tid;
+      float G = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < C; ++r) {
+        G += sm.Kh[r][i];
+        const float e = expf(G), ei = expf(-G);
+        const float kv = sm.Kt[r][i];
+        sm.Kt[r][i] = kv * e;
+        sm.Kh[r][i] = kv * ei;
+        sm.Qt[r][i] *= e;
+      }
+      sm.gl[i] = expf(G);
     }
     __syncthreads();
 
@@ -168,76 +248,148 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     }
     __syncthreads();
 
-    // ---- 2. N = (I + A)^-1 by forward substitution, one row at a time (rows past L:
-    //         A is zero there, so N is the identity)
-    if (tid < C) {
-      for (int r = L; r < C; ++r) sm.BN[r][tid] = (r == tid) ? 1.f : 0.f;
+    // ---- 2. N = (I + A)^-1 (lower triangular): the four 16x16 diagonal blocks by forward
+    //         substitution, one per half-warp; then 16 -> 32 and 32 -> 64 merges
+    //         N21 = -N22 (A21 N11), each product by all threads. A21 is overwritten by
+    //         A21 N11 (A is not needed afterwards); the upper blocks of N stay zero.
+    for (int e = tid; e < C * C; e += NT) {
+      const int r = e / C, c = e % C;
+      if ((r >> 4) != (c >> 4)) sm.BN[r][c] = 0.f;
     }
-    for (int r = 0; r < L; ++r) {
-      if (tid < C) {
-        const int c = tid;
+    if (tid < 64) {
+      const int base = 16 * (tid >> 4), c = tid & 15;
+      for (int r = 0; r < 16; ++r) {
         float val = (c == r) ? 1.f : 0.f;
-        for (int s2 = c; s2 < r; ++s2) val = fmaf(-sm.BA[r][s2], sm.BN[s2][c], val);
-        sm.BN[r][c] = (c <= r) ? val : 0.f;
+        for (int s2 = c; s2 < r; ++s2)
+          val = fmaf(-sm.BA[base + r][base + s2], sm.BN[base + s2][base + c], val);
+        sm.BN[base + r][base + c] = (c <= r) ? val : 0.f;
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    {  // 16 -> 32, both 32-blocks at once: thread -> block o = 32 (tid >> 7), two elements
+      const int o = 32 * (tid >> 7);
+      float xv[2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m, r = idx >> 4, c = idx & 15;
+        float acc = 0.f;
+        for (int s2 = c; s2 < 16; ++s2)
+          acc = fmaf(sm.BA[o + 16 + r][o + s2], sm.BN[o + s2][o + c], acc);
+        xv[m] = acc;
       }
       __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m;
+        sm.BA[o + 16 + (idx >> 4)][o + (idx & 15)] = xv[m];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m, r = idx >> 4, c = idx & 15;
+        float acc = 0.f;
+        for (int s2 = 0; s2 <= r; ++s2)
+          acc = fmaf(sm.BN[o + 16 + r][o + 16 + s2], sm.BA[o + 16 + s2][o + c], acc);
+        sm.BN[o + 16 + r][o + c] = -acc;
+      }
     }
+    __syncthreads();
+    {  // 32 -> 64: four elements per thread
+      float xv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m, r = idx >> 5, c = idx & 31;
+        float acc = 0.f;
+        for (int s2 = c; s2 < 32; ++s2) acc = fmaf(sm.BA[32 + r][s2], sm.BN[s2][c], acc);
+        xv[m] = acc;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m;
+        sm.BA[32 + (idx >> 5)][idx & 31] = xv[m];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m, r = idx >> 5, c = idx & 31;
+        float acc = 0.f;
+        for (int s2 = 0; s2 <= r; ++s2) acc = fmaf(sm.BN[32 + r][32 + s2], sm.BA[32 + s2][c], acc);
+        sm.BN[32 + r][c] = -acc;
+      }
+    }
+    __syncthreads();
 
-    // ---- 3. Y = V - K~ S, then U = N Diag(beta) Y
+    // ---- 3. Y = V - K~ S, then U = N Diag(beta) Y            (C x DVS tiles, 2 x 4)
     {
-      float acc[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+      float acc[2][4] = {};
       for (int i = 0; i < DK; ++i) {
-        const float kt = sm.Kt[r4][i];
+        const float k0 = sm.Kt[rcr][i], k1 = sm.Kt[rcr + 1][i];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(kt, sm.S[i][cb + c], acc[c]);
+        for (int x = 0; x < 4; ++x) {
+          const float sv = sm.S[i][rcc + 8 * x];
+          acc[0][x] = fmaf(k0, sv, acc[0][x]);
+          acc[1][x] = fmaf(k1, sv, acc[1][x]);
+        }
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) sm.Y[r4][cb + c] -= acc[c];
+      for (int y = 0; y < 2; ++y)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sm.Y[rcr + y][rcc + 8 * x] -= acc[y][x];
     }
     __syncthreads();
     {
-      float acc[8];
+      float acc[2][4] = {};
+      for (int s2 = 0; s2 <= rcr + 1; ++s2) {  // N is lower triangular
+        const float b = sm.bet[s2];
+        const float n0 = sm.BN[rcr][s2] * b, n1 = sm.BN[rcr + 1][s2] * b;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-      for (int s2 = 0; s2 <= r4; ++s2) {
-        const float t = sm.BN[r4][s2] * sm.bet[s2];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(t, sm.Y[s2][cb + c], acc[c]);
+        for (int x = 0; x < 4; ++x) {
+          const float yv = sm.Y[s2][rcc + 8 * x];
+          acc[0][x] = fmaf(n0, yv, acc[0][x]);
+          acc[1][x] = fmaf(n1, yv, acc[1][x]);
+        }
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) sm.U[r4][cb + c] = acc[c];
+      for (int y = 0; y < 2; ++y)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sm.U[rcr + y][rcc + 8 * x] = acc[y][x];
     }
     __syncthreads();
 
     // ---- 4. dU = (K^ gl) dS' + scale P^T dO
     {
-      float acc[8], acc2[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = acc2[c] = 0.f;
+      float acc[2][4] = {}, acc2[2][4] = {};
       for (int i = 0; i < DK; ++i) {
-        const float kb = sm.Kh[r4][i] * sm.gl[i];
+        const float gi = sm.gl[i];
+        const float k0 = sm.Kh[rcr][i] * gi, k1 = sm.Kh[rcr + 1][i] * gi;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(kb, sm.dS[i][cb + c], acc[c]);
+        for (int x = 0; x < 4; ++x) {
+          const float dv0 = sm.dS[i][rcc + 8 * x];
+          acc[0][x] = fmaf(k0, dv0, acc[0][x]);
+          acc[1][x] = fmaf(k1, dv0, acc[1][x]);
+        }
       }
-      for (int t = r4; t < C; ++t) {
-        const float p = sm.BP[t][r4];
+      for (int t = rcr; t < C; ++t) {  // P[t][r] = 0 for t < r
+        const float p0 = sm.BP[t][rcr], p1 = sm.BP[t][rcr + 1];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc2[c] = fmaf(p, sm.dO[t][cb + c], acc2[c]);
+        for (int x = 0; x < 4; ++x) {
+          const float o = sm.dO[t][rcc + 8 * x];
+          acc2[0][x] = fmaf(p0, o, acc2[0][x]);
+          acc2[1][x] = fmaf(p1, o, acc2[1][x]);
+        }
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) sm.dU[r4][cb + c] = fmaf(scale, acc2[c], acc[c]);
+      for (int y = 0; y < 2; ++y)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sm.dU[rcr + y][rcc + 8 * x] = fmaf(scale, acc2[y][x], acc[y][x]);
     }
     __syncthreads();
 
-    // ---- 5. dT = dU Y^T (over P, which is dead)
+    // ---- 5. dT = dU Y^T (over P, which is dead)                 (C x C tiles, 4 x 4)
     {
-      float acc[4][4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+      float acc[4][4] = {};
       for (int j = 0; j < DVS; ++j) {
         float du[4], yy[4];
 #pragma unroll
@@ -254,26 +406,39 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
       for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) sm.BP[ty * 4 + x][tx * 4 + y] = acc[x][y];
+      // sum_j S[i][j] dS'[i][j], NT / DK threads per channel
+      constexpr int TPR = NT / DK, JPT = DVS / TPR;
+      const int i = tid / TPR, j0p = (tid % TPR) * JPT;
+      float sd = 0.f;
+#pragma unroll
+      for (int j = 0; j < JPT; ++j) sd = fmaf(sm.S[i][j0p + j], sm.dS[i][j0p + j], sd);
+#pragma unroll
+      for (int o2 = 1; o2 < TPR; o2 <<= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o2);
+      if (tid % TPR == 0) sm.sdS[i] = sd;
     }
     __syncthreads();
 
     // ---- 6. Z = Diag(beta) N^T dU (= dL/dV, over Y); dbeta from T = N Diag(beta)
     {
-      float acc[8];
+      float acc[2][4] = {};
+      for (int t = rcr; t < C; ++t) {  // N[t][r] = 0 for t < r
+        const float n0 = sm.BN[t][rcr], n1 = sm.BN[t][rcr + 1];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-      for (int t = r4; t < C; ++t) {
-        const float nv = sm.BN[t][r4];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(nv, sm.dU[t][cb + c], acc[c]);
+        for (int x = 0; x < 4; ++x) {
+          const float d = sm.dU[t][rcc + 8 * x];
+          acc[0][x] = fmaf(n0, d, acc[0][x]);
+          acc[1][x] = fmaf(n1, d, acc[1][x]);
+        }
       }
-      const float b = sm.bet[r4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) sm.Y[r4][cb + c] = b * acc[c];
-      if (r4 < L) {
-        Tin* o = dvo + ((c0 + r4) * H + h) * DV + j0 + cb;
+      for (int y = 0; y < 2; ++y) {
+        const int r = rcr + y;
+        const float b = sm.bet[r];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) st_out(o + c, b * acc[c]);
+        for (int x = 0; x < 4; ++x) {
+          sm.Y[r][rcc + 8 * x] = b * acc[y][x];
+          if (r < L) st_out(dvo + ((c0 + r) * H + h) * DV + j0 + rcc + 8 * x, b * acc[y][x]);
+        }
       }
       if (tid < C) {
         const int r = tid;
@@ -291,11 +456,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     }
     __syncthreads();
     {
-      float acc[4][4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+      float acc[4][4] = {};
       for (int c = 0; c < C; ++c) {  // (N^T dN)[r][s] = sum_c N[c][r] dN[c][s]
         float nv[4], dn[4];
 #pragma unroll
@@ -315,11 +476,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     }
     __syncthreads();
     {
-      float acc[4][4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+      float acc[4][4] = {};
       for (int c = 0; c < C; ++c) {  // dA[r][s] = -sum_c (N^T dN)[r][c] N[s][c]
         float tv[4], nv[4];
 #pragma unroll
@@ -342,11 +499,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     // ---- 8. dG = strict_lower(Diag(beta) dA) in place, with dbeta += sum_s G dA (G = K~ K^^T
     //         recomputed); dP = scale lower_incl(dO U^T) over (N^T dN)
     {
-      float accG[4][4], accP[4][4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) accG[x][y] = accP[x][y] = 0.f;
+      float accG[4][4] = {}, accP[4][4] = {};
       for (int i = 0; i < DK; ++i) {
         float kt[4], kh[4];
 #pragma unroll
@@ -390,92 +543,241 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     __syncthreads();
     if (tid < L) atomicAdd(a.acc_b + (c0 + tid) * H + h, sm.dbet[tid]);
 
-    // ---- 9. per (row group, channel i): dQ~, dK~, dK^ -> dq, dk; dGamma -> dg
+    // ---- 9. per element of the C x DK tiles (4 rows x CT channels per thread): dQ~, dK~,
+    //         dK^ -> dq, dk; dGamma -> dg. N is dead: its buffer holds the row-group scans.
     {
-      const int i = tid % DK, rg = tid / DK, rb = rg * RPT;
-      float E[RPT], dgam[RPT], dkk[RPT];
-      uint32_t live = 0;  // bit rr: g >= lb (the clamp passes the gradient)
-      {
+      float* scan = &sm.BN[0][0];           // [16][DK]: prefix / suffix totals per row group
+      float* dglp_all = scan + 16 * DK;     // [16][DK]: dgl parts per row group
+      const int rg = tid >> 4, cg = tid & 15, rb = 4 * rg;
+      // 9a. Gamma of the thread's rows: its rows' clamped decay sums, then the earlier groups'
+      float gsum[CT] = {}, graw[4][CT];
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) {
+          const int r = rb + y, c = cg + 16 * x;
+          graw[y][x] = r < L ? ld_in(g + ((c0 + r) * H + h) * DK + c) : 0.f;
+          gsum[x] += r < L ? fmaxf(graw[y][x], lb) : 0.f;
+        }
+#pragma unroll
+      for (int x = 0; x < CT; ++x) scan[rg * DK + cg + 16 * x] = gsum[x];
+      __syncthreads();
+      float E[4][CT];
+      uint32_t live = 0;  // bit y * CT + x: g >= lb (the clamp passes the gradient)
+#pragma unroll
+      for (int x = 0; x < CT; ++x) {
         float G = 0.f;
-        for (int r = 0; r < rb + RPT; ++r) {
-          float gr = 0.f;
-          if (r < L) gr = ld_in(g + ((c0 + r) * H + h) * DK + i);
-          G += r < L ? fmaxf(gr, lb) : 0.f;
-          if (r >= rb) {
-            E[r - rb] = expf(G);
-            if (gr >= lb) live |= 1u << (r - rb);
-          }
+        for (int q2 = 0; q2 < rg; ++q2) G += scan[q2 * DK + cg + 16 * x];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          G += rb + y < L ? fmaxf(graw[y][x], lb) : 0.f;
+          E[y][x] = expf(G);
+          if (graw[y][x] >= lb) live |= 1u << (y * CT + x);
         }
       }
-      const float gli = sm.gl[i];
-      float dglp = 0.f;
-#pragma unroll 1
-      for (int rr = 0; rr < RPT; ++rr) {
-        const int r = rb + rr;
-        // dQ~ = scale dO S^T + dP K^
-        float a1 = 0.f, a2 = 0.f;
-        for (int j = 0; j < DVS; ++j) a1 = fmaf(sm.dO[r][j], sm.S[i][j], a1);
-        for (int t = 0; t <= r; ++t) a2 = fmaf(sm.BA[r][t], sm.Kh[t][i], a2);
-        const float dqt = fmaf(scale, a1, a2);
-        // dK~ = -Z S^T + dG K^
-        float b1 = 0.f, b2 = 0.f;
-        for (int j = 0; j < DVS; ++j) b1 = fmaf(sm.Y[r][j], sm.S[i][j], b1);
-        for (int t = 0; t < r; ++t) b2 = fmaf(sm.BP[r][t], sm.Kh[t][i], b2);
-        const float dkt = b2 - b1;
-        // dK^ = dP^T Q~ + dG^T K~ + (U dS'^T) gl
-        float c1 = 0.f, c2 = 0.f, dkb = 0.f;
-        for (int t = r; t < C; ++t) c1 = fmaf(sm.BA[t][r], sm.Qt[t][i], c1);
-        for (int t = r + 1; t < C; ++t) c2 = fmaf(sm.BP[t][r], sm.Kt[t][i], c2);
-        for (int j = 0; j < DVS; ++j) dkb = fmaf(sm.U[r][j], sm.dS[i][j], dkb);
-        const float dkh = c1 + c2 + dkb * gli;
-        const float kh = sm.Kh[r][i];
-        dglp = fmaf(kh, dkb, dglp);
-        dgam[rr] = dkt * sm.Kt[r][i] - dkh * kh + dqt * sm.Qt[r][i];
-        dkk[rr] = dkt * E[rr] + dkh / E[rr];
-        if (r < L) atomicAdd(a.acc_q + ((c0 + r) * H + h) * DK + i, dqt * E[rr]);
-      }
-      if (rg == 0) {
-        for (int j = 0; j < DVS; ++j) dglp = fmaf(sm.S[i][j], sm.dS[i][j], dglp);
-      }
-      sm.part[rg][i] = dglp;
-      __syncthreads();
-      float dgl = 0.f;
+      float dgam[4][CT], dkk[4][CT], acc[4][CT];
+      // 9b. dQ~ = scale dO S^T + dP K^  ->  dq, dGamma
 #pragma unroll
-      for (int q2 = 0; q2 < RG; ++q2) dgl += sm.part[q2][i];
-      // the end-of-chunk decay gl = E[L - 1] feeds the last live row's dGamma
-      if (L - 1 >= rb && L - 1 < rb + RPT) dgam[L - 1 - rb] = fmaf(dgl, gli, dgam[L - 1 - rb]);
-      // reverse cumulative sum over the live rows: local suffix sums, then the later groups
-      float suf = 0.f;
+      for (int y = 0; y < 4; ++y)
 #pragma unroll
-      for (int rr = RPT - 1; rr >= 0; --rr) {
-        if (rb + rr < L) suf += dgam[rr];
-        dgam[rr] = suf;
+        for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
+      for (int j = 0; j < DVS; ++j) {
+        float o[4], sv[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) o[y] = sm.dO[rb + y][j];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) sv[x] = sm.S[cg + 16 * x][j];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(o[y], sv[x], acc[y][x]);
       }
-      __syncthreads();  // every group has read part[] as dgl parts
-      sm.part[rg][i] = suf;
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) acc[y][x] *= scale;
+      for (int t = 0; t < rb + 4; ++t) {  // dP[r][t] = 0 for t > r
+        float p[4], kh[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) p[y] = sm.BA[rb + y][t];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) kh[x] = sm.Kh[t][cg + 16 * x];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(p[y], kh[x], acc[y][x]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) {
+          const int r = rb + y, c = cg + 16 * x;
+          dgam[y][x] = acc[y][x] * sm.Qt[r][c];
+          if (r < L) atomicAdd(a.acc_q + ((c0 + r) * H + h) * DK + c, acc[y][x] * E[y][x]);
+        }
+      // 9c. dK~ = -Z S^T + dG K^  ->  dk (first part), dGamma
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
+      for (int j = 0; j < DVS; ++j) {
+        float z[4], sv[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) z[y] = sm.Y[rb + y][j];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) sv[x] = sm.S[cg + 16 * x][j];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(-z[y], sv[x], acc[y][x]);
+      }
+      for (int t = 0; t < rb + 3; ++t) {  // dG[r][t] = 0 for t >= r
+        float dg4[4], kh[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) dg4[y] = sm.BP[rb + y][t];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) kh[x] = sm.Kh[t][cg + 16 * x];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(dg4[y], kh[x], acc[y][x]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) {
+          const int r = rb + y, c = cg + 16 * x;
+          dkk[y][x] = acc[y][x] * E[y][x];
+          dgam[y][x] = fmaf(acc[y][x], sm.Kt[r][c], dgam[y][x]);
+        }
+      // 9d. dK^ = (U dS'^T) gl + dP^T Q~ + dG^T K~  ->  dk, dGamma, dgl parts
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
+      for (int j = 0; j < DVS; ++j) {
+        float u[4], d[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) u[y] = sm.U[rb + y][j];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) d[x] = sm.dS[cg + 16 * x][j];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(u[y], d[x], acc[y][x]);
+      }
+      float dglp[CT];
+#pragma unroll
+      for (int x = 0; x < CT; ++x) {
+        const int c = cg + 16 * x;
+        const float gi = sm.gl[c];
+        float part = rg == 0 ? sm.sdS[c] : 0.f;  // the decay of S itself
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          part = fmaf(sm.Kh[rb + y][c], acc[y][x], part);  // K^ (U dS'^T)
+          acc[y][x] *= gi;
+        }
+        dglp[x] = part;
+      }
+      for (int t = rb; t < C; ++t) {  // dP[t][r] = 0 for t < r, dG[t][r] = 0 for t <= r
+        float p[4], dg4[4], qt[CT], kt[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          p[y] = sm.BA[t][rb + y];
+          dg4[y] = sm.BP[t][rb + y];
+        }
+#pragma unroll
+        for (int x = 0; x < CT; ++x) {
+          qt[x] = sm.Qt[t][cg + 16 * x];
+          kt[x] = sm.Kt[t][cg + 16 * x];
+        }
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x)
+            acc[y][x] = fmaf(p[y], qt[x], fmaf(dg4[y], kt[x], acc[y][x]));
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+#pragma unroll
+        for (int x = 0; x < CT; ++x) {
+          const int r = rb + y, c = cg + 16 * x;
+          dgam[y][x] = fmaf(-acc[y][x], sm.Kh[r][c], dgam[y][x]);
+          if (r < L)
+            atomicAdd(a.acc_k + ((c0 + r) * H + h) * DK + c, dkk[y][x] + acc[y][x] / E[y][x]);
+        }
+#pragma unroll
+      for (int x = 0; x < CT; ++x) dglp_all[rg * DK + cg + 16 * x] = dglp[x];
       __syncthreads();
-      float later = 0.f;
-      for (int q2 = rg + 1; q2 < RG; ++q2) later += sm.part[q2][i];
-#pragma unroll 1
-      for (int rr = 0; rr < RPT; ++rr) {
-        const int r = rb + rr;
-        if (r >= L) break;
-        const int64_t off = ((c0 + r) * H + h) * DK + i;
-        atomicAdd(a.acc_k + off, dkk[rr]);
-        atomicAdd(a.acc_g + off, ((live >> rr) & 1u) ? dgam[rr] + later : 0.f);
+      // 9e. gl = E[L - 1] feeds the last live row; then the reverse cumulative sum over the
+      //     live rows: local suffix sums plus the later groups' totals
+#pragma unroll
+      for (int x = 0; x < CT; ++x) {
+        const int c = cg + 16 * x;
+        float dgl = 0.f;
+        for (int q2 = 0; q2 < 16; ++q2) dgl += dglp_all[q2 * DK + c];
+        float suf = 0.f;
+#pragma unroll
+        for (int y = 3; y >= 0; --y) {
+          const int r = rb + y;
+          if (r == L - 1) dgam[y][x] = fmaf(dgl, sm.gl[c], dgam[y][x]);
+          if (r < L) suf += dgam[y][x];
+          dgam[y][x] = suf;
+        }
+        scan[rg * DK + c] = suf;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int x = 0; x < CT; ++x) {
+        const int c = cg + 16 * x;
+        float later = 0.f;
+        for (int q2 = rg + 1; q2 < 16; ++q2) later += scan[q2 * DK + c];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int r = rb + y;
+          if (r < L)
+            atomicAdd(a.acc_g + ((c0 + r) * H + h) * DK + c,
+                      ((live >> (y * CT + x)) & 1u) ? dgam[y][x] + later : 0.f);
+        }
       }
     }
-    __syncthreads();  // dS' is read above; it is updated below
+    __syncthreads();  // dS' and S are read above; dS is updated below
 
-    // ---- 10. dS <- Diag(gl) dS' + scale Q~^T dO - K~^T Z (the start state's gradient)
-    for (int e = tid; e < DK * DVS; e += NT) {
-      const int i = e / DVS, j = e % DVS;
-      float a1 = 0.f, a2 = 0.f;
+    // ---- 10. dS <- Diag(gl) dS' + scale Q~^T dO - K~^T Z        (DK x DVS tiles, IT x 4)
+    {
+      constexpr int IT = DK / 32;
+      const int ib = (tid >> 3) * IT, jc = tid & 7;
+      float a1[IT][4] = {}, a2[IT][4] = {};
       for (int r = 0; r < C; ++r) {
-        a1 = fmaf(sm.Qt[r][i], sm.dO[r][j], a1);
-        a2 = fmaf(sm.Kt[r][i], sm.Y[r][j], a2);
+        float qt[IT], kt[IT], o[4], z[4];
+#pragma unroll
+        for (int y = 0; y < IT; ++y) {
+          qt[y] = sm.Qt[r][ib + y];
+          kt[y] = sm.Kt[r][ib + y];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          o[x] = sm.dO[r][jc + 8 * x];
+          z[x] = sm.Y[r][jc + 8 * x];
+        }
+#pragma unroll
+        for (int y = 0; y < IT; ++y)
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            a1[y][x] = fmaf(qt[y], o[x], a1[y][x]);
+            a2[y][x] = fmaf(kt[y], z[x], a2[y][x]);
+          }
       }
-      sm.dS[i][j] = fmaf(sm.gl[i], sm.dS[i][j], fmaf(scale, a1, -a2));
+#pragma unroll
+      for (int y = 0; y < IT; ++y) {
+        const int i = ib + y;
+        const float gi = sm.gl[i];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int j = jc + 8 * x;
+          sm.dS[i][j] = fmaf(gi, sm.dS[i][j], fmaf(scale, a1[y][x], -a2[y][x]));
+        }
+      }
     }
   }
   __syncthreads();
