@@ -38,6 +38,19 @@ def prefill_flops_per_token_head(dk: int, dv: int, chunk: int = C) -> float:
     return 2 * chunk * (3 * dk + 2 * dv) + 6 * dk * dv + chunk * chunk / 3
 
 
+def backward_flops_per_token_head(dk: int, dv: int, chunk: int = C) -> float:
+    """Algorithmic FLOPs of the chunked backward per (token, head), counting the products
+    of its formulas as dense: 2 (7 dk dv + 7 C dk + 5 C dv + 7 C^2 / 3) (seven d_k x d_v
+    products such as K~ S, Q~^T dO, dO S^T; seven C x C x d_k ones such as K~ K^^T, dP K^;
+    five C x C x d_v ones such as T Y, dU Y^T; the inverse and dA = -N^T dN N^T)."""
+    return 2 * (7 * dk * dv + 7 * chunk * dk + 5 * chunk * dv + 7 * chunk * chunk / 3)
+
+
+def fp32_alu_peak_tflops(sms: int = 148, lanes: int = 128, ghz: float = 1.965) -> float:
+    """fp32 FMA peak of the CUDA cores: SMs x fp32 lanes per SM x 2 FLOP x max clock."""
+    return round(sms * lanes * 2 * ghz / 1e3, 1)
+
+
 def prefill_bytes_per_token_head(dk: int, dv: int, elem: int = 2) -> int:
     """Compulsory HBM bytes per (token, head): read q, k, g, v, beta; write out."""
     return elem * (3 * dk + dv + 1) + elem * dv
@@ -284,9 +297,42 @@ def bench_ours(args, world, rank, local):
                            "bytes_per_step": state_bytes + tok_bytes,
                            "traffic": measured_traffic("decode_n256_h32_d128")},
               "gpu_launches": dsteps}
+    # ---- backward leg (kda_chunk_bwd on the prefill workload; CUDA-core fp32)
+    d_out = torch.randn(x.v.shape, generator=torch.Generator(device=dev).manual_seed(7),
+                        device=dev).to(w.dtype)
+    bws = torch.empty(int(kda.lib.kda_chunk_bwd_workspace_size(kda.ctypes.byref(shape))),
+                      dtype=torch.uint8, device=dev)
+    grads = [torch.empty_like(t) for t in (x.q, x.k, x.v, x.g, x.beta)]
+    ds0 = torch.empty_like(x.initial_state)
+
+    def bstep():
+        rc = kda.lib.kda_chunk_bwd(
+            *(kda._ptr(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.initial_state)), None,
+            kda._ptr(d_out), None, *(kda._ptr(t) for t in grads), kda._ptr(ds0),
+            kda.ctypes.byref(shape), kda._ptr(bws), bws.numel(), kda._stream(stream))
+        assert rc == kda.KDA_OK, rc
+
+    for _ in range(3):
+        bstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    bsteps = 5
+    b_total, _ = time_region(bstep, bsteps, stream)
+    b_ms = max_over_ranks(b_total, world) / bsteps
+    b_flops = (backward_flops_per_token_head(dk, dv) + prefill_flops_per_token_head(dk, dv)) * T * H
+    b_tf = b_flops / (b_ms / 1e3) / 1e12
+    fp32_peak = fp32_alu_peak_tflops()
+    backward = {"workload": PREFILL, "ms_per_call": round(b_ms, 3),
+                "tokens_per_s": round(T * world / (b_ms / 1e3), 1),
+                "roofline": {"bound": "alu", "achieved": round(b_tf, 2), "peak": fp32_peak,
+                             "unit": "TFLOP/s", "frac": round(b_tf / fp32_peak, 4),
+                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                             "flops_per_call": b_flops, "traffic": None},
+                "gpu_launches": bsteps * (kda_launches_per_step(kda, shape) + 5)}
+    del bws, grads
     return {
         "value": round(value, 1), "ms_per_step": round(ms_step, 4), "clocks": clk,
-        "roofline": roofline, "e2e": e2e, "decode": decode,
+        "roofline": roofline, "e2e": e2e, "decode": decode, "backward": backward,
         "gpu_launches": launches_per_step * args.steps,
         "tflops": round(tc_tflops * world, 2),
     }
@@ -430,7 +476,7 @@ def main():
             "dtype": "bf16", "data": "synthetic (seeded; no weights, no dataset)",
             "config": cfg, "impl": "ours", "tflops": r["tflops"], "roofline": r["roofline"],
             "cpu_baseline": cpu, "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
-            "clocks": r["clocks"], "decode": r["decode"],
+            "clocks": r["clocks"], "decode": r["decode"], "backward": r["backward"],
         }
         print(json.dumps(line))
     if world > 1:

@@ -87,3 +87,10 @@ def test_backward_without_upstream_state_grad(kda):
     x = make_inputs(None, H=4, dk=128, dv=128, dtype=torch.bfloat16, seed=507,
                     lengths=[257, 3], state_std=0.02)
     _check(kda, x, torch.bfloat16, "no dS_final", with_final=False)
+
+
+def test_full_bf16_h32_t8192_d128_backward(kda):
+    """The 8K-token, 32-head workload: every gradient of every element."""
+    from kimi_delta_attention_19_b200.inputs import WORKLOADS, workload_inputs
+    x = workload_inputs(WORKLOADS["bf16_h32_t8192_d128"])
+    _check(kda, x, torch.bfloat16, "8K x 32 heads", seed=7)
