@@ -390,15 +390,22 @@ def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: 
 
 def kernels_only(args):
     """Profiler driver: `warmup + steps` calls of one path on its benchmark workload on
-    cuda:0 (prefill: kda_chunk_fwd on the 8K x 32-head inputs with one workspace; decode:
-    chained decode steps on the 256 x 32-head state), no timing and no CPU leg. ncu
-    captures select launches with -s/-c on this run."""
+    cuda:0 (prefill: kda_chunk_fwd on the 8K x 32-head inputs with one workspace; backward:
+    kda_chunk_bwd on the same inputs; decode: chained decode steps on the 256 x 32-head
+    state), no timing and no CPU leg. ncu captures select launches with -s/-c on this run."""
     from kimi_delta_attention_19_b200 import kda
     from kimi_delta_attention_19_b200.inputs import (WORKLOADS, decode_state, decode_tokens,
                                                       workload_inputs)
     dev = "cuda:0"
     n = args.warmup + args.steps
-    if args.kernels_only == "prefill":
+    if args.kernels_only == "backward":
+        w = WORKLOADS[PREFILL]
+        x = workload_inputs(w, device=dev)
+        d_out = torch.randn(x.v.shape, generator=torch.Generator(device=dev).manual_seed(7),
+                            device=dev).to(w.dtype)
+        for _ in range(n):
+            kda.chunk_bwd(x.q, x.k, x.v, x.g, x.beta, d_out, initial_state=x.initial_state)
+    elif args.kernels_only == "prefill":
         w = WORKLOADS[PREFILL]
         x = workload_inputs(w, device=dev)
         shape = kda.make_shape(w.T, w.H, w.dk, w.dv, w.dtype)
@@ -426,7 +433,7 @@ def main():
                     help="tokens per reference-arm step (bounded oracle sample)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum timed oracle work for the cpu_baseline object")
-    ap.add_argument("--kernels-only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--kernels-only", choices=["prefill", "backward", "decode"], default=None,
                     help="profiler driver: run warmup + steps calls of one path, print no "
                          "measurement (for ncu -s/-c captures)")
     args = ap.parse_args()
