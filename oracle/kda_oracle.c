@@ -350,15 +350,19 @@ typedef struct {
     const double *initial_state, *d_out, *d_final;
     double lb, scale;
     double *dq, *dkk, *dvv, *dg, *dbeta, *ds0;
+    int prologue;      /* KDA_ORACLE_* prologue flags: raw inputs, chain rule through them */
     int64_t next_item;
     pthread_mutex_t lock;
 } bjob_t;
 
 #define KDA_ORACLE_BWD_BLOCK 64
 
-/* Inputs of token t (head h): k, q, v, beta, the clamped decay and the raw log decay. */
+/* Inputs of token t (head h) as the recurrence uses them: k, q (unit length with the
+ * L2 prologue; their norms in *nk, *nq), v, beta, the log decay before the clamp (the gate's
+ * output with the gate prologue; sig = sigmoid(a) then) and the clamped decay. */
 static void load_token(const bjob_t *J, int64_t t, int h, double *kt, double *qt, double *vt,
-                       double *decay, double *graw, double *b)
+                       double *decay, double *graw, double *b, double *nk, double *nq,
+                       double *sig)
 {
     const int dk = J->dk, dv = J->dv, H = J->H;
     const int64_t tok_k = (t * H + h) * dk, tok_v = (t * H + h) * dv;
@@ -366,7 +370,25 @@ static void load_token(const bjob_t *J, int64_t t, int h, double *kt, double *qt
         kt[i] = load_elem(J->k, J->dtype, tok_k + i);
         qt[i] = load_elem(J->q, J->dtype, tok_k + i);
         graw[i] = load_elem(J->g, J->dtype, tok_k + i);
+        if (J->prologue & KDA_ORACLE_GATE_SIGMOID) {
+            sig[i] = 1.0 / (1.0 + exp(-graw[i]));
+            graw[i] = J->lb * sig[i];
+        }
         decay[i] = exp(graw[i] < J->lb ? J->lb : graw[i]);
+    }
+    *nk = *nq = 1.0;
+    if (J->prologue & KDA_ORACLE_QK_L2NORM) {
+        double a = 0.0, c = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            a += kt[i] * kt[i];
+            c += qt[i] * qt[i];
+        }
+        *nk = sqrt(a) < 1e-12 ? 1e-12 : sqrt(a);
+        *nq = sqrt(c) < 1e-12 ? 1e-12 : sqrt(c);
+        for (int i = 0; i < dk; ++i) {
+            kt[i] /= *nk;
+            qt[i] /= *nq;
+        }
     }
     for (int j = 0; j < dv; ++j) vt[j] = load_elem(J->v, J->dtype, tok_v + j);
     *b = load_elem(J->beta, J->dtype, t * H + h);
@@ -397,14 +419,15 @@ static int bwd_one(const bjob_t *J, int seq, int h)
     double *S = (double *)malloc(sizeof(double) * st);
     double *Sb = (double *)malloc(sizeof(double) * st);
     double *dS = (double *)malloc(sizeof(double) * st);
-    double *buf = (double *)malloc(sizeof(double) * (size_t)(5 * dk + 6 * dv));
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(6 * dk + 6 * dv));
     if (!ckpt || !pre || !S || !Sb || !dS || !buf) {
         free(ckpt); free(pre); free(S); free(Sb); free(dS); free(buf);
         return 1;
     }
     double *kt = buf, *qt = kt + dk, *decay = qt + dk, *graw = decay + dk, *dgp = graw + dk;
-    double *vt = dgp + dk, *w = vt + dv, *u = w + dv, *du = u + dv, *dw = du + dv, *dov = dw + dv;
-    double b;
+    double *sig = dgp + dk;
+    double *vt = sig + dk, *w = vt + dv, *u = w + dv, *du = u + dv, *dw = du + dv, *dov = dw + dv;
+    double b, nk, nq;
 
     /* forward sweep: the state at the start of every block */
     if (J->initial_state) memcpy(S, J->initial_state + state_off, sizeof(double) * st);
@@ -413,7 +436,7 @@ static int bwd_one(const bjob_t *J, int seq, int h)
         memcpy(ckpt + (size_t)blk * st, S, sizeof(double) * st);
         const int64_t e = t0 + (blk + 1) * B < t1 ? t0 + (blk + 1) * B : t1;
         for (int64_t t = t0 + blk * B; t < e; ++t) {
-            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b, &nk, &nq, sig);
             step_state(S, dk, dv, kt, vt, decay, b, w);
         }
     }
@@ -425,11 +448,11 @@ static int bwd_one(const bjob_t *J, int seq, int h)
         memcpy(S, ckpt + (size_t)blk * st, sizeof(double) * st);
         for (int64_t t = s; t < e; ++t) {
             memcpy(pre + (size_t)(t - s) * st, S, sizeof(double) * st);
-            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b, &nk, &nq, sig);
             step_state(S, dk, dv, kt, vt, decay, b, w);
         }
         for (int64_t t = e - 1; t >= s; --t) {
-            load_token(J, t, h, kt, qt, vt, decay, graw, &b);
+            load_token(J, t, h, kt, qt, vt, decay, graw, &b, &nk, &nq, sig);
             const double *Sp = pre + (size_t)(t - s) * st;
             /* recompute the step: Sb, w, u and S_t (in S) */
             for (int i = 0; i < dk; ++i)
@@ -486,6 +509,23 @@ static int bwd_one(const bjob_t *J, int seq, int h)
                 J->dg[tk + i] = graw[i] >= J->lb ? dgp[i] : 0.0;
                 for (int j = 0; j < dv; ++j) dS[i * dv + j] *= decay[i];
             }
+            /* through the prologue, to the raw inputs */
+            if (J->prologue & KDA_ORACLE_GATE_SIGMOID)
+                for (int i = 0; i < dk; ++i) J->dg[tk + i] *= J->lb * sig[i] * (1.0 - sig[i]);
+            if (J->prologue & KDA_ORACLE_QK_L2NORM) {
+                /* x = r / max(|r|, eps): dr = (dx - x (x . dx)) / |r| above eps, dx / eps below */
+                double pk = 0.0, pq = 0.0;
+                for (int i = 0; i < dk; ++i) {
+                    pk += kt[i] * J->dkk[tk + i];
+                    pq += qt[i] * J->dq[tk + i];
+                }
+                if (nk <= 1e-12) pk = 0.0;
+                if (nq <= 1e-12) pq = 0.0;
+                for (int i = 0; i < dk; ++i) {
+                    J->dkk[tk + i] = (J->dkk[tk + i] - kt[i] * pk) / nk;
+                    J->dq[tk + i] = (J->dq[tk + i] - qt[i] * pq) / nq;
+                }
+            }
         }
     }
     if (J->ds0) memcpy(J->ds0 + state_off, dS, sizeof(double) * st);
@@ -511,7 +551,9 @@ static void *bwd_worker(void *arg)
  * Gradients of the recurrence (see the block comment above). Layouts as in the forward;
  * d_out [T, H, dv] fp64 (NULL = 0), d_final [n_seqs, H, dk, dv] fp64 (NULL = 0); outputs
  * dq, dk, dg [T, H, dk], dv [T, H, dv], dbeta [T, H], ds0 [n_seqs, H, dk, dv] (NULL to
- * skip), all fp64. Returns 0, -1 on a bad argument, -2 when a thread failed.
+ * skip), all fp64. With prologue flags the inputs are raw (as in kda_oracle_recurrent_ex)
+ * and the gradients are those of the raw q, k and gate pre-activations.
+ * Returns 0, -1 on a bad argument, -2 when a thread failed.
  */
 int kda_oracle_backward(int64_t T, int H, int dk, int dv, int n_seqs,
                         const int64_t *cu_seqlens, int dtype,
@@ -520,7 +562,7 @@ int kda_oracle_backward(int64_t T, int H, int dk, int dv, int n_seqs,
                         const double *initial_state, double lb, double scale,
                         const double *d_out, const double *d_final,
                         double *dq, double *dkk, double *dvv, double *dg, double *dbeta,
-                        double *ds0, int n_threads)
+                        double *ds0, int prologue, int n_threads)
 {
     if (T < 0 || H <= 0 || dk <= 0 || dv <= 0 || n_seqs <= 0 || !cu_seqlens) return -1;
     if (dtype != KDA_ORACLE_F32 && dtype != KDA_ORACLE_BF16) return -1;
@@ -529,6 +571,7 @@ int kda_oracle_backward(int64_t T, int H, int dk, int dv, int n_seqs,
         if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
     if (T > 0 && (!q || !k || !v || !g || !beta || !dq || !dkk || !dvv || !dg || !dbeta))
         return -1;
+    if (prologue & ~(KDA_ORACLE_QK_L2NORM | KDA_ORACLE_GATE_SIGMOID)) return -1;
 
     bjob_t J;
     memset(&J, 0, sizeof J);
@@ -538,6 +581,7 @@ int kda_oracle_backward(int64_t T, int H, int dk, int dv, int n_seqs,
     J.initial_state = initial_state; J.d_out = d_out; J.d_final = d_final;
     J.lb = lb; J.scale = scale;
     J.dq = dq; J.dkk = dkk; J.dvv = dvv; J.dg = dg; J.dbeta = dbeta; J.ds0 = ds0;
+    J.prologue = prologue;
     pthread_mutex_init(&J.lock, NULL);
 
     const int64_t n_items = (int64_t)n_seqs * H;

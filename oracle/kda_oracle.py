@@ -77,7 +77,7 @@ def _bind(path: str):
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                   p, ctypes.c_int, p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
-                  p, p, p, p, p, p, p, p, ctypes.c_int]
+                  p, p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int]
     return lib
 
 
@@ -244,8 +244,11 @@ def recurrent_snapshots(q, k, v, g, beta, *, snapshot_tokens: int, cu_seqlens=No
 
 def backward(q, k, v, g, beta, *, d_out=None, d_final=None, cu_seqlens=None,
              initial_state=None, lb: float = -1.0, scale: float | None = None,
-             n_threads: int | None = None, lib=None) -> dict:
+             prologue: int = 0, n_threads: int | None = None, lib=None) -> dict:
     """fp64 reverse-mode gradients of the token recurrence (kda_oracle.c, "backward").
+
+    prologue: 0, or QK_L2NORM | GATE_SIGMOID: raw inputs; gradients of the raw q, k and
+    gate pre-activations.
 
     d_out: dL/do [T, H, dv] (None = 0); d_final: dL/dS_final [n, H, dk, dv] (None = 0).
     Returns dict dq, dk, dg [T, H, dk], dv [T, H, dv], dbeta [T, H], ds0 [n, H, dk, dv],
@@ -287,7 +290,7 @@ def backward(q, k, v, g, beta, *, d_out=None, d_final=None, cu_seqlens=None,
                                  ptr(ga), ptr(ba), ptr(s0), float(lb), float(scale), ptr(do),
                                  ptr(dS), ptr(res["dq"]), ptr(res["dk"]), ptr(res["dv"]),
                                  ptr(res["dg"]), ptr(res["dbeta"]), ptr(res["ds0"]),
-                                 int(n_threads))
+                                 int(prologue), int(n_threads))
     if rc != 0:
         raise ValueError(f"kda_oracle_backward failed with code {rc}")
     return res

@@ -424,11 +424,53 @@ def pin_backward_beta_zero(lib):
     assert np.all(got["dk"] == 0.0) and np.all(got["dv"] == 0.0)
 
 
+def pin_backward_prologue_finite_differences(lib):
+    """With the raw-input prologue the gradients are those of the raw q, k and gate
+    pre-activations: central finite differences of the chunked fp64 form fed with
+    q / |q|, k / |k| and lb * sigmoid(a) formed in fp64 here."""
+    rng = np.random.default_rng(95)
+    lb = -0.8
+    x = make_inputs(None, H=1, dk=3, dv=2, dtype=torch.float32, seed=95, lengths=[5, 3],
+                    state_std=0.5, raw=True)
+    cu = x.cu_seqlens.tolist()
+    T = cu[-1]
+    do = rng.standard_normal((T, 1, 2))
+    dS = rng.standard_normal((2, 1, 3, 2))
+    got = ko.backward(x.q, x.k, x.v, x.g, x.beta, d_out=do, d_final=dS, cu_seqlens=cu,
+                      initial_state=x.initial_state, lb=lb,
+                      prologue=ko.QK_L2NORM | ko.GATE_SIGMOID, lib=lib)
+    vals = {n: ko._widen(getattr(x, n)).copy() for n in ("q", "k", "g")}
+    fixed = {n: ko._widen(getattr(x, n)) for n in ("v", "beta")}
+
+    def loss():
+        qn = vals["q"] / np.linalg.norm(vals["q"], axis=-1, keepdims=True)
+        kn = vals["k"] / np.linalg.norm(vals["k"], axis=-1, keepdims=True)
+        gg = lb / (1.0 + np.exp(-vals["g"]))
+        o, s = ko.chunked(qn, kn, fixed["v"], gg, fixed["beta"], chunk=2, cu_seqlens=cu,
+                          initial_state=x.initial_state.double().numpy(), lb=lb)
+        return float(np.sum(do * o) + np.sum(dS * s))
+    h = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("g", "dg")):
+        arr = vals[name]
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            x0 = arr[idx]
+            arr[idx] = x0 + h
+            lp = loss()
+            arr[idx] = x0 - h
+            lm = loss()
+            arr[idx] = x0
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - got[key]))
+        assert err <= 1e-6 * max(1.0, np.max(np.abs(fd))), (name, err)
+
+
 ALL_PINS = [pin_golden, pin_chunked_agreement, pin_beta_zero_pure_decay, pin_delta_rule_reach,
             pin_general_beta_reach, pin_associative_memory, pin_one_token_expansion,
             pin_linearity, pin_contraction_bound, pin_resume_and_varlen, pin_decay_clamp,
             pin_sampled_rows, pin_snapshots_are_prefix_states, pin_prologue_l2norm,
-            pin_prologue_gate, pin_backward_finite_differences, pin_backward_beta_zero]
+            pin_prologue_gate, pin_backward_finite_differences, pin_backward_beta_zero,
+            pin_backward_prologue_finite_differences]
 
 
 def failing_pins(lib_path: str) -> list[str]:

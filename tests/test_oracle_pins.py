@@ -66,6 +66,10 @@ MUTANTS = {
     "bwd_dq_from_decayed_prev_state": ("a += S[i * dv + j] * dov[j];",
                                        "a += Sb[i * dv + j] * dov[j];"),
     "bwd_dbeta_without_recall": ("db += du[j] * (vt[j] - w[j]);", "db += du[j] * vt[j];"),
+    "bwd_l2norm_without_projection": ("J->dq[tk + i] = (J->dq[tk + i] - qt[i] * pq) / nq;",
+                                      "J->dq[tk + i] = J->dq[tk + i] / nq;"),
+    "bwd_gate_without_sigmoid_slope": (
+        "J->dg[tk + i] *= J->lb * sig[i] * (1.0 - sig[i]);", "J->dg[tk + i] *= J->lb;"),
 }
 
 
