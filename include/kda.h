@@ -78,7 +78,7 @@ typedef struct {
 
 /*
  * Optional input prologue, fused into every entry point's kernels (prefill, snapshots,
- * no-alloc prefill, decode). With 0 the inputs are used as given.
+ * no-alloc prefill, decode, backward). With 0 the inputs are used as given.
  *  KDA_PROLOGUE_QK_L2NORM   q and k are raw: each (token, head) row is divided by
  *                           max(||row||_2, 1e-12) in fp32 before use ("Kimi K3 深度拆解",
  *                           section 4.2: the delta rule takes L2-normalised q and k).
@@ -161,8 +161,7 @@ int64_t kda_snapshot_count(const kda_shape *shape, int32_t snapshot_chunks);
 
 /*
  * Bytes of device scratch kda_chunk_bwd needs for this shape (a pure function of the
- * shape fields). Returns 0 for an invalid shape or a shape the backward does not
- * support (a nonzero prologue).
+ * shape fields). Returns 0 for an invalid shape.
  */
 size_t kda_chunk_bwd_workspace_size(const kda_shape *shape);
 
@@ -174,7 +173,8 @@ size_t kda_chunk_bwd_workspace_size(const kda_shape *shape);
  * from a forward pass with per-chunk snapshots that this call runs first.
  *
  *  q, k, v, g, beta, initial_state, cu_seqlens, shape: as in kda_chunk_fwd (the same
- *               forward inputs). shape->prologue must be 0 (KDA_ERR_UNSUPPORTED).
+ *               forward inputs). With shape->prologue set the inputs are raw and dq, dk,
+ *               dg are the gradients of the raw q, k and gate pre-activations.
  *  d_out        [B*T, H, dv] dtype, or NULL for zeros
  *  d_final_state[n, H, dk, dv] fp32, or NULL for zeros
  *  dq, dk, dg   [B*T, H, dk] dtype (written)     dv [B*T, H, dv] dtype (written)

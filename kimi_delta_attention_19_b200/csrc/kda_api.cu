@@ -173,7 +173,7 @@ struct BwdPlan {
 };
 
 bool bwd_plan(const kda_shape* shape, BwdPlan& p) {
-  if (check_shape(shape, true) != KDA_OK || shape->prologue != 0) return false;
+  if (check_shape(shape, true) != KDA_OK) return false;
   const size_t fwd = kda_chunk_fwd_workspace_size(shape);
   if (fwd == 0) return false;
   int64_t T_total, max_len;
@@ -211,7 +211,6 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
                          void* workspace, size_t workspace_bytes, kda_stream_t stream) {
   kda_status st = check_shape(shape, true);
   if (st != KDA_OK) return st;
-  if (shape->prologue != 0) return KDA_ERR_UNSUPPORTED;
   const kda_shape& s = *shape;
   if ((cu_seqlens != nullptr) != (s.n_seqs > 0)) return KDA_ERR_INVALID_ARG;
   if (cu_seqlens != nullptr && s.B != 1) return KDA_ERR_INVALID_ARG;
@@ -262,12 +261,9 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
   a.H = s.H; a.dk = s.dk; a.dv = s.dv;
   a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
   a.lb = s.g_lower_bound;
+  a.prologue = s.prologue;
   cudaError_t e = launch_backward(a, s.dtype, cs);
-  const int64_t nk = T_total * s.H * s.dk, nb = T_total * s.H;
-  if (e == cudaSuccess) e = launch_backward_convert(a.acc_q, dq, nk, s.dtype, cs);
-  if (e == cudaSuccess) e = launch_backward_convert(a.acc_k, dk, nk, s.dtype, cs);
-  if (e == cudaSuccess) e = launch_backward_convert(a.acc_g, dg, nk, s.dtype, cs);
-  if (e == cudaSuccess) e = launch_backward_convert(a.acc_b, dbeta, nb, s.dtype, cs);
+  if (e == cudaSuccess) e = launch_backward_finish(a, dq, dk, dg, dbeta, s.dtype, cs);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -74,7 +74,10 @@ __device__ __forceinline__ void unpack_vec<__nv_bfloat16>(const uint4& u, float 
   }
 }
 
-template <typename Tin, int DK>
+// PRO: the raw-input prologue flags (KDA_PROLOGUE_*); the kernel then works on the
+// normalised q, k and the gate's log decays, and the finishing pass carries the gradients
+// through the prologue to the raw inputs.
+template <typename Tin, int DK, int PRO>
 __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem<DK>& sm = *reinterpret_cast<BwdSmem<DK>*>(smem_raw);
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         oq[m] = (in && dout) ? *reinterpret_cast<const uint4*>(dout + off) : z;
       }
       if (tid < C) sm.bet[tid] = tid < L ? ld_in(beta + (c0 + tid) * H + h) : 0.f;
-      // unpack into shared memory (raw k -> Kt, raw q -> Qt, clamped g -> Kh; rows past
+      // unpack into shared memory (k -> Kt, q -> Qt, clamped log decay -> Kh; rows past
       // L are zero: no key, no decay)
 #pragma unroll
       for (int m = 0; m < NV; ++m) {
@@ -167,11 +170,33 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         unpack_vec<Tin>(kq[m], kf);
         unpack_vec<Tin>(qq[m], qf);
         unpack_vec<Tin>(gq[m], gf);
+        if (PRO & KDA_PROLOGUE_QK_L2NORM) {
+          // a row is VR consecutive lanes (VR divides 32): its norms by shuffles
+          float sk = 0.f, sq2 = 0.f;
+#pragma unroll
+          for (int x = 0; x < EV; ++x) {
+            sk = fmaf(kf[x], kf[x], sk);
+            sq2 = fmaf(qf[x], qf[x], sq2);
+          }
+#pragma unroll
+          for (int o2 = VR / 2; o2 > 0; o2 >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, o2);
+            sq2 += __shfl_xor_sync(0xffffffffu, sq2, o2);
+          }
+          const float rk = inv_l2(sk), rq = inv_l2(sq2);
+#pragma unroll
+          for (int x = 0; x < EV; ++x) {
+            kf[x] *= rk;
+            qf[x] *= rq;
+          }
+        }
 #pragma unroll
         for (int x = 0; x < EV; ++x) {
+          float gx = gf[x];
+          if (PRO & KDA_PROLOGUE_GATE_SIGMOID) gx = gate_from_preact(gx, lb);
           sm.Kt[r][i0 + x] = kf[x];
           sm.Qt[r][i0 + x] = qf[x];
-          sm.Kh[r][i0 + x] = r < L ? fmaxf(gf[x], lb) : 0.f;
+          sm.Kh[r][i0 + x] = r < L ? fmaxf(gx, lb) : 0.f;
         }
       }
 #pragma unroll
@@ -557,6 +582,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         for (int x = 0; x < CT; ++x) {
           const int r = rb + y, c = cg + 16 * x;
           graw[y][x] = r < L ? ld_in(g + ((c0 + r) * H + h) * DK + c) : 0.f;
+          if ((PRO & KDA_PROLOGUE_GATE_SIGMOID) && r < L) graw[y][x] = gate_from_preact(graw[y][x], lb);
           gsum[x] += r < L ? fmaxf(graw[y][x], lb) : 0.f;
         }
 #pragma unroll
@@ -798,15 +824,104 @@ __global__ void bwd_convert_kernel(const float* __restrict__ acc, Tout* __restri
     st_out(out + e, acc[e]);
 }
 
+// Through q = r / max(|r|, 1e-12): dr = (dq - q (q . dq)) / |r| (dq / 1e-12 at the floor).
+// One warp per (token, head) row of the raw input r.
 template <typename Tin, int DK>
-cudaError_t launch_typed(const BackwardArgs& a, cudaStream_t st) {
+__global__ void bwd_l2norm_kernel(const float* __restrict__ acc, const Tin* __restrict__ raw,
+                                  Tin* __restrict__ out, int64_t rows) {
+  constexpr int PL = DK / 32;
+  const int lane = threadIdx.x & 31;
+  for (int64_t row = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; row < rows;
+       row += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    float x[PL], d[PL], ss = 0.f, dot = 0.f;
+#pragma unroll
+    for (int p = 0; p < PL; ++p) {
+      x[p] = ld_in(raw + row * DK + lane + 32 * p);
+      d[p] = acc[row * DK + lane + 32 * p];
+      ss = fmaf(x[p], x[p], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float n = fmaxf(sqrtf(ss), 1e-12f), rn = 1.f / n;
+#pragma unroll
+    for (int p = 0; p < PL; ++p) dot = fmaf(x[p] * rn, d[p], dot);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (sqrtf(ss) <= 1e-12f) dot = 0.f;
+#pragma unroll
+    for (int p = 0; p < PL; ++p) st_out(out + row * DK + lane + 32 * p, (d[p] - x[p] * rn * dot) * rn);
+  }
+}
+
+// Through g = lb * sigmoid(a): da = dg lb sigmoid(a) (1 - sigmoid(a)).
+template <typename Tin>
+__global__ void bwd_gate_kernel(const float* __restrict__ acc, const Tin* __restrict__ raw,
+                                Tin* __restrict__ out, int64_t n, float lb) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const float a = ld_in(raw + e);
+    const float ex = __expf(-fabsf(a)), s = 1.f / (1.f + ex);
+    const float sg = a >= 0.f ? s : ex * s;  // sigmoid(a)
+    st_out(out + e, acc[e] * lb * sg * (1.f - sg));
+  }
+}
+
+template <typename Tin, int DK, int PRO>
+cudaError_t launch_kernel(const BackwardArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(BwdSmem<DK>);
-  cudaError_t e = cudaFuncSetAttribute(bwd_simt_kernel<Tin, DK>,
+  cudaError_t e = cudaFuncSetAttribute(bwd_simt_kernel<Tin, DK, PRO>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)a.n_seqs * a.H * (a.dv / DVS);
   if (blocks == 0) return cudaSuccess;
-  bwd_simt_kernel<Tin, DK><<<(unsigned)blocks, NT, smem, st>>>(a);
+  bwd_simt_kernel<Tin, DK, PRO><<<(unsigned)blocks, NT, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename Tin, int DK>
+cudaError_t launch_typed(const BackwardArgs& a, cudaStream_t st) {
+  switch (a.prologue) {
+    case 0: return launch_kernel<Tin, DK, 0>(a, st);
+    case 1: return launch_kernel<Tin, DK, 1>(a, st);
+    case 2: return launch_kernel<Tin, DK, 2>(a, st);
+    default: return launch_kernel<Tin, DK, 3>(a, st);
+  }
+}
+
+unsigned grid_for(int64_t n, int threads) {
+  const int64_t want = (n + threads - 1) / threads;
+  return (unsigned)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+}
+
+template <typename Tin>
+cudaError_t finish_typed(const BackwardArgs& a, void* dq, void* dk, void* dg, void* dbeta,
+                         cudaStream_t st) {
+  const int64_t rows = a.T_total * a.H, nk = rows * a.dk;
+  if (rows == 0) return cudaSuccess;
+  const int threads = 256;
+  Tin* oq = static_cast<Tin*>(dq);
+  Tin* ok = static_cast<Tin*>(dk);
+  Tin* og = static_cast<Tin*>(dg);
+  if (a.prologue & KDA_PROLOGUE_QK_L2NORM) {
+    const unsigned gr = grid_for(rows * 32, threads);
+    if (a.dk == 64) {
+      bwd_l2norm_kernel<Tin, 64><<<gr, threads, 0, st>>>(a.acc_q, static_cast<const Tin*>(a.q), oq, rows);
+      bwd_l2norm_kernel<Tin, 64><<<gr, threads, 0, st>>>(a.acc_k, static_cast<const Tin*>(a.k), ok, rows);
+    } else {
+      bwd_l2norm_kernel<Tin, 128><<<gr, threads, 0, st>>>(a.acc_q, static_cast<const Tin*>(a.q), oq, rows);
+      bwd_l2norm_kernel<Tin, 128><<<gr, threads, 0, st>>>(a.acc_k, static_cast<const Tin*>(a.k), ok, rows);
+    }
+  } else {
+    bwd_convert_kernel<Tin><<<grid_for(nk, threads), threads, 0, st>>>(a.acc_q, oq, nk);
+    bwd_convert_kernel<Tin><<<grid_for(nk, threads), threads, 0, st>>>(a.acc_k, ok, nk);
+  }
+  if (a.prologue & KDA_PROLOGUE_GATE_SIGMOID)
+    bwd_gate_kernel<Tin><<<grid_for(nk, threads), threads, 0, st>>>(
+        a.acc_g, static_cast<const Tin*>(a.g), og, nk, a.lb);
+  else
+    bwd_convert_kernel<Tin><<<grid_for(nk, threads), threads, 0, st>>>(a.acc_g, og, nk);
+  bwd_convert_kernel<Tin><<<grid_for(rows, threads), threads, 0, st>>>(
+      a.acc_b, static_cast<Tin*>(dbeta), rows);
   return cudaGetLastError();
 }
 
@@ -819,18 +934,10 @@ cudaError_t launch_backward(const BackwardArgs& a, kda_dtype dtype, cudaStream_t
                     : launch_typed<__nv_bfloat16, 128>(a, st);
 }
 
-cudaError_t launch_backward_convert(const float* acc, void* out, int64_t n, kda_dtype dtype,
-                                    cudaStream_t st) {
-  if (n == 0) return cudaSuccess;
-  const int threads = 256;
-  const int64_t want = (n + threads - 1) / threads;
-  const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
-  if (dtype == KDA_F32)
-    bwd_convert_kernel<float><<<blocks, threads, 0, st>>>(acc, static_cast<float*>(out), n);
-  else
-    bwd_convert_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>(
-        acc, static_cast<__nv_bfloat16*>(out), n);
-  return cudaGetLastError();
+cudaError_t launch_backward_finish(const BackwardArgs& a, void* dq, void* dk, void* dg,
+                                   void* dbeta, kda_dtype dtype, cudaStream_t st) {
+  return dtype == KDA_F32 ? finish_typed<float>(a, dq, dk, dg, dbeta, st)
+                          : finish_typed<__nv_bfloat16>(a, dq, dk, dg, dbeta, st);
 }
 
 }  // namespace kda

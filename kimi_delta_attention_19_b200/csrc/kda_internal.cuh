@@ -85,6 +85,7 @@ struct BackwardArgs {
   int H, dk, dv;
   float scale;
   float lb;
+  int prologue;             // KDA_PROLOGUE_* flags (raw inputs)
 };
 
 // Sequence bounds [t0, t1) of sequence s; false (and status set) when the
@@ -154,7 +155,8 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, kda_dtype dtype, cudaStrea
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, kda_dtype dtype, cudaStream_t st);
 cudaError_t launch_backward(const BackwardArgs& a, kda_dtype dtype, cudaStream_t st);
-cudaError_t launch_backward_convert(const float* acc, void* out, int64_t n, kda_dtype dtype,
-                                    cudaStream_t st);
+// dq, dk, dg, dbeta from the fp32 accumulators, through the prologue when it is on
+cudaError_t launch_backward_finish(const BackwardArgs& a, void* dq, void* dk, void* dg,
+                                   void* dbeta, kda_dtype dtype, cudaStream_t st);
 
 }  // namespace kda

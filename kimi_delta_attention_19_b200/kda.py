@@ -214,13 +214,14 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
               initial_state: torch.Tensor | None = None,
               cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
               scale: float | None = None, lb: float = -1.0, want_d_initial: bool = True,
-              workspace: torch.Tensor | None = None, stream=None):
+              workspace: torch.Tensor | None = None, prologue: int = 0, stream=None):
     """Gradients of chunk_fwd: (dq, dk, dv, dg, dbeta, d_initial_state).
 
     Same layouts as chunk_fwd; d_out like out, d_final_state like final_state (fp32).
-    d_initial_state is fp32 [n, H, dk, dv] (None unless want_d_initial).
+    d_initial_state is fp32 [n, H, dk, dv] (None unless want_d_initial). With prologue
+    flags the inputs are raw and dq, dk, dg are the raw inputs' gradients.
     """
-    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb)
+    shape, n = _prefill_shape(q, v, cu_seqlens, max_seqlen, scale, lb, prologue)
     H, dk, dv_ = shape.H, shape.dk, shape.dv
     dq, dkk, dg = (torch.empty_like(q) for _ in range(3))
     dvv = torch.empty_like(v)

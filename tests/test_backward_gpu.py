@@ -31,7 +31,7 @@ def kda():
     return k
 
 
-def _check(kda, x, dtype, what, lb=-1.0, seed=0, with_final=True):
+def _check(kda, x, dtype, what, lb=-1.0, seed=0, with_final=True, prologue=0):
     rng = np.random.default_rng(seed)
     T, H, dv = x.v.shape
     n = len(x.lengths)
@@ -43,11 +43,11 @@ def _check(kda, x, dtype, what, lb=-1.0, seed=0, with_final=True):
                         d_final_state=None if d_fin is None else d_fin.to(DEV),
                         initial_state=x.initial_state.to(DEV),
                         cu_seqlens=None if cu is None else cu.to(DEV),
-                        max_seqlen=max(x.lengths), lb=lb)
+                        max_seqlen=max(x.lengths), lb=lb, prologue=prologue)
     torch.cuda.synchronize()
     ref = ko.backward(x.q, x.k, x.v, x.g, x.beta, d_out=d_out.double(), d_final=d_fin,
                       cu_seqlens=None if cu is None else cu.tolist(),
-                      initial_state=x.initial_state, lb=lb)
+                      initial_state=x.initial_state, lb=lb, prologue=prologue)
     for name, gt in zip(NAMES, got):
         rel, mx = errors(gt, ref[name])
         assert rel <= TOL[dtype], f"{what} {name}: rel-L2 {rel:.3e} > {TOL[dtype]:.0e} (max-abs {mx:.3e})"
@@ -94,3 +94,19 @@ def test_full_bf16_h32_t8192_d128_backward(kda):
     from kimi_delta_attention_19_b200.inputs import WORKLOADS, workload_inputs
     x = workload_inputs(WORKLOADS["bf16_h32_t8192_d128"])
     _check(kda, x, torch.bfloat16, "8K x 32 heads", seed=7)
+
+
+@pytest.mark.parametrize("dtype,d,prologue", [(torch.bfloat16, 128, 3), (torch.float32, 64, 3),
+                                              (torch.float32, 128, 1), (torch.bfloat16, 64, 2)])
+def test_backward_prologue(kda, dtype, d, prologue):
+    """Raw inputs through the fused prologue: gradients of the raw q, k (L2 normalisation)
+    and gate pre-activations (lb * sigmoid), against the oracle's chain rule."""
+    raw = make_inputs(None, H=2, dk=d, dv=d, dtype=dtype, seed=508 + d, lengths=[140, 0, 64],
+                      state_std=0.02, raw=True)
+    ref = make_inputs(None, H=2, dk=d, dv=d, dtype=dtype, seed=508 + d, lengths=[140, 0, 64],
+                      state_std=0.02)
+    if not prologue & 1:
+        raw.q, raw.k = ref.q, ref.k
+    if not prologue & 2:
+        raw.g = ref.g
+    _check(kda, raw, dtype, f"prologue={prologue} {dtype} d={d}", lb=-0.9, prologue=prologue)
