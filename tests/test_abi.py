@@ -122,6 +122,35 @@ def test_snapshot_count_and_argument_errors(kda):
         kda.KDA_ERR_UNSUPPORTED
 
 
+def test_backward_workspace_and_argument_errors(kda):
+    """kda_chunk_bwd: workspace size is pure and larger than the forward's; bad arguments
+    return before any CUDA call (the addresses are never dereferenced)."""
+    P = ctypes.c_void_p
+    sh = kda.make_shape(1000, 2, 64, 64, torch.float32, B=3)
+    nb = int(kda.lib.kda_chunk_bwd_workspace_size(ctypes.byref(sh)))
+    assert nb > kda.workspace_size(sh) and nb % 256 == 0
+    assert int(kda.lib.kda_chunk_bwd_workspace_size(ctypes.byref(sh))) == nb
+    bad = kda.make_shape(1000, 2, 64, 48, torch.float32, B=3)
+    assert int(kda.lib.kda_chunk_bwd_workspace_size(ctypes.byref(bad))) == 0
+    pro = kda.make_shape(1000, 2, 64, 64, torch.float32, B=3, prologue=3)
+    assert int(kda.lib.kda_chunk_bwd_workspace_size(ctypes.byref(pro))) == nb
+
+    def call(shape=sh, q=4096, dq=4096, dstate=None, ws=256 * 1000, wsb=nb):
+        return kda.lib.kda_chunk_bwd(P(q), P(4096), P(4096), P(4096), P(4096), None, None,
+                                     P(4096), None, P(dq), P(4096), P(4096), P(4096), P(4096),
+                                     P(dstate), ctypes.byref(shape), P(ws), wsb, None)
+
+    assert call(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(dq=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(dq=4100) == kda.KDA_ERR_INVALID_ARG            # misaligned gradient
+    assert call(dstate=4104) == kda.KDA_ERR_INVALID_ARG        # misaligned d_initial_state
+    assert call(wsb=nb - 256) == kda.KDA_ERR_INVALID_ARG       # workspace one step short
+    assert call(ws=256 * 1000 + 16) == kda.KDA_ERR_INVALID_ARG
+    assert call(shape=bad) == kda.KDA_ERR_UNSUPPORTED
+    assert call(shape=kda.make_shape(1000, 2, 64, 64, torch.float32, B=3, prologue=4)) == \
+        kda.KDA_ERR_INVALID_ARG
+
+
 def test_decode_argument_errors(kda):
     P = ctypes.c_void_p
     sh = kda.make_shape(1, 4, 128, 128, torch.bfloat16, B=8)

@@ -110,3 +110,35 @@ def test_backward_prologue(kda, dtype, d, prologue):
     if not prologue & 2:
         raw.g = ref.g
     _check(kda, raw, dtype, f"prologue={prologue} {dtype} d={d}", lb=-0.9, prologue=prologue)
+
+
+def test_backward_batched_layout_and_no_dout(kda):
+    """[B, T, H, d] inputs without cu_seqlens, and d_out = None (only dS_final drives L)."""
+    x = make_inputs(100, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=512, batch=3,
+                    state_std=0.02)
+    rng = np.random.default_rng(5)
+    d_fin = torch.tensor(rng.standard_normal((3, 2, 128, 128)), dtype=torch.float32)
+    args = [t.to(DEV).view(3, 100, *t.shape[1:]) for t in (x.q, x.k, x.v, x.g, x.beta)]
+    got = kda.chunk_bwd(*args, None, d_final_state=d_fin.to(DEV),
+                        initial_state=x.initial_state.to(DEV))
+    torch.cuda.synchronize()
+    ref = ko.backward(x.q, x.k, x.v, x.g, x.beta, d_out=None, d_final=d_fin,
+                      cu_seqlens=x.cu_seqlens.tolist(), initial_state=x.initial_state)
+    for name, gt in zip(NAMES, got):
+        rel, mx = errors(gt.reshape(ref[name].shape), ref[name])
+        assert rel <= TOL[torch.bfloat16], f"batched {name}: rel-L2 {rel:.3e}"
+
+
+def test_backward_bad_cu_seqlens_reports_without_trap(kda):
+    """A malformed cu_seqlens is skipped and reported in the workspace status word."""
+    x = make_inputs(None, H=2, dk=64, dv=64, dtype=torch.float32, seed=513,
+                    lengths=[100, 60], state_std=0.02)
+    cu = torch.tensor([0, 120, 100], dtype=torch.int32, device=DEV)  # not monotone
+    shape = kda.make_shape(160, 2, 64, 64, torch.float32, n_seqs=2, max_seqlen=120)
+    ws = torch.empty(int(kda.lib.kda_chunk_bwd_workspace_size(kda.ctypes.byref(shape))),
+                     dtype=torch.uint8, device=DEV)
+    d_out = torch.ones_like(x.v).to(DEV)
+    kda.chunk_bwd(*(t.to(DEV) for t in (x.q, x.k, x.v, x.g, x.beta)), d_out, cu_seqlens=cu,
+                  max_seqlen=120, workspace=ws)
+    rc, code = kda.workspace_status(ws)
+    assert rc == kda.KDA_ERR_DEVICE and code != 0
