@@ -12,7 +12,7 @@
 //   dT  = dU Y^T,        Z = T^T dU = dV
 //   dS  = Diag(gl) dS' + scale Q~^T dO - K~^T Z          (carried to the previous chunk)
 //   dN  = dT Diag(beta), dA = -N^T dN N^T,  dG = strict_lower(Diag(beta) dA)
-//   dbeta_r = sum_c N_cr dT_cr + sum_{s<r} (K~ K^^T)_rs dA_rs
+//   dbeta_r = sum_c N_cr dT_cr + sum_{s<r} (K~ K^^T)_rs dA_rs = ... + K~_r . (dA K^)_r
 //   dP  = scale lower_incl(dO U^T)
 //   dQ~ = scale dO S^T + dP K^,   dK~ = -Z S^T + dG K^
 //   dK^ = dP^T Q~ + dG^T K~ + (U dS'^T) gl,   dgl = rowsum(S dS') + colsum(K^ (U dS'^T))
@@ -521,22 +521,10 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     }
     __syncthreads();
 
-    // ---- 8. dG = strict_lower(Diag(beta) dA) in place, with dbeta += sum_s G dA (G = K~ K^^T
-    //         recomputed); dP = scale lower_incl(dO U^T) over (N^T dN)
+    // ---- 8. dA keeps its strict lower part (dG = Diag(beta) dA is applied where it is used);
+    //         dP = scale lower_incl(dO U^T) over (N^T dN)
     {
-      float accG[4][4] = {}, accP[4][4] = {};
-      for (int i = 0; i < DK; ++i) {
-        float kt[4], kh[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          kt[x] = sm.Kt[ty * 4 + x][i];
-          kh[x] = sm.Kh[tx * 4 + x][i];
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) accG[x][y] = fmaf(kt[x], kh[y], accG[x][y]);
-      }
+      float accP[4][4] = {};
       for (int j = 0; j < DVS; ++j) {
         float d[4], u[4];
 #pragma unroll
@@ -552,17 +540,12 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
         const int r = ty * 4 + x;
-        const float br = sm.bet[r];
-        float db = 0.f;
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
           const int c = tx * 4 + y;
-          const float da = sm.BP[r][c];
-          if (c < r) db = fmaf(accG[x][y], da, db);
-          sm.BP[r][c] = (c < r) ? br * da : 0.f;
+          if (c >= r) sm.BP[r][c] = 0.f;
           sm.BA[r][c] = (c <= r) ? scale * accP[x][y] : 0.f;
         }
-        atomicAdd(&sm.dbet[r], db);
       }
     }
     __syncthreads();
@@ -641,11 +624,36 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
           dgam[y][x] = acc[y][x] * sm.Qt[r][c];
           if (r < L) atomicAdd(a.acc_q + ((c0 + r) * H + h) * DK + c, acc[y][x] * E[y][x]);
         }
-      // 9c. dK~ = -Z S^T + dG K^  ->  dk (first part), dGamma
+      // 9c. dK~ = -Z S^T + Diag(beta) (dA K^)  ->  dk (first part), dGamma; and the A part
+      //     of dbeta, sum_s (K~ K^^T)_rs dA_rs = K~_r . (dA K^)_r
 #pragma unroll
       for (int y = 0; y < 4; ++y)
 #pragma unroll
         for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
+      for (int t = 0; t < rb + 3; ++t) {  // dA[r][t] = 0 for t >= r
+        float da4[4], kh[CT];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) da4[y] = sm.BP[rb + y][t];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) kh[x] = sm.Kh[t][cg + 16 * x];
+#pragma unroll
+        for (int y = 0; y < 4; ++y)
+#pragma unroll
+          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(da4[y], kh[x], acc[y][x]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int r = rb + y;
+        float db = 0.f;
+#pragma unroll
+        for (int x = 0; x < CT; ++x) db = fmaf(sm.Kt[r][cg + 16 * x], acc[y][x], db);
+#pragma unroll
+        for (int o2 = 8; o2 > 0; o2 >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o2);
+        if (cg == 0 && r < L) atomicAdd(a.acc_b + (c0 + r) * H + h, db);
+        const float br = sm.bet[r];
+#pragma unroll
+        for (int x = 0; x < CT; ++x) acc[y][x] *= br;
+      }
       for (int j = 0; j < DVS; ++j) {
         float z[4], sv[CT];
 #pragma unroll
@@ -656,17 +664,6 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         for (int y = 0; y < 4; ++y)
 #pragma unroll
           for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(-z[y], sv[x], acc[y][x]);
-      }
-      for (int t = 0; t < rb + 3; ++t) {  // dG[r][t] = 0 for t >= r
-        float dg4[4], kh[CT];
-#pragma unroll
-        for (int y = 0; y < 4; ++y) dg4[y] = sm.BP[rb + y][t];
-#pragma unroll
-        for (int x = 0; x < CT; ++x) kh[x] = sm.Kh[t][cg + 16 * x];
-#pragma unroll
-        for (int y = 0; y < 4; ++y)
-#pragma unroll
-          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(dg4[y], kh[x], acc[y][x]);
       }
 #pragma unroll
       for (int y = 0; y < 4; ++y)
@@ -705,12 +702,13 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         }
         dglp[x] = part;
       }
-      for (int t = rb; t < C; ++t) {  // dP[t][r] = 0 for t < r, dG[t][r] = 0 for t <= r
+      for (int t = rb; t < C; ++t) {  // dP[t][r] = 0 for t < r, dA[t][r] = 0 for t <= r
         float p[4], dg4[4], qt[CT], kt[CT];
+        const float bt = sm.bet[t];  // dG = Diag(beta) dA
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
           p[y] = sm.BA[t][rb + y];
-          dg4[y] = sm.BP[t][rb + y];
+          dg4[y] = bt * sm.BP[t][rb + y];
         }
 #pragma unroll
         for (int x = 0; x < CT; ++x) {
