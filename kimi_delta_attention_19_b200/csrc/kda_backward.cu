@@ -112,7 +112,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
   const int64_t snap0 = t0 / C;  // snapshot index of this sequence's first chunk end
   const int rcr = 2 * (tid >> 3), rcc = tid & 7;  // C x DVS tiles: rows rcr, rcr + 1;
                                                   // columns rcc + 8 x
-  const int tx = tid % 16, ty = tid / 16;         // 4x4 blocks of C x C tiles
+  const int tx = tid % 16, ty = tid / 16;         // C x C tiles: rows 4 ty + x, columns
+                                                  // tx + 16 y (conflict-free loads)
 
   for (int64_t cc = n_chunks - 1; cc >= 0; --cc) {
     const int64_t c0 = t0 + cc * C;
@@ -252,7 +253,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         for (int x = 0; x < 4; ++x) {
           kt[x] = sm.Kt[ty * 4 + x][i];
           qt[x] = sm.Qt[ty * 4 + x][i];
-          kh[x] = sm.Kh[tx * 4 + x][i];
+          kh[x] = sm.Kh[tx + 16 * x][i];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -266,7 +267,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
       for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
-          const int r = ty * 4 + x, c = tx * 4 + y;
+          const int r = ty * 4 + x, c = tx + 16 * y;
           sm.BA[r][c] = (c < r) ? sm.bet[r] * accA[x][y] : 0.f;
           sm.BP[r][c] = (c <= r) ? accP[x][y] : 0.f;
         }
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           du[x] = sm.dU[ty * 4 + x][j];
-          yy[x] = sm.Y[tx * 4 + x][j];
+          yy[x] = sm.Y[tx + 16 * x][j];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -430,7 +431,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
       for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int y = 0; y < 4; ++y) sm.BP[ty * 4 + x][tx * 4 + y] = acc[x][y];
+        for (int y = 0; y < 4; ++y) sm.BP[ty * 4 + x][tx + 16 * y] = acc[x][y];
       // sum_j S[i][j] dS'[i][j], NT / DK threads per channel
       constexpr int TPR = NT / DK, JPT = DVS / TPR;
       const int i = tid / TPR, j0p = (tid % TPR) * JPT;
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           nv[x] = sm.BN[c][ty * 4 + x];
-          dn[x] = sm.BP[c][tx * 4 + x];
+          dn[x] = sm.BP[c][tx + 16 * x];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
       for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int y = 0; y < 4; ++y) sm.BA[ty * 4 + x][tx * 4 + y] = acc[x][y];
+        for (int y = 0; y < 4; ++y) sm.BA[ty * 4 + x][tx + 16 * y] = acc[x][y];
     }
     __syncthreads();
     {
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           tv[x] = sm.BA[ty * 4 + x][c];
-          nv[x] = sm.BN[tx * 4 + x][c];
+          nv[x] = sm.BN[tx + 16 * x][c];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
       for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int y = 0; y < 4; ++y) sm.BP[ty * 4 + x][tx * 4 + y] = -acc[x][y];
+        for (int y = 0; y < 4; ++y) sm.BP[ty * 4 + x][tx + 16 * y] = -acc[x][y];
     }
     __syncthreads();
 
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
           d[x] = sm.dO[ty * 4 + x][j];
-          u[x] = sm.U[tx * 4 + x][j];
+          u[x] = sm.U[tx + 16 * x][j];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -542,7 +543,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         const int r = ty * 4 + x;
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
-          const int c = tx * 4 + y;
+          const int c = tx + 16 * y;
           if (c >= r) sm.BP[r][c] = 0.f;
           sm.BA[r][c] = (c <= r) ? scale * accP[x][y] : 0.f;
         }
