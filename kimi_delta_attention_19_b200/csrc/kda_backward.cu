@@ -41,12 +41,14 @@ struct BwdSmem {
   float BA[C][C + 1];    // A, then N^T dN, then dP
   float BN[C][C + 1];    // N = (I + A)^-1
   float BP[C][C + 1];    // P, then dT -> dN -> dA -> dG
-  float S[DK][DVS + 1];  // chunk start state (slice)
-  float dS[DK][DVS + 1]; // dL/d(chunk end state), updated in place to the chunk start
-  float Y[C][DVS + 1];   // V - K~ S, then Z = T^T dU (= dL/dV)
-  float U[C][DVS + 1];
-  float dO[C][DVS + 1];
-  float dU[C][DVS + 1];
+  // d_v-slice arrays: rows of DVS + 4 floats, 16-byte aligned, so products over the slice's
+  // columns read float4s (conflict-free with the stride of 36 words)
+  alignas(16) float S[DK][DVS + 4];  // chunk start state (slice)
+  alignas(16) float dS[DK][DVS + 4]; // dL/d(chunk end state), updated in place to the start
+  alignas(16) float Y[C][DVS + 4];   // V - K~ S, then Z = T^T dU (= dL/dV)
+  alignas(16) float U[C][DVS + 4];
+  alignas(16) float dO[C][DVS + 4];
+  alignas(16) float dU[C][DVS + 4];
   float gl[DK];
   float sdS[DK];         // sum_j S[i][j] dS'[i][j]: the decay of S's part of dgl
   float bet[C];
@@ -77,6 +79,11 @@ __device__ __forceinline__ void unpack_vec<__nv_bfloat16>(const uint4& u, float 
 // PRO: the raw-input prologue flags (KDA_PROLOGUE_*); the kernel then works on the
 // normalised q, k and the gate's log decays, and the finishing pass carries the gradients
 // through the prologue to the raw inputs.
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float dot4(const float4& a, const float4& b, float c) {
+  return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, c))));
+}
+
 template <typename Tin, int DK, int PRO>
 __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -203,10 +210,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
       for (int m = 0; m < NS; ++m) {
         const int e = tid + NT * m, i = e / SV, j = 4 * (e % SV);
-        sm.S[i][j] = sq[m].x;
-        sm.S[i][j + 1] = sq[m].y;
-        sm.S[i][j + 2] = sq[m].z;
-        sm.S[i][j + 3] = sq[m].w;
+        *reinterpret_cast<float4*>(&sm.S[i][j]) = sq[m];
       }
 #pragma unroll
       for (int m = 0; m < NO; ++m) {
@@ -416,17 +420,17 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     // ---- 5. dT = dU Y^T (over P, which is dead)                 (C x C tiles, 4 x 4)
     {
       float acc[4][4] = {};
-      for (int j = 0; j < DVS; ++j) {
-        float du[4], yy[4];
+      for (int j = 0; j < DVS; j += 4) {
+        float4 du[4], yy[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          du[x] = sm.dU[ty * 4 + x][j];
-          yy[x] = sm.Y[tx + 16 * x][j];
+          du[x] = ld4(&sm.dU[ty * 4 + x][j]);
+          yy[x] = ld4(&sm.Y[tx + 16 * x][j]);
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(du[x], yy[y], acc[x][y]);
+          for (int y = 0; y < 4; ++y) acc[x][y] = dot4(du[x], yy[y], acc[x][y]);
       }
 #pragma unroll
       for (int x = 0; x < 4; ++x)
@@ -526,17 +530,17 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     //         dP = scale lower_incl(dO U^T) over (N^T dN)
     {
       float accP[4][4] = {};
-      for (int j = 0; j < DVS; ++j) {
-        float d[4], u[4];
+      for (int j = 0; j < DVS; j += 4) {
+        float4 d[4], u[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          d[x] = sm.dO[ty * 4 + x][j];
-          u[x] = sm.U[tx + 16 * x][j];
+          d[x] = ld4(&sm.dO[ty * 4 + x][j]);
+          u[x] = ld4(&sm.U[tx + 16 * x][j]);
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
 #pragma unroll
-          for (int y = 0; y < 4; ++y) accP[x][y] = fmaf(d[x], u[y], accP[x][y]);
+          for (int y = 0; y < 4; ++y) accP[x][y] = dot4(d[x], u[y], accP[x][y]);
       }
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
@@ -591,16 +595,16 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
       for (int y = 0; y < 4; ++y)
 #pragma unroll
         for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
-      for (int j = 0; j < DVS; ++j) {
-        float o[4], sv[CT];
+      for (int j = 0; j < DVS; j += 4) {
+        float4 o[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) o[y] = sm.dO[rb + y][j];
+        for (int y = 0; y < 4; ++y) o[y] = ld4(&sm.dO[rb + y][j]);
 #pragma unroll
-        for (int x = 0; x < CT; ++x) sv[x] = sm.S[cg + 16 * x][j];
+        for (int x = 0; x < CT; ++x) {
+          const float4 sv = ld4(&sm.S[cg + 16 * x][j]);
 #pragma unroll
-        for (int y = 0; y < 4; ++y)
-#pragma unroll
-          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(o[y], sv[x], acc[y][x]);
+          for (int y = 0; y < 4; ++y) acc[y][x] = dot4(o[y], sv, acc[y][x]);
+        }
       }
 #pragma unroll
       for (int y = 0; y < 4; ++y)
@@ -655,16 +659,19 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 #pragma unroll
         for (int x = 0; x < CT; ++x) acc[y][x] *= br;
       }
-      for (int j = 0; j < DVS; ++j) {
-        float z[4], sv[CT];
+      for (int j = 0; j < DVS; j += 4) {
+        float4 z[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) z[y] = sm.Y[rb + y][j];
+        for (int y = 0; y < 4; ++y) {
+          z[y] = ld4(&sm.Y[rb + y][j]);
+          z[y] = make_float4(-z[y].x, -z[y].y, -z[y].z, -z[y].w);
+        }
 #pragma unroll
-        for (int x = 0; x < CT; ++x) sv[x] = sm.S[cg + 16 * x][j];
+        for (int x = 0; x < CT; ++x) {
+          const float4 sv = ld4(&sm.S[cg + 16 * x][j]);
 #pragma unroll
-        for (int y = 0; y < 4; ++y)
-#pragma unroll
-          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(-z[y], sv[x], acc[y][x]);
+          for (int y = 0; y < 4; ++y) acc[y][x] = dot4(z[y], sv, acc[y][x]);
+        }
       }
 #pragma unroll
       for (int y = 0; y < 4; ++y)
@@ -679,16 +686,16 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
       for (int y = 0; y < 4; ++y)
 #pragma unroll
         for (int x = 0; x < CT; ++x) acc[y][x] = 0.f;
-      for (int j = 0; j < DVS; ++j) {
-        float u[4], d[CT];
+      for (int j = 0; j < DVS; j += 4) {
+        float4 u[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) u[y] = sm.U[rb + y][j];
+        for (int y = 0; y < 4; ++y) u[y] = ld4(&sm.U[rb + y][j]);
 #pragma unroll
-        for (int x = 0; x < CT; ++x) d[x] = sm.dS[cg + 16 * x][j];
+        for (int x = 0; x < CT; ++x) {
+          const float4 d = ld4(&sm.dS[cg + 16 * x][j]);
 #pragma unroll
-        for (int y = 0; y < 4; ++y)
-#pragma unroll
-          for (int x = 0; x < CT; ++x) acc[y][x] = fmaf(u[y], d[x], acc[y][x]);
+          for (int y = 0; y < 4; ++y) acc[y][x] = dot4(u[y], d, acc[y][x]);
+        }
       }
       float dglp[CT];
 #pragma unroll
