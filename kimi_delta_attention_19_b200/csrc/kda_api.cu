@@ -166,9 +166,12 @@ namespace kda {
 namespace {
 
 // Backward workspace: [forward workspace (status word first) | per-chunk snapshots |
-// forward output scratch | fp32 accumulators dq, dk, dg, dbeta], each 256-byte aligned.
+// forward output scratch], each 256-byte aligned. The fp32 accumulators of dq, dk, dg,
+// dbeta reuse the forward workspace after its status header: they are zeroed only after
+// the forward has run (same stream), when its tiles are dead; the first region is as large
+// as the larger of the two.
 struct BwdPlan {
-  size_t fwd, snaps, out, acc_q, acc_k, acc_g, acc_b, total;
+  size_t snaps, out, acc_q, acc_k, acc_g, acc_b, total;
   int64_t n_snaps;
 };
 
@@ -182,14 +185,14 @@ bool bwd_plan(const kda_shape* shape, BwdPlan& p) {
   const size_t elem = shape->dtype == KDA_F32 ? 4 : 2;
   const size_t th = static_cast<size_t>(T_total) * shape->H;
   p.n_snaps = T_total / kChunk;
-  p.fwd = 0;
-  p.snaps = align_up(fwd, 256);
-  p.out = align_up(p.snaps + static_cast<size_t>(p.n_snaps) * shape->H * shape->dk * shape->dv * 4, 256);
-  p.acc_q = align_up(p.out + th * shape->dv * elem, 256);
+  p.acc_q = align_up(kWorkspaceHeader, 256);
   p.acc_k = p.acc_q + align_up(th * shape->dk * 4, 256);
   p.acc_g = p.acc_k + align_up(th * shape->dk * 4, 256);
   p.acc_b = p.acc_g + align_up(th * shape->dk * 4, 256);
-  p.total = p.acc_b + align_up(th * 4, 256);
+  const size_t acc_end = p.acc_b + align_up(th * 4, 256);
+  p.snaps = align_up(fwd > acc_end ? fwd : acc_end, 256);
+  p.out = align_up(p.snaps + static_cast<size_t>(p.n_snaps) * shape->H * shape->dk * shape->dv * 4, 256);
+  p.total = align_up(p.out + th * shape->dv * elem, 256);
   return true;
 }
 
@@ -239,7 +242,7 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
   st = chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, ws + p.out, nullptr, 1, snaps,
                  p.n_snaps, shape, ws, p.snaps, stream);
   if (st != KDA_OK) return st;
-  if (cudaMemsetAsync(ws + p.acc_q, 0, p.total - p.acc_q, cs) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaMemsetAsync(ws + p.acc_q, 0, p.snaps - p.acc_q, cs) != cudaSuccess) return KDA_ERR_CUDA;
 
   BackwardArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;

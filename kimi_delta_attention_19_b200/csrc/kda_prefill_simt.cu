@@ -41,8 +41,27 @@ struct SimtSmem {
   float U[C][DVS];
   float gl[DK];         // exp(Gamma_L) per channel
   float bet[C];
-  float rk[C], rq[C];   // prologue: 1 / |k row|, 1 / |q row|
 };
+
+// A 16-byte vector of inputs as floats
+template <typename T>
+__device__ __forceinline__ void unpack_vec(const uint4& u, float (&f)[16 / sizeof(T)]);
+template <>
+__device__ __forceinline__ void unpack_vec<float>(const uint4& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+template <>
+__device__ __forceinline__ void unpack_vec<__nv_bfloat16>(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(w[e] << 16);
+    f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
 
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
@@ -78,56 +97,88 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
 
     const bool l2n = (a.prologue & KDA_PROLOGUE_QK_L2NORM) != 0;
     const bool gsig = (a.prologue & KDA_PROLOGUE_GATE_SIGMOID) != 0;
-    if (l2n) {
-      // prologue: inverse L2 norms of the chunk's raw k and q rows, one warp per row
-      const int warp = tid >> 5, lane = tid & 31;
-      for (int rr = warp; rr < 2 * C; rr += NT / 32) {
-        const int r = rr % C;
-        const bool isq = rr >= C;
-        float ss = 0.f;
-        if (r < L) {
-          const Tin* src = (isq ? q : k) + ((c0 + r) * H + h) * DK;
-          for (int i = lane; i < DK; i += 32) {
-            const float x = ld_in(src + i);
-            ss = fmaf(x, x, ss);
+    // 1. Stage the chunk's k, q (unit rows with the prologue) and clamped log decays, the V
+    //    slice and beta: 16-byte vectors, every load issued before any store; rows past L
+    //    are zero (no key, no decay). Then the decay tiles in place, one channel per thread.
+    {
+      constexpr int EV = 16 / sizeof(Tin), VR = DK / EV, NV = C * VR / NT;
+      constexpr int OV = DVS / EV, NO = (C * OV + NT - 1) / NT;
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      uint4 kq[NV], qq[NV], gq[NV], vq[NO];
+#pragma unroll
+      for (int m = 0; m < NV; ++m) {
+        const int e = tid + NT * m, r = e / VR, vi = e % VR;
+        const int64_t off = ((c0 + r) * H + h) * DK + vi * EV;
+        kq[m] = r < L ? *reinterpret_cast<const uint4*>(k + off) : z;
+        qq[m] = r < L ? *reinterpret_cast<const uint4*>(q + off) : z;
+        gq[m] = r < L ? *reinterpret_cast<const uint4*>(g + off) : z;
+      }
+#pragma unroll
+      for (int m = 0; m < NO; ++m) {
+        const int e = tid + NT * m, r = e / OV, vj = e % OV;
+        const bool in = e < C * OV && r < L;
+        vq[m] = in ? *reinterpret_cast<const uint4*>(v + ((c0 + r) * H + h) * DV + j0 + vj * EV) : z;
+      }
+      if (tid < C) sm.bet[tid] = tid < L ? ld_in(beta + (c0 + tid) * H + h) : 0.f;
+#pragma unroll
+      for (int m = 0; m < NV; ++m) {
+        const int e = tid + NT * m, r = e / VR, i0 = (e % VR) * EV;
+        float kf[EV], qf[EV], gf[EV];
+        unpack_vec<Tin>(kq[m], kf);
+        unpack_vec<Tin>(qq[m], qf);
+        unpack_vec<Tin>(gq[m], gf);
+        if (l2n) {  // a row is VR consecutive lanes (VR divides 32): norms by shuffles
+          float sk = 0.f, sq2 = 0.f;
+#pragma unroll
+          for (int x = 0; x < EV; ++x) {
+            sk = fmaf(kf[x], kf[x], sk);
+            sq2 = fmaf(qf[x], qf[x], sq2);
+          }
+#pragma unroll
+          for (int o2 = VR / 2; o2 > 0; o2 >>= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, o2);
+            sq2 += __shfl_xor_sync(0xffffffffu, sq2, o2);
+          }
+          const float rk = inv_l2(sk), rq = inv_l2(sq2);
+#pragma unroll
+          for (int x = 0; x < EV; ++x) {
+            kf[x] *= rk;
+            qf[x] *= rq;
           }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) (isq ? sm.rq : sm.rk)[r] = inv_l2(ss);
+        for (int x = 0; x < EV; ++x) {
+          const float gx = gsig ? gate_from_preact(gf[x], a.lb) : gf[x];
+          sm.Kt[r][i0 + x] = kf[x];
+          sm.Qt[r][i0 + x] = qf[x];
+          sm.Kh[r][i0 + x] = r < L ? fmaxf(gx, a.lb) : 0.f;
+        }
       }
-      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < NO; ++m) {
+        const int e = tid + NT * m, r = e / OV, j = (e % OV) * EV;
+        if (e < C * OV) {
+          float vf[EV];
+          unpack_vec<Tin>(vq[m], vf);
+#pragma unroll
+          for (int x = 0; x < EV; ++x) sm.Y[r][j + x] = vf[x];
+        }
+      }
     }
-
-    // 1. Prefix sums of the clamped log decay and the decayed operands.
+    __syncthreads();
     if (tid < DK) {
       const int i = tid;
       float G = 0.f;
+#pragma unroll 8
       for (int r = 0; r < C; ++r) {
-        float kt = 0.f, kh = 0.f, qt = 0.f;
-        if (r < L) {
-          const int64_t off = ((c0 + r) * H + h) * DK + i;
-          float gr = ld_in(g + off);
-          if (gsig) gr = gate_from_preact(gr, a.lb);
-          G += fmaxf(gr, a.lb);
-          const float e = expf(G), ei = expf(-G);
-          const float kv = ld_in(k + off) * (l2n ? sm.rk[r] : 1.f);
-          kt = kv * e;
-          kh = kv * ei;
-          qt = ld_in(q + off) * (l2n ? sm.rq[r] : 1.f) * e;
-        }
-        sm.Kt[r][i] = kt;
-        sm.Kh[r][i] = kh;
-        sm.Qt[r][i] = qt;
+        G += sm.Kh[r][i];
+        const float e = expf(G), ei = expf(-G);
+        const float kv = sm.Kt[r][i];
+        sm.Kt[r][i] = kv * e;
+        sm.Kh[r][i] = kv * ei;
+        sm.Qt[r][i] *= e;
       }
       sm.gl[i] = expf(G);
-    } else {
-      for (int e = tid - DK; e < C * DVS; e += NT - DK) {
-        const int r = e / DVS, c = e % DVS;
-        sm.Y[r][c] = (r < L) ? ld_in(v + ((c0 + r) * H + h) * DV + j0 + c) : 0.f;
-      }
-      for (int r = tid - DK; r < C; r += NT - DK)
-        sm.bet[r] = (r < L) ? ld_in(beta + (c0 + r) * H + h) : 0.f;
     }
     __syncthreads();
 
@@ -145,7 +196,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
         for (int x = 0; x < 4; ++x) {
           kt[x] = sm.Kt[ty * 4 + x][i];
           qt[x] = sm.Qt[ty * 4 + x][i];
-          kh[x] = sm.Kh[tx * 4 + x][i];
+          kh[x] = sm.Kh[tx + 16 * x][i];
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x)
@@ -159,29 +210,84 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       for (int x = 0; x < 4; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
-          const int r = ty * 4 + x, c = tx * 4 + y;
+          const int r = ty * 4 + x, c = tx + 16 * y;
           sm.A[r][c] = (c < r) ? sm.bet[r] * accA[x][y] : 0.f;
           sm.P[r][c] = (c <= r) ? accP[x][y] : 0.f;
         }
     }
     __syncthreads();
 
-    // 3. T = (I + A)^{-1} Diag(beta) by forward substitution, one row at a time.
-    if (tid < C) {
-      for (int r = L; r < C; ++r) sm.Tm[r][tid] = 0.f;
+    // 3. N = (I + A)^{-1} into Tm (T = N Diag(beta) is applied in step 5): the four 16x16
+    //    diagonal blocks by forward substitution, one per half-warp; then 16 -> 32 and
+    //    32 -> 64 merges N21 = -N22 (A21 N11) by all threads (A21 is overwritten by A21 N11;
+    //    A is not needed afterwards). Rows past L: A is zero there, N the identity.
+    for (int e = tid; e < C * C; e += NT) {
+      const int rr = e / C, cc = e % C;
+      if ((rr >> 4) != (cc >> 4)) sm.Tm[rr][cc] = 0.f;
     }
-    for (int r = 0; r < L; ++r) {
-      if (tid < C) {
-        const int c = tid;
-        float val = 0.f;
-        if (c <= r) {
-          val = (c == r) ? sm.bet[r] : 0.f;
-          for (int s2 = c; s2 < r; ++s2) val = fmaf(-sm.A[r][s2], sm.Tm[s2][c], val);
-        }
-        sm.Tm[r][c] = val;
+    if (tid < 64) {
+      const int base = 16 * (tid >> 4), c = tid & 15;
+      for (int rr = 0; rr < 16; ++rr) {
+        float val = (c == rr) ? 1.f : 0.f;
+        for (int s2 = c; s2 < rr; ++s2)
+          val = fmaf(-sm.A[base + rr][base + s2], sm.Tm[base + s2][base + c], val);
+        sm.Tm[base + rr][base + c] = (c <= rr) ? val : 0.f;
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    {
+      const int o = 32 * (tid >> 7);
+      float xv[2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m, rr = idx >> 4, cc = idx & 15;
+        float acc = 0.f;
+        for (int s2 = cc; s2 < 16; ++s2) acc = fmaf(sm.A[o + 16 + rr][o + s2], sm.Tm[o + s2][o + cc], acc);
+        xv[m] = acc;
       }
       __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m;
+        sm.A[o + 16 + (idx >> 4)][o + (idx & 15)] = xv[m];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int idx = (tid & 127) + 128 * m, rr = idx >> 4, cc = idx & 15;
+        float acc = 0.f;
+        for (int s2 = 0; s2 <= rr; ++s2)
+          acc = fmaf(sm.Tm[o + 16 + rr][o + 16 + s2], sm.A[o + 16 + s2][o + cc], acc);
+        sm.Tm[o + 16 + rr][o + cc] = -acc;
+      }
     }
+    __syncthreads();
+    {
+      float xv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m, rr = idx >> 5, cc = idx & 31;
+        float acc = 0.f;
+        for (int s2 = cc; s2 < 32; ++s2) acc = fmaf(sm.A[32 + rr][s2], sm.Tm[s2][cc], acc);
+        xv[m] = acc;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m;
+        sm.A[32 + (idx >> 5)][idx & 31] = xv[m];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int idx = tid + NT * m, rr = idx >> 5, cc = idx & 31;
+        float acc = 0.f;
+        for (int s2 = 0; s2 <= rr; ++s2) acc = fmaf(sm.Tm[32 + rr][32 + s2], sm.A[32 + s2][cc], acc);
+        sm.Tm[32 + rr][cc] = -acc;
+      }
+    }
+    __syncthreads();
 
     const int r = tid / 4, cb = (tid % 4) * 8;
     // 4. Y = V - K~ S
@@ -204,7 +310,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = 0.f;
       for (int s2 = 0; s2 <= r; ++s2) {
-        const float t = sm.Tm[r][s2];
+        const float t = sm.Tm[r][s2] * sm.bet[s2];  // T = N Diag(beta)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] = fmaf(t, sm.Y[s2][cb + c], acc[c]);
       }
