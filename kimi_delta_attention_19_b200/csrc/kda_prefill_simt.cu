@@ -36,12 +36,21 @@ struct SimtSmem {
   float A[C][C + 1];
   float P[C][C + 1];
   float Tm[C][C + 1];
-  float S[DK][DVS];     // state slice
-  float Y[C][DVS];      // V slice, then V - K~ S
-  float U[C][DVS];
+  alignas(16) float S[DK][DVS];  // state slice
+  alignas(16) float Y[C][DVS];   // V slice, then V - K~ S
+  alignas(16) float U[C][DVS];
   float gl[DK];         // exp(Gamma_L) per channel
   float bet[C];
 };
+
+// acc[0..3] += a * v (S, Y and U rows are 32 floats, 16-byte aligned: float4 reads)
+__device__ __forceinline__ void axpy4(float a, const float* v, float* acc) {
+  const float4 x = *reinterpret_cast<const float4*>(v);
+  acc[0] = fmaf(a, x.x, acc[0]);
+  acc[1] = fmaf(a, x.y, acc[1]);
+  acc[2] = fmaf(a, x.z, acc[2]);
+  acc[3] = fmaf(a, x.w, acc[3]);
+}
 
 // A 16-byte vector of inputs as floats
 template <typename T>
@@ -297,8 +306,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       for (int c = 0; c < 8; ++c) acc[c] = 0.f;
       for (int i = 0; i < DK; ++i) {
         const float kt = sm.Kt[r][i];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(kt, sm.S[i][cb + c], acc[c]);
+        axpy4(kt, &sm.S[i][cb], acc);
+        axpy4(kt, &sm.S[i][cb + 4], acc + 4);
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) sm.Y[r][cb + c] -= acc[c];
@@ -311,8 +320,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       for (int c = 0; c < 8; ++c) acc[c] = 0.f;
       for (int s2 = 0; s2 <= r; ++s2) {
         const float t = sm.Tm[r][s2] * sm.bet[s2];  // T = N Diag(beta)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(t, sm.Y[s2][cb + c], acc[c]);
+        axpy4(t, &sm.Y[s2][cb], acc);
+        axpy4(t, &sm.Y[s2][cb + 4], acc + 4);
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) sm.U[r][cb + c] = acc[c];
@@ -325,13 +334,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       for (int c = 0; c < 8; ++c) acc[c] = 0.f;
       for (int i = 0; i < DK; ++i) {
         const float qt = sm.Qt[r][i];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(qt, sm.S[i][cb + c], acc[c]);
+        axpy4(qt, &sm.S[i][cb], acc);
+        axpy4(qt, &sm.S[i][cb + 4], acc + 4);
       }
       for (int s2 = 0; s2 <= r; ++s2) {
         const float p = sm.P[r][s2];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = fmaf(p, sm.U[s2][cb + c], acc[c]);
+        axpy4(p, &sm.U[s2][cb], acc);
+        axpy4(p, &sm.U[s2][cb + 4], acc + 4);
       }
       if (r < L) {
         Tin* o = out + ((c0 + r) * H + h) * DV + j0 + cb;
@@ -351,7 +360,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_simt_kernel(PrefillArgs a) {
       for (int rr = 0; rr < L; ++rr) {
         const float kb = sm.Kh[rr][i] * gli;
 #pragma unroll
-        for (int c = 0; c < PER; ++c) acc[c] = fmaf(kb, sm.U[rr][cs + c], acc[c]);
+        for (int c = 0; c < PER; c += 4) axpy4(kb, &sm.U[rr][cs + c], acc + c);
       }
       __syncthreads();
 #pragma unroll
