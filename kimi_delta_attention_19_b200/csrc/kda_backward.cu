@@ -22,8 +22,9 @@
 // One CTA per (sequence, head, 32-column slice of d_v) walks the chunks backwards. The
 // columns of S and dS evolve independently, so dv, dS and dS0 of a slice are complete in
 // its CTA; dq, dk, dg and dbeta are sums over the slices and are added, in fp32, into
-// accumulators that a final pass converts to the input dtype. The chunk start states
-// come from a forward pass that keeps the state after every chunk.
+// accumulators that a finishing pass converts to the input dtype (carrying them through
+// the raw-input prologue when it is on). The chunk start states come from a forward pass
+// that keeps the state after every chunk.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -40,7 +41,8 @@ struct BwdSmem {
   float Qt[C][DK + 1];   // Q~
   float BA[C][C + 1];    // A, then N^T dN, then dP
   float BN[C][C + 1];    // N = (I + A)^-1
-  float BP[C][C + 1];    // P, then dT -> dN -> dA -> dG
+  float BP[C][C + 1];    // P, then dT -> dN -> dA (strict lower; dG = Diag(beta) dA is
+                         // applied where it is used)
   // d_v-slice arrays: rows of DVS + 4 floats, 16-byte aligned, so products over the slice's
   // columns read float4s (conflict-free with the stride of 36 words)
   alignas(16) float S[DK][DVS + 4];  // chunk start state (slice)
@@ -127,9 +129,10 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     const int L = (t1 - c0) < C ? (int)(t1 - c0) : C;
     __syncthreads();  // the previous chunk's reads are done
 
-    // ---- 0. stage the chunk's raw k, q and clamped g (all threads, coalesced; rows past L
-    //         are zero: no key, no decay) and the slice's S, V, dO and beta; then the decay
-    //         tiles in place, one channel per thread
+    // ---- 0. stage the chunk's k, q and clamped log decays (normalised and gated with the
+    //         prologue; all threads, coalesced; rows past L are zero: no key, no decay) and
+    //         the slice's S, V, dO and beta; then the decay tiles in place, one channel per
+    //         thread
     {
       // k, q, g rows: 16-byte vectors, all of a thread's loads issued before any store
       constexpr int EV = 16 / sizeof(Tin);        // elements per vector
