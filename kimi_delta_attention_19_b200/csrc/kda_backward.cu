@@ -31,10 +31,11 @@ namespace kda {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int DVS = 32;   // d_v columns per CTA
 constexpr int NT = 256;   // threads per CTA
 
-template <int DK>
+// DVS: the d_v columns of one CTA (32, or 16 when the sequences and heads alone give too
+// few CTAs to fill the GPU)
+template <int DK, int DVS>
 struct BwdSmem {
   float Kt[C][DK + 1];   // K~
   float Kh[C][DK + 1];   // K^
@@ -86,10 +87,10 @@ __device__ __forceinline__ float dot4(const float4& a, const float4& b, float c)
   return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, c))));
 }
 
-template <typename Tin, int DK, int PRO>
+template <typename Tin, int DK, int DVS, int PRO>
 __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  BwdSmem<DK>& sm = *reinterpret_cast<BwdSmem<DK>*>(smem_raw);
+  BwdSmem<DK, DVS>& sm = *reinterpret_cast<BwdSmem<DK, DVS>*>(smem_raw);
   constexpr int CT = DK / 16;   // channels per thread in the per-element pass
   const int n_slices = a.dv / DVS;
   const int slice = blockIdx.x % n_slices;
@@ -119,8 +120,9 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 
   const int64_t n_chunks = (t1 - t0 + C - 1) / C;
   const int64_t snap0 = t0 / C;  // snapshot index of this sequence's first chunk end
-  const int rcr = 2 * (tid >> 3), rcc = tid & 7;  // C x DVS tiles: rows rcr, rcr + 1;
-                                                  // columns rcc + 8 x
+  // C x DVS tiles: RR rows from rcr, columns rcc + RCW x (x < 4)
+  constexpr int RCW = DVS / 4, RR = C * DVS / (NT * 4);
+  const int rcr = RR * (tid / RCW), rcc = tid % RCW;
   const int tx = tid % 16, ty = tid / 16;         // C x C tiles: rows 4 ty + x, columns
                                                   // tx + 16 y (conflict-free loads)
 
@@ -354,69 +356,78 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
     }
     __syncthreads();
 
-    // ---- 3. Y = V - K~ S, then U = N Diag(beta) Y            (C x DVS tiles, 2 x 4)
+    // ---- 3. Y = V - K~ S, then U = N Diag(beta) Y            (C x DVS tiles, RR x 4)
     {
-      float acc[2][4] = {};
+      float acc[RR][4] = {};
       for (int i = 0; i < DK; ++i) {
-        const float k0 = sm.Kt[rcr][i], k1 = sm.Kt[rcr + 1][i];
+        float kr[RR];
+#pragma unroll
+        for (int y = 0; y < RR; ++y) kr[y] = sm.Kt[rcr + y][i];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const float sv = sm.S[i][rcc + 8 * x];
-          acc[0][x] = fmaf(k0, sv, acc[0][x]);
-          acc[1][x] = fmaf(k1, sv, acc[1][x]);
+          const float sv = sm.S[i][rcc + RCW * x];
+#pragma unroll
+          for (int y = 0; y < RR; ++y) acc[y][x] = fmaf(kr[y], sv, acc[y][x]);
         }
       }
 #pragma unroll
-      for (int y = 0; y < 2; ++y)
+      for (int y = 0; y < RR; ++y)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) sm.Y[rcr + y][rcc + 8 * x] -= acc[y][x];
+        for (int x = 0; x < 4; ++x) sm.Y[rcr + y][rcc + RCW * x] -= acc[y][x];
     }
     __syncthreads();
     {
-      float acc[2][4] = {};
-      for (int s2 = 0; s2 <= rcr + 1; ++s2) {  // N is lower triangular
+      float acc[RR][4] = {};
+      for (int s2 = 0; s2 < rcr + RR; ++s2) {  // N is lower triangular
         const float b = sm.bet[s2];
-        const float n0 = sm.BN[rcr][s2] * b, n1 = sm.BN[rcr + 1][s2] * b;
+        float nr[RR];
+#pragma unroll
+        for (int y = 0; y < RR; ++y) nr[y] = sm.BN[rcr + y][s2] * b;
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const float yv = sm.Y[s2][rcc + 8 * x];
-          acc[0][x] = fmaf(n0, yv, acc[0][x]);
-          acc[1][x] = fmaf(n1, yv, acc[1][x]);
+          const float yv = sm.Y[s2][rcc + RCW * x];
+#pragma unroll
+          for (int y = 0; y < RR; ++y) acc[y][x] = fmaf(nr[y], yv, acc[y][x]);
         }
       }
 #pragma unroll
-      for (int y = 0; y < 2; ++y)
+      for (int y = 0; y < RR; ++y)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) sm.U[rcr + y][rcc + 8 * x] = acc[y][x];
+        for (int x = 0; x < 4; ++x) sm.U[rcr + y][rcc + RCW * x] = acc[y][x];
     }
     __syncthreads();
 
     // ---- 4. dU = (K^ gl) dS' + scale P^T dO
     {
-      float acc[2][4] = {}, acc2[2][4] = {};
+      float acc[RR][4] = {}, acc2[RR][4] = {};
       for (int i = 0; i < DK; ++i) {
         const float gi = sm.gl[i];
-        const float k0 = sm.Kh[rcr][i] * gi, k1 = sm.Kh[rcr + 1][i] * gi;
+        float kr[RR];
+#pragma unroll
+        for (int y = 0; y < RR; ++y) kr[y] = sm.Kh[rcr + y][i] * gi;
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const float dv0 = sm.dS[i][rcc + 8 * x];
-          acc[0][x] = fmaf(k0, dv0, acc[0][x]);
-          acc[1][x] = fmaf(k1, dv0, acc[1][x]);
+          const float dv0 = sm.dS[i][rcc + RCW * x];
+#pragma unroll
+          for (int y = 0; y < RR; ++y) acc[y][x] = fmaf(kr[y], dv0, acc[y][x]);
         }
       }
       for (int t = rcr; t < C; ++t) {  // P[t][r] = 0 for t < r
-        const float p0 = sm.BP[t][rcr], p1 = sm.BP[t][rcr + 1];
+        float pr[RR];
+#pragma unroll
+        for (int y = 0; y < RR; ++y) pr[y] = sm.BP[t][rcr + y];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const float o = sm.dO[t][rcc + 8 * x];
-          acc2[0][x] = fmaf(p0, o, acc2[0][x]);
-          acc2[1][x] = fmaf(p1, o, acc2[1][x]);
+          const float o = sm.dO[t][rcc + RCW * x];
+#pragma unroll
+          for (int y = 0; y < RR; ++y) acc2[y][x] = fmaf(pr[y], o, acc2[y][x]);
         }
       }
 #pragma unroll
-      for (int y = 0; y < 2; ++y)
+      for (int y = 0; y < RR; ++y)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) sm.dU[rcr + y][rcc + 8 * x] = fmaf(scale, acc2[y][x], acc[y][x]);
+        for (int x = 0; x < 4; ++x)
+          sm.dU[rcr + y][rcc + RCW * x] = fmaf(scale, acc2[y][x], acc[y][x]);
     }
     __syncthreads();
 
@@ -453,24 +464,26 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 
     // ---- 6. Z = Diag(beta) N^T dU (= dL/dV, over Y); dbeta from T = N Diag(beta)
     {
-      float acc[2][4] = {};
+      float acc[RR][4] = {};
       for (int t = rcr; t < C; ++t) {  // N[t][r] = 0 for t < r
-        const float n0 = sm.BN[t][rcr], n1 = sm.BN[t][rcr + 1];
+        float nr[RR];
+#pragma unroll
+        for (int y = 0; y < RR; ++y) nr[y] = sm.BN[t][rcr + y];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const float d = sm.dU[t][rcc + 8 * x];
-          acc[0][x] = fmaf(n0, d, acc[0][x]);
-          acc[1][x] = fmaf(n1, d, acc[1][x]);
+          const float d = sm.dU[t][rcc + RCW * x];
+#pragma unroll
+          for (int y = 0; y < RR; ++y) acc[y][x] = fmaf(nr[y], d, acc[y][x]);
         }
       }
 #pragma unroll
-      for (int y = 0; y < 2; ++y) {
+      for (int y = 0; y < RR; ++y) {
         const int r = rcr + y;
         const float b = sm.bet[r];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          sm.Y[r][rcc + 8 * x] = b * acc[y][x];
-          if (r < L) st_out(dvo + ((c0 + r) * H + h) * DV + j0 + rcc + 8 * x, b * acc[y][x]);
+          sm.Y[r][rcc + RCW * x] = b * acc[y][x];
+          if (r < L) st_out(dvo + ((c0 + r) * H + h) * DV + j0 + rcc + RCW * x, b * acc[y][x]);
         }
       }
       if (tid < C) {
@@ -780,8 +793,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
 
     // ---- 10. dS <- Diag(gl) dS' + scale Q~^T dO - K~^T Z        (DK x DVS tiles, IT x 4)
     {
-      constexpr int IT = DK / 32;
-      const int ib = (tid >> 3) * IT, jc = tid & 7;
+      constexpr int JG = DVS / 4, IT = DK * DVS / (NT * 4);
+      const int ib = (tid / JG) * IT, jc = tid % JG;
       float a1[IT][4] = {}, a2[IT][4] = {};
       for (int r = 0; r < C; ++r) {
         float qt[IT], kt[IT], o[4], z[4];
@@ -792,8 +805,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         }
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          o[x] = sm.dO[r][jc + 8 * x];
-          z[x] = sm.Y[r][jc + 8 * x];
+          o[x] = sm.dO[r][jc + JG * x];
+          z[x] = sm.Y[r][jc + JG * x];
         }
 #pragma unroll
         for (int y = 0; y < IT; ++y)
@@ -809,7 +822,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_simt_kernel(BackwardArgs a) {
         const float gi = sm.gl[i];
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-          const int j = jc + 8 * x;
+          const int j = jc + JG * x;
           sm.dS[i][j] = fmaf(gi, sm.dS[i][j], fmaf(scale, a1[y][x], -a2[y][x]));
         }
       }
@@ -875,26 +888,34 @@ __global__ void bwd_gate_kernel(const float* __restrict__ acc, const Tin* __rest
   }
 }
 
-template <typename Tin, int DK, int PRO>
+template <typename Tin, int DK, int DVS, int PRO>
 cudaError_t launch_kernel(const BackwardArgs& a, cudaStream_t st) {
-  const size_t smem = sizeof(BwdSmem<DK>);
-  cudaError_t e = cudaFuncSetAttribute(bwd_simt_kernel<Tin, DK, PRO>,
+  const size_t smem = sizeof(BwdSmem<DK, DVS>);
+  cudaError_t e = cudaFuncSetAttribute(bwd_simt_kernel<Tin, DK, DVS, PRO>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)a.n_seqs * a.H * (a.dv / DVS);
   if (blocks == 0) return cudaSuccess;
-  bwd_simt_kernel<Tin, DK, PRO><<<(unsigned)blocks, NT, smem, st>>>(a);
+  bwd_simt_kernel<Tin, DK, DVS, PRO><<<(unsigned)blocks, NT, smem, st>>>(a);
   return cudaGetLastError();
 }
 
+template <typename Tin, int DK, int DVS>
+cudaError_t launch_width(const BackwardArgs& a, cudaStream_t st) {
+  switch (a.prologue) {
+    case 0: return launch_kernel<Tin, DK, DVS, 0>(a, st);
+    case 1: return launch_kernel<Tin, DK, DVS, 1>(a, st);
+    case 2: return launch_kernel<Tin, DK, DVS, 2>(a, st);
+    default: return launch_kernel<Tin, DK, DVS, 3>(a, st);
+  }
+}
+
+// One CTA per SM at most: 32-column slices unless they leave more than half the SMs idle,
+// then 16-column slices (twice the CTAs; each recomputes the chunk's decay tiles and inverse)
 template <typename Tin, int DK>
 cudaError_t launch_typed(const BackwardArgs& a, cudaStream_t st) {
-  switch (a.prologue) {
-    case 0: return launch_kernel<Tin, DK, 0>(a, st);
-    case 1: return launch_kernel<Tin, DK, 1>(a, st);
-    case 2: return launch_kernel<Tin, DK, 2>(a, st);
-    default: return launch_kernel<Tin, DK, 3>(a, st);
-  }
+  const int64_t wide = (int64_t)a.n_seqs * a.H * (a.dv / 32);
+  return 2 * wide <= 148 ? launch_width<Tin, DK, 16>(a, st) : launch_width<Tin, DK, 32>(a, st);
 }
 
 unsigned grid_for(int64_t n, int threads) {
