@@ -182,7 +182,7 @@ size_t kda_chunk_bwd_workspace_size(const kda_shape *shape);
  *  d_initial_state [n, H, dk, dv] fp32 (written), or NULL to skip
  *  workspace    >= kda_chunk_bwd_workspace_size(shape) bytes, 256-byte aligned.
  * g enters through max(g, lb): where g < lb its gradient is 0 (at g == lb it passes).
- * Computed in fp32 on CUDA cores (one CTA per sequence, head and 32-column slice of dv);
+ * Computed in fp32 on CUDA cores (one CTA per sequence, head and 32- or 16-column slice of dv);
  * dq, dk, dg and dbeta sum the slices' contributions with fp32 atomics, so their last
  * bits may differ between runs. Errors as in kda_chunk_fwd.
  */

@@ -19,7 +19,7 @@
 //   dGamma = dK~ K~ - dK^ K^ + dQ~ Q~ (+ dgl gl on the last row), dg' = reverse cumsum,
 //   dg = dg' where g >= lb,   dq = dQ~ E,   dk = dK~ E + dK^ / E
 //
-// One CTA per (sequence, head, 32-column slice of d_v) walks the chunks backwards. The
+// One CTA per (sequence, head, slice of 32 or 16 columns of d_v) walks the chunks backwards. The
 // columns of S and dS evolve independently, so dv, dS and dS0 of a slice are complete in
 // its CTA; dq, dk, dg and dbeta are sums over the slices and are added, in fp32, into
 // accumulators that a finishing pass converts to the input dtype (carrying them through
