@@ -184,7 +184,9 @@ size_t kda_chunk_bwd_workspace_size(const kda_shape *shape);
  * g enters through max(g, lb): where g < lb its gradient is 0 (at g == lb it passes).
  * Computed in fp32 on CUDA cores (one CTA per sequence, head and 32- or 16-column slice of dv);
  * dq, dk, dg and dbeta sum the slices' contributions with fp32 atomics, so their last
- * bits may differ between runs. Errors as in kda_chunk_fwd.
+ * bits may differ between runs. Errors as in kda_chunk_fwd; when its forward pass skips a
+ * sequence (malformed cu_seqlens, or longer than max_seqlen) KDA_ERR_DEVICE is recorded and
+ * that sequence's gradients are unspecified.
  */
 kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
                          const void *beta, const float *initial_state,
