@@ -289,6 +289,7 @@ def bench_ours(args, world, rank, local):
     tok_bytes = N * Hd * (3 * d + d + 1) * 2 + N * Hd * d * 2
     d_gbs = (state_bytes + tok_bytes) / (d_ms / 1e3) / 1e9
     decode = {"workload": DECODE, "steps": dsteps, "ms_per_step": round(d_ms, 5),
+              "launch": "eager: one kda_decode_step per step, no CUDA graph",
               "state_gbs": round(d_gbs * world, 1), "unit": "GB/s",
               "tokens_per_s": round(N * world / (d_ms / 1e3), 1),
               "roofline": {"bound": "hbm", "achieved": round(d_gbs, 1), "peak": peaks["hbm_gbs"],
