@@ -88,7 +88,13 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _ptr(t: torch.Tensor | None):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor argument; the C ABI takes contiguous token-major tensors."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError(f"KDA tensors must be contiguous (got strides {tuple(t.stride())} "
+                         f"for shape {tuple(t.shape)})")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:

@@ -171,6 +171,16 @@ def test_decode_argument_errors(kda):
         kda.KDA_ERR_INVALID_ARG
 
 
+def test_binding_rejects_non_contiguous_tensors(kda):
+    """A strided view would be read as the wrong memory: the binding refuses it before any
+    library call."""
+    q = torch.zeros(8, 2, 64).transpose(0, 1)
+    with pytest.raises(ValueError, match="contiguous"):
+        kda._ptr(q)
+    assert kda._ptr(None) is None
+    assert kda._ptr(torch.zeros(4, 4)).value is not None
+
+
 def test_binding_refuses_without_library(tmp_path, monkeypatch):
     """With libkda.so absent the binding raises instead of falling back."""
     import importlib.util
