@@ -249,6 +249,42 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     return dq, dkk, dvv, dg, dbeta, ds0
 
 
+class _ChunkKDA(torch.autograd.Function):
+    """chunk_fwd with chunk_bwd as its backward (both in the library's kernels)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, beta, initial_state, cu_seqlens, max_seqlen, scale, lb,
+                prologue):
+        out, fin = chunk_fwd(q, k, v, g, beta, initial_state=initial_state,
+                             cu_seqlens=cu_seqlens, max_seqlen=max_seqlen, scale=scale, lb=lb,
+                             prologue=prologue)
+        ctx.save_for_backward(q, k, v, g, beta, initial_state, cu_seqlens)
+        ctx.opts = (max_seqlen, scale, lb, prologue)
+        return out, fin
+
+    @staticmethod
+    def backward(ctx, d_out, d_fin):
+        q, k, v, g, beta, s0, cu = ctx.saved_tensors
+        max_seqlen, scale, lb, prologue = ctx.opts
+        dq, dk, dv, dg, dbeta, ds0 = chunk_bwd(
+            q, k, v, g, beta, None if d_out is None else d_out.contiguous(),
+            d_final_state=None if d_fin is None else d_fin.contiguous(), initial_state=s0,
+            cu_seqlens=cu, max_seqlen=max_seqlen, scale=scale, lb=lb,
+            want_d_initial=s0 is not None and ctx.needs_input_grad[5], prologue=prologue)
+        return dq, dk, dv, dg, dbeta, ds0, None, None, None, None, None
+
+
+def kda_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, *, initial_state: torch.Tensor | None = None,
+                  cu_seqlens: torch.Tensor | None = None, max_seqlen: int = 0,
+                  scale: float | None = None, lb: float = -1.0, prologue: int = 0):
+    """Differentiable chunked prefill: (out, final_state) as chunk_fwd returns them, with
+    gradients for q, k, v, g, beta and initial_state from kda_chunk_bwd (for training).
+    Same layouts and options as chunk_fwd."""
+    return _ChunkKDA.apply(q, k, v, g, beta, initial_state, cu_seqlens, max_seqlen, scale, lb,
+                           prologue)
+
+
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 

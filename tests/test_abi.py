@@ -181,6 +181,46 @@ def test_binding_rejects_non_contiguous_tensors(kda):
     assert kda._ptr(torch.zeros(4, 4)).value is not None
 
 
+def test_autograd_plumbing_with_stand_in_calls(kda, monkeypatch):
+    """kda_attention's autograd wiring on CPU, with stand-ins for the two library calls:
+    the options reach both calls, dL/dout and dL/dfinal_state reach the backward call, and
+    its six gradients come back to the right inputs (dS0 only when asked for)."""
+    seen = {}
+
+    def fwd(q, k, v, g, beta, **kw):
+        seen["fwd"] = kw
+        return torch.zeros(v.shape), torch.zeros(1, q.shape[1], q.shape[2], v.shape[2])
+
+    def bwd(q, k, v, g, beta, d_out, **kw):
+        seen["bwd"] = (d_out.clone(), kw)
+        ds0 = torch.full((1, q.shape[1], q.shape[2], v.shape[2]), 6.0)
+        return (torch.full_like(q, 1.0), torch.full_like(k, 2.0), torch.full_like(v, 3.0),
+                torch.full_like(g, 4.0), torch.full_like(beta, 5.0),
+                ds0 if kw["want_d_initial"] else None)
+
+    monkeypatch.setattr(kda, "chunk_fwd", fwd)
+    monkeypatch.setattr(kda, "chunk_bwd", bwd)
+    q, k, g = (torch.randn(10, 2, 4, requires_grad=True) for _ in range(3))
+    v = torch.randn(10, 2, 3, requires_grad=True)
+    b = torch.rand(10, 2, requires_grad=True)
+    s0 = torch.randn(1, 2, 4, 3, requires_grad=True)
+    out, fin = kda.kda_attention(q, k, v, g, b, initial_state=s0, scale=0.3, lb=-0.5,
+                                 prologue=1)
+    (2.0 * out.sum() + 3.0 * fin.sum()).backward()
+    assert seen["fwd"]["scale"] == 0.3 and seen["fwd"]["lb"] == -0.5
+    assert seen["fwd"]["prologue"] == 1
+    d_out, kw = seen["bwd"]
+    assert torch.equal(d_out, torch.full((10, 2, 3), 2.0))
+    assert torch.equal(kw["d_final_state"], torch.full((1, 2, 4, 3), 3.0))
+    assert kw["want_d_initial"] and kw["initial_state"] is not None and kw["prologue"] == 1
+    for t, val in ((q, 1.0), (k, 2.0), (v, 3.0), (g, 4.0), (b, 5.0), (s0, 6.0)):
+        assert torch.equal(t.grad, torch.full_like(t, val))
+    # no initial state: no dS0 asked for
+    out, fin = kda.kda_attention(q, k, v, g, b)
+    out.sum().backward()
+    assert not seen["bwd"][1]["want_d_initial"]
+
+
 def test_binding_refuses_without_library(tmp_path, monkeypatch):
     """With libkda.so absent the binding raises instead of falling back."""
     import importlib.util

@@ -142,3 +142,25 @@ def test_backward_bad_cu_seqlens_reports_without_trap(kda):
                   max_seqlen=120, workspace=ws)
     rc, code = kda.workspace_status(ws)
     assert rc == kda.KDA_ERR_DEVICE and code != 0
+
+
+def test_autograd_function_matches_oracle(kda):
+    """kda_attention under torch autograd: loss.backward() gives the oracle's gradients."""
+    x = make_inputs(None, H=2, dk=64, dv=64, dtype=torch.float32, seed=520,
+                    lengths=[100, 40], state_std=0.02)
+    q, k, v, g, b = (t.to(DEV).requires_grad_() for t in (x.q, x.k, x.v, x.g, x.beta))
+    s0 = x.initial_state.to(DEV).requires_grad_()
+    out, fin = kda.kda_attention(q, k, v, g, b, initial_state=s0,
+                                 cu_seqlens=x.cu_seqlens.to(DEV), max_seqlen=100)
+    rng = np.random.default_rng(9)
+    w_out = torch.tensor(rng.standard_normal(tuple(out.shape)), dtype=torch.float32).to(DEV)
+    w_fin = torch.tensor(rng.standard_normal(tuple(fin.shape)), dtype=torch.float32).to(DEV)
+    loss = (out * w_out).sum() + (fin * w_fin).sum()
+    loss.backward()
+    torch.cuda.synchronize()
+    ref = ko.backward(x.q, x.k, x.v, x.g, x.beta, d_out=w_out.cpu().double(),
+                      d_final=w_fin.cpu(), cu_seqlens=x.cu_seqlens.tolist(),
+                      initial_state=x.initial_state)
+    for name, t in zip(NAMES, (q, k, v, g, b, s0)):
+        rel, mx = errors(t.grad, ref[name])
+        assert rel <= TOL[torch.float32], f"autograd {name}: rel-L2 {rel:.3e}"
