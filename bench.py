@@ -89,7 +89,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.index = index
         self.period = period_s
         self.samples = []
@@ -124,15 +124,23 @@ class ClockSampler:
         self._thread = threading.Thread(target=run, daemon=True)
         self._thread.start()
 
+    def mark(self) -> int:
+        """Index of the next sample: summary(since=mark()) covers what follows."""
+        return len(self.samples)
+
+    def summary(self, since: int = 0) -> dict | None:
+        xs = self.samples[since:]
+        if not xs:
+            return None
+        return {"sm_mhz": statistics.median(xs), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(xs)}
+
     def stop(self) -> dict | None:
         if self._thread is None:
             return None
         self._stop.set()
         self._thread.join()
-        if not self.samples:
-            return None
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        return self.summary()
 
 
 def dist_setup(n_gpus: int):
@@ -206,14 +214,16 @@ def bench_ours(args, world, rank, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # one sampler over every leg below; `clocks` is the prefill's timed region alone
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
+    mark = clocks.mark()
     total_ms, per = time_region(step, args.steps, stream)
     barrier(world)
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    clk = clocks.summary(mark)
     total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / args.steps
     tokens_per_step = T * world
@@ -330,13 +340,68 @@ def bench_ours(args, world, rank, local):
                              "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
                              "flops_per_call": b_flops, "traffic": None},
                 "gpu_launches": bsteps * (kda_launches_per_step(kda, shape) + 5)}
-    del bws, grads
+    del bws, grads, x, ws, out, fin
+    torch.cuda.empty_cache()
+    # ---- the other two prefill workloads north of the 8K one: one long sequence, and
+    #      packed variable-length sequences (device-resident inputs, CUDA events)
+    others = {}
+    for name, reps in (("bf16_h16_t1m_d128", 3), ("varlen8_h32_d128", 5)):
+        others[name] = bench_prefill_workload(kda, WORKLOADS[name], reps, world, rank, dev,
+                                              stream, peaks)
+        torch.cuda.empty_cache()
+    clk_all = clocks.stop()
     return {
         "value": round(value, 1), "ms_per_step": round(ms_step, 4), "clocks": clk,
+        "clocks_all_legs": clk_all,
         "roofline": roofline, "e2e": e2e, "decode": decode, "backward": backward,
+        "prefill_1m": others["bf16_h16_t1m_d128"], "prefill_varlen": others["varlen8_h32_d128"],
         "gpu_launches": launches_per_step * args.steps,
         "tflops": round(tc_tflops * world, 2),
     }
+
+
+def bench_prefill_workload(kda, w, reps: int, world: int, rank: int, dev: str, stream,
+                           peaks: dict) -> dict:
+    """kda_chunk_fwd on workload `w` (inputs drawn on the device, one workspace), one
+    untimed call then `reps` timed ones; tokens/s, algorithmic TFLOP/s and the fraction
+    of the measured bf16 peak, like the headline line."""
+    from kimi_delta_attention_19_b200.inputs import workload_inputs
+    x = workload_inputs(w, seed=rank, device=dev)
+    T_total, H, dk, dv = x.q.shape[0], w.H, w.dk, w.dv
+    n = len(x.lengths)
+    varlen = x.cu_seqlens is not None
+    shape = kda.make_shape(T_total, H, dk, dv, w.dtype, n_seqs=n if varlen else 0,
+                           max_seqlen=max(x.lengths) if varlen else 0)
+    ws = kda.alloc_workspace(shape, dev)
+    out = torch.empty(T_total, H, dv, dtype=w.dtype, device=dev)
+    fin = torch.empty(n, H, dk, dv, dtype=torch.float32, device=dev)
+
+    def call():
+        kda.chunk_fwd(x.q, x.k, x.v, x.g, x.beta, initial_state=x.initial_state,
+                      cu_seqlens=x.cu_seqlens, max_seqlen=max(x.lengths) if varlen else 0,
+                      out=out, final_state=fin, workspace=ws, stream=stream)
+
+    call()
+    torch.cuda.synchronize()
+    barrier(world)
+    total, _ = time_region(call, reps, stream)
+    ms = max_over_ranks(total, world) / reps
+    flops = prefill_flops_per_token_head(dk, dv) * T_total * H
+    tf = flops / (ms / 1e3) / 1e12
+    algo_bytes = prefill_bytes_per_token_head(dk, dv) * T_total * H + 2 * 4 * n * H * dk * dv
+    gbs = algo_bytes / (ms / 1e3) / 1e9
+    res = {"workload": w.name, "tokens": T_total, "sequences": n, "heads": H,
+           "ms_per_call": round(ms, 4), "calls_timed": reps,
+           "tokens_per_s": round(T_total * world / (ms / 1e3), 1),
+           "tflops": round(tf * world, 2),
+           "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                        "peak_source": peaks["source"],
+                        "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4)}},
+           "gpu_launches": reps * kda_launches_per_step(kda, shape)}
+    del x, ws, out, fin
+    return res
 
 
 def kda_launches_per_step(kda, shape) -> int:
@@ -384,6 +449,7 @@ def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: 
         dt += time.perf_counter() - t0
         done += tokens
     return {"value": round(done / dt, 2), "unit": "tokens/s", "cores": threads,
+            "host_cores": os.cpu_count(),
             "kind": "oracle", "seconds": round(dt, 3),
             "sample": f"{done // tokens} pass(es) over {tokens} of {w.T} tokens of {PREFILL} "
                       f"(all {w.H} heads), fp64 token-by-token recurrence, {threads} threads"}
@@ -484,7 +550,9 @@ def main():
             "dtype": "bf16", "data": "synthetic (seeded; no weights, no dataset)",
             "config": cfg, "impl": "ours", "tflops": r["tflops"], "roofline": r["roofline"],
             "cpu_baseline": cpu, "e2e": r["e2e"], "gpu_launches": r["gpu_launches"],
-            "clocks": r["clocks"], "decode": r["decode"], "backward": r["backward"],
+            "clocks": r["clocks"], "clocks_all_legs": r["clocks_all_legs"],
+            "decode": r["decode"], "backward": r["backward"],
+            "prefill_1m": r["prefill_1m"], "prefill_varlen": r["prefill_varlen"],
         }
         print(json.dumps(line))
     if world > 1:

@@ -215,6 +215,12 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void
  *  - All calls on a device share the array and it keeps the previous call's
  *    contents (the prefill clears what must start at zero). Calls whose work
  *    overlaps on the GPU, e.g. on unordered streams, race on the array.
+ *  - The array's address is looked up per CUDA context: after a device reset, or
+ *    with another context current, the next call looks it up again (again a call
+ *    to make before any stream capture in that context).
+ *  - Device-side errors (malformed cu_seqlens, a sequence longer than
+ *    max_seqlen) are recorded in the array's status word: read it with
+ *    kda_workspace_status(NULL, 0, stream, &code) on the same device.
  */
 #define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
@@ -236,19 +242,29 @@ kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, co
  *  n_slots     number of state slots (>= N when state_slots is NULL)
  *  out         [N, H, dv] dtype (written)
  *  shape       B = N, T = 1; n_seqs, max_seqlen and chunk are ignored.
+ *  status      int32 device word, or NULL. A state_slots entry outside [0, n_slots)
+ *              (only visible on the device) is not trapped: that sequence's state is
+ *              left untouched, its out rows are set to NaN, and, when status is not
+ *              NULL, 3 is written to *status. The library never clears *status (zero it
+ *              before the steps it should cover); kda_workspace_status(status, 4, ...)
+ *              reads it back.
  * Allocates nothing; safe to capture in a CUDA graph.
  */
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *g,
                            const void *beta, float *state, const int32_t *state_slots,
                            int64_t n_slots, void *out, const kda_shape *shape,
-                           kda_stream_t stream);
+                           int32_t *status, kda_stream_t stream);
 
 /*
  * Synchronises `stream` and reads the device-side status word a previous
- * kda_chunk_fwd left in `workspace`: KDA_OK, or KDA_ERR_DEVICE when a
- * malformed cu_seqlens (or an expired bounded wait) was detected. The word is
- * cleared by the next kda_chunk_fwd on that workspace. Diagnostic only: the
- * compute path never calls it.
+ * kda_chunk_fwd (or kda_chunk_bwd) left in `workspace`: KDA_OK, or KDA_ERR_DEVICE
+ * when a malformed cu_seqlens, a sequence longer than max_seqlen or an expired
+ * bounded wait was detected (*device_code: 1 cu_seqlens or max_seqlen, 2 wait,
+ * 3 decode slot). The word is cleared by the next kda_chunk_fwd on that workspace.
+ * workspace == NULL reads the word of kda_chunk_fwd_noalloc's fixed array on the
+ * current device (workspace_bytes is then ignored). A decode status word (see
+ * kda_decode_step) is read the same way, with workspace_bytes = 4. Diagnostic only:
+ * the compute path never calls it.
  */
 kda_status kda_workspace_status(const void *workspace, size_t workspace_bytes,
                                 kda_stream_t stream, int32_t *device_code);

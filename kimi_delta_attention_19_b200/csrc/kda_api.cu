@@ -281,7 +281,7 @@ int64_t kda_snapshot_count(const kda_shape* shape, int32_t snapshot_chunks) {
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* g,
                            const void* beta, float* state, const int32_t* state_slots,
                            int64_t n_slots, void* out, const kda_shape* shape,
-                           kda_stream_t stream) {
+                           int32_t* status, kda_stream_t stream) {
   kda_status st = check_shape(shape, false);
   if (st != KDA_OK) return st;
   const kda_shape& s = *shape;
@@ -292,6 +292,7 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
     if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (state_slots != nullptr && (reinterpret_cast<uintptr_t>(state_slots) & 3u))
     return KDA_ERR_INVALID_ARG;
+  if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u)) return KDA_ERR_INVALID_ARG;
 
   DecodeArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
@@ -299,6 +300,7 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
   a.slots = state_slots;
   a.n_slots = n_slots;
   a.out = out;
+  a.status = status;
   a.N = s.B; a.H = s.H; a.dk = s.dk; a.dv = s.dv;
   a.scale = s.scale > 0.f ? s.scale : 1.0f / sqrtf((float)s.dk);
   a.lb = s.g_lower_bound;
@@ -309,7 +311,15 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v, const vo
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
                                 kda_stream_t stream, int32_t* device_code) {
-  if (workspace == nullptr || workspace_bytes < sizeof(int32_t)) return KDA_ERR_INVALID_ARG;
+  if (workspace == nullptr) {
+    // the status word of kda_chunk_fwd_noalloc's fixed array on the current device
+    void* p = nullptr;
+    const kda_status st = noalloc_scratch_address(&p);
+    if (st != KDA_OK) return st;
+    workspace = p;
+  } else if (workspace_bytes < sizeof(int32_t)) {
+    return KDA_ERR_INVALID_ARG;
+  }
   int32_t code = 0;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(&code, workspace, sizeof code, cudaMemcpyDeviceToHost, cs) != cudaSuccess)

@@ -58,7 +58,17 @@ __global__ void __launch_bounds__(NW * 32, 2) decode_kernel(DecodeArgs a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n = blockIdx.x / a.H, h = blockIdx.x % a.H;
   const int64_t slot = a.slots ? (int64_t)a.slots[n] : (int64_t)n;
-  if (slot < 0 || slot >= a.n_slots) return;  // host validates the common case
+  if (slot < 0 || slot >= a.n_slots) {
+    // a state_slots entry the host could not see: no state is touched, the output row
+    // becomes NaN (never stale values) and the caller's status word, if any, says why
+    if (warp == 0) {
+      Tin* o = static_cast<Tin*>(a.out) + ((int64_t)n * a.H + h) * DV + lane * V;
+#pragma unroll
+      for (int c = 0; c < V; ++c) st_out(o + c, __int_as_float(0x7fc00000));
+      if (lane == 0 && a.status != nullptr) atomicExch(a.status, kDevBadSlot);
+    }
+    return;
+  }
   float* S = a.state + (slot * a.H + h) * (int64_t)DK * DV;
 
   // Issue the state loads first so they are in flight while the token loads land.

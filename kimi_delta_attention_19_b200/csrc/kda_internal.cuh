@@ -17,6 +17,7 @@ constexpr int kWorkspaceHeader = 256;  // bytes: status word + scheduler counter
 constexpr int32_t kDevOk = 0;
 constexpr int32_t kDevBadSeqlens = 1;   // cu_seqlens not monotone / out of [0, T]
 constexpr int32_t kDevWaitTimeout = 2;  // a bounded wait on another CTA gave up
+constexpr int32_t kDevBadSlot = 3;      // a decode state_slots entry outside [0, n_slots)
 
 // Everything a prefill launch needs, resolved on the host.
 struct PrefillArgs {
@@ -54,6 +55,7 @@ struct DecodeArgs {
   const int32_t* slots;
   int64_t n_slots;
   void* out;
+  int32_t* status;          // caller's device status word, or null
   int N, H, dk, dv;
   float scale;
   float lb;
@@ -158,5 +160,7 @@ cudaError_t launch_backward(const BackwardArgs& a, kda_dtype dtype, cudaStream_t
 // dq, dk, dg, dbeta from the fp32 accumulators, through the prologue when it is on
 cudaError_t launch_backward_finish(const BackwardArgs& a, void* dq, void* dk, void* dg,
                                    void* dbeta, kda_dtype dtype, cudaStream_t st);
+// Device address of the no-alloc entry point's fixed scratch array in the current context.
+kda_status noalloc_scratch_address(void** out);
 
 }  // namespace kda

@@ -61,7 +61,7 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(Shape), p]
     L.kda_decode_step.restype = st
     L.kda_decode_step.argtypes = [p, p, p, p, p, p, p, ctypes.c_int64, p,
-                                  ctypes.POINTER(Shape), p]
+                                  ctypes.POINTER(Shape), p, p]
     L.kda_workspace_status.restype = st
     L.kda_workspace_status.argtypes = [p, sz, p, ctypes.POINTER(ctypes.c_int32)]
     L.kda_status_string.restype = ctypes.c_char_p
@@ -320,10 +320,13 @@ def chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, state: torch.Tensor, *, state_slots: torch.Tensor | None = None,
                 scale: float | None = None, lb: float = -1.0, out: torch.Tensor | None = None,
-                prologue: int = 0, stream=None) -> torch.Tensor:
+                prologue: int = 0, status: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
     """One token per sequence: q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H].
 
     Updates fp32 `state` [n_slots, H, dk, dv] in place; returns out [N, H, dv].
+    `status` (int32 device tensor, optional) receives 3 when a state_slots entry is
+    out of range (that sequence's out rows are NaN and its state is untouched).
     """
     N, H, dk = q.shape
     dv = v.shape[-1]
@@ -332,17 +335,19 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
         out = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
     rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
                              _ptr(state_slots), state.shape[0], _ptr(out), ctypes.byref(shape),
-                             _stream(stream))
+                             _ptr(status), _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step")
     return out
 
 
-def workspace_status(workspace: torch.Tensor, stream=None) -> tuple[int, int]:
-    """(status, device code) left in `workspace` by the last kda_chunk_fwd (synchronises)."""
+def workspace_status(workspace: torch.Tensor | None, stream=None) -> tuple[int, int]:
+    """(status, device code) left in `workspace` by the last kda_chunk_fwd (synchronises).
+    None reads the status word of chunk_fwd_noalloc's fixed array on the current device;
+    a decode status tensor is read the same way as a workspace."""
     code = ctypes.c_int32(0)
-    rc = lib.kda_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream),
-                                  ctypes.byref(code))
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.kda_workspace_status(_ptr(workspace), nbytes, _stream(stream), ctypes.byref(code))
     return rc, code.value
 
 

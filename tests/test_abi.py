@@ -155,14 +155,16 @@ def test_decode_argument_errors(kda):
     P = ctypes.c_void_p
     sh = kda.make_shape(1, 4, 128, 128, torch.bfloat16, B=8)
 
-    def call(state=4096, slots=None, n_slots=8, shape=sh, q=4096):
+    def call(state=4096, slots=None, n_slots=8, shape=sh, q=4096, status=None):
         return kda.lib.kda_decode_step(P(q), P(4096), P(4096), P(4096), P(4096), P(state),
-                                       P(slots), n_slots, P(4096), ctypes.byref(shape), None)
+                                       P(slots), n_slots, P(4096), ctypes.byref(shape),
+                                       P(status), None)
 
     assert call(state=None) == kda.KDA_ERR_INVALID_ARG
     assert call(n_slots=4) == kda.KDA_ERR_INVALID_ARG          # fewer slots than sequences
     assert call(q=4097) == kda.KDA_ERR_INVALID_ARG
     assert call(slots=4098) == kda.KDA_ERR_INVALID_ARG         # int32 slots misaligned
+    assert call(status=4098) == kda.KDA_ERR_INVALID_ARG        # int32 status misaligned
     assert call(shape=kda.make_shape(2, 4, 128, 128, torch.bfloat16, B=8)) == \
         kda.KDA_ERR_INVALID_ARG                                 # decode is one token
     assert call(shape=kda.make_shape(1, 4, 128, 80, torch.bfloat16, B=8)) == \

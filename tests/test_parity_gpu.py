@@ -250,6 +250,39 @@ def test_decode_state_slots(kda):
     assert torch.equal(state[untouched].cpu(), S0[untouched])
 
 
+def test_decode_bad_slot_reports_without_trap(kda):
+    """A state_slots entry outside [0, n_slots) only exists on the device: that sequence's
+    state is left alone, its out rows are NaN, the status word says 3, and every other
+    sequence is updated as usual."""
+    N, H, d = 4, 2, 128
+    tok = decode_tokens(1, N, H, d, d, seed=33)
+    S0 = decode_state(6, H, d, d, seed=34)
+    slots = torch.tensor([4, 6, 1, -1], dtype=torch.int32)  # 6 and -1 are out of range
+    state = S0.to(DEV).clone()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = kda.decode_step(tok.q[0].to(DEV), tok.k[0].to(DEV), tok.v[0].to(DEV),
+                          tok.g[0].to(DEV), tok.beta[0].to(DEV), state,
+                          state_slots=slots.to(DEV), status=status)
+    torch.cuda.synchronize()
+    assert kda.workspace_status(status) == (kda.KDA_ERR_DEVICE, 3)
+    assert torch.isnan(out[1].float()).all() and torch.isnan(out[3].float()).all()
+    good = [0, 2]
+    ro, rs = ko.recurrent(tok.q[0][good], tok.k[0][good], tok.v[0][good], tok.g[0][good],
+                          tok.beta[0][good], cu_seqlens=list(range(len(good) + 1)),
+                          initial_state=S0[slots[good].long()])
+    assert_close(out[good], ro, torch.bfloat16, "good slots out")
+    assert_close(state[slots[good].long()], rs, torch.bfloat16, "good slots state")
+    untouched = [0, 2, 3, 5]
+    assert torch.equal(state[untouched].cpu(), S0[untouched])
+    # without a status word the bad rows are still NaN and nothing else changes
+    out2 = kda.decode_step(tok.q[0].to(DEV), tok.k[0].to(DEV), tok.v[0].to(DEV),
+                           tok.g[0].to(DEV), tok.beta[0].to(DEV), S0.to(DEV).clone(),
+                           state_slots=slots.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.isnan(out2[1].float()).all()
+    assert torch.equal(out2[good], out[good])
+
+
 def test_decode_equals_prefill_one_token(kda):
     x = make_inputs(None, H=4, dk=128, dv=128, dtype=torch.bfloat16, seed=41,
                     lengths=[1] * 6, state_std=0.02)
