@@ -157,11 +157,21 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
 }
+// Limit, in SM clocks, of the first wait on a kernel's inputs (the intra-chunk kernel's
+// TMA loads, the walks' first stage, the combine's first M and L). A test-only build of
+// the library sets it to a few clocks so that the wait runs out and each kernel's
+// bail-out path (record the error, let the copies and products in flight finish, free
+// tensor memory, return) runs on the GPU; every other wait keeps its own limit.
+#ifndef KDA_FIRST_WAIT_LIMIT
+#define KDA_FIRST_WAIT_LIMIT 4000000000LL
+#endif
+
 // Bounded wait by thread 0 alone (the others sleep in the barrier instead of polling),
 // then a uniform decision: true when it timed out. The other threads then observe the
 // completed phase themselves, which orders the data it guards before their reads.
-__device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity) {
-  const bool ok = threadIdx.x != 0 || mbar_wait(bar, parity);
+__device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity,
+                                                long long limit = 4000000000LL) {
+  const bool ok = threadIdx.x != 0 || mbar_wait(bar, parity, limit);
   if (__syncthreads_or(!ok)) return true;
   if (threadIdx.x != 0) mbar_try_wait(bar, parity);
   return false;
@@ -284,7 +294,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   };
 
   do {
-    if (cta_wait_failed(bar_in, 0)) { failed = true; break; }
+    if (cta_wait_failed(bar_in, 0, KDA_FIRST_WAIT_LIMIT)) { failed = true; break; }
     in_done = true;
     if (L < C) {
       // a sequence's ragged last chunk: rows past L (the next sequence's tokens, or the
@@ -929,7 +939,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       group_sync(half_bar, 128);
       if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + hc);
       if (n_chunks > 0) {
-        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0))) {
+        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0, KDA_FIRST_WAIT_LIMIT))) {
           failed = true;
         } else {
           rescale_all(0, v0, v1);
@@ -1243,7 +1253,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
   }
   bool failed = false, ld_pending = true;
   for (int sg = 1; sg < nseg - 1; ++sg) {
-    if (cta_wait_failed(bar_ld, (sg - 1) & 1)) {
+    if (cta_wait_failed(bar_ld, (sg - 1) & 1, sg == 1 ? KDA_FIRST_WAIT_LIMIT : 4000000000LL)) {
       failed = true;
       break;
     }

@@ -37,11 +37,11 @@ class Shape(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("prologue", ctypes.c_int32)]
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python -m kimi_delta_attention_19_b200.build` (no fallback exists)")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     p, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     L.kda_chunk_fwd_workspace_size.restype = sz
     L.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
@@ -72,6 +72,12 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Another build of the same C ABI (e.g. the test-only short-wait variant), with the
+    argument types declared as for `lib`."""
+    return _load(path)
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
             "kda_chunk_fwd_snapshots", "kda_snapshot_count", "kda_chunk_bwd_workspace_size",
