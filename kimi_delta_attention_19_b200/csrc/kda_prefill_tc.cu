@@ -16,8 +16,8 @@
 //   U  = U0 - W S                                O = scale (Q~ S + P U)
 //   S <- Diag(gl) S + Kb^T U
 // Everything above the last two lines depends on the chunk alone. An intra-chunk
-// kernel computes it for every (chunk, head) at once and leaves -W, U0, Kb, Q~,
-// P^T and gl in the workspace. The walk over the chunks of a sequence, which
+// kernel computes it for every (chunk, head) at once and leaves -W^T, U0^T, Kb^T,
+// Q~^T, P and gl in the workspace. The walk over the chunks of a sequence, which
 // carries S, is then four tensor-core products per chunk in the transposed frame
 // (M = 128, the d_v index of S):
 //   U^T = U0^T + S^T (-W)^T,  (Q~ S)^T = S^T Q~^T,  O^T += U^T P^T,  S^T += U^T Kb
@@ -46,11 +46,15 @@ constexpr int C = kChunk;  // 64
 constexpr int D = 128;     // d_k = d_v on this path
 constexpr uint32_t K8 = 8192, K16 = 16384, K32 = 32768;
 
-// Workspace tiles per (chunk slot, head); rows are the chunk's tokens except for U0.
-//   wn, kb, qt: [64][128] bf16  (-W, Kb, Q~)
-//   u0:         [128][64] bf16  (U0^T: row j, column r)
-//   pt:         [64][64]  bf16  (P^T: row s, column r)
-//   gl:         [128]     fp32
+// Workspace tiles per (chunk slot, head), every one a row-major array of 64-element
+// (128-byte) bf16 rows, the layout the walk's products take as operands:
+//   wt:  [128][64] -W^T  (row i = key channel, column r = token of the chunk)
+//   qt:  [128][64] Q~^T  (row i, column r)
+//   u0:  [128][64] U0^T  (row j = value channel, column r)
+//   kbt: [128][64] Kb^T  (row i, column s)
+//   p:   [64][64]  P     (row r, column s)
+//   gl:  [128]     fp32
+// Each row is written whole by one thread (16-byte stores) and read by TMA.
 constexpr size_t kTileBig = size_t(C) * D * 2;
 constexpr size_t kTilePt = size_t(C) * C * 2;
 constexpr size_t kTileGl = size_t(D) * 4;
@@ -102,22 +106,34 @@ __device__ __forceinline__ int64_t seg_offset(int seg, int first_tokens, int seg
   return seg == 0 ? 0 : first_tokens + static_cast<int64_t>(seg - 1) * seg_tokens;
 }
 
+// Sequence owning chunk slot u: the last one whose first slot is <= u.
+__device__ __forceinline__ int owner_seq(const SeqTable& q, int64_t u) {
+  int lo = 0, hi = q.n_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (slot_base(seq_start(q, mid), mid) <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 struct IntraArgs {
-  CUtensorMap tm_q, tm_k, tm_g;  // [T_total][H*128] bf16, 64x64 boxes, no swizzle
-  CUtensorMap tm_v;              // the same shape, 128-byte swizzle (an MMA operand as loaded)
-  CUtensorMap tm_qt, tm_kb;      // workspace Q~ and Kb, [tiles*64][128], 128-byte swizzle
+  CUtensorMap tm_q, tm_k, tm_g;  // [T_total][H*128] bf16, 64x128 boxes, no swizzle
+  CUtensorMap tm_v;              // the same shape, 64x64 boxes, 128-byte swizzle (an MMA operand as loaded)
+  // workspace tiles (layouts above), stored from 128-byte-swizzled staging tiles:
+  CUtensorMap tm_wt, tm_qt, tm_u0, tm_kbt;  // [tiles*128][64] bf16, 128x64 boxes
+  CUtensorMap tm_p;                         // [tiles*64][64], 64x64 boxes
   SeqTable seq;
   const __nv_bfloat16* beta;
-  __nv_bfloat16 *wn, *u0, *pt;
   float* gl;
   int H;
   float lb;
 };
 
 struct WalkArgs {
-  CUtensorMap tm_wn, tm_u0, tm_kb, tm_qt;  // [tiles*64][128] bf16, 64x64 boxes, 128-byte swizzle
-  CUtensorMap tm_pt;                       // [tiles*64][64]
-  CUtensorMap tm_o;                        // out [T_total][H*128], 64x64 boxes, no swizzle
+  CUtensorMap tm_wt, tm_qt, tm_u0, tm_kbt;  // [tiles*128][64] bf16, 128x64 boxes, 128-byte swizzle
+  CUtensorMap tm_p;                         // [tiles*64][64], 64x64 boxes
+  CUtensorMap tm_o;                         // out [T_total][H*128], 64x64 boxes, no swizzle
   SeqTable seq;
   const float* gl;
   __nv_bfloat16* out;
@@ -147,10 +163,24 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   __nv_bfloat162 t = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(t);
 }
+// (x, y) as bf16 pairs hi + lo: hi = bf16(x), lo = bf16(x - hi), so hi + lo carries
+// about 16 bits of x; products of split factors keep fp32 accuracy on the tensor cores.
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_bf16(x - hf.x, y - hf.y);
+}
 // 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error ~2^-22).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 1/x by the hardware approximation (rcp.approx.ftz.f32: relative error ~2^-23).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ uint4 pack8(const float* f) {
@@ -181,38 +211,35 @@ __device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity,
 // ------------------------------------------------------------------ intra-chunk kernel
 // One CTA of 8 warps per (chunk slot, head); two CTAs per SM. Everything of a chunk
 // that does not depend on the state: decay tiles, the Gram products on the tensor
-// cores, T = (I + A)^{-1} Diag(beta) by blocked forward substitution in fp32, and
-// the WY factors W = T K~, U0 = T V on the tensor cores.
+// cores, T = (I + A)^{-1} Diag(beta) by blocked forward substitution (16x16 diagonal
+// blocks on the CUDA cores, the off-diagonal merges as tensor-core products), and the
+// WY factors W = T K~, U0 = T V on the tensor cores.
 constexpr int kIntraThreads = 256;
 struct IntraSm {
   // Raw inputs as loaded by TMA; each region is reused once its contents are read.
-  // fp32 64x64 matrices (A, N) use a padded row of 68 floats: conflict-free row and
-  // column access with plain addressing.
-  static constexpr int FP = 68;
-  static constexpr uint32_t FP_BYTES = 64 * FP * 4;  // 17 KB
   static constexpr uint32_t SV = 0;        // V, swizzled: [64 s][64 j] boxes (U0's A operand)
   static constexpr uint32_t KQ = K16;      // [K~ a0 | Q~ a0 | K~ a1 | Q~ a1], 8 KB each
-  static constexpr uint32_t SK = 3 * K16;  // raw k, then K^, then T and the merge scratch
-  static constexpr uint32_t SG = 4 * K16;  // raw g, then Kb (store staging), then N
-  static constexpr uint32_t SQ = 5 * K16;  // raw q, then A
-  static constexpr uint32_t KH = SK, T = SK, BT = SK + K8;
-  static constexpr uint32_t NS = SG - 1024;  // N spans [63 KB, 80 KB)
-  static constexpr uint32_t A = SQ;          // A spans [80 KB, 97 KB)
-  static constexpr uint32_t TOT = SQ + FP_BYTES;  // float[4][128] partial decay sums
+  static constexpr uint32_t SK = 3 * K16;  // raw k, then K^, then T
+  static constexpr uint32_t SG = 4 * K16;  // raw g, then the N_d / N1 tile pair (hi, lo)
+  static constexpr uint32_t SQ = 5 * K16;  // raw q, then the Y / Z tile pair (hi, lo)
+  static constexpr uint32_t KH = SK, T = SK, NB = SG, YB = SQ;
+  // 128-byte-swizzled staging tiles of the TMA stores to the workspace: Q~^T and Kb^T
+  // (phase 2, over the raw g and q), P (phase 4, after K^), -W^T and U0^T (phase 8)
+  static constexpr uint32_t QTS = SG, KBS = SQ, PS = SK + K8, WTS = SG, U0S = SQ;
+  // float[2][64]: 1/|k row|, 1/|q row| (prologue)
+  static constexpr uint32_t RN = SQ + K16;
+  static constexpr uint32_t TOT = RN + 512;       // float[4][128] partial decay sums
   static constexpr uint32_t BET = TOT + 2048;     // float[64]
   static constexpr uint32_t BARS = BET + 256;
-  // float[2][64]: 1/|k row|, 1/|q row| (prologue), in the gap after raw q that A only
-  // reaches in phase 4, after the last use of RN
-  static constexpr uint32_t RN = SQ + K16;
   static constexpr uint32_t TPTR = BARS + 64;
   static constexpr uint32_t BYTES = TPTR + 16;
-  // tensor-memory columns: [K~;Q~] K^^T, W^T, U0^T
+  // tensor-memory columns: [K~;Q~] K^^T (G), W^T, U0^T; while T is formed: the A
+  // operands A_off and N_d / N1 (hi | lo, 32 columns each) over W and U, and the
+  // merge products over the free columns and G
   static constexpr uint32_t G = 0, W = 64, U = 128, COLS = 256;
+  static constexpr uint32_t AOP = 64, NOP = 128, DA = 192, DB = 0;
 };
 static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTAs per SM");
-static_assert(IntraSm::BT + 4096 <= IntraSm::NS && IntraSm::NS + IntraSm::FP_BYTES == IntraSm::SQ,
-              "intra-chunk shared-memory regions overlap");
-static_assert(IntraSm::RN + 512 <= IntraSm::TOT, "prologue norms overlap the decay sums");
 
 // PRO: the raw-input prologue flags (KDA_PROLOGUE_*), a template parameter so the plain
 // instance carries no trace of it.
@@ -227,13 +254,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   const int h = static_cast<int>(blockIdx.x % a.H);
 
   // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
-  int lo = 0, hi = a.seq.n_seqs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (slot_base(seq_start(a.seq, mid), mid) <= u) lo = mid;
-    else hi = mid - 1;
-  }
-  const int s = lo;
+  const int s = owner_seq(a.seq, u);
   int64_t t0, t1;
   if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
   const int64_t c = u - slot_base(t0, s);
@@ -244,7 +265,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 
   float* tot = reinterpret_cast<float*>(sm + L_::TOT);
   float* bet = reinterpret_cast<float*>(sm + L_::BET);
-  float* bt = reinterpret_cast<float*>(sm + L_::BT);
   float* rn = reinterpret_cast<float*>(sm + L_::RN);
   uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);  // g, k, q
   uint64_t* bar_v = bar_in + 1;
@@ -271,7 +291,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     for (int bx = 0; bx < 2; ++bx)
       tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_v, h * D + 64 * bx, static_cast<int>(r0));
   }
-  if (tid < C) bet[tid] = tid < L ? __bfloat162float(a.beta[(r0 + tid) * a.H + h]) : 0.f;
+  // beta of this thread's row, kept in a register until phase 1 is done (its load then
+  // overlaps the TMA wait and phase 1 instead of delaying them)
+  const float beta_r = tid < L ? __bfloat162float(a.beta[(r0 + tid) * a.H + h]) : 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -280,18 +302,6 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   int mma_issued = 0, mma_done = 0;
   bool in_done = false, v_done = false, failed = false;
 
-  float* const Am = reinterpret_cast<float*>(sm + L_::A);
-  float* const Nm = reinterpret_cast<float*>(sm + L_::NS);
-  auto a_ptr = [&](int r, int cc) -> float* { return Am + r * L_::FP + cc; };
-  auto n_ptr = [&](int r, int cc) -> float* { return Nm + r * L_::FP + cc; };
-  auto a4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(a_ptr(r, cc)); };
-  auto n4 = [&](int r, int cc) -> float4 { return *reinterpret_cast<const float4*>(n_ptr(r, cc)); };
-  auto fma4 = [](float sv, const float4& v, float4& acc) {
-    acc.x = fmaf(sv, v.x, acc.x);
-    acc.y = fmaf(sv, v.y, acc.y);
-    acc.z = fmaf(sv, v.z, acc.z);
-    acc.w = fmaf(sv, v.w, acc.w);
-  };
 
   do {
     if (cta_wait_failed(bar_in, 0, KDA_FIRST_WAIT_LIMIT)) { failed = true; break; }
@@ -334,16 +344,17 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       if (hf == 0) rn[which * 64 + r] = inv_l2(ss);
       __syncthreads();
     }
-    // ---- 1. raw k, q into registers; prefix sums of the clamped log decay in log2 units.
+    // ---- 1. raw k, q into registers; the per-token decay factors e_i = exp(max(g_i, lb))
+    //         (one exponential each) and their product over this thread's rows.
     //         Thread = (channel pair p, quarter qr of 16 rows).
     const int p = tid & 63, qr = tid >> 6;
     const int ch = 2 * p, bx = p >> 5;
     constexpr float kLog2e = 1.4426950408889634f;
     const float lb2 = a.lb * kLog2e;
     uint32_t kraw[16], qraw[16];
-    float G0[16], G1[16];
+    float E0[16], E1[16];
     {
-      float acc0 = 0.f, acc1 = 0.f;
+      float pr0 = 1.f, pr1 = 1.f;
       const uint32_t off0 = 16 * qr * 256 + 4 * p;  // raw rows are 256 bytes
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -358,41 +369,54 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
           gg.x = live ? gate_from_preact(gg.x, a.lb) : 0.f;
           gg.y = live ? gate_from_preact(gg.y, a.lb) : 0.f;
         }
-        acc0 += fmaxf(gg.x * kLog2e, lb2);
-        acc1 += fmaxf(gg.y * kLog2e, lb2);
-        G0[i] = acc0;
-        G1[i] = acc1;
+        E0[i] = ex2_approx(fmaxf(gg.x * kLog2e, lb2));
+        E1[i] = ex2_approx(fmaxf(gg.y * kLog2e, lb2));
+        pr0 *= E0[i];
+        pr1 *= E1[i];
       }
-      *reinterpret_cast<float2*>(tot + qr * 128 + ch) = make_float2(acc0, acc1);
+      *reinterpret_cast<float2*>(tot + qr * 128 + ch) = make_float2(pr0, pr1);
     }
+    if (tid < C) bet[tid] = beta_r;
     __syncthreads();  // every raw read is done: SK, SG and SQ may be overwritten
-    // ---- 2. decay tiles: K~, Q~, K^ (MMA operands), Kb (store staging); gl to the workspace.
+    // ---- 2. decay tiles: K~, Q~, K^ (MMA operands); Q~^T and Kb^T rows 2p, 2p + 1 (this
+    //         thread's 16 tokens, 32 contiguous bytes each) and gl to the workspace.
+    //         With gamma_i = exp(Gamma_i) the running product of the e's: gamma_i is the
+    //         product of the earlier quarters' totals and this quarter's e's up to i;
+    //         1 / gamma_i and gl / gamma_i are the product of this quarter's e's after i
+    //         times 1 / (product up to this quarter's end) or the later quarters' totals.
+    //         No reciprocal of a small number is taken per element, and each factor stays
+    //         within [exp(64 lb), exp(-64 lb)] (finite: lb * 64 >= -80).
     //         Rows 16 qr + i: the swizzle term depends on i % 8 only.
     {
-      float o0 = 0.f, o1 = 0.f, s0 = 0.f, s1 = 0.f;
+      uint32_t qt0[8], qt1[8], kb0[8], kb1[8];  // bf16 pairs along the token index
+      float2 tq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tq[q] = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
+      float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float2 tq = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
         if (q < qr) {
-          o0 += tq.x;
-          o1 += tq.y;
+          pre0 *= tq[q].x;
+          pre1 *= tq[q].y;
+        } else if (q > qr) {
+          suf0 *= tq[q].x;
+          suf1 *= tq[q].y;
         }
-        s0 += tq.x;
-        s1 += tq.y;
       }
-      const float gl0 = ex2_approx(s0), gl1 = ex2_approx(s1);
+      const float gl0 = ((tq[0].x * tq[1].x) * tq[2].x) * tq[3].x;
+      const float gl1 = ((tq[0].y * tq[1].y) * tq[2].y) * tq[3].y;
       if (qr == 3) *reinterpret_cast<float2*>(a.gl + tile * D + ch) = make_float2(gl0, gl1);
+      const float inv0 = rcp_approx(pre0 * (qr == 0 ? tq[0].x : qr == 1 ? tq[1].x : qr == 2 ? tq[2].x : tq[3].x));
+      const float inv1 = rcp_approx(pre1 * (qr == 0 ? tq[0].y : qr == 1 ? tq[1].y : qr == 2 ? tq[2].y : tq[3].y));
       const int c3 = (ch & 63) >> 3;
       const uint32_t row0 = 2 * qr * 1024 + (ch & 7) * 2;
-      const uint32_t kq0 = L_::KQ + bx * K16 + row0, kh0b = L_::KH + bx * K8 + row0,
-                     kb0b = L_::SG + bx * K8 + row0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t ro = (i >> 3) * 1024 + (i & 7) * 128 + ((c3 ^ (i & 7)) << 4);
-        const float g0 = G0[i] + o0, g1 = G1[i] + o1;
-        const float e0 = ex2_approx(g0), e1 = ex2_approx(g1);
-        const float ei0 = ex2_approx(-g0), ei1 = ex2_approx(-g1);
-        float2 kk = unpack_bf16(kraw[i]), qq = unpack_bf16(qraw[i]);
+      const uint32_t kq0 = L_::KQ + bx * K16 + row0, kh0b = L_::KH + bx * K8 + row0;
+      auto row_off = [&](int i) -> uint32_t {
+        return (i >> 3) * 1024 + (i & 7) * 128 + ((c3 ^ (i & 7)) << 4);
+      };
+      auto kq_in = [&](int i, float2& kk, float2& qq) {
+        kk = unpack_bf16(kraw[i]);
+        qq = unpack_bf16(qraw[i]);
         if (PRO & KDA_PROLOGUE_QK_L2NORM) {
           const float rk = rn[16 * qr + i], rq = rn[64 + 16 * qr + i];
           kk.x *= rk;
@@ -400,17 +424,68 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
           qq.x *= rq;
           qq.y *= rq;
         }
-        const float kh0 = kk.x * ei0, kh1 = kk.y * ei1;
-        *reinterpret_cast<uint32_t*>(sm + kq0 + ro) = pack_bf16(kk.x * e0, kk.y * e1);
-        *reinterpret_cast<uint32_t*>(sm + kq0 + K8 + ro) = pack_bf16(qq.x * e0, qq.y * e1);
-        *reinterpret_cast<uint32_t*>(sm + kh0b + ro) = pack_bf16(kh0, kh1);
-        *reinterpret_cast<uint32_t*>(sm + kb0b + ro) = pack_bf16(kh0 * gl0, kh1 * gl1);
+      };
+      // forward over the rows: K~ = k gamma, Q~ = q gamma
+      float gm0 = pre0, gm1 = pre1, qprev0 = 0.f, qprev1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        gm0 *= E0[i];
+        gm1 *= E1[i];
+        float2 kk, qq;
+        kq_in(i, kk, qq);
+        const float qt0f = qq.x * gm0, qt1f = qq.y * gm1;
+        *reinterpret_cast<uint32_t*>(sm + kq0 + row_off(i)) = pack_bf16(kk.x * gm0, kk.y * gm1);
+        *reinterpret_cast<uint32_t*>(sm + kq0 + K8 + row_off(i)) = pack_bf16(qt0f, qt1f);
+        if (i & 1) {
+          qt0[i >> 1] = pack_bf16(qprev0, qt0f);
+          qt1[i >> 1] = pack_bf16(qprev1, qt1f);
+        } else {
+          qprev0 = qt0f;
+          qprev1 = qt1f;
+        }
       }
+      // rows ch, ch + 1 of the Q~^T staging tile (raw g is dead): tokens 16 qr .. + 15
+      auto stage2 = [&](uint32_t base, const uint32_t* r0w, const uint32_t* r1w) {
+        *reinterpret_cast<uint4*>(sm + base + sw128_chunk(ch, 2 * qr, 0)) =
+            make_uint4(r0w[0], r0w[1], r0w[2], r0w[3]);
+        *reinterpret_cast<uint4*>(sm + base + sw128_chunk(ch, 2 * qr + 1, 0)) =
+            make_uint4(r0w[4], r0w[5], r0w[6], r0w[7]);
+        *reinterpret_cast<uint4*>(sm + base + sw128_chunk(ch + 1, 2 * qr, 0)) =
+            make_uint4(r1w[0], r1w[1], r1w[2], r1w[3]);
+        *reinterpret_cast<uint4*>(sm + base + sw128_chunk(ch + 1, 2 * qr + 1, 0)) =
+            make_uint4(r1w[4], r1w[5], r1w[6], r1w[7]);
+      };
+      stage2(L_::QTS, qt0, qt1);
+      // backward over the rows: K^ = k / gamma, Kb = k gl / gamma
+      float rs0 = 1.f, rs1 = 1.f, kprev0 = 0.f, kprev1 = 0.f;
+#pragma unroll
+      for (int i = 15; i >= 0; --i) {
+        float2 kk, qq;
+        kq_in(i, kk, qq);
+        const float kh0 = kk.x * (rs0 * inv0), kh1 = kk.y * (rs1 * inv1);
+        const float kb0f = kk.x * (rs0 * suf0), kb1f = kk.y * (rs1 * suf1);
+        *reinterpret_cast<uint32_t*>(sm + kh0b + row_off(i)) = pack_bf16(kh0, kh1);
+        if (!(i & 1)) {
+          kb0[i >> 1] = pack_bf16(kb0f, kprev0);
+          kb1[i >> 1] = pack_bf16(kb1f, kprev1);
+        } else {
+          kprev0 = kb0f;
+          kprev1 = kb1f;
+        }
+        rs0 *= E0[i];
+        rs1 *= E1[i];
+      }
+      stage2(L_::KBS, kb0, kb1);
     }
     fence_async_smem();
     __syncthreads();
-    // ---- 3. Q~ (its two boxes inside the Gram operand) and Kb to the workspace by TMA;
-    //         MMA-g: [K~; Q~] K^^T, M = 128 (64 rows of K~, then 64 of Q~), N = 64
+    // ---- 3. MMA-g: [K~; Q~] K^^T, M = 128 (64 rows of K~, then 64 of Q~), N = 64;
+    //         Q~^T and Kb^T to the workspace by TMA
+    if (tid == 32) {
+      tma_store_2d(&a.tm_qt, sm + L_::QTS, 0, static_cast<int>(tile * D));
+      tma_store_2d(&a.tm_kbt, sm + L_::KBS, 0, static_cast<int>(tile * D));
+      bulk_commit();
+    }
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ig = idesc_bf16(128, 64, 0, 0);
@@ -422,161 +497,195 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
                   sdesc_sw128(sb + L_::KH + kho, 16, 1024), ig, k > 0);
       }
       umma_commit(bar_mma);
-    } else if (tid == 32) {
-      const int y = static_cast<int>(tile * C);
-      tma_store_2d(&a.tm_qt, sm + L_::KQ + K8, 0, y);
-      tma_store_2d(&a.tm_qt, sm + L_::KQ + K8 + K16, 64, y);
-      tma_store_2d(&a.tm_kb, sm + L_::SG, 0, y);
-      tma_store_2d(&a.tm_kb, sm + L_::SG + K8, 64, y);
-      bulk_commit();
     }
     mma_issued = 1;
+    if (tid == 32) bulk_wait_read();  // the staging tiles are rewritten from phase 4 on
     if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
     mma_done = 1;
     tc_fence_after();
-    // ---- 4. A (fp32, beta-scaled strict lower) to shared memory; P^T to the workspace
+    // ---- 4-6. T = (I + A)^{-1} Diag(beta) by blocked forward substitution with two
+    //   32x32 diagonal blocks: N = [[N_lo, 0], [N_21, N_hi]], N_21 = -N_hi A_21 N_lo.
+    //   Rows r < 64 of the Gram accumulator (tensor-memory lanes 0..63) hold K~_r K^^T:
+    //   warps 0, 1, 4, 5 take one row each and a half hh of its 64 columns, so the
+    //   diagonal block of rows 0..31 is in the half of warp 0 and that of rows 32..63 in
+    //   the half of warp 5 (the "owners", one block per warp, a row per lane). Warps 2, 3,
+    //   6, 7 write P from lanes 64..127.
+    //   Diagonal blocks on the CUDA cores: N_bb = (I + A_bb)^{-1} in fp32 (a column per
+    //   lane, rows of A broadcast from shared memory).
+    //   The off-diagonal block on the tensor cores, two products at fp32 accuracy through
+    //   a bf16 split of both factors (x = hi + lo, the lo x lo term dropped), the left
+    //   factor an A operand in tensor memory, the right one a row-major (MN-major) tile:
+    //     R1: Z = A_21 N_lo (A restricted to rows 32..63 / columns 0..31: K steps 0, 1)
+    //     R2: D = N_d Z     (Z nonzero in rows 32..63: K steps 2, 3), N_21 = -D
+    //   and T = (N_d - D) Diag(beta), the WY products' bf16 operand. Rows 64..127 of
+    //   every product (lanes the left factor does not fill) are never read.
+    const bool rowt = (warp & 3) < 2;                       // rows r < 64 of A
+    const int hh = warp >> 2;                               // column half 32 hh ..
+    const int rr = (warp & 3) * 32 + lane;                  // row (when rowt)
+    const bool owner = rowt && hh == (warp & 3);            // warps 0 and 5
+    float nrow[32];                                         // owners: N_d row (block-local)
+    // this thread's 32 columns of a row-major 64x64 bf16 hi/lo tile pair (lo K8 after hi)
+    auto put_tile = [&](uint32_t tile_off, const float* f) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_bf16(f[8 * q + 2 * e], f[8 * q + 2 * e + 1], hi[e], lo[e]);
+        const uint32_t off = tile_off + sw128_chunk(rr, 4 * hh + q, K8);
+        *reinterpret_cast<uint4*>(sm + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(sm + off + K8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    };
+    // ... and as a tensor-memory A operand (K pairs per column: hi at col, lo at col + 32)
+    auto put_aop = [&](uint32_t col, const float* f) {
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) split_bf16(f[2 * t], f[2 * t + 1], hi[t], lo[t]);
+      tmem_st16(tb + lane_base + col + 16 * hh, hi);
+      tmem_st16(tb + lane_base + col + 32 + 16 * hh, lo);
+    };
+    // d = left right over the K steps in kmask, left = the A operand at aop (tensor
+    // memory), right = the tile pair at btile; then a commit on bar_mma
+    auto merge_mma = [&](uint32_t d, uint32_t aop, uint32_t btile, int kmask) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, 0, 1);
+      uint32_t acc = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (!(kmask >> k & 1)) continue;
+        const uint64_t bh = sdesc_sw128(sb + btile + k * 2048, K8, 1024);
+        const uint64_t bl = sdesc_sw128(sb + btile + K8 + k * 2048, K8, 1024);
+        umma_bf16_tmem_a(tb + d, tb + aop + 8 * k, bh, id, acc);
+        umma_bf16_tmem_a(tb + d, tb + aop + 8 * k, bl, id, 1);
+        umma_bf16_tmem_a(tb + d, tb + aop + 32 + 8 * k, bh, id, 1);
+        acc = 1;
+      }
+      umma_commit(bar_mma);
+    };
     {
-      const int wq = warp & 3, cb = (warp >> 2) * 32;
       uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::G + cb, v);
+      tmem_ld32(tb + lane_base + L_::G + 32 * hh, v);
       tmem_ld_wait(v);
-      if (wq < 2) {
-        const int r = wq * 32 + lane;
-        const float br = bet[r];
+      if (rowt) {
+        // A = Diag(beta) strict_lower(K~ K^^T); A_21 (rows 32..63, columns 0..31, held
+        // by warp 1) as an A operand; the owners keep their diagonal block's row in v
+        const float br = bet[rr];
+        float f[32];
 #pragma unroll
-        for (int g4 = 0; g4 < 8; ++g4) {
-          float4 f;
-          const int cc = cb + 4 * g4;
-          f.x = (cc + 0 < r) ? br * __uint_as_float(v[4 * g4 + 0]) : 0.f;
-          f.y = (cc + 1 < r) ? br * __uint_as_float(v[4 * g4 + 1]) : 0.f;
-          f.z = (cc + 2 < r) ? br * __uint_as_float(v[4 * g4 + 2]) : 0.f;
-          f.w = (cc + 3 < r) ? br * __uint_as_float(v[4 * g4 + 3]) : 0.f;
-          *reinterpret_cast<float4*>(a_ptr(r, cc)) = f;
+        for (int t = 0; t < 32; ++t) {
+          const int c = 32 * hh + t;
+          const float a_rc = c < rr ? br * __uint_as_float(v[t]) : 0.f;
+          f[t] = (rr >= 32 && hh == 0) ? a_rc : 0.f;
+          v[t] = __float_as_uint(a_rc);
         }
-      } else {
-        const int r = (wq - 2) * 32 + lane;
-        __nv_bfloat16* po = a.pt + (tile * C + cb) * C + r;
+        put_aop(L_::AOP, f);
+        if (owner) {
+          // N_bb by forward substitution, a column per lane: the block's rows of A go to a
+          // per-warp fp32 scratch (rows of 36 floats) in the Y tile's region, free until
+          // R1; lane c forms column c of N_bb, x_r = [r == c] - sum_{s<r} A_rs x_s, row by
+          // row from broadcast float4 reads of A (entries s >= r are zero); the columns go
+          // back through the scratch so that lane l ends with row l of N_bb.
+          float* scr = reinterpret_cast<float*>(sm + L_::YB) + (warp == 0 ? 0 : 32 * 36);
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          po[t * C] = __float2bfloat16_rn(cb + t <= r ? __uint_as_float(v[t]) : 0.f);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(scr + lane * 36 + 4 * q) =
+                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          __syncwarp();
+          float x[32];
+#pragma unroll
+          for (int r = 0; r < 32; ++r) x[r] = 0.f;
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            float acc[4] = {r == lane ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; 4 * q < r; ++q) {
+              const float4 a4 = *reinterpret_cast<const float4*>(scr + r * 36 + 4 * q);
+              acc[0] = fmaf(-a4.x, x[4 * q], acc[0]);
+              acc[1] = fmaf(-a4.y, x[4 * q + 1], acc[1]);
+              acc[2] = fmaf(-a4.z, x[4 * q + 2], acc[2]);
+              acc[3] = fmaf(-a4.w, x[4 * q + 3], acc[3]);
+            }
+            x[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 32; ++r) scr[r * 36 + lane] = x[r];
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 n4 = *reinterpret_cast<const float4*>(scr + lane * 36 + 4 * q);
+            nrow[4 * q] = n4.x;
+            nrow[4 * q + 1] = n4.y;
+            nrow[4 * q + 2] = n4.z;
+            nrow[4 * q + 3] = n4.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) nrow[c] = 0.f;
+        }
+        put_tile(L_::NB, nrow);
+        put_aop(L_::NOP, nrow);
+      } else {
+        // P = lower_incl(Q~ K^^T): row r, columns 32 hh .. 32 hh + 31
+        const int r = (warp & 3) * 32 + lane - 64;
+        float f[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) f[t] = 32 * hh + t <= r ? __uint_as_float(v[t]) : 0.f;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          *reinterpret_cast<uint4*>(sm + L_::PS + sw128_chunk(r, 4 * hh + q8, 0)) = pack8(f + 8 * q8);
       }
     }
-    if (tid == 32) bulk_wait_read();  // Kb staging is read before N overwrites it
+    tmem_st_wait();
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    // ---- 5. N = (I + A)^{-1}: 16x16 diagonal blocks, then 16->32 and 32->64 merges
-    if (warp < 4 && lane < 16) {
-      const int base = 16 * warp, l = lane;
-      float nv[16];
-#pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        float arow[16];
-#pragma unroll
-        for (int g4 = 0; g4 < (rr + 3) / 4; ++g4) {
-          const float4 v4 = a4(base + rr, base + 4 * g4);
-          arow[4 * g4 + 0] = v4.x;
-          arow[4 * g4 + 1] = v4.y;
-          arow[4 * g4 + 2] = v4.z;
-          arow[4 * g4 + 3] = v4.w;
-        }
-        float e0 = (rr == l) ? 1.f : 0.f, e1 = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < rr; kk += 2) {
-          e0 = fmaf(-arow[kk], nv[kk], e0);
-          if (kk + 1 < rr) e1 = fmaf(-arow[kk + 1], nv[kk + 1], e1);
-        }
-        nv[rr] = (rr < l) ? 0.f : e0 + e1;
-        *n_ptr(base + rr, base + l) = nv[rr];
-      }
+    if (tid == 32) {  // P to the workspace
+      tma_store_2d(&a.tm_p, sm + L_::PS, 0, static_cast<int>(tile * C));
+      bulk_commit();
     }
+    // R1: Z = A_21 N_lo (K steps 0, 1)
+    if (tid == 0) merge_mma(L_::DA, L_::AOP, L_::NB, 0x3);
+    mma_issued = 2;
+    if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
+    mma_done = 2;
+    tc_fence_after();
+    if (rowt) {
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::DA + 32 * hh, v);
+      tmem_ld_wait(v);
+      float f[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) f[t] = rr >= 32 && hh == 0 ? __uint_as_float(v[t]) : 0.f;
+      put_tile(L_::YB, f);
+    }
+    fence_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // Merges. Column c of an off-diagonal block N21 = -N22 (A21 N11) needs only column
-    // c of N11, so each warp owns a few columns: it forms P = A21 N11 for them, hands P
-    // round through its own scratch (a warp barrier), then writes -N22 P.
-    {
-      float* pw = bt + warp * 128;  // per-warp scratch, 512 bytes
-      // 16 -> 32: blocks b = warp / 4 (rows and columns 32b..32b+31), four columns per warp
-      {
-        const int b = warp >> 2, R0 = 32 * b, R1 = R0 + 16;
-        const int r = lane & 15, c0 = 4 * (warp & 3) + 2 * (lane >> 4);
-        float p0 = 0.f, p1 = 0.f;
+    // R2: D = N_d Z (K steps 2, 3)
+    if (tid == 0) merge_mma(L_::DB, L_::NOP, L_::YB, 0xC);
+    mma_issued = 3;
+    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
+    mma_done = 3;
+    tc_fence_after();
+    // T = (N_d - D) Diag(beta), lower triangle, bf16 rows of the WY products' operand
+    if (rowt) {
+      uint32_t d4[32];
+      tmem_ld32(tb + lane_base + L_::DB + 32 * hh, d4);
+      tmem_ld_wait(d4);
+      float f[32];
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const float4 av = a4(R1 + r, R0 + 4 * g4);
-          const float af[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 nn = *reinterpret_cast<const float2*>(n_ptr(R0 + 4 * g4 + e, R0 + c0));
-            p0 = fmaf(af[e], nn.x, p0);
-            p1 = fmaf(af[e], nn.y, p1);
-          }
-        }
-        *reinterpret_cast<float2*>(pw + r * 4 + (c0 & 3)) = make_float2(p0, p1);
-        __syncwarp();
-        float o0 = 0.f, o1 = 0.f;
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const float4 nv4 = n4(R1 + r, R1 + 4 * g4);
-          const float nf[4] = {nv4.x, nv4.y, nv4.z, nv4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 pp = *reinterpret_cast<const float2*>(pw + (4 * g4 + e) * 4 + (c0 & 3));
-            o0 = fmaf(nf[e], pp.x, o0);
-            o1 = fmaf(nf[e], pp.y, o1);
-          }
-        }
-        *reinterpret_cast<float2*>(n_ptr(R1 + r, R0 + c0)) = make_float2(-o0, -o1);
-        *reinterpret_cast<float2*>(n_ptr(R0 + r, R1 + c0)) = make_float2(0.f, 0.f);
+      for (int t = 0; t < 32; ++t) {
+        const int c = 32 * hh + t;
+        const float nrc = nrow[t] - __uint_as_float(d4[t]);
+        f[t] = c <= rr ? nrc * bet[c] : 0.f;
       }
-      __syncthreads();
-      // 32 -> 64: rows 32..63, columns 0..31, four columns per warp, lane = row
-      {
-        const int r = lane, cc = 4 * warp;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int g4 = 0; g4 < 8; ++g4) {
-          const float4 av = a4(32 + r, 4 * g4);
-          fma4(av.x, n4(4 * g4 + 0, cc), acc);
-          fma4(av.y, n4(4 * g4 + 1, cc), acc);
-          fma4(av.z, n4(4 * g4 + 2, cc), acc);
-          fma4(av.w, n4(4 * g4 + 3, cc), acc);
-        }
-        __syncwarp();  // the 16 -> 32 scratch of this warp is no longer read
-        *reinterpret_cast<float4*>(pw + r * 4) = acc;
-        __syncwarp();
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int g4 = 0; g4 < 8; ++g4) {
-          const float4 nv4 = n4(32 + r, 32 + 4 * g4);
-          fma4(nv4.x, *reinterpret_cast<const float4*>(pw + (4 * g4 + 0) * 4), o);
-          fma4(nv4.y, *reinterpret_cast<const float4*>(pw + (4 * g4 + 1) * 4), o);
-          fma4(nv4.z, *reinterpret_cast<const float4*>(pw + (4 * g4 + 2) * 4), o);
-          fma4(nv4.w, *reinterpret_cast<const float4*>(pw + (4 * g4 + 3) * 4), o);
-        }
-        *reinterpret_cast<float4*>(n_ptr(32 + r, cc)) = make_float4(-o.x, -o.y, -o.z, -o.w);
-      }
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(rr, 4 * hh + q, K8)) = pack8(f + 8 * q);
     }
-    __syncthreads();
-    // ---- 6. T = N Diag(beta), lower triangle, bf16 operand: two 16-byte chunks per thread
-    {
-      const int r = tid >> 2;
-#pragma unroll
-      for (int q8 = 0; q8 < 2; ++q8) {
-        const int c8 = (tid & 3) * 2 + q8;
-        float f[8];
-#pragma unroll
-        for (int h4 = 0; h4 < 2; ++h4) {
-          const int cc = 8 * c8 + 4 * h4;
-          const float4 nn = n4(r, cc);
-          const float4 bb = *reinterpret_cast<const float4*>(bet + cc);
-          f[4 * h4 + 0] = (cc + 0 <= r) ? nn.x * bb.x : 0.f;
-          f[4 * h4 + 1] = (cc + 1 <= r) ? nn.y * bb.y : 0.f;
-          f[4 * h4 + 2] = (cc + 2 <= r) ? nn.z * bb.z : 0.f;
-          f[4 * h4 + 3] = (cc + 3 <= r) ? nn.w * bb.w : 0.f;
-        }
-        *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(r, c8, K8)) = pack8(f);
-      }
-    }
+    tc_fence_before();
     fence_async_smem();
     if (cta_wait_failed(bar_v, 0)) { failed = true; break; }  // also the barrier for T
     v_done = true;
@@ -594,29 +703,39 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       umma_commit(bar_mma);
     }
-    mma_issued = 2;
+    mma_issued = 4;
     if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
-    mma_done = 2;
+    mma_done = 4;
     tc_fence_after();
-    // ---- 8. -W and U0 to the workspace: tensor-memory lane i holds column i of both
+    // ---- 8. -W^T and U0^T to the workspace through staging tiles (the merge tiles are
+    //         dead): tensor-memory lane i holds row i of both
     {
       const int i = (warp & 3) * 32 + lane, cb = (warp >> 2) * 32;
       uint32_t v[32];
       tmem_ld32(tb + lane_base + L_::W + cb, v);
       tmem_ld_wait(v);
-      __nv_bfloat16* wo = a.wn + (tile * C + cb) * D + i;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) wo[t * D] = __float2bfloat16_rn(-__uint_as_float(v[t]));
-      tmem_ld32(tb + lane_base + L_::U + cb, v);
-      tmem_ld_wait(v);
-      // U0 is stored transposed ([j][r] per tile): this lane's 32 values are contiguous
-      uint4* uo = reinterpret_cast<uint4*>(a.u0 + (tile * D + i) * C + cb);
+      for (int t = 0; t < 32; ++t) v[t] ^= 0x80000000u;  // -W
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        uo[q] = pack8(reinterpret_cast<const float*>(v) + 8 * q);
+        *reinterpret_cast<uint4*>(sm + L_::WTS + sw128_chunk(i, (cb >> 3) + q, 0)) =
+            pack8(reinterpret_cast<const float*>(v) + 8 * q);
+      tmem_ld32(tb + lane_base + L_::U + cb, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(sm + L_::U0S + sw128_chunk(i, (cb >> 3) + q, 0)) =
+            pack8(reinterpret_cast<const float*>(v) + 8 * q);
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 32) {
+      tma_store_2d(&a.tm_wt, sm + L_::WTS, 0, static_cast<int>(tile * D));
+      tma_store_2d(&a.tm_u0, sm + L_::U0S, 0, static_cast<int>(tile * D));
+      bulk_commit();
     }
   } while (0);
-  if (tid == 32) bulk_wait_all();  // workspace stores complete
+  if (tid == 32) bulk_wait_all();  // the workspace stores complete before the CTA exits
   if (failed && tid == 0) {
     atomicExch(a.seq.status, kDevWaitTimeout);
     // copies and products in flight finish before the CTA releases its memory
@@ -650,11 +769,13 @@ constexpr int kConvBar = 1;  // named barrier of the conversion warps; 2 + half 
 template <bool PC>
 struct WalkSm {
   static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks: [S] or [M | L]
-  // One input stage; every [64][128] tile is two 64-column boxes.
-  //   output walk, even stage: WQ = [-W a0 | Q~ a0 | -W a1 | Q~ a1], PK = [P^T | Kb a0 | Kb a1]
-  //   output walk, odd stage:  WQ = [Q~ a0 | -W a0 | Q~ a1 | -W a1], PK = [Kb a0 | Kb a1 | P^T]
-  //   summary walk: WQ = -W, PK = Kb.
-  // The order follows the tensor-memory order of the accumulators in the two products.
+  // One input stage of 128-byte-swizzled tiles as TMA lands them (rows of 64 elements):
+  //   output walk, even stage: WQ = [-W^T | Q~^T] (128 rows each), PK = [P (64 rows) | Kb^T]
+  //   output walk, odd stage:  WQ = [Q~^T | -W^T],                  PK = [Kb^T | P]
+  //   summary walk: WQ = -W^T, PK = Kb^T.
+  // WQ is MMA-1's B operand, MN-major (rows = the state row i, 64 tokens each; the two
+  // 64-token groups 16 KB apart); PK is MMA-2's, K-major (rows = output columns, 64
+  // tokens each). The order follows the tensor-memory order of the accumulators.
   static constexpr uint32_t WQ = 0;
   static constexpr uint32_t U0 = PC ? K32 : K16;
   static constexpr uint32_t PK = U0 + K16;
@@ -669,13 +790,13 @@ struct WalkSm {
   // S at 128..255 (so MMA-2's accumulator [O | S] is 64..255); p = 1: S at 128..255,
   // [O | U] at 256..383 (MMA-2's [S | O] is 128..319). Summary walk: S per block at
   // 128 b, U per block at 256 + 64 b. The bf16 S^T operand (64 columns of pairs) per
-  // block at 384 + 64 b; the bf16 U^T operand is packed in place over U: thread half hc
-  // packs its 32 columns into the first 16, so K step k sits at U + uk(k).
+  // block at 384 + 64 b; the bf16 U^T operand is packed in place over U: K step k (16
+  // columns of U) is packed into the first 8 of them, at U + uk(k).
   __device__ static constexpr uint32_t st(int b) { return PC ? 128 : 128 * b; }
   __device__ static constexpr uint32_t uc(int b, int p) { return PC ? (p ? 320 : 0) : 256 + 64 * b; }
   __device__ static constexpr uint32_t yo(int p) { return p ? 256 : 64; }
   __device__ static constexpr uint32_t sbf(int b) { return 384 + 64 * b; }
-  __device__ static constexpr uint32_t uk(int k) { return (k >> 1) * 32 + (k & 1) * 8; }
+  __device__ static constexpr uint32_t uk(int k) { return 16 * k; }
   static constexpr uint32_t COLS = 512;
 };
 static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
@@ -739,12 +860,12 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
   if (warp == kWalkLoadWarp) {
     // ============================================================ stage loads
     if (lane == 0 && n_chunks > 0) {
-      tma_prefetch_desc(&a.tm_wn);
+      tma_prefetch_desc(&a.tm_wt);
       tma_prefetch_desc(&a.tm_u0);
-      tma_prefetch_desc(&a.tm_kb);
+      tma_prefetch_desc(&a.tm_kbt);
       if (PC) {
         tma_prefetch_desc(&a.tm_qt);
-        tma_prefetch_desc(&a.tm_pt);
+        tma_prefetch_desc(&a.tm_p);
       }
       int issued = 0;
       bool ok = true;
@@ -753,23 +874,20 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         if (n >= 2 && !(ok = mbar_wait(bar_empty + st, ((n - 2) >> 1) & 1))) break;
         unsigned char* dst = sm + st * L_::STAGE;
         const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
-        const int y = static_cast<int>(tile * C);
+        const int y = static_cast<int>(tile * D);  // row of the [tiles * 128][64] arrays
         mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
-        for (int bx = 0; bx < 2; ++bx) {
-          if (PC) {
-            // even stages: [-W | Q~] rows, odd stages: [Q~ | -W]
-            tma_load_2d(dst + L_::WQ + st * K8 + bx * K16, &a.tm_wn, bar_full + st, 64 * bx, y);
-            tma_load_2d(dst + L_::WQ + (st ^ 1) * K8 + bx * K16, &a.tm_qt, bar_full + st, 64 * bx, y);
-            // even stages: [P^T | Kb], odd stages: [Kb | P^T]
-            tma_load_2d(dst + L_::PK + (st ? 0 : K8) + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
-          } else {
-            tma_load_2d(dst + L_::WQ + bx * K8, &a.tm_wn, bar_full + st, 64 * bx, y);
-            tma_load_2d(dst + L_::PK + bx * K8, &a.tm_kb, bar_full + st, 64 * bx, y);
-          }
-          tma_load_2d(dst + L_::U0 + bx * K8, &a.tm_u0, bar_full + st, 0,
-                      static_cast<int>(tile * D) + 64 * bx);
+        if (PC) {
+          // even stages: [-W^T | Q~^T], [P | Kb^T]; odd stages: [Q~^T | -W^T], [Kb^T | P]
+          tma_load_2d(dst + L_::WQ + st * K16, &a.tm_wt, bar_full + st, 0, y);
+          tma_load_2d(dst + L_::WQ + (st ^ 1) * K16, &a.tm_qt, bar_full + st, 0, y);
+          tma_load_2d(dst + L_::PK + (st ? 0 : K8), &a.tm_kbt, bar_full + st, 0, y);
+          tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_p, bar_full + st, 0,
+                      static_cast<int>(tile * C));
+        } else {
+          tma_load_2d(dst + L_::WQ, &a.tm_wt, bar_full + st, 0, y);
+          tma_load_2d(dst + L_::PK, &a.tm_kbt, bar_full + st, 0, y);
         }
-        if (PC) tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_pt, bar_full + st, 0, y);
+        tma_load_2d(dst + L_::U0, &a.tm_u0, bar_full + st, 0, y);
         bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
         ++issued;
       }
@@ -788,8 +906,9 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         const uint32_t stg = sb + st * L_::STAGE;
         if (!(ok = mbar_wait(bar_full + st, (n >> 1) & 1))) break;
         // MMA-1: U^T (output walk: with (Q~ S)^T in the same accumulator) = S^T [-W; Q~]^T,
-        // K = the 128 state rows in two halves, each started once its half of S^T is packed
-        const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 0);
+        // K = the 128 state rows in two halves, each started once its half of S^T is packed;
+        // B MN-major: 16 rows of the stage tiles per K step
+        const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 1);
         const uint32_t d1 = PC ? (st ? L_::yo(1) : L_::uc(0, 0)) : 0;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -800,38 +919,38 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int k = 4 * half + kk;
-              const uint32_t ko_w = half * (PC ? K16 : K8) + kk * 32;
               umma_bf16_tmem_a(tb + (PC ? d1 : L_::uc(b, 0)), tb + L_::sbf(b) + 8 * k,
-                               sdesc_sw128(stg + L_::WQ + ko_w, 16, 1024), i_k, k > 0);
+                               sdesc_sw128(stg + L_::WQ + k * 2048, K16, 1024), i_k, k > 0);
             }
         }
         if (!ok) break;
         umma_commit(bar_m1);
         ++m_issued;
         // MMA-2: output walk: [O^T | S^T] (or [S^T | O^T]) += U^T [P^T | Kb] in one N = 192
-        // product; summary walk: S^T += U^T Kb per block (B operands MN-major)
+        // product; summary walk: S^T += U^T Kb per block (B operands K-major: the stage's
+        // rows of P and Kb^T, 16 tokens = 32 bytes per K step)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!(ok = mbar_wait(bar_yready + half, n & 1))) break;
           tc_fence_after();
           if (PC) {
-            const uint32_t i2 = idesc_bf16(128, 192, 0, 1);
+            const uint32_t i2 = idesc_bf16(128, 192, 0, 0);
             const uint32_t d2 = st ? L_::st(0) : L_::yo(0);
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               const int k = 2 * half + kk;
               umma_bf16_tmem_a(tb + d2, tb + L_::uc(0, st) + L_::uk(k),
-                               sdesc_sw128(stg + L_::PK + k * 2048, K8, 1024), i2, 1);
+                               sdesc_sw128(stg + L_::PK + k * 32, 16, 1024), i2, 1);
             }
           } else {
-            const uint32_t i2 = idesc_bf16(128, 128, 0, 1);
+            const uint32_t i2 = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
             for (int b = 0; b < NB; ++b)
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk) {
                 const int k = 2 * half + kk;
                 umma_bf16_tmem_a(tb + L_::st(b), tb + L_::uc(b, 0) + L_::uk(k),
-                                 sdesc_sw128(stg + L_::PK + k * 2048, K8, 1024), i2, 1);
+                                 sdesc_sw128(stg + L_::PK + k * 32, 16, 1024), i2, 1);
               }
           }
         }
@@ -852,17 +971,18 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     // ============================================================ conversion warps
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
-    const int hc = warp >> 2;                // column half this thread converts
-    const int half_bar = 2 + hc;             // named barrier of this half's 128 threads
-    const bool half_lead = (warp & 3) == 0 && lane == 0;
+    const int hc = warp >> 2;                // which columns this thread converts (below)
+    // A thread's 64 columns of S^T (state rows i) are i = 32 hc .. + 31 (in v0) and
+    // 64 + 32 hc .. + 31 (in v1): every warp packs its part of the first K half of the
+    // bf16 operand before any of the second, so MMA-1's first half can start early.
     // S <- Diag(gl) S on this thread's 64 fp32 columns of block b (held in v0, v1),
     // written back to tensor memory: the decay of the chunk about to be walked
     auto rescale = [&](int b, int st, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
-      const float* gl = gls + st * D + 64 * hc;
+      const float* gl = gls + st * D + 32 * hc;
 #pragma unroll
       for (int t4 = 0; t4 < 8; ++t4) {
         const float4 g0 = *reinterpret_cast<const float4*>(gl + 4 * t4);
-        const float4 g1 = *reinterpret_cast<const float4*>(gl + 32 + 4 * t4);
+        const float4 g1 = *reinterpret_cast<const float4*>(gl + 64 + 4 * t4);
         v0[4 * t4 + 0] = __float_as_uint(g0.x * __uint_as_float(v0[4 * t4 + 0]));
         v0[4 * t4 + 1] = __float_as_uint(g0.y * __uint_as_float(v0[4 * t4 + 1]));
         v0[4 * t4 + 2] = __float_as_uint(g0.z * __uint_as_float(v0[4 * t4 + 2]));
@@ -872,8 +992,8 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         v1[4 * t4 + 2] = __float_as_uint(g1.z * __uint_as_float(v1[4 * t4 + 2]));
         v1[4 * t4 + 3] = __float_as_uint(g1.w * __uint_as_float(v1[4 * t4 + 3]));
       }
-      tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, v0);
-      tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+      tmem_st32(tb + lane_base + L_::st(b) + 32 * hc, v0);
+      tmem_st32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
     };
     // The decay of stage st on every block: the output walk's single block is still in
     // v0, v1; the summary walk's blocks are reloaded from tensor memory.
@@ -883,8 +1003,8 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       } else {
 #pragma unroll 1
         for (int b = 0; b < NB; ++b) {
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, v0);
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+          tmem_ld32(tb + lane_base + L_::st(b) + 32 * hc, v0);
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
           tmem_ld_wait(v0);
           tmem_ld_wait(v1);
           rescale(b, st, v0, v1);
@@ -892,15 +1012,12 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       }
       tmem_st_wait();
     };
-    // S^T of block b (this thread's 64 columns, in v0, v1) into the bf16 operand
-    auto pack_state = [&](int b, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
-      uint32_t pk[32];
+    // this thread's 32 columns of K half kh of S^T (block b, in v) into the bf16 operand
+    auto pack_half = [&](int b, int kh, const uint32_t (&v)[32]) {
+      uint32_t pk[16];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        pk[t] = pack_bf16(__uint_as_float(v0[2 * t]), __uint_as_float(v0[2 * t + 1]));
-        pk[16 + t] = pack_bf16(__uint_as_float(v1[2 * t]), __uint_as_float(v1[2 * t + 1]));
-      }
-      tmem_st32(tb + lane_base + L_::sbf(b) + 32 * hc, pk);
+      for (int t = 0; t < 16; ++t) pk[t] = pack_bf16(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1]));
+      tmem_st16(tb + lane_base + L_::sbf(b) + 32 * kh + 16 * hc, pk);
     };
     bool failed = false, pend_store = false;
     // initial state: fp32 into tensor memory, bf16 copy as the MMA operand; then the
@@ -916,7 +1033,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       for (int b = 0; b < NB; ++b) {
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const int c0 = 64 * hc + t, c1 = 64 * hc + 32 + t;
+          const int c0 = 32 * hc + t, c1 = 64 + 32 * hc + t;
           float x0, x1;
           if (PC) {
             x0 = src ? src[static_cast<int64_t>(c0) * D + row] : 0.f;
@@ -928,16 +1045,20 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
           v0[t] = __float_as_uint(x0);
           v1[t] = __float_as_uint(x1);
         }
-        pack_state(b, v0, v1);
+        pack_half(b, 0, v0);
+        pack_half(b, 1, v1);
         if (NB > 1 || n_chunks == 0) {  // the unscaled fp32 state (reloaded below / final)
-          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc, v0);
-          tmem_st32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+          tmem_st32(tb + lane_base + L_::st(b) + 32 * hc, v0);
+          tmem_st32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
         }
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(half_bar, 128);
-      if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + hc);
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0 && n_chunks > 0) {
+        mbar_arrive(bar_sready);
+        mbar_arrive(bar_sready + 1);
+      }
       if (n_chunks > 0) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0, KDA_FIRST_WAIT_LIMIT))) {
           failed = true;
@@ -983,11 +1104,11 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       const int64_t done = off / C + n + 1;  // chunks of the sequence walked so far
       if (done % a.snap_every != 0 || done * C > len) return;
       const int64_t idx = t0 / (static_cast<int64_t>(C) * a.snap_every) + done / a.snap_every - 1;
-      float* dst = a.snap + (idx * a.H + h) * D * D + static_cast<int64_t>(64 * hc) * D + row;
+      float* dst = a.snap + (idx * a.H + h) * D * D + static_cast<int64_t>(32 * hc) * D + row;
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
         dst[t * D] = __uint_as_float(v0[t]);
-        dst[(32 + t) * D] = __uint_as_float(v1[t]);
+        dst[(64 + t) * D] = __uint_as_float(v1[t]);
       }
     };
 
@@ -996,14 +1117,15 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     // MMA-1(n + 1), then the fp32 state rescaled by the next chunk's decay.
     for (int n = 0; n < n_chunks && !failed; ++n) {
       const int st = n & 1;
-      // U0^T[j][r] for this thread's rows r = 32 hc .. 32 hc + 31 (four 16-byte chunks
-      // of row j of the swizzled [64 j][64 r] box)
+      // U0^T[j][r] for this thread's tokens r = 32 p + 16 hc .. + 15, p = 0, 1 (16-byte
+      // chunks 4 p + 2 hc, 4 p + 2 hc + 1 of row j of the swizzled [128 j][64 r] tile)
       float u0v[32];
       {
-        const unsigned char* u0r = sm + st * L_::STAGE + L_::U0 + (row >> 6) * K8;
+        const unsigned char* u0r = sm + st * L_::STAGE + L_::U0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row & 63, 4 * hc + q, K8));
+          const int c8 = 4 * (q >> 1) + 2 * hc + (q & 1);
+          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row, c8, 0));
           const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1018,28 +1140,48 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         break;
       }
       tc_fence_after();
-      // ---- U^T (+ U0^T) -> bf16 operand, packed in place (this thread's 32 columns)
+      // ---- U^T (+ U0^T) -> bf16 operand, packed in place: K half p (tokens 32 p ..
+      //      32 p + 31) by every warp before the next, so MMA-2's first half starts early;
+      //      this thread's 16 columns 32 p + 16 hc .. + 15 are K step 2 p + hc
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        uint32_t v[32], pk[16];
-        tmem_ld32(tb + lane_base + L_::uc(b, st) + 32 * hc, v);
+        // both K halves' columns of this block are loaded before the first wait
+        uint32_t v[32];
+        uint32_t (&v_lo)[16] = *reinterpret_cast<uint32_t (*)[16]>(v);
+        uint32_t (&v_hi)[16] = *reinterpret_cast<uint32_t (*)[16]>(v + 16);
+        tmem_ld16(tb + lane_base + L_::uc(b, st) + 16 * hc, v_lo);
+        tmem_ld16(tb + lane_base + L_::uc(b, st) + 32 + 16 * hc, v_hi);
         tmem_ld_wait(v);
         const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          float x0 = __uint_as_float(v[2 * t]), x1 = __uint_as_float(v[2 * t + 1]);
-          if (with_u0) {
-            x0 += u0v[2 * t];
-            x1 += u0v[2 * t + 1];
+        for (int p2 = 0; p2 < 2; ++p2) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            float x0 = __uint_as_float(v[16 * p2 + 2 * t]), x1 = __uint_as_float(v[16 * p2 + 2 * t + 1]);
+            if (with_u0) {
+              x0 += u0v[16 * p2 + 2 * t];
+              x1 += u0v[16 * p2 + 2 * t + 1];
+            }
+            pk[t] = pack_bf16(x0, x1);
           }
-          pk[t] = pack_bf16(x0, x1);
+          tmem_st8(tb + lane_base + L_::uc(b, st) + 32 * p2 + 16 * hc, pk);
+          if (NB == 1 && p2 == 0) {
+            // the first K half of the single block is in place: MMA-2's first half may go
+            tmem_st_wait();
+            tc_fence_before();
+            group_sync(kConvBar, kWalkConvThreads);
+            if (tid == 0) mbar_arrive(bar_yready);
+          }
         }
-        tmem_st16(tb + lane_base + L_::uc(b, st) + 32 * hc, pk);
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(half_bar, 128);
-      if (half_lead) mbar_arrive(bar_yready + hc);
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0) {
+        if (NB > 1) mbar_arrive(bar_yready);
+        mbar_arrive(bar_yready + 1);
+      }
       // ---- while MMA-2(n) runs: the previous chunk's outputs
       if (PC && n > 0) {
         const bool staged = emit_out(n - 1);
@@ -1055,20 +1197,42 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         break;
       }
       tc_fence_after();
-      // ---- bf16 S^T operand for MMA-1(n + 1), then the next chunk's decay on the fp32 state
+      // ---- bf16 S^T operand for MMA-1(n + 1), K half 0 (state rows 0..63) from every
+      //      warp first, then K half 1; then the next chunk's decay on the fp32 state
       uint32_t v0[32], v1[32];
-#pragma unroll 1
-      for (int b = 0; b < NB; ++b) {
-        tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc, v0);
-        tmem_ld32(tb + lane_base + L_::st(b) + 64 * hc + 32, v1);
+      if (NB == 1) {
+        // both halves' loads in flight before the first wait
+        tmem_ld32(tb + lane_base + L_::st(0) + 32 * hc, v0);
+        tmem_ld32(tb + lane_base + L_::st(0) + 64 + 32 * hc, v1);
         tmem_ld_wait(v0);
         tmem_ld_wait(v1);
-        pack_state(b, v0, v1);
+        pack_half(0, 0, v0);
+      } else {
+#pragma unroll 1
+        for (int b = 0; b < NB; ++b) {
+          tmem_ld32(tb + lane_base + L_::st(b) + 32 * hc, v0);
+          tmem_ld_wait(v0);
+          pack_half(b, 0, v0);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(half_bar, 128);
-      if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + hc);
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready);
+      if (NB == 1) {
+        pack_half(0, 1, v1);
+      } else {
+#pragma unroll 1
+        for (int b = 0; b < NB; ++b) {
+          tmem_ld32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
+          tmem_ld_wait(v1);
+          pack_half(b, 1, v1);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      group_sync(kConvBar, kWalkConvThreads);
+      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready + 1);
       if (PC && SNAP) store_snapshot(n, v0, v1);  // while MMA-1(n + 1) runs
       if (n + 1 < n_chunks) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
@@ -1169,12 +1333,6 @@ struct CombTm {
   static constexpr uint32_t D = 0, AH = 128, AL = 192, COLS = 256;
 };
 
-__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
-  const float2 hf = __bfloat1622float2(h);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = pack_bf16(x - hf.x, y - hf.y);
-}
 
 __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_constant__ WalkArgs a) {
   extern __shared__ unsigned char smem_raw[];
@@ -1369,15 +1527,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D bf16 tensor map over `rows` rows of `cols` elements, `pitch` bytes apart,
-// moved in boxes of 64 rows x `box_cols`; with `swizzle` (64 columns) a box lands in
-// the 128-byte-swizzled operand layout.
+// moved in boxes of `box_rows` rows x `box_cols`; with `swizzle` (64 columns) a box
+// lands in the 128-byte-swizzled operand layout.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t pitch,
-              bool swizzle, uint32_t box_cols = 64) {
+              bool swizzle, uint32_t box_cols = 64, uint32_t box_rows = 64) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch)};
-  cuuint32_t box[2] = {box_cols, 64};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1435,14 +1593,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   const SeqTable seq{pa.cu, pa.status, pa.T, pa.T_total, pa.n_seqs};
   // workspace: header | M, L, S_start (segmented walks only) | per-chunk tiles
   unsigned char* tp = pa.ws + plan.tiles_off;
-  auto* wn = reinterpret_cast<__nv_bfloat16*>(tp);
-  __nv_bfloat16* u0 = wn + tiles * C * D;
-  __nv_bfloat16* kb = u0 + tiles * C * D;
-  __nv_bfloat16* qt = kb + tiles * C * D;
-  __nv_bfloat16* pt = qt + tiles * C * D;
-  auto* gl = reinterpret_cast<float*>(pt + tiles * C * C);
+  auto* wt = reinterpret_cast<__nv_bfloat16*>(tp);
+  __nv_bfloat16* qt = wt + tiles * C * D;
+  __nv_bfloat16* u0 = qt + tiles * C * D;
+  __nv_bfloat16* kbt = u0 + tiles * C * D;
+  __nv_bfloat16* pm = kbt + tiles * C * D;
+  auto* gl = reinterpret_cast<float*>(pm + tiles * C * C);
   const uint64_t in_cols = static_cast<uint64_t>(pa.H) * D, in_pitch = in_cols * 2;
-  const uint64_t rows_t = static_cast<uint64_t>(tiles) * C;
+  const uint64_t rows_big = static_cast<uint64_t>(tiles) * D;  // [tiles * 128][64] arrays
+  const uint64_t rows_p = static_cast<uint64_t>(tiles) * C;    // [tiles * 64][64]
 
   IntraArgs ia;
   memset(&ia, 0, sizeof ia);
@@ -1452,21 +1611,21 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
       !make_map(&ia.tm_k, pa.k, in_cols, pa.T_total, in_pitch, false, D) ||
       !make_map(&ia.tm_g, pa.g, in_cols, pa.T_total, in_pitch, false, D) ||
       !make_map(&ia.tm_v, pa.v, in_cols, pa.T_total, in_pitch, true) ||
-      !make_map(&ia.tm_qt, qt, D, rows_t, D * 2, true) ||
-      !make_map(&ia.tm_kb, kb, D, rows_t, D * 2, true) ||
+      !make_map(&ia.tm_wt, wt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&ia.tm_qt, qt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&ia.tm_u0, u0, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&ia.tm_kbt, kbt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&ia.tm_p, pm, C, rows_p, C * 2, true) ||
 
-      !make_map(&wa.tm_wn, wn, D, rows_t, D * 2, true) ||
-      !make_map(&wa.tm_u0, u0, C, static_cast<uint64_t>(tiles) * D, C * 2, true) ||
-      !make_map(&wa.tm_kb, kb, D, rows_t, D * 2, true) ||
-      !make_map(&wa.tm_qt, qt, D, rows_t, D * 2, true) ||
-      !make_map(&wa.tm_pt, pt, C, rows_t, C * 2, true) ||
+      !make_map(&wa.tm_wt, wt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&wa.tm_qt, qt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&wa.tm_u0, u0, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&wa.tm_kbt, kbt, C, rows_big, C * 2, true, C, D) ||
+      !make_map(&wa.tm_p, pm, C, rows_p, C * 2, true) ||
       !make_map(&wa.tm_o, pa.out, in_cols, pa.T_total, in_pitch, false))
     return cudaErrorInvalidValue;
   ia.seq = seq;
   ia.beta = static_cast<const __nv_bfloat16*>(pa.beta);
-  ia.wn = wn;
-  ia.u0 = u0;
-  ia.pt = pt;
   ia.gl = gl;
   ia.H = pa.H;
   ia.lb = pa.lb;
