@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t u = blockIdx.x / a.H;
-  const int h = static_cast<int>(blockIdx.x % a.H);
+  const int64_t u = static_cast<int64_t>(blockIdx.x / static_cast<unsigned>(a.H));
+  const int h = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.H));
 
   // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
   const int s = owner_seq(a.seq, u);
@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   if (warp == 0) {
     tmem_alloc(tptr, L_::COLS);
     tmem_relinquish();
-  }
-  if (tid == 0) {
+  } else if (tid == 32) {
+    // barriers and input loads from warp 1, while warp 0 allocates tensor memory
     mbar_init(bar_in, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
@@ -754,18 +754,20 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 
 // ------------------------------------------------------------------ walk over chunks
 // One CTA per (sequence, head, segment), warp-specialized:
-//   warps 0..7  conversion: warps w and w + 4 share the tensor-memory lanes 32 (w % 4)..+31
-//               (state columns j); warps 0..3 own the first half of the columns, warps
-//               4..7 the second. They rescale the fp32 state, add U0 and pack U^T and S^T
-//               into bf16 MMA operands kept in tensor memory, and write the outputs;
-//   warp 8      issues the MMAs (one thread);
-//   warp 9      streams each chunk's workspace tiles into two stages by TMA (one thread).
-// Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and per column
-// half s_ready/y_ready (that half of the bf16 S^T or U^T operand is in tensor memory), so
-// the first half of a product starts while the second half is still being packed.
-constexpr int kWalkConvThreads = 256, kWalkThreads = 320;
-constexpr int kWalkMmaWarp = 8, kWalkLoadWarp = 9;
-constexpr int kConvBar = 1;  // named barrier of the conversion warps; 2 + half for a half
+//   warps 0..15 conversion: warps w, w + 4, w + 8, w + 12 share the tensor-memory lanes
+//               32 (w % 4)..+31 (state columns j) and split their columns four ways;
+//               warps 0..7 own K half 0 of the products' operands, warps 8..15 K half 1.
+//               They rescale the fp32 state, add U0 and pack U^T and S^T into bf16 MMA
+//               operands kept in tensor memory, and write the outputs;
+//   warp 16     issues the MMAs (one thread);
+//   warp 17     streams each chunk's workspace tiles into two stages by TMA (one thread).
+// Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and per K half
+// s_ready/y_ready (that half of the bf16 S^T or U^T operand is in tensor memory), so the
+// first half of a product starts while the second half is still being packed.
+constexpr int kWalkConvThreads = 512, kWalkThreads = 576;
+constexpr int kWalkMmaWarp = 16, kWalkLoadWarp = 17;
+constexpr int kConvBar = 1;   // named barrier of all the conversion warps
+constexpr int kHalfBar0 = 2;  // named barriers of the two K halves' warps: 2, 3
 template <bool PC>
 struct WalkSm {
   static constexpr int NB = PC ? 1 : 2;  // 128-column state blocks: [S] or [M | L]
@@ -905,11 +907,13 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         const int st = n & 1;
         const uint32_t stg = sb + st * L_::STAGE;
         if (!(ok = mbar_wait(bar_full + st, (n >> 1) & 1))) break;
-        // MMA-1: U^T (output walk: with (Q~ S)^T in the same accumulator) = S^T [-W; Q~]^T,
-        // K = the 128 state rows in two halves, each started once its half of S^T is packed;
-        // B MN-major: 16 rows of the stage tiles per K step
-        const uint32_t i_k = idesc_bf16(128, PC ? 128 : 64, 0, 1);
-        const uint32_t d1 = PC ? (st ? L_::yo(1) : L_::uc(0, 0)) : 0;
+        // MMA-1: U^T = S^T (-W)^T and (output walk) (Q~ S)^T = S^T Q~^T, K = the 128 state
+        // rows in two halves, each started once its half of S^T is packed; B MN-major: 16
+        // rows of the stage tiles per K step
+        // The U^T part (B = the -W^T tile) is committed on m1 by itself, so that the
+        // conversion warps pack it while the (Q~ S)^T part (output walk) still runs.
+        const uint32_t i_k = idesc_bf16(128, 64, 0, 1);
+        const uint32_t wt_off = PC ? st * K16 : 0;  // -W^T tile in the stage
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!(ok = mbar_wait(bar_sready + half, n & 1))) break;
@@ -919,13 +923,21 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int k = 4 * half + kk;
-              umma_bf16_tmem_a(tb + (PC ? d1 : L_::uc(b, 0)), tb + L_::sbf(b) + 8 * k,
-                               sdesc_sw128(stg + L_::WQ + k * 2048, K16, 1024), i_k, k > 0);
+              umma_bf16_tmem_a(tb + L_::uc(b, st), tb + L_::sbf(b) + 8 * k,
+                               sdesc_sw128(stg + L_::WQ + wt_off + k * 2048, K16, 1024), i_k, k > 0);
             }
         }
         if (!ok) break;
         umma_commit(bar_m1);
         ++m_issued;
+        if (PC) {
+          // (Q~ S)^T into this chunk's O columns (B = the Q~^T tile); MMA-2 adds U^T P^T
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_bf16_tmem_a(tb + L_::yo(st), tb + L_::sbf(0) + 8 * k,
+                             sdesc_sw128(stg + L_::WQ + (K16 - wt_off) + k * 2048, K16, 1024), i_k,
+                             k > 0);
+        }
         // MMA-2: output walk: [O^T | S^T] (or [S^T | O^T]) += U^T [P^T | Kb] in one N = 192
         // product; summary walk: S^T += U^T Kb per block (B operands K-major: the stage's
         // rows of P and Kb^T, 16 tokens = 32 bytes per K step)
@@ -969,55 +981,37 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     }
   } else {
     // ============================================================ conversion warps
+    // Warp w holds tensor-memory lanes 32 (w % 4) .. + 31 (state columns j) and part
+    // pt = w / 4 of the columns: state rows i = 32 pt .. + 31, U^T and O^T columns (the
+    // chunk's tokens) 16 pt .. + 15. Warps 0..7 (parts 0, 1) own K half 0 of both MMA
+    // operands (state rows 0..63, tokens 0..31), warps 8..15 K half 1; each half has its
+    // own named barrier and releases its half of each product as soon as it is packed.
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
-    const int hc = warp >> 2;                // which columns this thread converts (below)
-    // A thread's 64 columns of S^T (state rows i) are i = 32 hc .. + 31 (in v0) and
-    // 64 + 32 hc .. + 31 (in v1): every warp packs its part of the first K half of the
-    // bf16 operand before any of the second, so MMA-1's first half can start early.
-    // S <- Diag(gl) S on this thread's 64 fp32 columns of block b (held in v0, v1),
-    // written back to tensor memory: the decay of the chunk about to be walked
-    auto rescale = [&](int b, int st, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
-      const float* gl = gls + st * D + 32 * hc;
+    const int pt = warp >> 2;                // column part
+    const int kh = pt >> 1;                  // the K half this warp's columns belong to
+    const int half_bar = kHalfBar0 + kh;     // named barrier of this half's 256 threads
+    const bool half_lead = (warp & 7) == 0 && lane == 0;
+    // S <- Diag(gl) S on this thread's 32 fp32 state rows of block b (held in v), written
+    // back to tensor memory: the decay of the chunk about to be walked
+    auto rescale = [&](int b, int st, uint32_t (&v)[32]) {
+      const float* gl = gls + st * D + 32 * pt;
 #pragma unroll
       for (int t4 = 0; t4 < 8; ++t4) {
-        const float4 g0 = *reinterpret_cast<const float4*>(gl + 4 * t4);
-        const float4 g1 = *reinterpret_cast<const float4*>(gl + 64 + 4 * t4);
-        v0[4 * t4 + 0] = __float_as_uint(g0.x * __uint_as_float(v0[4 * t4 + 0]));
-        v0[4 * t4 + 1] = __float_as_uint(g0.y * __uint_as_float(v0[4 * t4 + 1]));
-        v0[4 * t4 + 2] = __float_as_uint(g0.z * __uint_as_float(v0[4 * t4 + 2]));
-        v0[4 * t4 + 3] = __float_as_uint(g0.w * __uint_as_float(v0[4 * t4 + 3]));
-        v1[4 * t4 + 0] = __float_as_uint(g1.x * __uint_as_float(v1[4 * t4 + 0]));
-        v1[4 * t4 + 1] = __float_as_uint(g1.y * __uint_as_float(v1[4 * t4 + 1]));
-        v1[4 * t4 + 2] = __float_as_uint(g1.z * __uint_as_float(v1[4 * t4 + 2]));
-        v1[4 * t4 + 3] = __float_as_uint(g1.w * __uint_as_float(v1[4 * t4 + 3]));
+        const float4 g = *reinterpret_cast<const float4*>(gl + 4 * t4);
+        v[4 * t4 + 0] = __float_as_uint(g.x * __uint_as_float(v[4 * t4 + 0]));
+        v[4 * t4 + 1] = __float_as_uint(g.y * __uint_as_float(v[4 * t4 + 1]));
+        v[4 * t4 + 2] = __float_as_uint(g.z * __uint_as_float(v[4 * t4 + 2]));
+        v[4 * t4 + 3] = __float_as_uint(g.w * __uint_as_float(v[4 * t4 + 3]));
       }
-      tmem_st32(tb + lane_base + L_::st(b) + 32 * hc, v0);
-      tmem_st32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
+      tmem_st32(tb + lane_base + L_::st(b) + 32 * pt, v);
     };
-    // The decay of stage st on every block: the output walk's single block is still in
-    // v0, v1; the summary walk's blocks are reloaded from tensor memory.
-    auto rescale_all = [&](int st, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
-      if (NB == 1) {
-        rescale(0, st, v0, v1);
-      } else {
-#pragma unroll 1
-        for (int b = 0; b < NB; ++b) {
-          tmem_ld32(tb + lane_base + L_::st(b) + 32 * hc, v0);
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
-          tmem_ld_wait(v0);
-          tmem_ld_wait(v1);
-          rescale(b, st, v0, v1);
-        }
-      }
-      tmem_st_wait();
-    };
-    // this thread's 32 columns of K half kh of S^T (block b, in v) into the bf16 operand
-    auto pack_half = [&](int b, int kh, const uint32_t (&v)[32]) {
+    // this thread's 32 state rows of block b (in v) into the bf16 S^T operand
+    auto pack_state = [&](int b, const uint32_t (&v)[32]) {
       uint32_t pk[16];
 #pragma unroll
       for (int t = 0; t < 16; ++t) pk[t] = pack_bf16(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1]));
-      tmem_st16(tb + lane_base + L_::sbf(b) + 32 * kh + 16 * hc, pk);
+      tmem_st16(tb + lane_base + L_::sbf(b) + 16 * pt, pk);
     };
     bool failed = false, pend_store = false;
     // initial state: fp32 into tensor memory, bf16 copy as the MMA operand; then the
@@ -1028,42 +1022,40 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         if (seg > 0) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
         else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
       }
-      uint32_t v0[32], v1[32];  // the last block's values (the only one in the output walk)
+      uint32_t v[32];  // the last block's values (the only one in the output walk)
 #pragma unroll 1
       for (int b = 0; b < NB; ++b) {
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const int c0 = 32 * hc + t, c1 = 64 + 32 * hc + t;
-          float x0, x1;
-          if (PC) {
-            x0 = src ? src[static_cast<int64_t>(c0) * D + row] : 0.f;
-            x1 = src ? src[static_cast<int64_t>(c1) * D + row] : 0.f;
-          } else {
-            x0 = (b == 0 && c0 == row) ? 1.f : 0.f;
-            x1 = (b == 0 && c1 == row) ? 1.f : 0.f;
-          }
-          v0[t] = __float_as_uint(x0);
-          v1[t] = __float_as_uint(x1);
+          const int c = 32 * pt + t;
+          float x;
+          if (PC) x = src ? src[static_cast<int64_t>(c) * D + row] : 0.f;
+          else x = (b == 0 && c == row) ? 1.f : 0.f;
+          v[t] = __float_as_uint(x);
         }
-        pack_half(b, 0, v0);
-        pack_half(b, 1, v1);
-        if (NB > 1 || n_chunks == 0) {  // the unscaled fp32 state (reloaded below / final)
-          tmem_st32(tb + lane_base + L_::st(b) + 32 * hc, v0);
-          tmem_st32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
-        }
+        pack_state(b, v);
+        if (NB > 1 || n_chunks == 0)  // the unscaled fp32 state (reloaded below / final)
+          tmem_st32(tb + lane_base + L_::st(b) + 32 * pt, v);
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0 && n_chunks > 0) {
-        mbar_arrive(bar_sready);
-        mbar_arrive(bar_sready + 1);
-      }
+      group_sync(half_bar, 256);
+      if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + kh);
       if (n_chunks > 0) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0, KDA_FIRST_WAIT_LIMIT))) {
           failed = true;
         } else {
-          rescale_all(0, v0, v1);
+          if (NB == 1) {
+            rescale(0, 0, v);
+          } else {
+#pragma unroll 1
+            for (int b = 0; b < NB; ++b) {
+              tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+              tmem_ld_wait(v);
+              rescale(b, 0, v);
+            }
+          }
+          tmem_st_wait();
         }
       }
     }
@@ -1073,21 +1065,21 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     auto emit_out = [&](int n) {
       const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
       const int L = (c_end - c0) < C ? static_cast<int>(c_end - c0) : C;
-      uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::yo(n & 1) + 32 * hc, v);
+      uint32_t v[16];
+      tmem_ld16(tb + lane_base + L_::yo(n & 1) + 16 * pt, v);
       tmem_ld_wait(v);
       if (L == C) {
         __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sm + L_::OS + (row >> 6) * K8) +
-                            32 * hc * 64 + (row & 63);
+                            16 * pt * 64 + (row & 63);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) ob[t * 64] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
+        for (int t = 0; t < 16; ++t) ob[t * 64] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
       } else {
         // a sequence's ragged last chunk: rows past L belong to the next sequence
-        __nv_bfloat16* o = a.out + ((c0 + 32 * hc) * a.H + h) * D + row;
+        __nv_bfloat16* o = a.out + ((c0 + 16 * pt) * a.H + h) * D + row;
         const int64_t ostride = static_cast<int64_t>(a.H) * D;
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (32 * hc + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
+        for (int t = 0; t < 16; ++t)
+          if (16 * pt + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
       }
       return L == C;
     };
@@ -1098,18 +1090,15 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       bulk_commit();
     };
 
-    // The fp32 state after chunk n (this thread's 64 state rows of column `row`, in v0,
-    // v1) when that chunk is full and closes a snapshot interval of the sequence
-    auto store_snapshot = [&](int n, const uint32_t (&v0)[32], const uint32_t (&v1)[32]) {
+    // The fp32 state after chunk n (this thread's 32 state rows of column `row`, in v)
+    // when that chunk is full and closes a snapshot interval of the sequence
+    auto store_snapshot = [&](int n, const uint32_t (&v)[32]) {
       const int64_t done = off / C + n + 1;  // chunks of the sequence walked so far
       if (done % a.snap_every != 0 || done * C > len) return;
       const int64_t idx = t0 / (static_cast<int64_t>(C) * a.snap_every) + done / a.snap_every - 1;
-      float* dst = a.snap + (idx * a.H + h) * D * D + static_cast<int64_t>(32 * hc) * D + row;
+      float* dst = a.snap + (idx * a.H + h) * D * D + static_cast<int64_t>(32 * pt) * D + row;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        dst[t * D] = __uint_as_float(v0[t]);
-        dst[(64 + t) * D] = __uint_as_float(v1[t]);
-      }
+      for (int t = 0; t < 32; ++t) dst[t * D] = __uint_as_float(v[t]);
     };
 
     // Per chunk n (stage st = n % 2 has landed): MMA-1(n) runs -> U^T (+ U0^T) packed ->
@@ -1117,15 +1106,14 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     // MMA-1(n + 1), then the fp32 state rescaled by the next chunk's decay.
     for (int n = 0; n < n_chunks && !failed; ++n) {
       const int st = n & 1;
-      // U0^T[j][r] for this thread's tokens r = 32 p + 16 hc .. + 15, p = 0, 1 (16-byte
-      // chunks 4 p + 2 hc, 4 p + 2 hc + 1 of row j of the swizzled [128 j][64 r] tile)
-      float u0v[32];
+      // U0^T[j][r] for this thread's tokens r = 16 pt .. + 15 (16-byte chunks 2 pt,
+      // 2 pt + 1 of row j of the swizzled [128 j][64 r] tile)
+      float u0v[16];
       {
         const unsigned char* u0r = sm + st * L_::STAGE + L_::U0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c8 = 4 * (q >> 1) + 2 * hc + (q & 1);
-          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row, c8, 0));
+        for (int q = 0; q < 2; ++q) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row, 2 * pt + q, 0));
           const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1140,48 +1128,30 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         break;
       }
       tc_fence_after();
-      // ---- U^T (+ U0^T) -> bf16 operand, packed in place: K half p (tokens 32 p ..
-      //      32 p + 31) by every warp before the next, so MMA-2's first half starts early;
-      //      this thread's 16 columns 32 p + 16 hc .. + 15 are K step 2 p + hc
+      // ---- U^T (+ U0^T) -> bf16 operand, packed in place: this thread's 16 columns are
+      //      K step pt, packed into their first 8
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        // both K halves' columns of this block are loaded before the first wait
-        uint32_t v[32];
-        uint32_t (&v_lo)[16] = *reinterpret_cast<uint32_t (*)[16]>(v);
-        uint32_t (&v_hi)[16] = *reinterpret_cast<uint32_t (*)[16]>(v + 16);
-        tmem_ld16(tb + lane_base + L_::uc(b, st) + 16 * hc, v_lo);
-        tmem_ld16(tb + lane_base + L_::uc(b, st) + 32 + 16 * hc, v_hi);
+        uint32_t v[16], pk[8];
+        const uint32_t col = L_::uc(b, st) + 16 * pt;
+        tmem_ld16(tb + lane_base + col, v);
         tmem_ld_wait(v);
         const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
 #pragma unroll
-        for (int p2 = 0; p2 < 2; ++p2) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            float x0 = __uint_as_float(v[16 * p2 + 2 * t]), x1 = __uint_as_float(v[16 * p2 + 2 * t + 1]);
-            if (with_u0) {
-              x0 += u0v[16 * p2 + 2 * t];
-              x1 += u0v[16 * p2 + 2 * t + 1];
-            }
-            pk[t] = pack_bf16(x0, x1);
+        for (int t = 0; t < 8; ++t) {
+          float x0 = __uint_as_float(v[2 * t]), x1 = __uint_as_float(v[2 * t + 1]);
+          if (with_u0) {
+            x0 += u0v[2 * t];
+            x1 += u0v[2 * t + 1];
           }
-          tmem_st8(tb + lane_base + L_::uc(b, st) + 32 * p2 + 16 * hc, pk);
-          if (NB == 1 && p2 == 0) {
-            // the first K half of the single block is in place: MMA-2's first half may go
-            tmem_st_wait();
-            tc_fence_before();
-            group_sync(kConvBar, kWalkConvThreads);
-            if (tid == 0) mbar_arrive(bar_yready);
-          }
+          pk[t] = pack_bf16(x0, x1);
         }
+        tmem_st8(tb + lane_base + col, pk);
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0) {
-        if (NB > 1) mbar_arrive(bar_yready);
-        mbar_arrive(bar_yready + 1);
-      }
+      group_sync(half_bar, 256);
+      if (half_lead) mbar_arrive(bar_yready + kh);
       // ---- while MMA-2(n) runs: the previous chunk's outputs
       if (PC && n > 0) {
         const bool staged = emit_out(n - 1);
@@ -1197,49 +1167,36 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         break;
       }
       tc_fence_after();
-      // ---- bf16 S^T operand for MMA-1(n + 1), K half 0 (state rows 0..63) from every
-      //      warp first, then K half 1; then the next chunk's decay on the fp32 state
-      uint32_t v0[32], v1[32];
-      if (NB == 1) {
-        // both halves' loads in flight before the first wait
-        tmem_ld32(tb + lane_base + L_::st(0) + 32 * hc, v0);
-        tmem_ld32(tb + lane_base + L_::st(0) + 64 + 32 * hc, v1);
-        tmem_ld_wait(v0);
-        tmem_ld_wait(v1);
-        pack_half(0, 0, v0);
-      } else {
+      // ---- bf16 S^T operand for MMA-1(n + 1) (each half released when packed), then the
+      //      next chunk's decay on the fp32 state
+      uint32_t v[32];
 #pragma unroll 1
-        for (int b = 0; b < NB; ++b) {
-          tmem_ld32(tb + lane_base + L_::st(b) + 32 * hc, v0);
-          tmem_ld_wait(v0);
-          pack_half(b, 0, v0);
-        }
+      for (int b = 0; b < NB; ++b) {
+        tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+        tmem_ld_wait(v);
+        pack_state(b, v);
       }
       tmem_st_wait();
       tc_fence_before();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready);
-      if (NB == 1) {
-        pack_half(0, 1, v1);
-      } else {
-#pragma unroll 1
-        for (int b = 0; b < NB; ++b) {
-          tmem_ld32(tb + lane_base + L_::st(b) + 64 + 32 * hc, v1);
-          tmem_ld_wait(v1);
-          pack_half(b, 1, v1);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0 && n + 1 < n_chunks) mbar_arrive(bar_sready + 1);
-      if (PC && SNAP) store_snapshot(n, v0, v1);  // while MMA-1(n + 1) runs
+      group_sync(half_bar, 256);
+      if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + kh);
+      if (PC && SNAP) store_snapshot(n, v);  // while MMA-1(n + 1) runs
       if (n + 1 < n_chunks) {
         if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
           failed = true;
           break;
         }
-        rescale_all(st ^ 1, v0, v1);
+        if (NB == 1) {
+          rescale(0, st ^ 1, v);
+        } else {
+#pragma unroll 1
+          for (int b = 0; b < NB; ++b) {
+            tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+            tmem_ld_wait(v);
+            rescale(b, st ^ 1, v);
+          }
+        }
+        tmem_st_wait();
       }
       if (tid == 0 && pend_store) {
         bulk_wait_read();  // the staging tile may be rewritten after the barrier below
@@ -1274,13 +1231,11 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
           dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
         }
         if (dst == nullptr) continue;
-        for (int c = 64 * hc; c < 64 * hc + 64; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + lane_base + L_::st(b) + c, v);
-          tmem_ld_wait(v);
+        uint32_t v[32];
+        tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+        tmem_ld_wait(v);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(c + t) * D + row] = __uint_as_float(v[t]);
-        }
+        for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(32 * pt + t) * D + row] = __uint_as_float(v[t]);
       }
     }
   }
