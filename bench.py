@@ -342,11 +342,13 @@ def bench_ours(args, world, rank, local):
                 "roofline": {"bound": "alu", "achieved": round(b_tf, 2), "peak": fp32_peak,
                              "unit": "TFLOP/s", "frac": round(b_tf / fp32_peak, 4),
                              "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
-                             "flops_per_call": b_flops, "traffic": None},
+                             "flops_per_call": b_flops,
+                             "traffic": measured_traffic("backward_bf16_h32_t8192_d128"),
+                             "traffic_scope": "the bwd_simt_kernel launch of one call"},
                 "gpu_launches": bsteps * (kda_launches_per_step(kda, shape) + 5)}
     del bws, grads, x, ws, out, fin
     torch.cuda.empty_cache()
-    # ---- the other two prefill workloads north of the 8K one: one long sequence, and
+    # ---- the other two prefill workloads beside the 8K one: one long sequence, and
     #      packed variable-length sequences (device-resident inputs, CUDA events)
     others = {}
     for name, reps in (("bf16_h16_t1m_d128", 3), ("varlen8_h32_d128", 5)):

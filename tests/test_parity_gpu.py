@@ -114,6 +114,24 @@ def test_decay_clamp_active(kda):
     _check_full(kda, x, torch.bfloat16, "clamp active")
 
 
+def test_correlated_keys_large_inverse_blocks(kda):
+    """Keys that share a common direction (pairwise cosine ~0.6) and a weak decay make the
+    strictly lower A = Diag(beta) (K~ K^^T) dense and large, so (I + A)^{-1} has large
+    off-diagonal blocks: the blocked inverse (32x32 diagonal blocks, tensor-core merge of the
+    off-diagonal block) must keep its accuracy where it matters most."""
+    x = make_inputs(None, H=4, dk=128, dv=128, dtype=torch.float32, seed=19,
+                    lengths=[192, 77], state_std=0.02)
+    gen = torch.Generator().manual_seed(20)
+    base = torch.randn(1, 4, 128, generator=gen)
+    k = base + 0.8 * torch.randn(x.k.shape, generator=gen)
+    x.k = (k / k.norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    x.q = x.q.to(torch.bfloat16)
+    x.v = x.v.to(torch.bfloat16)
+    x.g = (-0.05 * torch.sigmoid(torch.randn(x.g.shape, generator=gen))).to(torch.bfloat16)
+    x.beta = torch.sigmoid(torch.randn(x.beta.shape, generator=gen) + 1.0).to(torch.bfloat16)
+    _check_full(kda, x, torch.bfloat16, "correlated keys")
+
+
 def test_resume_split_and_alias(kda):
     """Prefill [0,T) == prefill [0,m) then [m,T) from its final state, in place."""
     x = make_inputs(333, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=13, state_std=0.02)
