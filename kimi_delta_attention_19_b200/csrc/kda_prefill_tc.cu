@@ -54,7 +54,7 @@ constexpr uint32_t K8 = 8192, K16 = 16384, K32 = 32768;
 //   kbt: [128][64] Kb^T  (row i, column s)
 //   p:   [64][64]  P     (row r, column s)
 //   gl:  [128]     fp32
-// Each row is written whole by one thread (16-byte stores) and read by TMA.
+// Written by TMA stores from 128-byte-swizzled staging tiles, read by TMA.
 constexpr size_t kTileBig = size_t(C) * D * 2;
 constexpr size_t kTilePt = size_t(C) * C * 2;
 constexpr size_t kTileGl = size_t(D) * 4;
@@ -211,21 +211,29 @@ __device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity,
 // ------------------------------------------------------------------ intra-chunk kernel
 // One CTA of 8 warps per (chunk slot, head); two CTAs per SM. Everything of a chunk
 // that does not depend on the state: decay tiles, the Gram products on the tensor
-// cores, T = (I + A)^{-1} Diag(beta) by blocked forward substitution (16x16 diagonal
-// blocks on the CUDA cores, the off-diagonal merges as tensor-core products), and the
-// WY factors W = T K~, U0 = T V on the tensor cores.
+// cores, the two 32x32 diagonal blocks of (I + A)^{-1} on the CUDA cores, and the WY
+// factors W = T K~, U0 = T V on the tensor cores, blocked on the two token halves so
+// that the off-diagonal block of the inverse is never formed.
 constexpr int kIntraThreads = 256;
+constexpr int kPStoreThread = 192;  // warp 6, lane 0: issues (and waits for) the P store
 struct IntraSm {
   // Raw inputs as loaded by TMA; each region is reused once its contents are read.
   static constexpr uint32_t SV = 0;        // V, swizzled: [64 s][64 j] boxes (U0's A operand)
   static constexpr uint32_t KQ = K16;      // [K~ a0 | Q~ a0 | K~ a1 | Q~ a1], 8 KB each
   static constexpr uint32_t SK = 3 * K16;  // raw k, then K^, then T
-  static constexpr uint32_t SG = 4 * K16;  // raw g, then the N_d / N1 tile pair (hi, lo)
-  static constexpr uint32_t SQ = 5 * K16;  // raw q, then the Y / Z tile pair (hi, lo)
-  static constexpr uint32_t KH = SK, T = SK, NB = SG, YB = SQ;
+  static constexpr uint32_t SG = 4 * K16;  // raw g, then the inverse's fp32 scratch
+  static constexpr uint32_t SQ = 5 * K16;
+  static constexpr uint32_t KH = SK, T = SK;
   // 128-byte-swizzled staging tiles of the TMA stores to the workspace: Q~^T and Kb^T
-  // (phase 2, over the raw g and q), P (phase 4, after K^), -W^T and U0^T (phase 8)
+  // (phase 2, over the raw g and q), P (phase 4, after K^), -W^T and U0^T (phases 8-9;
+  // their token columns 0..31 are also the A operands of the second WY product)
   static constexpr uint32_t QTS = SG, KBS = SQ, PS = SK + K8, WTS = SG, U0S = SQ;
+  // phase 4 scratch (fp32, free until the staging of -W^T and U0^T): the diagonal
+  // blocks' rows of A and the solves' transposition (rows of 36 floats), A_21 (rows of
+  // 32 floats)
+  static constexpr uint32_t NLO = SG, A22 = SG + 4608, NHT = SG + 9216, A21 = SQ;
+  // G = N_hi A_21 and -G, bf16 B operands of the second WY product, over the dead Q~ half
+  static constexpr uint32_t GP = KQ + K8, GN = KQ + K8 + 4096;
   // float[2][64]: 1/|k row|, 1/|q row| (prologue)
   static constexpr uint32_t RN = SQ + K16;
   static constexpr uint32_t TOT = RN + 512;       // float[4][128] partial decay sums
@@ -233,11 +241,8 @@ struct IntraSm {
   static constexpr uint32_t BARS = BET + 256;
   static constexpr uint32_t TPTR = BARS + 64;
   static constexpr uint32_t BYTES = TPTR + 16;
-  // tensor-memory columns: [K~;Q~] K^^T (G), W^T, U0^T; while T is formed: the A
-  // operands A_off and N_d / N1 (hi | lo, 32 columns each) over W and U, and the
-  // merge products over the free columns and G
+  // tensor-memory columns: [K~;Q~] K^^T (G), W^T, U0^T
   static constexpr uint32_t G = 0, W = 64, U = 128, COLS = 256;
-  static constexpr uint32_t AOP = 64, NOP = 128, DA = 192, DB = 0;
 };
 static_assert(2 * (IntraSm::BYTES + 1024 + 1024) <= 233472, "two intra-chunk CTAs per SM");
 
@@ -503,111 +508,92 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
     mma_done = 1;
     tc_fence_after();
-    // ---- 4-6. T = (I + A)^{-1} Diag(beta) by blocked forward substitution with two
-    //   32x32 diagonal blocks: N = [[N_lo, 0], [N_21, N_hi]], N_21 = -N_hi A_21 N_lo.
+    // ---- 4-6. T = (I + A)^{-1} Diag(beta), blocked on the two 32-token halves:
+    //   (I + A)^{-1} = [[N_lo, 0], [N_21, N_hi]], N_bb = (I + A_bb)^{-1},
+    //   N_21 = -N_hi A_21 N_lo. For X = T B (B = K~ or V: the WY factors W, U0) that is
+    //     X_lo = T_lo B_lo,   X_hi = T_hi B_hi - G X_lo,   G = N_hi A_21,
+    //   T_bb = N_bb Diag(beta_b): one product with the block-diagonal T, then a short
+    //   one that subtracts G X_lo from the upper half (N_21 is never formed).
     //   Rows r < 64 of the Gram accumulator (tensor-memory lanes 0..63) hold K~_r K^^T:
     //   warps 0, 1, 4, 5 take one row each and a half hh of its 64 columns, so the
-    //   diagonal block of rows 0..31 is in the half of warp 0 and that of rows 32..63 in
-    //   the half of warp 5 (the "owners", one block per warp, a row per lane). Warps 2, 3,
-    //   6, 7 write P from lanes 64..127.
-    //   Diagonal blocks on the CUDA cores: N_bb = (I + A_bb)^{-1} in fp32 (a column per
-    //   lane, rows of A broadcast from shared memory).
-    //   The off-diagonal block on the tensor cores, two products at fp32 accuracy through
-    //   a bf16 split of both factors (x = hi + lo, the lo x lo term dropped), the left
-    //   factor an A operand in tensor memory, the right one a row-major (MN-major) tile:
-    //     R1: Z = A_21 N_lo (A restricted to rows 32..63 / columns 0..31: K steps 0, 1)
-    //     R2: D = N_d Z     (Z nonzero in rows 32..63: K steps 2, 3), N_21 = -D
-    //   and T = (N_d - D) Diag(beta), the WY products' bf16 operand. Rows 64..127 of
-    //   every product (lanes the left factor does not fill) are never read.
+    //   diagonal block of rows 0..31 is in the half of warp 0, that of rows 32..63 in the
+    //   half of warp 5, and A_21 in warp 1's. Warps 2, 3, 6, 7 write P from lanes 64..127.
+    //   Forward substitution on the CUDA cores, a right-hand-side column per lane, rows
+    //   of the block broadcast from shared memory: warp 0 solves (I + A_11) N_lo = I,
+    //   warp 5 (I + A_22) N_hi = I and, beside it, warp 6 (I + A_22) G = A_21 (so G costs
+    //   no extra step on the chain; the three solvers sit on three different SM
+    //   sub-partitions, warp % 4).
     const bool rowt = (warp & 3) < 2;                       // rows r < 64 of A
     const int hh = warp >> 2;                               // column half 32 hh ..
     const int rr = (warp & 3) * 32 + lane;                  // row (when rowt)
-    const bool owner = rowt && hh == (warp & 3);            // warps 0 and 5
-    float nrow[32];                                         // owners: N_d row (block-local)
-    // this thread's 32 columns of a row-major 64x64 bf16 hi/lo tile pair (lo K8 after hi)
-    auto put_tile = [&](uint32_t tile_off, const float* f) {
+    // x = (I + A_bb)^{-1} rhs for this lane's column: x_r = rhs_r - sum_{s<r} A_rs x_s,
+    // row by row from broadcast float4 reads of the block's rows (entries s >= r are 0)
+    auto fsub = [&](const float* arows, auto rhs, float (&x)[32]) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t hi[4], lo[4];
+      for (int r = 0; r < 32; ++r) x[r] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split_bf16(f[8 * q + 2 * e], f[8 * q + 2 * e + 1], hi[e], lo[e]);
-        const uint32_t off = tile_off + sw128_chunk(rr, 4 * hh + q, K8);
-        *reinterpret_cast<uint4*>(sm + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sm + off + K8) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      for (int r = 0; r < 32; ++r) {
+        float acc[4] = {rhs(r), 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; 4 * q < r; ++q) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arows + r * 36 + 4 * q);
+          acc[0] = fmaf(-a4.x, x[4 * q], acc[0]);
+          acc[1] = fmaf(-a4.y, x[4 * q + 1], acc[1]);
+          acc[2] = fmaf(-a4.z, x[4 * q + 2], acc[2]);
+          acc[3] = fmaf(-a4.w, x[4 * q + 3], acc[3]);
+        }
+        x[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
       }
     };
-    // ... and as a tensor-memory A operand (K pairs per column: hi at col, lo at col + 32)
-    auto put_aop = [&](uint32_t col, const float* f) {
-      uint32_t hi[16], lo[16];
+    // this lane's row of A (in v) as a 36-float row of dst
+    float* const a22 = reinterpret_cast<float*>(sm + L_::A22);
+    float* const a21 = reinterpret_cast<float*>(sm + L_::A21);
+    auto put_rows = [&](float* dst, const uint32_t (&v)[32]) {
 #pragma unroll
-      for (int t = 0; t < 16; ++t) split_bf16(f[2 * t], f[2 * t + 1], hi[t], lo[t]);
-      tmem_st16(tb + lane_base + col + 16 * hh, hi);
-      tmem_st16(tb + lane_base + col + 32 + 16 * hh, lo);
-    };
-    // d = left right over the K steps in kmask, left = the A operand at aop (tensor
-    // memory), right = the tile pair at btile; then a commit on bar_mma
-    auto merge_mma = [&](uint32_t d, uint32_t aop, uint32_t btile, int kmask) {
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, 0, 1);
-      uint32_t acc = 0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (!(kmask >> k & 1)) continue;
-        const uint64_t bh = sdesc_sw128(sb + btile + k * 2048, K8, 1024);
-        const uint64_t bl = sdesc_sw128(sb + btile + K8 + k * 2048, K8, 1024);
-        umma_bf16_tmem_a(tb + d, tb + aop + 8 * k, bh, id, acc);
-        umma_bf16_tmem_a(tb + d, tb + aop + 8 * k, bl, id, 1);
-        umma_bf16_tmem_a(tb + d, tb + aop + 32 + 8 * k, bh, id, 1);
-        acc = 1;
-      }
-      umma_commit(bar_mma);
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(dst + lane * 36 + 4 * q) =
+            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
     };
     {
       uint32_t v[32];
       tmem_ld32(tb + lane_base + L_::G + 32 * hh, v);
       tmem_ld_wait(v);
       if (rowt) {
-        // A = Diag(beta) strict_lower(K~ K^^T); A_21 (rows 32..63, columns 0..31, held
-        // by warp 1) as an A operand; the owners keep their diagonal block's row in v
+        // A = Diag(beta) strict_lower(K~ K^^T), row rr, columns 32 hh ..
         const float br = bet[rr];
-        float f[32];
+        float f[32];  // this row of the block-diagonal T (zero off the blocks)
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
           const int c = 32 * hh + t;
-          const float a_rc = c < rr ? br * __uint_as_float(v[t]) : 0.f;
-          f[t] = (rr >= 32 && hh == 0) ? a_rc : 0.f;
-          v[t] = __float_as_uint(a_rc);
+          v[t] = __float_as_uint(c < rr ? br * __uint_as_float(v[t]) : 0.f);
+          f[t] = 0.f;
         }
-        put_aop(L_::AOP, f);
-        if (owner) {
-          // N_bb by forward substitution, a column per lane: the block's rows of A go to a
-          // per-warp fp32 scratch (rows of 36 floats) in the Y tile's region, free until
-          // R1; lane c forms column c of N_bb, x_r = [r == c] - sum_{s<r} A_rs x_s, row by
-          // row from broadcast float4 reads of A (entries s >= r are zero); the columns go
-          // back through the scratch so that lane l ends with row l of N_bb.
-          float* scr = reinterpret_cast<float*>(sm + L_::YB) + (warp == 0 ? 0 : 32 * 36);
+        if (warp == 1) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(scr + lane * 36 + 4 * q) =
+            *reinterpret_cast<float4*>(a21 + lane * 32 + 4 * q) =
                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-          __syncwarp();
-          float x[32];
-#pragma unroll
-          for (int r = 0; r < 32; ++r) x[r] = 0.f;
-#pragma unroll
-          for (int r = 0; r < 32; ++r) {
-            float acc[4] = {r == lane ? 1.f : 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int q = 0; 4 * q < r; ++q) {
-              const float4 a4 = *reinterpret_cast<const float4*>(scr + r * 36 + 4 * q);
-              acc[0] = fmaf(-a4.x, x[4 * q], acc[0]);
-              acc[1] = fmaf(-a4.y, x[4 * q + 1], acc[1]);
-              acc[2] = fmaf(-a4.z, x[4 * q + 2], acc[2]);
-              acc[3] = fmaf(-a4.w, x[4 * q + 3], acc[3]);
-            }
-            x[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          group_sync(1, 96);  // warps 1, 5, 6: A_21 and A_22's rows are in place
+        } else if (warp == 4) {
+          // the upper-right block of T is zero
+        } else {
+          // warps 0 and 5: N_bb column `lane`, back through a transposition scratch so
+          // that lane l ends with row l of N_bb; T_bb = N_bb Diag(beta_b)
+          float* const scr = reinterpret_cast<float*>(sm + (warp == 0 ? L_::NLO : L_::NHT));
+          const float* arows;
+          if (warp == 0) {
+            put_rows(scr, v);
+            __syncwarp();
+            arows = scr;
+          } else {
+            put_rows(a22, v);
+            group_sync(1, 96);
+            arows = a22;
           }
+          float x[32];
+          fsub(arows, [&](int r) { return r == lane ? 1.f : 0.f; }, x);
           __syncwarp();
 #pragma unroll
           for (int r = 0; r < 32; ++r) scr[r * 36 + lane] = x[r];
@@ -615,17 +601,14 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const float4 n4 = *reinterpret_cast<const float4*>(scr + lane * 36 + 4 * q);
-            nrow[4 * q] = n4.x;
-            nrow[4 * q + 1] = n4.y;
-            nrow[4 * q + 2] = n4.z;
-            nrow[4 * q + 3] = n4.w;
-          }
-        } else {
+            const float nq[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-          for (int c = 0; c < 32; ++c) nrow[c] = 0.f;
+            for (int e = 0; e < 4; ++e) f[4 * q + e] = nq[e] * bet[32 * hh + 4 * q + e];
+          }
         }
-        put_tile(L_::NB, nrow);
-        put_aop(L_::NOP, nrow);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(rr, 4 * hh + q, K8)) = pack8(f + 8 * q);
       } else {
         // P = lower_incl(Q~ K^^T): row r, columns 32 hh .. 32 hh + 31
         const int r = (warp & 3) * 32 + lane - 64;
@@ -635,63 +618,34 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8)
           *reinterpret_cast<uint4*>(sm + L_::PS + sw128_chunk(r, 4 * hh + q8, 0)) = pack8(f + 8 * q8);
+        fence_async_smem();
+        group_sync(2, 128);  // warps 2, 3, 6, 7: P is staged
+        if (tid == kPStoreThread) {  // P to the workspace
+          tma_store_2d(&a.tm_p, sm + L_::PS, 0, static_cast<int>(tile * C));
+          bulk_commit();
+        }
+        if (warp == 6) {
+          // G = N_hi A_21, column `lane`, as +G and -G rows (bf16, K-major B operands)
+          group_sync(1, 96);
+          float y[32];
+          fsub(a22, [&](int r) { return a21[r * 32 + lane]; }, y);
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            const uint32_t off = sw128_chunk(r, lane >> 3, 0) + (lane & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(sm + L_::GP + off) = __float2bfloat16_rn(y[r]);
+            *reinterpret_cast<__nv_bfloat16*>(sm + L_::GN + off) = __float2bfloat16_rn(-y[r]);
+          }
+        }
       }
     }
-    tmem_st_wait();
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (tid == 32) {  // P to the workspace
-      tma_store_2d(&a.tm_p, sm + L_::PS, 0, static_cast<int>(tile * C));
-      bulk_commit();
-    }
-    // R1: Z = A_21 N_lo (K steps 0, 1)
-    if (tid == 0) merge_mma(L_::DA, L_::AOP, L_::NB, 0x3);
-    mma_issued = 2;
-    if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
-    mma_done = 2;
-    tc_fence_after();
-    if (rowt) {
-      uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::DA + 32 * hh, v);
-      tmem_ld_wait(v);
-      float f[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) f[t] = rr >= 32 && hh == 0 ? __uint_as_float(v[t]) : 0.f;
-      put_tile(L_::YB, f);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // R2: D = N_d Z (K steps 2, 3)
-    if (tid == 0) merge_mma(L_::DB, L_::NOP, L_::YB, 0xC);
-    mma_issued = 3;
-    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
-    mma_done = 3;
-    tc_fence_after();
-    // T = (N_d - D) Diag(beta), lower triangle, bf16 rows of the WY products' operand
-    if (rowt) {
-      uint32_t d4[32];
-      tmem_ld32(tb + lane_base + L_::DB + 32 * hh, d4);
-      tmem_ld_wait(d4);
-      float f[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const int c = 32 * hh + t;
-        const float nrc = nrow[t] - __uint_as_float(d4[t]);
-        f[t] = c <= rr ? nrc * bet[c] : 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(rr, 4 * hh + q, K8)) = pack8(f + 8 * q);
-    }
-    tc_fence_before();
-    fence_async_smem();
-    if (cta_wait_failed(bar_v, 0)) { failed = true; break; }  // also the barrier for T
+    if (cta_wait_failed(bar_v, 0)) { failed = true; break; }  // also the barrier for T, P, +-G
     v_done = true;
-    // ---- 7. W^T = K~^T T^T and U0^T = V^T T^T. K~ (in the Gram operand) and V (as
-    //         loaded) serve as MN-major A operands: 64-element column groups LBO apart,
-    //         8-row groups 1024 bytes apart, 16 rows of K per instruction.
+    // ---- 7. W^T = K~^T T^T and U0^T = V^T T^T with the block-diagonal T: the lower token
+    //         half is final, the upper one still lacks -G X_lo. K~ (in the Gram operand)
+    //         and V (as loaded) serve as MN-major A operands: 64-element column groups LBO
+    //         apart, 8-row groups 1024 bytes apart, 16 rows of K per instruction.
     if (tid == 0) {
       tc_fence_after();
       const uint32_t iw = idesc_bf16(128, 64, 1, 0);
@@ -703,28 +657,57 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       umma_commit(bar_mma);
     }
-    mma_issued = 4;
+    mma_issued = 2;
     if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
-    mma_done = 4;
+    mma_done = 2;
     tc_fence_after();
-    // ---- 8. -W^T and U0^T to the workspace through staging tiles (the merge tiles are
-    //         dead): tensor-memory lane i holds row i of both
+    // ---- 8. token columns 0..31 of -W^T (warps 0..3) and U0^T (warps 4..7) to the staging
+    //         tiles: tensor-memory lane i holds row i
+    const int i = (warp & 3) * 32 + lane;
+    const uint32_t xcol = hh ? L_::U : L_::W;
+    const uint32_t xst = hh ? L_::U0S : L_::WTS;
+    const uint32_t xsign = hh ? 0u : 0x80000000u;
     {
-      const int i = (warp & 3) * 32 + lane, cb = (warp >> 2) * 32;
       uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::W + cb, v);
+      tmem_ld32(tb + lane_base + xcol, v);
       tmem_ld_wait(v);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] ^= 0x80000000u;  // -W
+      for (int t = 0; t < 32; ++t) v[t] ^= xsign;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(sm + L_::WTS + sw128_chunk(i, (cb >> 3) + q, 0)) =
+        *reinterpret_cast<uint4*>(sm + xst + sw128_chunk(i, q, 0)) =
             pack8(reinterpret_cast<const float*>(v) + 8 * q);
-      tmem_ld32(tb + lane_base + L_::U + cb, v);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- 9. the upper token half: W_hi^T += (-W_lo^T) G^T, U0_hi^T += U0_lo^T (-G)^T,
+    //         the staged lower halves as K-major A operands (K = 32 tokens)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ib = idesc_bf16(128, 32, 0, 0);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        umma_bf16(tb + L_::W + 32, sdesc_sw128(sb + L_::WTS + k * 32, 16, 1024),
+                  sdesc_sw128(sb + L_::GP + k * 32, 16, 1024), ib, 1);
+        umma_bf16(tb + L_::U + 32, sdesc_sw128(sb + L_::U0S + k * 32, 16, 1024),
+                  sdesc_sw128(sb + L_::GN + k * 32, 16, 1024), ib, 1);
+      }
+      umma_commit(bar_mma);
+    }
+    mma_issued = 3;
+    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
+    mma_done = 3;
+    tc_fence_after();
+    {
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + xcol + 32, v);
       tmem_ld_wait(v);
 #pragma unroll
+      for (int t = 0; t < 32; ++t) v[t] ^= xsign;
+#pragma unroll
       for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(sm + L_::U0S + sw128_chunk(i, (cb >> 3) + q, 0)) =
+        *reinterpret_cast<uint4*>(sm + xst + sw128_chunk(i, 4 + q, 0)) =
             pack8(reinterpret_cast<const float*>(v) + 8 * q);
     }
     fence_async_smem();
@@ -735,7 +718,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       bulk_commit();
     }
   } while (0);
-  if (tid == 32) bulk_wait_all();  // the workspace stores complete before the CTA exits
+  // the workspace stores have read their staging tiles before the CTA's shared memory is
+  // released (their writes are visible to the next kernel once this grid completes)
+  if (tid == 32 || tid == kPStoreThread) bulk_wait_read();
   if (failed && tid == 0) {
     atomicExch(a.seq.status, kDevWaitTimeout);
     // copies and products in flight finish before the CTA releases its memory
@@ -1213,7 +1198,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       group_sync(kConvBar, kWalkConvThreads);
       if (tid == 0 && staged) store_out(n_chunks - 1);
     }
-    if (PC && tid == 0) bulk_wait_all();  // outputs written before the kernel ends
+    if (PC && tid == 0) bulk_wait_read();  // the output stores have read the staging tile
     if (failed) {
       if (tid == 0) atomicExch(a.seq.status, kDevWaitTimeout);
     } else {

@@ -129,6 +129,25 @@ def make_inputs(T: int | None = None, H: int = 2, dk: int = 64, dv: int = 64, *,
     return Inputs(q, k, v, g, beta, s0, cu, list(lengths))
 
 
+def correlated_key_inputs(*, seed: int = 19, H: int = 4, lengths: list[int] | None = None,
+                          noise: float = 0.8, g_scale: float = 0.05) -> Inputs:
+    """bf16 inputs whose keys share one direction per head (unit rows of base + noise * N(0, 1):
+    pairwise cosine ~0.6 at noise 0.8) with a weak decay (g = -g_scale * sigmoid(N(0, 1))) and
+    beta = sigmoid(N(1, 1)): an ill-conditioned (I + A) with large off-diagonal inverse blocks.
+    d_k = d_v = 128; q, v and the initial state as in make_inputs."""
+    x = make_inputs(None, H=H, dk=128, dv=128, dtype=torch.float32, seed=seed,
+                    lengths=lengths or [192, 77], state_std=0.02)
+    gen = torch.Generator().manual_seed(seed + 1)
+    base = torch.randn(1, H, 128, generator=gen)
+    k = base + noise * torch.randn(x.k.shape, generator=gen)
+    x.k = _l2n(k).to(torch.bfloat16)
+    x.q = x.q.to(torch.bfloat16)
+    x.v = x.v.to(torch.bfloat16)
+    x.g = (-g_scale * torch.sigmoid(torch.randn(x.g.shape, generator=gen))).to(torch.bfloat16)
+    x.beta = torch.sigmoid(torch.randn(x.beta.shape, generator=gen) + 1.0).to(torch.bfloat16)
+    return x
+
+
 def workload_inputs(w: Workload, *, seed: int = 0, device: str = "cpu") -> Inputs:
     """Inputs for a named prefill workload (decode draws per step, see decode_token)."""
     if w.n_varlen:

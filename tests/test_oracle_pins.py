@@ -105,3 +105,34 @@ def test_pins_catch_planted_mistakes(tmp_path):
         if not caught:
             survivors.append(name)
     assert not survivors, f"pins missed planted mistakes: {survivors}"
+
+
+def test_correlated_key_bound_catches_dropped_inverse_block(monkeypatch):
+    """The GPU bound on the correlated-key inputs (rel-L2 1e-2) separates a correct blocked
+    inverse from one that drops the off-diagonal block: the oracle's chunked form with that
+    mistake planted (A_21 ignored in the 64-token solve) lands far outside the bound, while
+    the unmodified chunked form agrees with the token-by-token recurrence."""
+    import numpy as np
+    from kimi_delta_attention_19_b200.inputs import correlated_key_inputs
+
+    x = correlated_key_inputs(seed=19)
+    cu = x.cu_seqlens.tolist()
+    args = (x.q, x.k, x.v, x.g, x.beta)
+    ro, rs = ko.recurrent(*args, cu_seqlens=cu, initial_state=x.initial_state, lb=-1.0)
+    ro, rs = np.asarray(ro, np.float64), np.asarray(rs, np.float64)
+
+    def rel(a, b):
+        return float(np.linalg.norm(np.asarray(a) - b) / np.linalg.norm(b))
+
+    co, cs = ko.chunked(*args, chunk=64, cu_seqlens=cu, initial_state=x.initial_state, lb=-1.0)
+    assert rel(co, ro) < 1e-9 and rel(cs, rs) < 1e-9
+    solve = ko._forward_substitution
+
+    def without_off_diagonal(L, B):
+        L2 = L.copy()
+        L2[32:, :32] = 0.0
+        return solve(L2, B)
+
+    monkeypatch.setattr(ko, "_forward_substitution", without_off_diagonal)
+    bo, bs = ko.chunked(*args, chunk=64, cu_seqlens=cu, initial_state=x.initial_state, lb=-1.0)
+    assert rel(bo, ro) > 5e-2 and rel(bs, rs) > 5e-2, (rel(bo, ro), rel(bs, rs))
