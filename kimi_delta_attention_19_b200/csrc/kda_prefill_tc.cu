@@ -133,7 +133,6 @@ struct IntraArgs {
 struct WalkArgs {
   CUtensorMap tm_wt, tm_qt, tm_u0, tm_kbt;  // [tiles*128][64] bf16, 128x64 boxes, 128-byte swizzle
   CUtensorMap tm_p;                         // [tiles*64][64], 64x64 boxes
-  CUtensorMap tm_o;                         // out [T_total][H*128], 64x64 boxes, no swizzle
   SeqTable seq;
   const float* gl;
   __nv_bfloat16* out;
@@ -745,7 +744,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 //               They rescale the fp32 state, add U0 and pack U^T and S^T into bf16 MMA
 //               operands kept in tensor memory, and write the outputs;
 //   warp 16     issues the MMAs (one thread);
-//   warp 17     streams each chunk's workspace tiles into two stages by TMA (one thread).
+//   warp 17     streams each chunk's workspace tiles into three stages by TMA (one thread).
 // Hand-offs are mbarriers: full/empty per stage, m1/m2 (MMA groups done), and per K half
 // s_ready/y_ready (that half of the bf16 S^T or U^T operand is in tensor memory), so the
 // first half of a product starts while the second half is still being packed.
@@ -767,10 +766,9 @@ struct WalkSm {
   static constexpr uint32_t U0 = PC ? K32 : K16;
   static constexpr uint32_t PK = U0 + K16;
   static constexpr uint32_t STAGE = PK + (PC ? K16 + K8 : K16);
-  static constexpr uint32_t STAGE_TX = STAGE + 512;  // + gl
-  static constexpr uint32_t OS = 2 * STAGE;            // output staging: two [64 r][64 j] boxes
-  static constexpr uint32_t GL = OS + (PC ? K16 : 0);  // float[2][128]
-  static constexpr uint32_t BARS = GL + 1024;
+  static constexpr int NSTAGE = 3;  // chunk n in stage n % 3: two chunks' loads in flight
+  static constexpr uint32_t GL = NSTAGE * STAGE;  // float[3][128]: each stage's gl, own barrier
+  static constexpr uint32_t BARS = GL + NSTAGE * 512;
   static constexpr uint32_t TPTR = BARS + 128;
   static constexpr uint32_t BYTES = TPTR + 16;
   // Tensor-memory columns. Output walk, by chunk parity p: p = 0: [U | O] at 0..127,
@@ -822,12 +820,14 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 
   float* gls = reinterpret_cast<float*>(sm + L_::GL);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_::BARS);
-  uint64_t* bar_full = bars;       // two stages
-  uint64_t* bar_empty = bars + 2;  // two stages
-  uint64_t* bar_m1 = bars + 4;
-  uint64_t* bar_m2 = bars + 5;
-  uint64_t* bar_sready = bars + 6;  // two column halves
-  uint64_t* bar_yready = bars + 8;  // two column halves
+  constexpr int NS = L_::NSTAGE;
+  uint64_t* bar_full = bars;        // per stage: the tiles have landed
+  uint64_t* bar_empty = bars + NS;  // per stage: the products have read it
+  uint64_t* bar_gl = bars + 2 * NS; // per stage: the stage's gl has landed
+  uint64_t* bar_m1 = bars + 3 * NS;
+  uint64_t* bar_m2 = bars + 3 * NS + 1;
+  uint64_t* bar_sready = bars + 3 * NS + 2;  // two column halves
+  uint64_t* bar_yready = bars + 3 * NS + 4;  // two column halves
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
 
   if (warp == 0) {
@@ -835,7 +835,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 3 * NS + 6; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
   }
   tc_fence_before();
@@ -857,31 +857,35 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       int issued = 0;
       bool ok = true;
       for (int n = 0; n < n_chunks; ++n) {
-        const int st = n & 1;
-        if (n >= 2 && !(ok = mbar_wait(bar_empty + st, ((n - 2) >> 1) & 1))) break;
-        unsigned char* dst = sm + st * L_::STAGE;
+        const int st = n & 1, sg = n % NS;  // layout parity, stage
+        if (n >= NS && !(ok = mbar_wait(bar_empty + sg, ((n - NS) / NS) & 1))) break;
+        unsigned char* dst = sm + sg * L_::STAGE;
         const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
         const int y = static_cast<int>(tile * D);  // row of the [tiles * 128][64] arrays
-        mbar_arrive_expect_tx(bar_full + st, L_::STAGE_TX);
+        // gl first, on its own barrier: the conversion warps need only it to rescale
+        mbar_arrive_expect_tx(bar_gl + sg, 512);
+        bulk_load(gls + sg * D, a.gl + tile * D, 512, bar_gl + sg);
+        mbar_arrive_expect_tx(bar_full + sg, L_::STAGE);
         if (PC) {
           // even stages: [-W^T | Q~^T], [P | Kb^T]; odd stages: [Q~^T | -W^T], [Kb^T | P]
-          tma_load_2d(dst + L_::WQ + st * K16, &a.tm_wt, bar_full + st, 0, y);
-          tma_load_2d(dst + L_::WQ + (st ^ 1) * K16, &a.tm_qt, bar_full + st, 0, y);
-          tma_load_2d(dst + L_::PK + (st ? 0 : K8), &a.tm_kbt, bar_full + st, 0, y);
-          tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_p, bar_full + st, 0,
+          tma_load_2d(dst + L_::WQ + st * K16, &a.tm_wt, bar_full + sg, 0, y);
+          tma_load_2d(dst + L_::WQ + (st ^ 1) * K16, &a.tm_qt, bar_full + sg, 0, y);
+          tma_load_2d(dst + L_::PK + (st ? 0 : K8), &a.tm_kbt, bar_full + sg, 0, y);
+          tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_p, bar_full + sg, 0,
                       static_cast<int>(tile * C));
         } else {
-          tma_load_2d(dst + L_::WQ, &a.tm_wt, bar_full + st, 0, y);
-          tma_load_2d(dst + L_::PK, &a.tm_kbt, bar_full + st, 0, y);
+          tma_load_2d(dst + L_::WQ, &a.tm_wt, bar_full + sg, 0, y);
+          tma_load_2d(dst + L_::PK, &a.tm_kbt, bar_full + sg, 0, y);
         }
-        tma_load_2d(dst + L_::U0, &a.tm_u0, bar_full + st, 0, y);
-        bulk_load(gls + st * D, a.gl + tile * D, 512, bar_full + st);
+        tma_load_2d(dst + L_::U0, &a.tm_u0, bar_full + sg, 0, y);
         ++issued;
       }
       if (!ok) atomicExch(a.seq.status, kDevWaitTimeout);
       // the copies in flight land before the CTA can exit
-      for (int n = issued >= 2 ? issued - 2 : 0; n < issued; ++n)
-        mbar_wait(bar_full + (n & 1), (n >> 1) & 1, 400000000LL);
+      for (int n = issued >= NS ? issued - NS : 0; n < issued; ++n) {
+        mbar_wait(bar_gl + n % NS, (n / NS) & 1, 400000000LL);
+        mbar_wait(bar_full + n % NS, (n / NS) & 1, 400000000LL);
+      }
     }
   } else if (warp == kWalkMmaWarp) {
     // ============================================================ MMA issue
@@ -889,9 +893,9 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       int m_issued = 0;
       bool ok = true;
       for (int n = 0; n < n_chunks && ok; ++n) {
-        const int st = n & 1;
-        const uint32_t stg = sb + st * L_::STAGE;
-        if (!(ok = mbar_wait(bar_full + st, (n >> 1) & 1))) break;
+        const int st = n & 1, sg = n % NS;  // layout parity, stage
+        const uint32_t stg = sb + sg * L_::STAGE;
+        if (!(ok = mbar_wait(bar_full + sg, (n / NS) & 1))) break;
         // MMA-1: U^T = S^T (-W)^T and (output walk) (Q~ S)^T = S^T Q~^T, K = the 128 state
         // rows in two halves, each started once its half of S^T is packed; B MN-major: 16
         // rows of the stage tiles per K step
@@ -953,7 +957,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         }
         if (!ok) break;
         umma_commit(bar_m2);
-        umma_commit(bar_empty + st);
+        umma_commit(bar_empty + sg);
         ++m_issued;
       }
       if (!ok) {
@@ -978,9 +982,10 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     const int half_bar = kHalfBar0 + kh;     // named barrier of this half's 256 threads
     const bool half_lead = (warp & 7) == 0 && lane == 0;
     // S <- Diag(gl) S on this thread's 32 fp32 state rows of block b (held in v), written
-    // back to tensor memory: the decay of the chunk about to be walked
-    auto rescale = [&](int b, int st, uint32_t (&v)[32]) {
-      const float* gl = gls + st * D + 32 * pt;
+    // back to tensor memory: the decay of the chunk about to be walked. Not waited for
+    // here: the next U^T pack's store wait covers it, before MMA-2 accumulates onto it.
+    auto rescale = [&](int b, int sg, uint32_t (&v)[32]) {
+      const float* gl = gls + sg * D + 32 * pt;
 #pragma unroll
       for (int t4 = 0; t4 < 8; ++t4) {
         const float4 g = *reinterpret_cast<const float4*>(gl + 4 * t4);
@@ -998,7 +1003,25 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       for (int t = 0; t < 16; ++t) pk[t] = pack_bf16(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1]));
       tmem_st16(tb + lane_base + L_::sbf(b) + 16 * pt, pk);
     };
-    bool failed = false, pend_store = false;
+    bool failed = false;
+    // U0^T[j][r] of the next chunk for this thread's tokens r = 16 pt .. + 15 (16-byte
+    // chunks 2 pt, 2 pt + 1 of row j of the swizzled [128 j][64 r] tile of stage sg),
+    // read as soon as the stage has landed, a chunk before the U^T pack that adds it
+    float u0v[16];
+    auto load_u0 = [&](int sg) {
+      const unsigned char* u0r = sm + sg * L_::STAGE + L_::U0;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row, 2 * pt + q, 0));
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16(w[e]);
+          u0v[8 * q + 2 * e] = f.x;
+          u0v[8 * q + 2 * e + 1] = f.y;
+        }
+      }
+    };
     // initial state: fp32 into tensor memory, bf16 copy as the MMA operand; then the
     // first chunk's decay on the fp32 copy
     {
@@ -1027,7 +1050,8 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       group_sync(half_bar, 256);
       if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + kh);
       if (n_chunks > 0) {
-        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full, 0, KDA_FIRST_WAIT_LIMIT))) {
+        const bool ok = mbar_wait(bar_gl, 0, KDA_FIRST_WAIT_LIMIT) && mbar_wait(bar_full, 0);
+        if (group_any(kConvBar, kWalkConvThreads, !ok)) {
           failed = true;
         } else {
           if (NB == 1) {
@@ -1040,39 +1064,32 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
               rescale(b, 0, v);
             }
           }
-          tmem_st_wait();
+          load_u0(0);
         }
       }
     }
 
-    // O of chunk n (tensor-memory buffer yo(n & 1)) to global memory: full chunks
-    // through the staging tile and a TMA store, a ragged last chunk directly
+    // O of chunk n (tensor-memory buffer yo(n & 1)) straight to global memory: lane pairs
+    // (j, j + 1) trade values so that each lane writes two adjacent columns of one token
+    // (even lanes the tokens 16 pt + 2 t, odd lanes 16 pt + 2 t + 1); a sequence's ragged
+    // last chunk stops at its length (rows past it belong to the next sequence)
     auto emit_out = [&](int n) {
       const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
       const int L = (c_end - c0) < C ? static_cast<int>(c_end - c0) : C;
       uint32_t v[16];
       tmem_ld16(tb + lane_base + L_::yo(n & 1) + 16 * pt, v);
       tmem_ld_wait(v);
-      if (L == C) {
-        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(sm + L_::OS + (row >> 6) * K8) +
-                            16 * pt * 64 + (row & 63);
+      const int odd = lane & 1;
+      const int64_t ostride = static_cast<int64_t>(a.H) * D;
+      __nv_bfloat16* o = a.out + ((c0 + 16 * pt + odd) * a.H + h) * D + (row & ~1);
 #pragma unroll
-        for (int t = 0; t < 16; ++t) ob[t * 64] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
-      } else {
-        // a sequence's ragged last chunk: rows past L belong to the next sequence
-        __nv_bfloat16* o = a.out + ((c0 + 16 * pt) * a.H + h) * D + row;
-        const int64_t ostride = static_cast<int64_t>(a.H) * D;
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          if (16 * pt + t < L) o[t * ostride] = __float2bfloat16_rn(a.scale * __uint_as_float(v[t]));
+      for (int t = 0; t < 8; ++t) {
+        const float x0 = a.scale * __uint_as_float(v[2 * t]);
+        const float x1 = a.scale * __uint_as_float(v[2 * t + 1]);
+        const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
+        const uint32_t pr = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
+        if (16 * pt + 2 * t + odd < L) *reinterpret_cast<uint32_t*>(o + 2 * t * ostride) = pr;
       }
-      return L == C;
-    };
-    auto store_out = [&](int n) {  // thread 0, once the staging tile is visible
-      const int64_t c0 = c_begin + static_cast<int64_t>(n) * C;
-      tma_store_2d(&a.tm_o, sm + L_::OS, h * D, static_cast<int>(c0));
-      tma_store_2d(&a.tm_o, sm + L_::OS + K8, h * D + 64, static_cast<int>(c0));
-      bulk_commit();
     };
 
     // The fp32 state after chunk n (this thread's 32 state rows of column `row`, in v)
@@ -1086,28 +1103,11 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       for (int t = 0; t < 32; ++t) dst[t * D] = __uint_as_float(v[t]);
     };
 
-    // Per chunk n (stage st = n % 2 has landed): MMA-1(n) runs -> U^T (+ U0^T) packed ->
+    // Per chunk n (stage n % 3 has landed): MMA-1(n) runs -> U^T (+ U0^T) packed ->
     // MMA-2(n) runs while the previous chunk's outputs are written -> S^T packed for
     // MMA-1(n + 1), then the fp32 state rescaled by the next chunk's decay.
     for (int n = 0; n < n_chunks && !failed; ++n) {
       const int st = n & 1;
-      // U0^T[j][r] for this thread's tokens r = 16 pt .. + 15 (16-byte chunks 2 pt,
-      // 2 pt + 1 of row j of the swizzled [128 j][64 r] tile)
-      float u0v[16];
-      {
-        const unsigned char* u0r = sm + st * L_::STAGE + L_::U0;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const uint4 w4 = *reinterpret_cast<const uint4*>(u0r + sw128_chunk(row, 2 * pt + q, 0));
-          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16(w[e]);
-            u0v[8 * q + 2 * e] = f.x;
-            u0v[8 * q + 2 * e + 1] = f.y;
-          }
-        }
-      }
       if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_m1, n & 1))) {
         failed = true;
         break;
@@ -1138,22 +1138,22 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       group_sync(half_bar, 256);
       if (half_lead) mbar_arrive(bar_yready + kh);
       // ---- while MMA-2(n) runs: the previous chunk's outputs
-      if (PC && n > 0) {
-        const bool staged = emit_out(n - 1);
-        fence_async_smem();
-        group_sync(kConvBar, kWalkConvThreads);
-        if (tid == 0 && staged) {
-          store_out(n - 1);
-          pend_store = true;
+      if (PC && n > 0) emit_out(n - 1);
+      // MMA-2(n) done; the next chunk's gl and tiles (issued two chunks ahead) have landed
+      const bool more = n + 1 < n_chunks;
+      const int sg1 = (n + 1) % NS;
+      const uint32_t ph1 = ((n + 1) / NS) & 1;
+      {
+        bool ok = mbar_wait(bar_m2, n & 1);
+        if (more) ok = ok && mbar_wait(bar_gl + sg1, ph1) && mbar_wait(bar_full + sg1, ph1);
+        if (group_any(kConvBar, kWalkConvThreads, !ok)) {
+          failed = true;
+          break;
         }
-      }
-      if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_m2, n & 1))) {
-        failed = true;
-        break;
       }
       tc_fence_after();
       // ---- bf16 S^T operand for MMA-1(n + 1) (each half released when packed), then the
-      //      next chunk's decay on the fp32 state
+      //      next chunk's decay on the fp32 state and its U0^T, while MMA-1(n + 1) runs
       uint32_t v[32];
 #pragma unroll 1
       for (int b = 0; b < NB; ++b) {
@@ -1164,41 +1164,27 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       tmem_st_wait();
       tc_fence_before();
       group_sync(half_bar, 256);
-      if (half_lead && n + 1 < n_chunks) mbar_arrive(bar_sready + kh);
+      if (half_lead && more) mbar_arrive(bar_sready + kh);
       if (PC && SNAP) store_snapshot(n, v);  // while MMA-1(n + 1) runs
-      if (n + 1 < n_chunks) {
-        if (group_any(kConvBar, kWalkConvThreads, !mbar_wait(bar_full + (st ^ 1), ((n + 1) >> 1) & 1))) {
-          failed = true;
-          break;
-        }
+      if (more) {
         if (NB == 1) {
-          rescale(0, st ^ 1, v);
+          rescale(0, sg1, v);
         } else {
 #pragma unroll 1
           for (int b = 0; b < NB; ++b) {
             tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
             tmem_ld_wait(v);
-            rescale(b, st ^ 1, v);
+            rescale(b, sg1, v);
           }
         }
-        tmem_st_wait();
+        load_u0(sg1);
       }
-      if (tid == 0 && pend_store) {
-        bulk_wait_read();  // the staging tile may be rewritten after the barrier below
-        pend_store = false;
-      }
-      tc_fence_before();
-      group_sync(kConvBar, kWalkConvThreads);
     }
     if (PC && !failed && n_chunks > 0) {
-      // the last chunk's outputs
       tc_fence_after();
-      const bool staged = emit_out(n_chunks - 1);
-      fence_async_smem();
-      group_sync(kConvBar, kWalkConvThreads);
-      if (tid == 0 && staged) store_out(n_chunks - 1);
+      emit_out(n_chunks - 1);  // the last chunk's outputs
     }
-    if (PC && tid == 0) bulk_wait_read();  // the output stores have read the staging tile
+    tmem_st_wait();  // a decay store left in flight by a wait that ran out
     if (failed) {
       if (tid == 0) atomicExch(a.seq.status, kDevWaitTimeout);
     } else {
@@ -1561,8 +1547,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
       !make_map(&wa.tm_qt, qt, C, rows_big, C * 2, true, C, D) ||
       !make_map(&wa.tm_u0, u0, C, rows_big, C * 2, true, C, D) ||
       !make_map(&wa.tm_kbt, kbt, C, rows_big, C * 2, true, C, D) ||
-      !make_map(&wa.tm_p, pm, C, rows_p, C * 2, true) ||
-      !make_map(&wa.tm_o, pa.out, in_cols, pa.T_total, in_pitch, false))
+      !make_map(&wa.tm_p, pm, C, rows_p, C * 2, true))
     return cudaErrorInvalidValue;
   ia.seq = seq;
   ia.beta = static_cast<const __nv_bfloat16*>(pa.beta);
