@@ -898,11 +898,12 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         if (!(ok = mbar_wait(bar_full + sg, (n / NS) & 1))) break;
         // MMA-1: U^T = S^T (-W)^T and (output walk) (Q~ S)^T = S^T Q~^T, K = the 128 state
         // rows in two halves, each started once its half of S^T is packed; B MN-major: 16
-        // rows of the stage tiles per K step
-        // The U^T part (B = the -W^T tile) is committed on m1 by itself, so that the
-        // conversion warps pack it while the (Q~ S)^T part (output walk) still runs.
-        const uint32_t i_k = idesc_bf16(128, 64, 0, 1);
-        const uint32_t wt_off = PC ? st * K16 : 0;  // -W^T tile in the stage
+        // rows of the stage tiles per K step. The output walk takes both in one N = 128
+        // product (B = the stage's two 64-token tiles, 16 KB apart): an M = 128, K = 16
+        // tcgen05.mma costs about the same for N = 64 and N = 128, so one product per K step
+        // is half the tensor-pipe time of two.
+        const uint32_t i1 = idesc_bf16(128, PC ? 128 : 64, 0, 1);
+        const uint32_t d1 = PC ? (st ? L_::yo(1) : L_::uc(0, 0)) : 0;  // [U | O] or [O | U]
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!(ok = mbar_wait(bar_sready + half, n & 1))) break;
@@ -912,21 +913,13 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int k = 4 * half + kk;
-              umma_bf16_tmem_a(tb + L_::uc(b, st), tb + L_::sbf(b) + 8 * k,
-                               sdesc_sw128(stg + L_::WQ + wt_off + k * 2048, K16, 1024), i_k, k > 0);
+              umma_bf16_tmem_a(tb + (PC ? d1 : L_::uc(b, st)), tb + L_::sbf(b) + 8 * k,
+                               sdesc_sw128(stg + L_::WQ + k * 2048, K16, 1024), i1, k > 0);
             }
         }
         if (!ok) break;
         umma_commit(bar_m1);
         ++m_issued;
-        if (PC) {
-          // (Q~ S)^T into this chunk's O columns (B = the Q~^T tile); MMA-2 adds U^T P^T
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_bf16_tmem_a(tb + L_::yo(st), tb + L_::sbf(0) + 8 * k,
-                             sdesc_sw128(stg + L_::WQ + (K16 - wt_off) + k * 2048, K16, 1024), i_k,
-                             k > 0);
-        }
         // MMA-2: output walk: [O^T | S^T] (or [S^T | O^T]) += U^T [P^T | Kb] in one N = 192
         // product; summary walk: S^T += U^T Kb per block (B operands K-major: the stage's
         // rows of P and Kb^T, 16 tokens = 32 bytes per K step)
