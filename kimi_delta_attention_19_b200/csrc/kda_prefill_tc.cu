@@ -186,6 +186,23 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
   return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
                     pack_bf16(f[6], f[7]));
 }
+// Two fp32 values as one 64-bit register pair (first value in the low half), and the
+// packed fused multiply-add of sm_100 (two independent round-to-nearest fp32 FMAs).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f32x2_split(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 // Limit, in SM clocks, of the first wait on a kernel's inputs (the intra-chunk kernel's
 // TMA loads, the walks' first stage, the combine's first M and L). A test-only build of
 // the library sets it to a few clocks so that the wait runs out and each kernel's
@@ -526,22 +543,32 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     const int hh = warp >> 2;                               // column half 32 hh ..
     const int rr = (warp & 3) * 32 + lane;                  // row (when rowt)
     // x = (I + A_bb)^{-1} rhs for this lane's column: x_r = rhs_r - sum_{s<r} A_rs x_s,
-    // row by row from broadcast float4 reads of the block's rows (entries s >= r are 0)
+    // row by row from broadcast float4 reads of the block's rows (entries s >= r are 0).
+    // The sum runs in two packed fp32 pairs (fma.rn.f32x2: two independent fp32 FMAs per
+    // instruction), x held as pairs (x_2m, x_2m+1).
     auto fsub = [&](const float* arows, auto rhs, float (&x)[32]) {
+      uint64_t x2[16];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) x[r] = 0.f;
+      for (int m = 0; m < 16; ++m) x2[m] = 0ull;
 #pragma unroll
       for (int r = 0; r < 32; ++r) {
-        float acc[4] = {rhs(r), 0.f, 0.f, 0.f};
+        uint64_t s01 = 0ull, s23 = 0ull;
 #pragma unroll
         for (int q = 0; 4 * q < r; ++q) {
           const float4 a4 = *reinterpret_cast<const float4*>(arows + r * 36 + 4 * q);
-          acc[0] = fmaf(-a4.x, x[4 * q], acc[0]);
-          acc[1] = fmaf(-a4.y, x[4 * q + 1], acc[1]);
-          acc[2] = fmaf(-a4.z, x[4 * q + 2], acc[2]);
-          acc[3] = fmaf(-a4.w, x[4 * q + 3], acc[3]);
+          s01 = fma_f32x2(f32x2(a4.x, a4.y), x2[2 * q], s01);
+          s23 = fma_f32x2(f32x2(a4.z, a4.w), x2[2 * q + 1], s23);
         }
-        x[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const float2 p01 = f32x2_split(s01), p23 = f32x2_split(s23);
+        const float xr = rhs(r) - ((p01.x + p01.y) + (p23.x + p23.y));
+        const float2 old = f32x2_split(x2[r >> 1]);
+        x2[r >> 1] = (r & 1) ? f32x2(old.x, xr) : f32x2(xr, old.y);
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const float2 v2 = f32x2_split(x2[m]);
+        x[2 * m] = v2.x;
+        x[2 * m + 1] = v2.y;
       }
     };
     // this lane's row of A (in v) as a 36-float row of dst
