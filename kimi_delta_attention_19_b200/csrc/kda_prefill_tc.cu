@@ -198,6 +198,19 @@ __device__ __forceinline__ float2 f32x2_split(uint64_t v) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
   return r;
 }
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16 pair (lower half first) -> fp32 pair
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t u) {
+  return f32x2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(uint64_t v) {
+  const float2 f = f32x2_split(v);
+  return pack_bf16(f.x, f.y);
+}
 __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
@@ -372,10 +385,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     const int ch = 2 * p, bx = p >> 5;
     constexpr float kLog2e = 1.4426950408889634f;
     const float lb2 = a.lb * kLog2e;
+    // per-channel-pair arithmetic in packed fp32 pairs (mul.rn.f32x2: the same products)
     uint32_t kraw[16], qraw[16];
-    float E0[16], E1[16];
+    uint64_t E2[16];
     {
-      float pr0 = 1.f, pr1 = 1.f;
+      uint64_t pr = f32x2(1.f, 1.f);
       const uint32_t off0 = 16 * qr * 256 + 4 * p;  // raw rows are 256 bytes
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -390,12 +404,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
           gg.x = live ? gate_from_preact(gg.x, a.lb) : 0.f;
           gg.y = live ? gate_from_preact(gg.y, a.lb) : 0.f;
         }
-        E0[i] = ex2_approx(fmaxf(gg.x * kLog2e, lb2));
-        E1[i] = ex2_approx(fmaxf(gg.y * kLog2e, lb2));
-        pr0 *= E0[i];
-        pr1 *= E1[i];
+        const float2 gl2 = f32x2_split(mul_f32x2(f32x2(gg.x, gg.y), f32x2(kLog2e, kLog2e)));
+        E2[i] = f32x2(ex2_approx(fmaxf(gl2.x, lb2)), ex2_approx(fmaxf(gl2.y, lb2)));
+        pr = mul_f32x2(pr, E2[i]);
       }
-      *reinterpret_cast<float2*>(tot + qr * 128 + ch) = make_float2(pr0, pr1);
+      *reinterpret_cast<float2*>(tot + qr * 128 + ch) = f32x2_split(pr);
     }
     if (tid < C) bet[tid] = beta_r;
     __syncthreads();  // every raw read is done: SK, SG and SQ may be overwritten
@@ -410,52 +423,49 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     //         Rows 16 qr + i: the swizzle term depends on i % 8 only.
     {
       uint32_t qt0[8], qt1[8], kb0[8], kb1[8];  // bf16 pairs along the token index
-      float2 tq[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tq[q] = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
-      float pre0 = 1.f, pre1 = 1.f, suf0 = 1.f, suf1 = 1.f;
+      uint64_t tq[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        if (q < qr) {
-          pre0 *= tq[q].x;
-          pre1 *= tq[q].y;
-        } else if (q > qr) {
-          suf0 *= tq[q].x;
-          suf1 *= tq[q].y;
-        }
+        const float2 t2 = *reinterpret_cast<const float2*>(tot + q * 128 + ch);
+        tq[q] = f32x2(t2.x, t2.y);
       }
-      const float gl0 = ((tq[0].x * tq[1].x) * tq[2].x) * tq[3].x;
-      const float gl1 = ((tq[0].y * tq[1].y) * tq[2].y) * tq[3].y;
-      if (qr == 3) *reinterpret_cast<float2*>(a.gl + tile * D + ch) = make_float2(gl0, gl1);
-      const float inv0 = rcp_approx(pre0 * (qr == 0 ? tq[0].x : qr == 1 ? tq[1].x : qr == 2 ? tq[2].x : tq[3].x));
-      const float inv1 = rcp_approx(pre1 * (qr == 0 ? tq[0].y : qr == 1 ? tq[1].y : qr == 2 ? tq[2].y : tq[3].y));
+      uint64_t pre = f32x2(1.f, 1.f), suf = f32x2(1.f, 1.f);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q < qr) pre = mul_f32x2(pre, tq[q]);
+        else if (q > qr) suf = mul_f32x2(suf, tq[q]);
+      }
+      const uint64_t glp = mul_f32x2(mul_f32x2(mul_f32x2(tq[0], tq[1]), tq[2]), tq[3]);
+      if (qr == 3) *reinterpret_cast<float2*>(a.gl + tile * D + ch) = f32x2_split(glp);
+      const float2 pq = f32x2_split(mul_f32x2(pre, qr == 0 ? tq[0] : qr == 1 ? tq[1] : qr == 2 ? tq[2] : tq[3]));
+      const uint64_t inv = f32x2(rcp_approx(pq.x), rcp_approx(pq.y));
       const int c3 = (ch & 63) >> 3;
       const uint32_t row0 = 2 * qr * 1024 + (ch & 7) * 2;
       const uint32_t kq0 = L_::KQ + bx * K16 + row0, kh0b = L_::KH + bx * K8 + row0;
       auto row_off = [&](int i) -> uint32_t {
         return (i >> 3) * 1024 + (i & 7) * 128 + ((c3 ^ (i & 7)) << 4);
       };
-      auto kq_in = [&](int i, float2& kk, float2& qq) {
-        kk = unpack_bf16(kraw[i]);
-        qq = unpack_bf16(qraw[i]);
+      auto kq_in = [&](int i, uint64_t& kk, uint64_t& qq) {
+        kk = bf16x2_to_f32x2(kraw[i]);
+        qq = bf16x2_to_f32x2(qraw[i]);
         if (PRO & KDA_PROLOGUE_QK_L2NORM) {
           const float rk = rn[16 * qr + i], rq = rn[64 + 16 * qr + i];
-          kk.x *= rk;
-          kk.y *= rk;
-          qq.x *= rq;
-          qq.y *= rq;
+          kk = mul_f32x2(kk, f32x2(rk, rk));
+          qq = mul_f32x2(qq, f32x2(rq, rq));
         }
       };
       // forward over the rows: K~ = k gamma, Q~ = q gamma
-      float gm0 = pre0, gm1 = pre1, qprev0 = 0.f, qprev1 = 0.f;
+      uint64_t gm = pre;
+      float qprev0 = 0.f, qprev1 = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        gm0 *= E0[i];
-        gm1 *= E1[i];
-        float2 kk, qq;
+        gm = mul_f32x2(gm, E2[i]);
+        uint64_t kk, qq;
         kq_in(i, kk, qq);
-        const float qt0f = qq.x * gm0, qt1f = qq.y * gm1;
-        *reinterpret_cast<uint32_t*>(sm + kq0 + row_off(i)) = pack_bf16(kk.x * gm0, kk.y * gm1);
+        const uint64_t qtv = mul_f32x2(qq, gm);
+        const float2 qtf = f32x2_split(qtv);
+        const float qt0f = qtf.x, qt1f = qtf.y;
+        *reinterpret_cast<uint32_t*>(sm + kq0 + row_off(i)) = pack_bf16x2(mul_f32x2(kk, gm));
         *reinterpret_cast<uint32_t*>(sm + kq0 + K8 + row_off(i)) = pack_bf16(qt0f, qt1f);
         if (i & 1) {
           qt0[i >> 1] = pack_bf16(qprev0, qt0f);
@@ -478,14 +488,15 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       };
       stage2(L_::QTS, qt0, qt1);
       // backward over the rows: K^ = k / gamma, Kb = k gl / gamma
-      float rs0 = 1.f, rs1 = 1.f, kprev0 = 0.f, kprev1 = 0.f;
+      uint64_t rs = f32x2(1.f, 1.f);
+      float kprev0 = 0.f, kprev1 = 0.f;
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
-        float2 kk, qq;
+        uint64_t kk, qq;
         kq_in(i, kk, qq);
-        const float kh0 = kk.x * (rs0 * inv0), kh1 = kk.y * (rs1 * inv1);
-        const float kb0f = kk.x * (rs0 * suf0), kb1f = kk.y * (rs1 * suf1);
-        *reinterpret_cast<uint32_t*>(sm + kh0b + row_off(i)) = pack_bf16(kh0, kh1);
+        *reinterpret_cast<uint32_t*>(sm + kh0b + row_off(i)) = pack_bf16x2(mul_f32x2(kk, mul_f32x2(rs, inv)));
+        const float2 kbf = f32x2_split(mul_f32x2(kk, mul_f32x2(rs, suf)));
+        const float kb0f = kbf.x, kb1f = kbf.y;
         if (!(i & 1)) {
           kb0[i >> 1] = pack_bf16(kb0f, kprev0);
           kb1[i >> 1] = pack_bf16(kb1f, kprev1);
@@ -493,8 +504,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
           kprev0 = kb0f;
           kprev1 = kb1f;
         }
-        rs0 *= E0[i];
-        rs1 *= E1[i];
+        rs = mul_f32x2(rs, E2[i]);
       }
       stage2(L_::KBS, kb0, kb1);
     }
