@@ -198,6 +198,11 @@ __device__ __forceinline__ float2 f32x2_split(uint64_t v) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
   return r;
 }
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -1019,10 +1024,14 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
 #pragma unroll
       for (int t4 = 0; t4 < 8; ++t4) {
         const float4 g = *reinterpret_cast<const float4*>(gl + 4 * t4);
-        v[4 * t4 + 0] = __float_as_uint(g.x * __uint_as_float(v[4 * t4 + 0]));
-        v[4 * t4 + 1] = __float_as_uint(g.y * __uint_as_float(v[4 * t4 + 1]));
-        v[4 * t4 + 2] = __float_as_uint(g.z * __uint_as_float(v[4 * t4 + 2]));
-        v[4 * t4 + 3] = __float_as_uint(g.w * __uint_as_float(v[4 * t4 + 3]));
+        const float2 a0 = f32x2_split(mul_f32x2(f32x2(g.x, g.y),
+                                                f32x2(__uint_as_float(v[4 * t4]), __uint_as_float(v[4 * t4 + 1]))));
+        const float2 a1 = f32x2_split(mul_f32x2(f32x2(g.z, g.w),
+                                                f32x2(__uint_as_float(v[4 * t4 + 2]), __uint_as_float(v[4 * t4 + 3]))));
+        v[4 * t4 + 0] = __float_as_uint(a0.x);
+        v[4 * t4 + 1] = __float_as_uint(a0.y);
+        v[4 * t4 + 2] = __float_as_uint(a1.x);
+        v[4 * t4 + 3] = __float_as_uint(a1.y);
       }
       tmem_st32(tb + lane_base + L_::st(b) + 32 * pt, v);
     };
@@ -1114,8 +1123,9 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       __nv_bfloat16* o = a.out + ((c0 + 16 * pt + odd) * a.H + h) * D + (row & ~1);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const float x0 = a.scale * __uint_as_float(v[2 * t]);
-        const float x1 = a.scale * __uint_as_float(v[2 * t + 1]);
+        const float2 xs = f32x2_split(mul_f32x2(f32x2(a.scale, a.scale),
+                                                f32x2(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1]))));
+        const float x0 = xs.x, x1 = xs.y;
         const float recv = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
         const uint32_t pr = odd ? pack_bf16(recv, x1) : pack_bf16(x0, recv);
         if (16 * pt + 2 * t + odd < L) *reinterpret_cast<uint32_t*>(o + 2 * t * ostride) = pr;
@@ -1154,12 +1164,9 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         const bool with_u0 = PC || b == 1;  // the M block of the summary walk has V = 0
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          float x0 = __uint_as_float(v[2 * t]), x1 = __uint_as_float(v[2 * t + 1]);
-          if (with_u0) {
-            x0 += u0v[2 * t];
-            x1 += u0v[2 * t + 1];
-          }
-          pk[t] = pack_bf16(x0, x1);
+          uint64_t x = f32x2(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1]));
+          if (with_u0) x = add_f32x2(x, f32x2(u0v[2 * t], u0v[2 * t + 1]));
+          pk[t] = pack_bf16x2(x);
         }
         tmem_st8(tb + lane_base + col, pk);
       }
