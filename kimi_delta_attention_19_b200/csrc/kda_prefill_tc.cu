@@ -138,7 +138,7 @@ struct WalkArgs {
   __nv_bfloat16* out;
   const float* s0;
   float* sT;
-  float* mbuf;    // [pairs, max_segs, D, D]  summary of segment j: M (row-major [i][j])
+  float* mbuf;    // [pairs, max_segs, D, D]  summary of segment j: M, as bf16 hi/lo operand tiles
   float* lbuf;    // [pairs, max_segs, D, D]  summary of segment j: L
   float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 1
   float* snap;    // [floor(T_total / (snap_every C)), H, D, D] or null: prefix-cache snapshots
@@ -1242,6 +1242,23 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         uint32_t v[32];
         tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
         tmem_ld_wait(v);
+        if (!PC && b == 0) {
+          // M[i][j] (i = 32 pt + t, j = row) as the combine's B operand, already split: two
+          // 128x128 bf16 tiles hi = bf16(M), lo = bf16(M - hi), each two 64-column atoms of
+          // 128-byte-swizzled rows i, in the shared-memory layout a plain bulk copy keeps
+          unsigned char* mb = reinterpret_cast<unsigned char*>(dst);
+          const uint32_t cofs = (row >> 6) * K16 + (row & 7) * 2;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float x = __uint_as_float(v[t]);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+            const uint32_t o = cofs + sw128_chunk(32 * pt + t, (row & 63) >> 3, 0);
+            *reinterpret_cast<__nv_bfloat16*>(mb + o) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(mb + K32 + o) = lo;
+          }
+          continue;
+        }
 #pragma unroll
         for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(32 * pt + t) * D + row] = __uint_as_float(v[t]);
       }
@@ -1286,12 +1303,15 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid
 // x = hi + lo with hi = bf16(x), lo = bf16(x - hi):
 //   S^T M^T ~= S_hi^T M_hi^T + S_hi^T M_lo^T + S_lo^T M_hi^T
 // (the dropped lo x lo term is ~2^-16 of the product). S^T, the A operand, lives in tensor
-// memory; M_j, the B operand (row-major = K-major), in shared memory; L_j^T seeds the
-// accumulator. The next step's M and L (fp32) are copied into shared memory while the
-// current step's products run.
+// memory; M_j, the B operand (row-major = K-major), in shared memory, as the hi/lo tiles the
+// summary walk wrote already split; L_j^T seeds the accumulator. The next step's M tiles (into
+// the other of two buffers) and L (fp32) are copied into shared memory while the current
+// step's products run.
 constexpr int kCombThreads = 256;
-constexpr uint32_t kCombMS = 2 * K32, kCombLS = kCombMS + 4 * K16, kCombBars = kCombLS + 4 * K16;
-constexpr uint32_t kCombSmem = kCombBars + 64 + 1024;  // M hi/lo tiles, M and L staging, barriers
+// two buffers of M's hi/lo operand tiles (64 KB each: the step's and the next one's), the L
+// staging copy, barriers
+constexpr uint32_t kCombB = 0, kCombLS = 4 * K32, kCombBars = kCombLS + 4 * K16;
+constexpr uint32_t kCombSmem = kCombBars + 64 + 1024;
 struct CombTm {
   static constexpr uint32_t D = 0, AH = 128, AL = 192, COLS = 256;
 };
@@ -1304,7 +1324,6 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kCombBars);  // products done
   uint64_t* bar_ld = bar + 1;                                     // M, L staged
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + kCombBars + 16);
-  const float* Mst = reinterpret_cast<const float*>(sm + kCombMS);
   const float* Lst = reinterpret_cast<const float*>(sm + kCombLS);
   const int pair = blockIdx.x;
   const int s = pair / a.H;
@@ -1323,12 +1342,13 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     tmem_alloc(tptr, CombTm::COLS);
     tmem_relinquish();
   }
-  // M_sg and L_sg (64 KB each) into the staging buffers, in 16 KB pieces
+  // M_sg (its hi/lo operand tiles, into buffer (sg - 1) % 2) and L_sg (64 KB each), in 16 KB
+  // pieces
   auto stage_ml = [&](int sg) {
     const int64_t o = (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D;
     mbar_arrive_expect_tx(bar_ld, 2 * D * D * 4);
     for (int q = 0; q < 4; ++q) {
-      bulk_load(sm + kCombMS + q * K16, a.mbuf + o + q * (K16 / 4), K16, bar_ld);
+      bulk_load(sm + kCombB + ((sg - 1) & 1) * 2 * K32 + q * K16, a.mbuf + o + q * (K16 / 4), K16, bar_ld);
       bulk_load(sm + kCombLS + q * K16, a.lbuf + o + q * (K16 / 4), K16, bar_ld);
     }
   };
@@ -1379,24 +1399,6 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
       break;
     }
     ld_pending = false;
-    // M_sg -> split B operand tiles. Thread t takes the 16-byte pieces t + 256 q of the
-    // row-major staging copy (consecutive lanes, consecutive addresses: no bank
-    // conflicts): row (t >> 5) + 8 q, columns 4 (t & 31) .. + 3; each becomes an 8-byte
-    // half of a 16-byte chunk of the swizzled tiles.
-    {
-      const int c4 = 4 * (tid & 31);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int r = (tid >> 5) + 8 * q;
-        const float4 x = *reinterpret_cast<const float4*>(Mst + r * D + c4);
-        uint2 hi, lo;
-        split_bf16(x.x, x.y, hi.x, lo.x);
-        split_bf16(x.z, x.w, hi.y, lo.y);
-        const uint32_t off = sw128_chunk(r, c4 >> 3, K16) + (c4 & 7) * 2;
-        *reinterpret_cast<uint2*>(sm + off) = hi;
-        *reinterpret_cast<uint2*>(sm + K32 + off) = lo;
-      }
-    }
     // L_sg^T seeds the accumulator: lane j, columns c = 64 hc ..
     {
       const float* lr = Lst + row;
@@ -1414,16 +1416,17 @@ __global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_c
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      if (sg + 1 < nseg - 1) {  // every thread has read the staging buffers
+      if (sg + 1 < nseg - 1) {  // every thread has read the L staging; the other M buffer is free
         stage_ml(sg + 1);
         ld_pending = true;
       }
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128, 0, 0);
+      const uint32_t mb = sb + kCombB + ((sg - 1) & 1) * 2 * K32;  // this step's M tiles
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;
-        const uint64_t bh = sdesc_sw128(sb + ko, 16, 1024), bl = sdesc_sw128(sb + K32 + ko, 16, 1024);
+        const uint64_t bh = sdesc_sw128(mb + ko, 16, 1024), bl = sdesc_sw128(mb + K32 + ko, 16, 1024);
         umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bh, id, 1);
         umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bl, id, 1);
         umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AL + 8 * k, bh, id, 1);
