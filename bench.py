@@ -243,7 +243,7 @@ def bench_ours(args, world, rank, local):
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
                 "traffic": measured_traffic("prefill_bf16_h32_t8192_d128"),
-                "traffic_scope": "one kda_chunk_fwd call (intra-chunk + summary walk + combine + output walk)",
+                "traffic_scope": "one kda_chunk_fwd call (intra-chunk kernel + walk kernel)",
                 "peak_source": peaks["source"],
                 "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": algo_bytes},
@@ -448,26 +448,12 @@ def kda_launches_per_step(kda, shape) -> int:
     """Kernels one kda_chunk_fwd enqueues for `shape` (the header memset excluded).
 
     bf16 with d_k = d_v = 128 takes the tensor-core path: the intra-chunk kernel and the
-    first walk phase, plus the combine (three or more segments) and the second walk
-    phase (two or more). The segment rule is the library's: m = 148 // pairs later
-    segments of n = max(4, ceil(Lc / (m + 1.125))) chunks after a first segment of
-    ceil(1.125 n) chunks, one segment when m < 2 or the longest sequence has < 16 chunks.
-    Other shapes run one CUDA-core kernel."""
+    walk kernel (summary walks, combine steps and output walks of every segment in one
+    launch). Other shapes run one CUDA-core kernel."""
     T_total = shape.T * (1 if shape.n_seqs > 0 else shape.B)
-    n = shape.n_seqs if shape.n_seqs > 0 else shape.B
     if not (shape.dtype == kda.KDA_BF16 and shape.dk == 128 and shape.dv == 128 and T_total > 0):
         return 1
-    max_len = shape.max_seqlen if (shape.n_seqs > 0 and shape.max_seqlen > 0) else shape.T
-    pairs = n * shape.H
-    lc = -(-max_len // 64)
-    m = 148 // pairs if pairs > 0 else 1
-    if m < 2 or lc < 16:
-        segs = 1
-    else:
-        nch = max(4, -(-(8 * lc) // (8 * m + 9)))
-        first, seg = 64 * (-(-(9 * nch) // 8)), 64 * nch
-        segs = 1 if max_len <= first else 1 + -(-(max_len - first) // seg)
-    return 2 + (1 if segs > 2 else 0) + (1 if segs > 1 else 0)
+    return 2
 
 
 def cpu_oracle_rate(min_seconds: float = 10.0, tokens: int | None = None, seed: int = 0) -> dict:

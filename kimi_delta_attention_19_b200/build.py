@@ -44,7 +44,7 @@ def _compile(src: str, obj: str, extra: list[str] | None = None) -> str:
 # word set, copies and products drained, tensor memory freed) run on the GPU and the
 # context stay usable. The product never loads it.
 SHORTWAIT_LIB = os.path.join(PKG, "libkda_shortwait.so")
-SHORTWAIT_DEFINES = {"kda_prefill_tc.cu": ["-DKDA_FIRST_WAIT_LIMIT=64"]}
+SHORTWAIT_DEFINES = {"kda_prefill_tc.cu": ["-DKDA_FIRST_WAIT_LIMIT=64", "-DKDA_FIRST_WAIT_STUCK=1"]}
 
 
 def _link(lib: str, objs: list[str]) -> None:

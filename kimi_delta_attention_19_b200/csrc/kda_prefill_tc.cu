@@ -126,6 +126,8 @@ struct IntraArgs {
   SeqTable seq;
   const __nv_bfloat16* beta;
   float* gl;
+  int* flags;  // the walk kernel's hand-off flags, zeroed here (block 0)
+  int n_flags;
   int H;
   float lb;
 };
@@ -138,9 +140,8 @@ struct WalkArgs {
   __nv_bfloat16* out;
   const float* s0;
   float* sT;
-  float* mbuf;    // [pairs, max_segs, D, D]  summary of segment j: M, as bf16 hi/lo operand tiles
-  float* lbuf;    // [pairs, max_segs, D, D]  summary of segment j: L
-  float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 1
+  float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 2 (and of 1 when j = 2 exists)
+  int* flags;     // [pairs, max_segs]  sstart of segment j written (1) or never coming (2); zeroed per call
   float* snap;    // [floor(T_total / (snap_every C)), H, D, D] or null: prefix-cache snapshots
   int snap_every; // chunks between snapshots
   int H;
@@ -221,13 +222,18 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-// Limit, in SM clocks, of the first wait on a kernel's inputs (the intra-chunk kernel's
-// TMA loads, the walks' first stage, the combine's first M and L). A test-only build of
-// the library sets it to a few clocks so that the wait runs out and each kernel's
-// bail-out path (record the error, let the copies and products in flight finish, free
-// tensor memory, return) runs on the GPU; every other wait keeps its own limit.
+// Limit, in SM clocks, of the first wait on the inputs of the intra-chunk kernel (its TMA
+// loads) and of each walk (its first stage). A test-only build of the library sets it to a
+// few clocks and, with KDA_FIRST_WAIT_STUCK, points that wait at a spare mbarrier that
+// nothing arrives at (inputs that never land), so that it always runs out and each
+// kernel's bail-out path (record the error, tell the CTAs waiting for a state hand-off that
+// it is not coming, let the copies and products in flight finish, free tensor memory,
+// return) runs on the GPU; every other wait keeps its own limit.
 #ifndef KDA_FIRST_WAIT_LIMIT
 #define KDA_FIRST_WAIT_LIMIT 4000000000LL
+#endif
+#ifndef KDA_FIRST_WAIT_STUCK
+#define KDA_FIRST_WAIT_STUCK 0
 #endif
 
 // Bounded wait by thread 0 alone (the others sleep in the barrier instead of polling),
@@ -291,6 +297,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t u = static_cast<int64_t>(blockIdx.x / static_cast<unsigned>(a.H));
   const int h = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.H));
+  if (blockIdx.x == 0)  // the walk kernel's hand-off flags start cleared on every call
+    for (int i = tid; i < a.n_flags; i += kIntraThreads) a.flags[i] = 0;
 
   // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
   const int s = owner_seq(a.seq, u);
@@ -308,6 +316,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + L_::BARS);  // g, k, q
   uint64_t* bar_v = bar_in + 1;
   uint64_t* bar_mma = bar_in + 2;
+  uint64_t* bar_none = bar_in + 3;  // nothing arrives (the test-only stuck first wait)
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
 
   if (warp == 0) {
@@ -318,6 +327,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     mbar_init(bar_in, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_none, 1);
     fence_mbar_init();
     // v is needed last (by the WY products): its own barrier
     mbar_arrive_expect_tx(bar_in, 3 * K16);
@@ -343,7 +353,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 
 
   do {
-    if (cta_wait_failed(bar_in, 0, KDA_FIRST_WAIT_LIMIT)) { failed = true; break; }
+    if (cta_wait_failed(KDA_FIRST_WAIT_STUCK ? bar_none : bar_in, 0, KDA_FIRST_WAIT_LIMIT)) {
+      failed = true;
+      break;
+    }
     in_done = true;
     if (L < C) {
       // a sequence's ragged last chunk: rows past L (the next sequence's tokens, or the
@@ -779,7 +792,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 }
 
 // ------------------------------------------------------------------ walk over chunks
-// One CTA per (sequence, head, segment), warp-specialized:
+// One kernel walks every segment: per (sequence, head) pair, CTA 0 walks segments 0 and 1
+// with outputs, and CTA r >= 1 walks segment r's summary, combines its start state and
+// then walks segment r + 1 with outputs (the kernel itself is at the end of this part).
+// Each CTA is warp-specialized:
 //   warps 0..15 conversion: warps w, w + 4, w + 8, w + 12 share the tensor-memory lanes
 //               32 (w % 4)..+31 (state columns j) and split their columns four ways;
 //               warps 0..7 own K half 0 of the products' operands, warps 8..15 K half 1.
@@ -810,9 +826,7 @@ struct WalkSm {
   static constexpr uint32_t STAGE = PK + (PC ? K16 + K8 : K16);
   static constexpr int NSTAGE = 3;  // chunk n in stage n % 3: two chunks' loads in flight
   static constexpr uint32_t GL = NSTAGE * STAGE;  // float[3][128]: each stage's gl, own barrier
-  static constexpr uint32_t BARS = GL + NSTAGE * 512;
-  static constexpr uint32_t TPTR = BARS + 128;
-  static constexpr uint32_t BYTES = TPTR + 16;
+  static constexpr uint32_t END = GL + NSTAGE * 512;
   // Tensor-memory columns. Output walk, by chunk parity p: p = 0: [U | O] at 0..127,
   // S at 128..255 (so MMA-2's accumulator [O | S] is 64..255); p = 1: S at 128..255,
   // [O | U] at 256..383 (MMA-2's [S | O] is 128..319). Summary walk: S per block at
@@ -824,44 +838,101 @@ struct WalkSm {
   __device__ static constexpr uint32_t yo(int p) { return p ? 256 : 64; }
   __device__ static constexpr uint32_t sbf(int b) { return 384 + 64 * b; }
   __device__ static constexpr uint32_t uk(int k) { return 16 * k; }
-  static constexpr uint32_t COLS = 512;
 };
-static_assert(WalkSm<true>::BYTES + 1024 <= 232448, "output walk shared memory");
-static_assert(WalkSm<false>::BYTES + 1024 <= 232448, "summary walk shared memory");
+// mbarriers of one walk: full, empty and gl per stage; m1, m2; s_ready and y_ready per K
+// half (then a spare one that nothing arrives at, for the test-only stuck first wait)
+constexpr int kWalkBars = 3 * WalkSm<true>::NSTAGE + 6;
+// Shared memory of the walk kernel: the output walk's stages and gl (the summary walk's
+// smaller ones overlap them); the combine's M operand tiles, inside the output walk's
+// third stage, which is not loaded before the combine's products have read them; one
+// mbarrier set per walk and the combine's; the tensor-memory address.
+struct WalkKSm {
+  static constexpr uint32_t MT = 146 * 1024;           // M: bf16 hi tile | lo tile (2 x 32 KB)
+  static constexpr uint32_t BARS = WalkSm<true>::END;  // two sets of 16, then the combine's
+  static constexpr uint32_t TPTR = BARS + 2 * 16 * 8 + 16;
+  static constexpr uint32_t BYTES = TPTR + 16;
+  static constexpr uint32_t COLS = 512;                // tensor memory, allocated once
+};
+static_assert(kWalkBars + 1 <= 16, "walk barrier set");
+static_assert(WalkKSm::MT % 1024 == 0 && WalkKSm::MT >= WalkSm<false>::END &&
+                  WalkKSm::MT >= 2 * WalkSm<true>::STAGE && WalkKSm::MT + 2 * K32 <= WalkSm<true>::GL,
+              "M tiles: past the summary walk's buffers and the output walk's first two stages");
+static_assert(WalkKSm::BYTES + 1024 <= 232448, "walk shared memory");
 
-// One CTA walks segment `seg` of the (sequence, head) pair: the output walk (PC) from
-// the segment's true start state, writing outputs (and the state where a later step
-// needs it), or the summary walk of a middle segment.
+// Segment `seg` of the sequence [t0, t1), head h: its tokens [c_begin, c_end) and the
+// workspace tile of its first chunk (chunk n of the segment: tile0 + n H).
+struct Seg {
+  int64_t t0, len, off, c_begin, c_end, tile0;
+  int n_chunks, h;
+};
+__device__ __forceinline__ Seg seg_geom(const WalkArgs& a, int s, int h, int64_t t0, int64_t t1,
+                                        int seg) {
+  Seg g;
+  g.t0 = t0;
+  g.len = t1 - t0;
+  g.h = h;
+  g.off = seg_offset(seg, a.first_tokens, a.seg_tokens);
+  g.c_begin = t0 + g.off;
+  const int64_t c_next = t0 + seg_offset(seg + 1, a.first_tokens, a.seg_tokens);
+  g.c_end = c_next < t1 ? c_next : t1;
+  g.n_chunks = g.c_end > g.c_begin ? static_cast<int>((g.c_end - g.c_begin + C - 1) / C) : 0;
+  g.tile0 = (slot_base(t0, s) + g.off / C) * a.H + h;
+  return g;
+}
+
+// The loads of chunk n of a walk (barrier set `bars`) into stage n % 3, which the caller
+// knows to be free: gl first, on its own barrier (the conversion warps need only it to
+// rescale), then the tiles.
+template <bool PC>
+__device__ __forceinline__ void issue_chunk(const WalkArgs& a, unsigned char* sm, uint64_t* bars,
+                                            int64_t tile0, int n) {
+  using L_ = WalkSm<PC>;
+  constexpr int NS = L_::NSTAGE;
+  const int st = n & 1, sg = n % NS;  // layout parity, stage
+  uint64_t* const full = bars + sg;
+  uint64_t* const glb = bars + 2 * NS + sg;
+  unsigned char* dst = sm + sg * L_::STAGE;
+  const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
+  const int y = static_cast<int>(tile * D);  // row of the [tiles * 128][64] arrays
+  mbar_arrive_expect_tx(glb, 512);
+  bulk_load(reinterpret_cast<float*>(sm + L_::GL) + sg * D, a.gl + tile * D, 512, glb);
+  mbar_arrive_expect_tx(full, L_::STAGE);
+  if (PC) {
+    // even stages: [-W^T | Q~^T], [P | Kb^T]; odd stages: [Q~^T | -W^T], [Kb^T | P]
+    tma_load_2d(dst + L_::WQ + st * K16, &a.tm_wt, full, 0, y);
+    tma_load_2d(dst + L_::WQ + (st ^ 1) * K16, &a.tm_qt, full, 0, y);
+    tma_load_2d(dst + L_::PK + (st ? 0 : K8), &a.tm_kbt, full, 0, y);
+    tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_p, full, 0, static_cast<int>(tile * C));
+  } else {
+    tma_load_2d(dst + L_::WQ, &a.tm_wt, full, 0, y);
+    tma_load_2d(dst + L_::PK, &a.tm_kbt, full, 0, y);
+  }
+  tma_load_2d(dst + L_::U0, &a.tm_u0, full, 0, y);
+}
+
+// One walk over segment `seg` (geometry g) of the (sequence, head) pair with the barrier
+// set `bars`. The output walk (PC) starts from the segment's start state (already in
+// tensor memory when `from_tmem`, else the initial state or zero), writes the outputs,
+// the final state when `last` and its end state, as the next segment's start, when
+// `put_next`. The summary walk leaves M as the combine's bf16 hi/lo operand tiles in
+// shared memory and L in tensor memory (columns 128..255). The caller has issued the
+// loads of the first `pre` chunks. Ends with a CTA barrier; returns false (in every
+// thread) when a wait ran out.
 template <bool PC, bool SNAP>
-__device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* smem_raw, int pair,
-                                             int seg) {
+__device__ __forceinline__ bool walk_segment(const WalkArgs& a, unsigned char* sm, uint32_t tb,
+                                             uint64_t* bars, const Seg& g, int pair, int seg,
+                                             bool from_tmem, int pre, bool last, bool put_next) {
   using L_ = WalkSm<PC>;
   constexpr int NB = L_::NB;
-  unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = pair / a.H, h = pair % a.H;
-  int64_t t0, t1;
-  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
-  const int64_t len = t1 - t0;
-  const int nseg = seg_count(len, a.first_tokens, a.seg_tokens);
-  if (len > a.max_len || nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
-    if (seg == 0 && tid == 0) atomicExch(a.seq.status, kDevBadSeqlens);
-    return;
-  }
-  // output walks: every segment; summary walks: the middle ones (segment 0's end state
-  // comes from its output walk, the last segment's is never needed)
-  if (PC ? (seg >= nseg) : (seg < 1 || seg > nseg - 2)) return;
-  const int64_t off = seg_offset(seg, a.first_tokens, a.seg_tokens);
-  const int64_t c_begin = t0 + off;
-  const int64_t c_next = t0 + seg_offset(seg + 1, a.first_tokens, a.seg_tokens);
-  const int64_t c_end = c_next < t1 ? c_next : t1;
-  const int n_chunks = static_cast<int>((c_end - c_begin + C - 1) / C);
-  // workspace tile of chunk n of this segment: tile0 + n H
-  const int64_t tile0 = (slot_base(t0, s) + off / C) * a.H + h;
+  const int h = g.h;
+  const int64_t t0 = g.t0, len = g.len, off = g.off, c_begin = g.c_begin, c_end = g.c_end;
+  const int n_chunks = g.n_chunks;
+  const int64_t tile0 = g.tile0;
+  bool good = true;  // this thread's waits all completed
 
   float* gls = reinterpret_cast<float*>(sm + L_::GL);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L_::BARS);
   constexpr int NS = L_::NSTAGE;
   uint64_t* bar_full = bars;        // per stage: the tiles have landed
   uint64_t* bar_empty = bars + NS;  // per stage: the products have read it
@@ -870,21 +941,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
   uint64_t* bar_m2 = bars + 3 * NS + 1;
   uint64_t* bar_sready = bars + 3 * NS + 2;  // two column halves
   uint64_t* bar_yready = bars + 3 * NS + 4;  // two column halves
-  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
-
-  if (warp == 0) {
-    tmem_alloc(tptr, L_::COLS);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    for (int i = 0; i < 3 * NS + 6; ++i) mbar_init(bars + i, 1);
-    fence_mbar_init();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = *tptr;
-  griddep_wait();  // the workspace and start states come from the previous kernels
+  tc_fence_after();  // after the caller's barrier: tensor memory as the previous step left it
 
   if (warp == kWalkLoadWarp) {
     // ============================================================ stage loads
@@ -896,33 +953,18 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         tma_prefetch_desc(&a.tm_qt);
         tma_prefetch_desc(&a.tm_p);
       }
-      int issued = 0;
+      int issued = pre;
       bool ok = true;
-      for (int n = 0; n < n_chunks; ++n) {
-        const int st = n & 1, sg = n % NS;  // layout parity, stage
+      for (int n = pre; n < n_chunks; ++n) {
+        const int sg = n % NS;
         if (n >= NS && !(ok = mbar_wait(bar_empty + sg, ((n - NS) / NS) & 1))) break;
-        unsigned char* dst = sm + sg * L_::STAGE;
-        const int64_t tile = tile0 + static_cast<int64_t>(n) * a.H;
-        const int y = static_cast<int>(tile * D);  // row of the [tiles * 128][64] arrays
-        // gl first, on its own barrier: the conversion warps need only it to rescale
-        mbar_arrive_expect_tx(bar_gl + sg, 512);
-        bulk_load(gls + sg * D, a.gl + tile * D, 512, bar_gl + sg);
-        mbar_arrive_expect_tx(bar_full + sg, L_::STAGE);
-        if (PC) {
-          // even stages: [-W^T | Q~^T], [P | Kb^T]; odd stages: [Q~^T | -W^T], [Kb^T | P]
-          tma_load_2d(dst + L_::WQ + st * K16, &a.tm_wt, bar_full + sg, 0, y);
-          tma_load_2d(dst + L_::WQ + (st ^ 1) * K16, &a.tm_qt, bar_full + sg, 0, y);
-          tma_load_2d(dst + L_::PK + (st ? 0 : K8), &a.tm_kbt, bar_full + sg, 0, y);
-          tma_load_2d(dst + L_::PK + (st ? K16 : 0), &a.tm_p, bar_full + sg, 0,
-                      static_cast<int>(tile * C));
-        } else {
-          tma_load_2d(dst + L_::WQ, &a.tm_wt, bar_full + sg, 0, y);
-          tma_load_2d(dst + L_::PK, &a.tm_kbt, bar_full + sg, 0, y);
-        }
-        tma_load_2d(dst + L_::U0, &a.tm_u0, bar_full + sg, 0, y);
+        issue_chunk<PC>(a, sm, bars, tile0, n);
         ++issued;
       }
-      if (!ok) atomicExch(a.seq.status, kDevWaitTimeout);
+      if (!ok) {
+        atomicExch(a.seq.status, kDevWaitTimeout);
+        good = false;
+      }
       // the copies in flight land before the CTA can exit
       for (int n = issued >= NS ? issued - NS : 0; n < issued; ++n) {
         mbar_wait(bar_gl + n % NS, (n / NS) & 1, 400000000LL);
@@ -997,6 +1039,7 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       }
       if (!ok) {
         atomicExch(a.seq.status, kDevWaitTimeout);
+        good = false;
         // every product issued so far (committed or not) finishes before tensor memory
         // is released: one more commit on m1, whose phase count is (m_issued + 1) / 2
         umma_commit(bar_m1);
@@ -1061,27 +1104,28 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
         }
       }
     };
-    // initial state: fp32 into tensor memory, bf16 copy as the MMA operand; then the
-    // first chunk's decay on the fp32 copy
+    // initial state: fp32 into tensor memory (unless it is there already), bf16 copy as
+    // the MMA operand; then the first chunk's decay on the fp32 copy
     {
-      const float* src = nullptr;
-      if (PC) {
-        if (seg > 0) src = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + seg) * D * D;
-        else if (a.s0) src = a.s0 + static_cast<int64_t>(pair) * D * D;
-      }
+      const float* src = (PC && a.s0) ? a.s0 + static_cast<int64_t>(pair) * D * D : nullptr;
       uint32_t v[32];  // the last block's values (the only one in the output walk)
 #pragma unroll 1
       for (int b = 0; b < NB; ++b) {
+        if (PC && from_tmem) {
+          tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+          tmem_ld_wait(v);
+        } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const int c = 32 * pt + t;
-          float x;
-          if (PC) x = src ? src[static_cast<int64_t>(c) * D + row] : 0.f;
-          else x = (b == 0 && c == row) ? 1.f : 0.f;
-          v[t] = __float_as_uint(x);
+          for (int t = 0; t < 32; ++t) {
+            const int c = 32 * pt + t;
+            float x;
+            if (PC) x = src ? src[static_cast<int64_t>(c) * D + row] : 0.f;
+            else x = (b == 0 && c == row) ? 1.f : 0.f;
+            v[t] = __float_as_uint(x);
+          }
         }
         pack_state(b, v);
-        if (NB > 1 || n_chunks == 0)  // the unscaled fp32 state (reloaded below / final)
+        if (NB > 1 || (n_chunks == 0 && !from_tmem))  // the unscaled fp32 state (reloaded below / final)
           tmem_st32(tb + lane_base + L_::st(b) + 32 * pt, v);
       }
       tmem_st_wait();
@@ -1089,7 +1133,8 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
       group_sync(half_bar, 256);
       if (half_lead && n_chunks > 0) mbar_arrive(bar_sready + kh);
       if (n_chunks > 0) {
-        const bool ok = mbar_wait(bar_gl, 0, KDA_FIRST_WAIT_LIMIT) && mbar_wait(bar_full, 0);
+        const bool ok = mbar_wait(KDA_FIRST_WAIT_STUCK ? bars + kWalkBars : bar_gl, 0, KDA_FIRST_WAIT_LIMIT) &&
+                        mbar_wait(bar_full, 0);
         if (group_any(kConvBar, kWalkConvThreads, !ok)) {
           failed = true;
         } else {
@@ -1224,255 +1269,239 @@ __device__ __forceinline__ void walk_segment(const WalkArgs& a, unsigned char* s
     tmem_st_wait();  // a decay store left in flight by a wait that ran out
     if (failed) {
       if (tid == 0) atomicExch(a.seq.status, kDevWaitTimeout);
-    } else {
-      // ---- final / summary state (row-major [i][j], fp32)
-      for (int b = 0; b < NB; ++b) {
-        float* dst = nullptr;
-        if (PC) {
-          if (seg == nseg - 1) {
-            if (a.sT) dst = a.sT + static_cast<int64_t>(pair) * D * D;
-          } else if (seg == 0) {  // S at the end of segment 0 starts the combine
-            dst = a.sstart + (static_cast<int64_t>(pair) * a.max_segs + 1) * D * D;
-          }
-        } else {
-          const int64_t un = static_cast<int64_t>(pair) * a.max_segs + seg;
-          dst = (b == 0 ? a.mbuf : a.lbuf) + un * D * D;
-        }
-        if (dst == nullptr) continue;
+      good = false;
+    } else if (!PC) {
+      // ---- summary: M[i][j] (i = 32 pt + t, j = row) as the combine's B operand, already
+      //      split: two 128x128 bf16 tiles hi = bf16(M), lo = bf16(M - hi), each two
+      //      64-column atoms of 128-byte-swizzled rows i (K-major: row i holds M[i][:])
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + L_::st(0) + 32 * pt, v);
+      tmem_ld_wait(v);
+      unsigned char* mb = sm + WalkKSm::MT;
+      const uint32_t cofs = (row >> 6) * K16 + (row & 7) * 2;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const float x = __uint_as_float(v[t]);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+        const uint32_t o = cofs + sw128_chunk(32 * pt + t, (row & 63) >> 3, 0);
+        *reinterpret_cast<__nv_bfloat16*>(mb + o) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(mb + K32 + o) = lo;
+      }
+      fence_async_smem();  // read by the tensor cores next
+    } else if (last || put_next) {
+      // ---- final state, or the next segment's start state (row-major [i][j], fp32)
+      float* dst = last ? a.sT : a.sstart + static_cast<int64_t>(pair) * a.max_segs * D * D;
+      if (dst != nullptr) {
+        dst += last ? static_cast<int64_t>(pair) * D * D : static_cast<int64_t>(seg + 1) * D * D;
         uint32_t v[32];
-        tmem_ld32(tb + lane_base + L_::st(b) + 32 * pt, v);
+        tmem_ld32(tb + lane_base + L_::st(0) + 32 * pt, v);
         tmem_ld_wait(v);
-        if (!PC && b == 0) {
-          // M[i][j] (i = 32 pt + t, j = row) as the combine's B operand, already split: two
-          // 128x128 bf16 tiles hi = bf16(M), lo = bf16(M - hi), each two 64-column atoms of
-          // 128-byte-swizzled rows i, in the shared-memory layout a plain bulk copy keeps
-          unsigned char* mb = reinterpret_cast<unsigned char*>(dst);
-          const uint32_t cofs = (row >> 6) * K16 + (row & 7) * 2;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float x = __uint_as_float(v[t]);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-            const uint32_t o = cofs + sw128_chunk(32 * pt + t, (row & 63) >> 3, 0);
-            *reinterpret_cast<__nv_bfloat16*>(mb + o) = hi;
-            *reinterpret_cast<__nv_bfloat16*>(mb + K32 + o) = lo;
-          }
-          continue;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) dst[static_cast<int64_t>(32 * pt + t) * D + row] = __uint_as_float(v[t]);
+        for (int t = 0; t < 32; ++t) __stcg(dst + static_cast<int64_t>(32 * pt + t) * D + row, __uint_as_float(v[t]));
+        if (put_next) __threadfence();  // before the flag that publishes it
       }
     }
   }
   tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tb, L_::COLS);
-  }
-  griddep_launch_dependents();
-}
-
-// Phase 1, per (sequence, head): CTA 0 walks segment 0 with outputs (its end state is
-// S_1), CTA r >= 1 is the summary walk of segment r, in parallel.
-constexpr uint32_t kWalkFirstSmem =
-    (WalkSm<true>::BYTES > WalkSm<false>::BYTES ? WalkSm<true>::BYTES : WalkSm<false>::BYTES) + 1024;
-// SNAP: the output walks also write chunk-boundary snapshots (a separate instance, so
-// the plain walk carries no trace of them).
-template <bool SNAP>
-__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_first(const __grid_constant__ WalkArgs a) {
-  extern __shared__ unsigned char smem_raw[];
-  const int per = a.max_segs > 2 ? a.max_segs - 1 : 1;
-  const int role = blockIdx.x % per, pair = blockIdx.x / per;
-  if (role == 0) walk_segment<true, SNAP>(a, smem_raw, pair, 0);
-  else walk_segment<false, false>(a, smem_raw, pair, role);
-}
-// Phase 2 (after the combine): the output walks of segments 1 .. nseg - 1.
-template <bool SNAP>
-__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk_rest(const __grid_constant__ WalkArgs a) {
-  extern __shared__ unsigned char smem_raw[];
-  const int per = a.max_segs - 1;
-  walk_segment<true, SNAP>(a, smem_raw, blockIdx.x / per, 1 + blockIdx.x % per);
+  const bool bad = __syncthreads_or(!good);
+  tc_fence_after();
+  return !bad;
 }
 
 // ------------------------------------------------------------------ combine
-// Start state of every segment j >= 2 from S_1 (written by segment 0's output walk):
-// S_{j+1} = M_j S_j + L_j for j = 1 .. nseg - 2, one CTA per (sequence, head). Each step
-// is one 128x128x128 product on the tensor cores in the transposed frame,
-// S_{j+1}^T = S_j^T M_j^T + L_j^T, at fp32 accuracy through a bf16 split of both factors,
-// x = hi + lo with hi = bf16(x), lo = bf16(x - hi):
+// Start state of segment r + 1 from that of segment r, S_{r+1} = M_r S_r + L_r, by the CTA
+// that has just walked segment r's summary. One 128x128x128 product on the tensor cores in
+// the transposed frame, S_{r+1}^T = S_r^T M_r^T + L_r^T, at fp32 accuracy through a bf16
+// split of both factors, x = hi + lo with hi = bf16(x), lo = bf16(x - hi):
 //   S^T M^T ~= S_hi^T M_hi^T + S_hi^T M_lo^T + S_lo^T M_hi^T
-// (the dropped lo x lo term is ~2^-16 of the product). S^T, the A operand, lives in tensor
-// memory; M_j, the B operand (row-major = K-major), in shared memory, as the hi/lo tiles the
-// summary walk wrote already split; L_j^T seeds the accumulator. The next step's M tiles (into
-// the other of two buffers) and L (fp32) are copied into shared memory while the current
-// step's products run.
-constexpr int kCombThreads = 256;
-// two buffers of M's hi/lo operand tiles (64 KB each: the step's and the next one's), the L
-// staging copy, barriers
-constexpr uint32_t kCombB = 0, kCombLS = 4 * K32, kCombBars = kCombLS + 4 * K16;
-constexpr uint32_t kCombSmem = kCombBars + 64 + 1024;
+// (the dropped lo x lo term is ~2^-16 of the product). L_r^T is the accumulator already:
+// the summary walk's second state block, in the tensor-memory columns where the output
+// walk keeps its state, so S_{r+1} stays there as the next output walk's start state. M_r
+// is the B operand the summary walk left in shared memory; S_r^T, published by the CTA of
+// segment r - 1, is split into the A operand.
 struct CombTm {
-  static constexpr uint32_t D = 0, AH = 128, AL = 192, COLS = 256;
+  static constexpr uint32_t D = 128, AH = 256, AL = 320;
 };
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait, bounded, for another CTA's hand-off flag: true when it says published, false when
+// it says the state is not coming or the wait ran out.
+__device__ __forceinline__ bool flag_wait(const int* p, long long limit_cycles = 4000000000LL) {
+  const long long t0 = clock64();
+  int f;
+  while ((f = ld_acquire_gpu(p)) == 0) {
+    if (clock64() - t0 > limit_cycles) return false;
+    __nanosleep(64);
+  }
+  return f == 1;
+}
 
+// The whole CTA calls it; `publish`: segment r + 2 has a summary walk, whose CTA waits for
+// S_{r+1}. Returns false (in every thread) when S_r never came or a wait ran out.
+__device__ __forceinline__ bool combine_step(const WalkArgs& a, unsigned char* sm, uint32_t tb,
+                                             uint64_t* bar, int pair, int r, bool publish) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* const flags = a.flags + static_cast<int64_t>(pair) * a.max_segs;
+  float* const sst = a.sstart + static_cast<int64_t>(pair) * a.max_segs * D * D;
+  const bool ok_in = tid != 0 || flag_wait(flags + r);
+  if (__syncthreads_or(!ok_in)) return false;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
+  const int pt = warp >> 2;                // K part: state rows k = 32 pt .. + 31
+  if (warp < kWalkMmaWarp) {
+    // S_r^T[j][k] = S_r[k][j] -> hi/lo bf16 pairs, tensor-memory column k / 2 of each half
+    // (read from L2: another SM wrote it)
+    const float* src = sst + static_cast<int64_t>(r) * D * D + static_cast<int64_t>(32 * pt) * D + row;
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      split_bf16(__ldcg(src + (2 * t) * D), __ldcg(src + (2 * t + 1) * D), hi[t], lo[t]);
+    tmem_st16(tb + lane_base + CombTm::AH + 16 * pt, hi);
+    tmem_st16(tb + lane_base + CombTm::AL + 16 * pt, lo);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == kWalkMmaWarp * 32) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16(128, 128, 0, 0);
+    const uint32_t mb = smem_u32(sm + WalkKSm::MT);
+#pragma unroll
+    for (int k = 0; k < D / 16; ++k) {
+      const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;  // K step k: atom k / 4, 32 bytes each
+      const uint64_t bh = sdesc_sw128(mb + ko, 16, 1024), bl = sdesc_sw128(mb + K32 + ko, 16, 1024);
+      umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bh, id, 1);
+      umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bl, id, 1);
+      umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AL + 8 * k, bh, id, 1);
+    }
+    umma_commit(bar);
+  }
+  if (cta_wait_failed(bar, 0)) {
+    // the products finish before tensor memory can be released
+    if (tid == 0) mbar_wait(bar, 0, 400000000LL);
+    return false;
+  }
+  tc_fence_after();
+  if (publish) {
+    if (warp < kWalkMmaWarp) {
+      uint32_t v[32];
+      tmem_ld32(tb + lane_base + CombTm::D + 32 * pt, v);
+      tmem_ld_wait(v);
+      float* dst = sst + static_cast<int64_t>(r + 1) * D * D + static_cast<int64_t>(32 * pt) * D + row;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) __stcg(dst + t * D, __uint_as_float(v[t]));
+      __threadfence();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) st_release_gpu(flags + r + 1, 1);
+  }
+  return true;
+}
 
-__global__ void __launch_bounds__(kCombThreads, 1) kda_tc_combine(const __grid_constant__ WalkArgs a) {
+// ------------------------------------------------------------------ walk kernel
+// CTA r of the `per` CTAs of a (sequence, head) pair:
+//   r = 0:  the output walk of segment 0, whose end state S_1 it publishes (when segment 1
+//           has a summary walk), then the output walk of segment 1 from S_1 in tensor memory;
+//   r >= 1: the summary walk of segment r (in parallel with segment 0's walk), the
+//           combine step S_{r+1} = M_r S_r + L_r as soon as CTA r - 1 has published S_r
+//           (publishing S_{r+1} in turn), then the output walk of segment r + 1 from S_{r+1}
+//           in tensor memory.
+// The grid (pairs x per <= the SM count, one CTA per SM) is resident at once, which the
+// hand-off waits rely on; each is bounded, and a CTA whose walk failed publishes "not
+// coming" so that the later ones stop waiting. The first two chunks of a CTA's second
+// walk are loaded while the combine waits. SNAP: the output walks also write
+// chunk-boundary snapshots (a separate instance, so the plain walk carries no trace of
+// them).
+template <bool SNAP>
+__global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_constant__ WalkArgs a) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = align1024(smem_raw);
-  const uint32_t sb = smem_u32(sm);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kCombBars);  // products done
-  uint64_t* bar_ld = bar + 1;                                     // M, L staged
-  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + kCombBars + 16);
-  const float* Lst = reinterpret_cast<const float*>(sm + kCombLS);
-  const int pair = blockIdx.x;
-  const int s = pair / a.H;
-  griddep_wait();  // M, L and S_1 come from the first walk phase
-  int64_t t0, t1;
-  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
-  const int64_t len = t1 - t0;
-  const int nseg = seg_count(len, a.first_tokens, a.seg_tokens);
-  if (len > a.max_len || nseg <= 2 || nseg > a.max_segs) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row = (warp & 3) * 32 + lane, hc = warp >> 2;  // lane j; this thread's column half
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  float* st0 = a.sstart + static_cast<int64_t>(pair) * a.max_segs * D * D;
-
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int per = a.max_segs > 2 ? a.max_segs - 1 : 1;
+  const int r = blockIdx.x % per, pair = blockIdx.x / per;
+  const int s = pair / a.H, h = pair % a.H;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + WalkKSm::BARS);  // first walk
+  uint64_t* bars2 = bars + 16;                                         // second walk
+  uint64_t* bar_comb = bars + 32;
+  uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + WalkKSm::TPTR);
+  // tensor memory once for the CTA's lifetime (an allocation after the relinquish is not
+  // allowed)
   if (warp == 0) {
-    tmem_alloc(tptr, CombTm::COLS);
+    tmem_alloc(tptr, WalkKSm::COLS);
     tmem_relinquish();
   }
-  // M_sg (its hi/lo operand tiles, into buffer (sg - 1) % 2) and L_sg (64 KB each), in 16 KB
-  // pieces
-  auto stage_ml = [&](int sg) {
-    const int64_t o = (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D;
-    mbar_arrive_expect_tx(bar_ld, 2 * D * D * 4);
-    for (int q = 0; q < 4; ++q) {
-      bulk_load(sm + kCombB + ((sg - 1) & 1) * 2 * K32 + q * K16, a.mbuf + o + q * (K16 / 4), K16, bar_ld);
-      bulk_load(sm + kCombLS + q * K16, a.lbuf + o + q * (K16 / 4), K16, bar_ld);
-    }
-  };
   if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_init(bar_ld, 1);
-    fence_mbar_init();
-    stage_ml(1);
-  } else if (tid == 32) {
-    // every step's M and L into L2 now: the steps read them one after another
-    for (int sg = 1; sg < nseg - 1; ++sg) {
-      const int64_t o = (static_cast<int64_t>(pair) * a.max_segs + sg) * D * D;
-      bulk_prefetch_l2(a.mbuf + o, D * D * 4);
-      bulk_prefetch_l2(a.lbuf + o, D * D * 4);
+    for (int i = 0; i <= kWalkBars; ++i) {
+      mbar_init(bars + i, 1);
+      mbar_init(bars2 + i, 1);
     }
+    mbar_init(bar_comb, 1);
+    fence_mbar_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = *tptr;
+  griddep_wait();  // the workspace tiles and the cleared flags come from the intra-chunk kernel
 
-  // this thread's 64 values of S^T (row j, columns 64 hc ..) -> the split A operand
-  auto put_a = [&](const uint32_t (&v0)[32], const uint32_t (&v1)[32]) {
-    uint32_t h[32], l[32];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      split_bf16(__uint_as_float(v0[2 * t]), __uint_as_float(v0[2 * t + 1]), h[t], l[t]);
-      split_bf16(__uint_as_float(v1[2 * t]), __uint_as_float(v1[2 * t + 1]), h[16 + t], l[16 + t]);
+  int64_t t0 = 0, t1 = 0;
+  int nseg = 0;
+  if (seq_bounds_tc(a.seq, s, t0, t1)) {
+    nseg = seg_count(t1 - t0, a.first_tokens, a.seg_tokens);
+    if (t1 - t0 > a.max_len || nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
+      if (r == 0 && tid == 0) atomicExch(a.seq.status, kDevBadSeqlens);
+      nseg = 0;
     }
-    tmem_st32(tb + lane_base + CombTm::AH + 32 * hc, h);
-    tmem_st32(tb + lane_base + CombTm::AL + 32 * hc, l);
-  };
-  {
-    // S_1^T[j][k] = S_1[k][j]
-    uint32_t v0[32], v1[32];
-    const float* src = st0 + static_cast<int64_t>(D) * D + row;
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      v0[t] = __float_as_uint(src[(64 * hc + t) * D]);
-      v1[t] = __float_as_uint(src[(64 * hc + 32 + t) * D]);
-    }
-    put_a(v0, v1);
   }
-  bool failed = false, ld_pending = true;
-  for (int sg = 1; sg < nseg - 1; ++sg) {
-    if (cta_wait_failed(bar_ld, (sg - 1) & 1, sg == 1 ? KDA_FIRST_WAIT_LIMIT : 4000000000LL)) {
-      failed = true;
-      break;
+  int* const flags = a.flags + static_cast<int64_t>(pair) * a.max_segs;
+  const bool loader = tid == kWalkLoadWarp * 32;
+  if (nseg > 0 && r == 0) {
+    const bool ok = walk_segment<true, SNAP>(a, sm, tb, bars, seg_geom(a, s, h, t0, t1, 0), pair, 0,
+                                             false, 0, nseg == 1, nseg > 2);
+    if (nseg > 2 && tid == 0) st_release_gpu(flags + 1, ok ? 1 : 2);
+    if (ok && nseg > 1) {
+      const Seg g1 = seg_geom(a, s, h, t0, t1, 1);
+      const int pre = g1.n_chunks < 2 ? g1.n_chunks : 2;
+      if (loader)
+        for (int n = 0; n < pre; ++n) issue_chunk<true>(a, sm, bars2, g1.tile0, n);
+      walk_segment<true, SNAP>(a, sm, tb, bars2, g1, pair, 1, true, pre, nseg == 2, false);
     }
-    ld_pending = false;
-    // L_sg^T seeds the accumulator: lane j, columns c = 64 hc ..
-    {
-      const float* lr = Lst + row;
-      uint32_t v0[32], v1[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        v0[t] = __float_as_uint(lr[(64 * hc + t) * D]);
-        v1[t] = __float_as_uint(lr[(64 * hc + 32 + t) * D]);
+  } else if (nseg > 0 && r <= nseg - 2) {
+    bool ok = walk_segment<false, false>(a, sm, tb, bars, seg_geom(a, s, h, t0, t1, r), pair, r,
+                                         false, 0, false, false);
+    const Seg g2 = seg_geom(a, s, h, t0, t1, r + 1);
+    // the next walk's first two chunks into stages 0 and 1 (the summary walk is done with
+    // them; the M tiles sit in stage 2)
+    const int pre = !ok ? 0 : g2.n_chunks < 2 ? g2.n_chunks : 2;
+    if (loader)
+      for (int n = 0; n < pre; ++n) issue_chunk<true>(a, sm, bars2, g2.tile0, n);
+    const bool publish = r + 1 <= nseg - 2;
+    if (ok) ok = combine_step(a, sm, tb, bar_comb, pair, r, publish);
+    if (!ok && publish && tid == 0) st_release_gpu(flags + r + 1, 2);
+    if (ok) {
+      walk_segment<true, SNAP>(a, sm, tb, bars2, g2, pair, r + 1, true, pre, r + 1 == nseg - 1, false);
+    } else if (loader) {
+      // the loads issued for the walk that will not run land before the CTA exits
+      for (int n = 0; n < pre; ++n) {
+        mbar_wait(bars2 + 2 * WalkSm<true>::NSTAGE + n, 0, 400000000LL);
+        mbar_wait(bars2 + n, 0, 400000000LL);
       }
-      tmem_st32(tb + lane_base + CombTm::D + 64 * hc, v0);
-      tmem_st32(tb + lane_base + CombTm::D + 64 * hc + 32, v1);
     }
-    tmem_st_wait();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      if (sg + 1 < nseg - 1) {  // every thread has read the L staging; the other M buffer is free
-        stage_ml(sg + 1);
-        ld_pending = true;
-      }
-      tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 128, 0, 0);
-      const uint32_t mb = sb + kCombB + ((sg - 1) & 1) * 2 * K32;  // this step's M tiles
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ko = (k >> 2) * K16 + (k & 3) * 32;
-        const uint64_t bh = sdesc_sw128(mb + ko, 16, 1024), bl = sdesc_sw128(mb + K32 + ko, 16, 1024);
-        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bh, id, 1);
-        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AH + 8 * k, bl, id, 1);
-        umma_bf16_tmem_a(tb + CombTm::D, tb + CombTm::AL + 8 * k, bh, id, 1);
-      }
-      umma_commit(bar);
-    }
-    if (cta_wait_failed(bar, (sg - 1) & 1)) {
-      failed = true;
-      break;
-    }
-    tc_fence_after();
-    // S_{sg+1}^T: to the workspace (row-major [k][j]) and, for a further step, to A
-    {
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tb + lane_base + CombTm::D + 64 * hc, v0);
-      tmem_ld32(tb + lane_base + CombTm::D + 64 * hc + 32, v1);
-      tmem_ld_wait(v0);
-      tmem_ld_wait(v1);
-      float* dst = st0 + static_cast<int64_t>(sg + 1) * D * D + row;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        dst[(64 * hc + t) * D] = __uint_as_float(v0[t]);
-        dst[(64 * hc + 32 + t) * D] = __uint_as_float(v1[t]);
-      }
-      if (sg + 1 < nseg - 1) put_a(v0, v1);
-    }
-    // the next step rewrites the B tiles and the accumulator: every thread is done here
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
-  if (failed && tid == 0) {
-    atomicExch(a.seq.status, kDevWaitTimeout);
-    // copies and products in flight finish before the CTA releases its memory
-    if (ld_pending) {
-      mbar_wait(bar_ld, 0, 400000000LL);
-      mbar_wait(bar_ld, 1, 400000000LL);
-    }
-    mbar_wait(bar, 0, 400000000LL);
-    mbar_wait(bar, 1, 400000000LL);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tb, CombTm::COLS);
+    tmem_dealloc(tb, WalkKSm::COLS);
   }
   griddep_launch_dependents();
 }
@@ -1522,11 +1551,11 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   p.n_slots = (T_total + C - 1) / C + n_seqs;
   p.pairs = static_cast<int64_t>(n_seqs) * H;
   if (max_len < 1) max_len = 1;
-  // Segments: the walks run one CTA per SM, and a chunk costs about the same in every
-  // CTA, so a sequence of Lc chunks is cut into segment 0 plus m later segments with
-  // m = SMs / pairs: phase 1 = segment 0's output walk beside the summary walks of
-  // segments 1 .. m - 1, phase 2 = the output walks of segments 1 .. m. Segment 0 is
-  // 1.125 x longer, matching the summary walk's slower chunk step.
+  // Segments: the walk kernel runs one CTA per SM, and a chunk costs about the same in
+  // every CTA, so a sequence of Lc chunks is cut into segment 0 plus m later segments with
+  // m = SMs / pairs, walked by m CTAs: CTA 0 walks segments 0 and 1 with outputs, CTA
+  // r >= 1 the summary of segment r beside segment 0's walk, then segment r + 1 with
+  // outputs. Segment 0 is 1.125 x longer, matching the summary walk's slower chunk step.
   const int64_t Lc = (max_len + C - 1) / C;
   const int64_t m = p.pairs > 0 ? 148 / p.pairs : 1;
   if (m < 2 || Lc < 16) {
@@ -1545,8 +1574,8 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   }
   const size_t state = sizeof(float) * D * D;
   size_t off = kWorkspaceHeader;
-  if (p.max_segs > 1)  // M, L and the start state of every segment
-    off += state * static_cast<size_t>(p.pairs) * 3 * static_cast<size_t>(p.max_segs);
+  if (p.max_segs > 2)  // the start state of every segment and its hand-off flag
+    off += (state + sizeof(int)) * static_cast<size_t>(p.pairs) * static_cast<size_t>(p.max_segs);
   p.tiles_off = align_to(off, 1024);
   p.ws_bytes = p.tiles_off + kTileBytes * static_cast<size_t>(p.n_slots) * static_cast<size_t>(H);
   return p;
@@ -1602,11 +1631,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   wa.sT = pa.sT;
   wa.snap = pa.snap;
   wa.snap_every = pa.snap_every;
-  const size_t state = static_cast<size_t>(D) * D;
-  float* base = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
-  wa.mbuf = base;
-  wa.lbuf = wa.mbuf + state * plan.pairs * plan.max_segs;
-  wa.sstart = wa.lbuf + state * plan.pairs * plan.max_segs;
+  if (plan.max_segs > 2) {
+    const size_t units = static_cast<size_t>(plan.pairs) * plan.max_segs;
+    wa.sstart = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
+    wa.flags = reinterpret_cast<int*>(wa.sstart + units * D * D);
+    ia.flags = wa.flags;
+    ia.n_flags = static_cast<int>(units);
+  }
   wa.H = pa.H;
   wa.first_tokens = plan.first_tokens;
   wa.max_len = pa.max_len;
@@ -1622,28 +1653,21 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        IntraSm::BYTES + 1024);
   const bool snap = pa.snap != nullptr;
-  void (*walk_first)(WalkArgs) = snap ? kda_tc_walk_first<true> : kda_tc_walk_first<false>;
-  void (*walk_rest)(WalkArgs) = snap ? kda_tc_walk_rest<true> : kda_tc_walk_rest<false>;
+  void (*walk)(WalkArgs) = snap ? kda_tc_walk<true> : kda_tc_walk<false>;
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(walk_first, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kWalkFirstSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(walk_rest, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             WalkSm<true>::BYTES + 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_tc_combine, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kCombSmem);
+    e = cudaFuncSetAttribute(walk, cudaFuncAttributeMaxDynamicSharedMemorySize, WalkKSm::BYTES + 1024);
   if (e != cudaSuccess) return e;
 
   intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
-  // The later kernels are launched with programmatic serialization: their CTAs may be
-  // scheduled while the previous kernel's last CTAs finish; they set up (tensor memory,
-  // barriers) and then wait for it (griddepcontrol.wait) before touching its results.
-  auto launch_dep = [&](const void* fn, int64_t grid, int threads, uint32_t smem) {
+  // The walk kernel is launched with programmatic serialization: its CTAs may be scheduled
+  // while the intra-chunk kernel's last CTAs finish; they set up (tensor memory, barriers)
+  // and then wait for it (griddepcontrol.wait) before touching its results.
+  {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
+    const int64_t per = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.pairs * per));
+    cfg.blockDim = dim3(kWalkThreads);
+    cfg.dynamicSmemBytes = WalkKSm::BYTES + 1024;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1651,18 +1675,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&wa};
-    return cudaLaunchKernelExC(&cfg, fn, args);
-  };
-  const int64_t per_first = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
-  if (e == cudaSuccess)
-    e = launch_dep(reinterpret_cast<const void*>(walk_first), plan.pairs * per_first,
-                   kWalkThreads, kWalkFirstSmem);
-  if (e == cudaSuccess && plan.max_segs > 2)
-    e = launch_dep(reinterpret_cast<const void*>(kda_tc_combine), plan.pairs, kCombThreads,
-                   kCombSmem);
-  if (e == cudaSuccess && plan.max_segs > 1)
-    e = launch_dep(reinterpret_cast<const void*>(walk_rest), plan.pairs * (plan.max_segs - 1),
-                   kWalkThreads, WalkSm<true>::BYTES + 1024);
+    e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(walk), args);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -3,9 +3,11 @@
 Every mbarrier wait in the tensor-core kernels has a limit; when one runs out the CTA records
 KDA_ERR_DEVICE (device code 2) in the workspace status word, lets its own copies and
 products in flight finish, frees its tensor memory and returns. The test-only build
-libkda_shortwait.so cuts the limit of the first wait on the inputs in each kernel (the
-intra-chunk kernel's TMA loads, the walks' first stage, the combine's first M and L) to 64
-clocks, which always runs out; every other wait keeps its limit. A prefill through it must
+libkda_shortwait.so points the first wait on the inputs of the intra-chunk kernel (its TMA
+loads) and of each walk (its first stage) at a spare mbarrier that nothing arrives at, with a
+limit of 64 clocks, so it always runs out however fast the real copies land; every other wait
+keeps its limit (a walk that failed tells the CTAs waiting for its state
+hand-off that it is not coming). A prefill through it must
 return with the status word set and no fault, and afterwards the regular library's prefill
 on the same device must still match the oracle.
 """
@@ -39,7 +41,7 @@ def kda():
 @pytest.mark.parametrize("T,H", [(64, 1), (3000, 2)])
 def test_first_wait_running_out_is_reported_and_context_stays_usable(kda, T, H):
     """(64, 1): one chunk of one head (intra-chunk kernel and one output walk);
-    (3000, 2): twelve segments per head (summary walks, combine, later output walks)."""
+    (3000, 2): twelve segments per head (summary walks, combine steps, later output walks)."""
     from kimi_delta_attention_19_b200 import build as kbuild
     assert os.path.exists(kbuild.SHORTWAIT_LIB), "build() makes the short-wait variant"
     short = kda.load_library(kbuild.SHORTWAIT_LIB)
