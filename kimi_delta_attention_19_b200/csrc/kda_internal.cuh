@@ -142,7 +142,8 @@ __device__ __forceinline__ void st_out<__nv_bfloat16>(__nv_bfloat16* p, float x)
 // Segment plan of the tensor-core prefill (a pure function of the shape).
 struct TcPlan {
   int first_tokens;  // tokens of a sequence's first segment (a multiple of the chunk length)
-  int seg_tokens;    // tokens of every later segment (a multiple of the chunk length)
+  int seg_tokens;    // tokens of segment 1 (a multiple of the chunk length)
+  int seg_dec;       // segment j >= 1 holds seg_tokens - (j - 1) seg_dec tokens
   int max_segs;      // segments of the longest sequence
   int64_t pairs;     // (sequence, head) pairs
   int64_t n_slots;   // chunk slots: ceil(T_total / chunk) + n_seqs

@@ -96,14 +96,22 @@ __device__ __forceinline__ bool seq_bounds_tc(const SeqTable& q, int s, int64_t&
 // ceil(T_total/64) + n_seqs.
 __device__ __forceinline__ int64_t slot_base(int64_t t0, int s) { return t0 / C + s; }
 
-// Segments of a sequence: segment 0 holds first_tokens tokens, every later one
-// seg_tokens (both multiples of the chunk length; the last segment may be shorter).
-__device__ __forceinline__ int seg_count(int64_t len, int first_tokens, int seg_tokens) {
-  if (len <= first_tokens) return 1;
-  return 1 + static_cast<int>((len - first_tokens + seg_tokens - 1) / seg_tokens);
+// Segments of a sequence: segment 0 holds first_tokens tokens, segment j >= 1
+// seg_tokens - (j - 1) seg_dec (all multiples of the chunk length; a sequence's last
+// segment may be shorter). Segment j starts at token seg_offset(j) of the sequence.
+__host__ __device__ __forceinline__ int64_t seg_offset(int seg, int first_tokens, int seg_tokens,
+                                                       int seg_dec) {
+  if (seg == 0) return 0;
+  const int64_t j = seg - 1;
+  return first_tokens + j * seg_tokens - static_cast<int64_t>(seg_dec) * (j * (j - 1) / 2);
 }
-__device__ __forceinline__ int64_t seg_offset(int seg, int first_tokens, int seg_tokens) {
-  return seg == 0 ? 0 : first_tokens + static_cast<int64_t>(seg - 1) * seg_tokens;
+// Segments that hold len tokens, counted up to max_segs + 1 (a sequence longer than the
+// plan covers).
+__host__ __device__ __forceinline__ int seg_count(int64_t len, int first_tokens, int seg_tokens,
+                                                  int seg_dec, int max_segs) {
+  int k = 1;
+  while (k <= max_segs && seg_offset(k, first_tokens, seg_tokens, seg_dec) < len) ++k;
+  return k;
 }
 
 // Sequence owning chunk slot u: the last one whose first slot is <= u.
@@ -145,7 +153,7 @@ struct WalkArgs {
   float* snap;    // [floor(T_total / (snap_every C)), H, D, D] or null: prefix-cache snapshots
   int snap_every; // chunks between snapshots
   int H;
-  int first_tokens, seg_tokens;  // segment 0, then every later segment (the last may be short)
+  int first_tokens, seg_tokens, seg_dec;  // segment 0; segment j >= 1: seg_tokens - (j - 1) seg_dec
   int max_segs;
   int64_t max_len;  // the caller's bound on a sequence's length
   float scale;
@@ -871,9 +879,9 @@ __device__ __forceinline__ Seg seg_geom(const WalkArgs& a, int s, int h, int64_t
   g.t0 = t0;
   g.len = t1 - t0;
   g.h = h;
-  g.off = seg_offset(seg, a.first_tokens, a.seg_tokens);
+  g.off = seg_offset(seg, a.first_tokens, a.seg_tokens, a.seg_dec);
   g.c_begin = t0 + g.off;
-  const int64_t c_next = t0 + seg_offset(seg + 1, a.first_tokens, a.seg_tokens);
+  const int64_t c_next = t0 + seg_offset(seg + 1, a.first_tokens, a.seg_tokens, a.seg_dec);
   g.c_end = c_next < t1 ? c_next : t1;
   g.n_chunks = g.c_end > g.c_begin ? static_cast<int>((g.c_end - g.c_begin + C - 1) / C) : 0;
   g.tile0 = (slot_base(t0, s) + g.off / C) * a.H + h;
@@ -1299,7 +1307,6 @@ __device__ __forceinline__ bool walk_segment(const WalkArgs& a, unsigned char* s
         tmem_ld_wait(v);
 #pragma unroll
         for (int t = 0; t < 32; ++t) __stcg(dst + static_cast<int64_t>(32 * pt + t) * D + row, __uint_as_float(v[t]));
-        if (put_next) __threadfence();  // before the flag that publishes it
       }
     }
   }
@@ -1336,22 +1343,36 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 __device__ __forceinline__ bool flag_wait(const int* p, long long limit_cycles = 4000000000LL) {
   const long long t0 = clock64();
   int f;
-  while ((f = ld_acquire_gpu(p)) == 0) {
+  while ((f = ld_acquire_gpu(p)) == 0)  // one thread per CTA polls: a load per L2 round trip
     if (clock64() - t0 > limit_cycles) return false;
-    __nanosleep(64);
-  }
   return f == 1;
 }
 
 // The whole CTA calls it; `publish`: segment r + 2 has a summary walk, whose CTA waits for
-// S_{r+1}. Returns false (in every thread) when S_r never came or a wait ran out.
+// S_{r+1}. `prefetch()`, called by the load warp's thread, issues the next walk's first
+// loads: before the wait when S_r is at least a hop away (r >= 2, flag not yet set), else
+// at the end, once S_{r+1} is published: with the walks streaming from HBM an SM takes
+// its 144 KB in ~4 us, and copies still landing slow every step of the combine down
+// (S_1, for r = 1, is planned to arrive with the summary's end).
+// Returns false (in every thread) when S_r never came or a wait ran out.
+template <typename F>
 __device__ __forceinline__ bool combine_step(const WalkArgs& a, unsigned char* sm, uint32_t tb,
-                                             uint64_t* bar, int pair, int r, bool publish) {
+                                             uint64_t* bar, int pair, int r, bool publish,
+                                             F&& prefetch) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* const flags = a.flags + static_cast<int64_t>(pair) * a.max_segs;
   float* const sst = a.sstart + static_cast<int64_t>(pair) * a.max_segs * D * D;
+  const bool loader = tid == kWalkLoadWarp * 32;
+  bool fetched = false;
+  if (loader && r >= 2 && ld_acquire_gpu(flags + r) == 0) {
+    prefetch();
+    fetched = true;
+  }
   const bool ok_in = tid != 0 || flag_wait(flags + r);
-  if (__syncthreads_or(!ok_in)) return false;
+  if (__syncthreads_or(!ok_in)) {
+    if (loader && !fetched) prefetch();  // the caller drains what it asked for
+    return false;
+  }
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const int row = (warp & 3) * 32 + lane;  // tensor-memory lane = state column j
   const int pt = warp >> 2;                // K part: state rows k = 32 pt .. + 31
@@ -1384,6 +1405,7 @@ __device__ __forceinline__ bool combine_step(const WalkArgs& a, unsigned char* s
     umma_commit(bar);
   }
   if (cta_wait_failed(bar, 0)) {
+    if (loader && !fetched) prefetch();  // the caller drains what it asked for
     // the products finish before tensor memory can be released
     if (tid == 0) mbar_wait(bar, 0, 400000000LL);
     return false;
@@ -1397,13 +1419,15 @@ __device__ __forceinline__ bool combine_step(const WalkArgs& a, unsigned char* s
       float* dst = sst + static_cast<int64_t>(r + 1) * D * D + static_cast<int64_t>(32 * pt) * D + row;
 #pragma unroll
       for (int t = 0; t < 32; ++t) __stcg(dst + t * D, __uint_as_float(v[t]));
-      __threadfence();
     }
+    // every thread's stores, then the flag by a gpu-scope release, which the CTA barrier
+    // makes cumulative over the other threads' stores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0) st_release_gpu(flags + r + 1, 1);
   }
+  if (loader && !fetched) prefetch();
   return true;
 }
 
@@ -1456,7 +1480,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
   int64_t t0 = 0, t1 = 0;
   int nseg = 0;
   if (seq_bounds_tc(a.seq, s, t0, t1)) {
-    nseg = seg_count(t1 - t0, a.first_tokens, a.seg_tokens);
+    nseg = seg_count(t1 - t0, a.first_tokens, a.seg_tokens, a.seg_dec, a.max_segs);
     if (t1 - t0 > a.max_len || nseg > a.max_segs) {  // the caller's max_seqlen bound was too small
       if (r == 0 && tid == 0) atomicExch(a.seq.status, kDevBadSeqlens);
       nseg = 0;
@@ -1467,6 +1491,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
   if (nseg > 0 && r == 0) {
     const bool ok = walk_segment<true, SNAP>(a, sm, tb, bars, seg_geom(a, s, h, t0, t1, 0), pair, 0,
                                              false, 0, nseg == 1, nseg > 2);
+    // after the walk's closing barrier, so the release covers S_1's stores by every thread
     if (nseg > 2 && tid == 0) st_release_gpu(flags + 1, ok ? 1 : 2);
     if (ok && nseg > 1) {
       const Seg g1 = seg_geom(a, s, h, t0, t1, 1);
@@ -1480,12 +1505,13 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
                                          false, 0, false, false);
     const Seg g2 = seg_geom(a, s, h, t0, t1, r + 1);
     // the next walk's first two chunks into stages 0 and 1 (the summary walk is done with
-    // them; the M tiles sit in stage 2)
+    // them; the M tiles sit in stage 2), issued during the combine step
     const int pre = !ok ? 0 : g2.n_chunks < 2 ? g2.n_chunks : 2;
-    if (loader)
-      for (int n = 0; n < pre; ++n) issue_chunk<true>(a, sm, bars2, g2.tile0, n);
     const bool publish = r + 1 <= nseg - 2;
-    if (ok) ok = combine_step(a, sm, tb, bar_comb, pair, r, publish);
+    if (ok)
+      ok = combine_step(a, sm, tb, bar_comb, pair, r, publish, [&] {
+        for (int n = 0; n < pre; ++n) issue_chunk<true>(a, sm, bars2, g2.tile0, n);
+      });
     if (!ok && publish && tid == 0) st_release_gpu(flags + r + 1, 2);
     if (ok) {
       walk_segment<true, SNAP>(a, sm, tb, bars2, g2, pair, r + 1, true, pre, r + 1 == nseg - 1, false);
@@ -1551,26 +1577,37 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   p.n_slots = (T_total + C - 1) / C + n_seqs;
   p.pairs = static_cast<int64_t>(n_seqs) * H;
   if (max_len < 1) max_len = 1;
-  // Segments: the walk kernel runs one CTA per SM, and a chunk costs about the same in
+  // Segments: the walk kernel runs one CTA per SM and a chunk costs about the same in
   // every CTA, so a sequence of Lc chunks is cut into segment 0 plus m later segments with
   // m = SMs / pairs, walked by m CTAs: CTA 0 walks segments 0 and 1 with outputs, CTA
-  // r >= 1 the summary of segment r beside segment 0's walk, then segment r + 1 with
-  // outputs. Segment 0 is 1.125 x longer, matching the summary walk's slower chunk step.
+  // r >= 1 the summary of segment r beside segment 0's walk, then (after the combine
+  // steps of CTAs 1 .. r, one after another) segment r + 1 with outputs. Segment 0 is
+  // 1.2 n chunks, as the summary walk's chunk step is ~1.2x the output walk's, so S_1 is
+  // ready when the summaries are; segment j >= 1 is n - (j - 1) delta chunks, delta = 2
+  // chunks (about one combine hop of output walk), so that the later segments, whose
+  // output walks start a hop later each, finish together. delta drops to 1, then 0, where
+  // it would take the last planned segment below max(4, n / 2) chunks.
   const int64_t Lc = (max_len + C - 1) / C;
   const int64_t m = p.pairs > 0 ? 148 / p.pairs : 1;
+  p.seg_dec = 0;
   if (m < 2 || Lc < 16) {
     p.first_tokens = p.seg_tokens = 1 << 30;  // one segment per sequence
     p.max_segs = 1;
   } else {
-    int64_t n = (8 * Lc + 8 * m + 9 - 1) / (8 * m + 9);  // ceil(Lc / (m + 1.125))
-    if (n < 4) n = 4;
-    const int64_t n0 = (9 * n + 7) / 8;  // ceil(1.125 n)
+    int64_t n = 4, delta = 2;
+    for (; delta >= 0; --delta) {
+      // n = ceil((Lc + delta m (m - 1) / 2) / (1.2 + m)): the segments cover Lc chunks
+      n = (5 * (Lc + delta * (m * (m - 1) / 2)) + 5 * m + 6 - 1) / (5 * m + 6);
+      if (n < 4) n = 4;
+      const int64_t lo = n / 2 > 4 ? (n + 1) / 2 : 4;
+      if (n - (m - 1) * delta >= lo) break;
+    }
+    if (delta < 0) delta = 0;
+    const int64_t n0 = (6 * n + 4) / 5;  // ceil(1.2 n)
     p.first_tokens = static_cast<int>(n0 * C);
     p.seg_tokens = static_cast<int>(n * C);
-    p.max_segs = max_len <= p.first_tokens
-                     ? 1
-                     : 1 + static_cast<int>((max_len - p.first_tokens + p.seg_tokens - 1) /
-                                            p.seg_tokens);
+    p.seg_dec = static_cast<int>(delta * C);
+    p.max_segs = seg_count(max_len, p.first_tokens, p.seg_tokens, p.seg_dec, static_cast<int>(m) + 1);
   }
   const size_t state = sizeof(float) * D * D;
   size_t off = kWorkspaceHeader;
@@ -1642,6 +1679,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   wa.first_tokens = plan.first_tokens;
   wa.max_len = pa.max_len;
   wa.seg_tokens = plan.seg_tokens;
+  wa.seg_dec = plan.seg_dec;
   wa.max_segs = plan.max_segs;
   wa.scale = pa.scale;
 
