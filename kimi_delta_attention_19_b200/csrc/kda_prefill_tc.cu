@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     //   warps 0, 1, 4, 5 take one row each and a half hh of its 64 columns, so the
     //   diagonal block of rows 0..31 is in the half of warp 0, that of rows 32..63 in the
     //   half of warp 5, and A_21 in warp 1's. Warps 2, 3, 6, 7 write P from lanes 64..127.
-    //   Forward substitution on the CUDA cores, a right-hand-side column per lane, rows
+    //   Forward substitution on the CUDA cores, a right-hand-side column per lane, columns
     //   of the block broadcast from shared memory: warp 0 solves (I + A_11) N_lo = I,
     //   warp 5 (I + A_22) N_hi = I and, beside it, warp 6 (I + A_22) G = A_21 (so G costs
     //   no extra step on the chain; the three solvers sit on three different SM
@@ -579,26 +579,27 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     const int hh = warp >> 2;                               // column half 32 hh ..
     const int rr = (warp & 3) * 32 + lane;                  // row (when rowt)
     // x = (I + A_bb)^{-1} rhs for this lane's column: x_r = rhs_r - sum_{s<r} A_rs x_s,
-    // row by row from broadcast float4 reads of the block's rows (entries s >= r are 0).
-    // The sum runs in two packed fp32 pairs (fma.rn.f32x2: two independent fp32 FMAs per
+    // column by column: once x_s is final, every later row takes its term -A_rs x_s, so
+    // the dependent chain is one fused multiply-add per column (the loads of column s do
+    // not depend on x and run ahead). `ncols` holds -A^T as rows of 36 floats (row s =
+    // -column s of A; entries r <= s are zero, so the pair that holds x_s itself is
+    // updated by zero). Packed fp32 pairs (fma.rn.f32x2: two independent fp32 FMAs per
     // instruction), x held as pairs (x_2m, x_2m+1).
-    auto fsub = [&](const float* arows, auto rhs, float (&x)[32]) {
+    auto fsub = [&](const float* ncols, auto rhs, float (&x)[32]) {
       uint64_t x2[16];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) x2[m] = 0ull;
+      for (int m = 0; m < 16; ++m) x2[m] = f32x2(rhs(2 * m), rhs(2 * m + 1));
 #pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        uint64_t s01 = 0ull, s23 = 0ull;
+      for (int c = 0; c < 31; ++c) {
+        const float2 pc = f32x2_split(x2[c >> 1]);
+        const float xc = (c & 1) ? pc.y : pc.x;
+        const uint64_t xx = f32x2(xc, xc);
 #pragma unroll
-        for (int q = 0; 4 * q < r; ++q) {
-          const float4 a4 = *reinterpret_cast<const float4*>(arows + r * 36 + 4 * q);
-          s01 = fma_f32x2(f32x2(a4.x, a4.y), x2[2 * q], s01);
-          s23 = fma_f32x2(f32x2(a4.z, a4.w), x2[2 * q + 1], s23);
+        for (int q = c >> 2; q < 8; ++q) {
+          const float4 a4 = *reinterpret_cast<const float4*>(ncols + c * 36 + 4 * q);
+          if (2 * q + 1 >= (c >> 1)) x2[2 * q + 1] = fma_f32x2(f32x2(a4.z, a4.w), xx, x2[2 * q + 1]);
+          if (2 * q >= (c >> 1)) x2[2 * q] = fma_f32x2(f32x2(a4.x, a4.y), xx, x2[2 * q]);
         }
-        const float2 p01 = f32x2_split(s01), p23 = f32x2_split(s23);
-        const float xr = rhs(r) - ((p01.x + p01.y) + (p23.x + p23.y));
-        const float2 old = f32x2_split(x2[r >> 1]);
-        x2[r >> 1] = (r & 1) ? f32x2(old.x, xr) : f32x2(xr, old.y);
       }
 #pragma unroll
       for (int m = 0; m < 16; ++m) {
@@ -607,15 +608,12 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
         x[2 * m + 1] = v2.y;
       }
     };
-    // this lane's row of A (in v) as a 36-float row of dst
+    // this lane's row r of A (in v) as column r of -A^T in dst (rows of 36 floats)
     float* const a22 = reinterpret_cast<float*>(sm + L_::A22);
     float* const a21 = reinterpret_cast<float*>(sm + L_::A21);
-    auto put_rows = [&](float* dst, const uint32_t (&v)[32]) {
+    auto put_cols = [&](float* dst, const uint32_t (&v)[32]) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(dst + lane * 36 + 4 * q) =
-            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+      for (int c = 0; c < 32; ++c) dst[c * 36 + lane] = -__uint_as_float(v[c]);
     };
     {
       uint32_t v[32];
@@ -637,25 +635,25 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
             *reinterpret_cast<float4*>(a21 + lane * 32 + 4 * q) =
                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-          group_sync(1, 96);  // warps 1, 5, 6: A_21 and A_22's rows are in place
+          group_sync(1, 96);  // warps 1, 5, 6: A_21's rows and A_22's columns are in place
         } else if (warp == 4) {
           // the upper-right block of T is zero
         } else {
           // warps 0 and 5: N_bb column `lane`, back through a transposition scratch so
           // that lane l ends with row l of N_bb; T_bb = N_bb Diag(beta_b)
           float* const scr = reinterpret_cast<float*>(sm + (warp == 0 ? L_::NLO : L_::NHT));
-          const float* arows;
+          const float* ncols;
           if (warp == 0) {
-            put_rows(scr, v);
+            put_cols(scr, v);
             __syncwarp();
-            arows = scr;
+            ncols = scr;
           } else {
-            put_rows(a22, v);
+            put_cols(a22, v);
             group_sync(1, 96);
-            arows = a22;
+            ncols = a22;
           }
           float x[32];
-          fsub(arows, [&](int r) { return r == lane ? 1.f : 0.f; }, x);
+          fsub(ncols, [&](int r) { return r == lane ? 1.f : 0.f; }, x);
           __syncwarp();
 #pragma unroll
           for (int r = 0; r < 32; ++r) scr[r * 36 + lane] = x[r];
