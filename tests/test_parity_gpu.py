@@ -12,6 +12,7 @@ from kimi_delta_attention_19_b200.inputs import (WORKLOADS, correlated_key_input
                                                   make_inputs, workload_inputs)
 from oracle import kda_oracle as ko
 from tests.parity import assert_close, errors
+from tests.plan import segment_plan
 
 pytestmark = pytest.mark.gpu
 
@@ -173,27 +174,11 @@ def test_tensor_core_segments(kda):
     assert_close(fin, rs, torch.bfloat16, "varlen segments final_state")
 
 
-def _segment_plan(n_seqs, H, max_len):
-    """The library's segment rule: segment 0, segment 1, and the shrink of each later
-    segment, in tokens (segment j >= 1 holds seg - (j - 1) dec tokens)."""
-    pairs = n_seqs * H
-    lc = -(-max_len // 64)
-    m = 148 // pairs
-    if m < 2 or lc < 16:
-        return None
-    for d in (2, 1, 0):
-        n = max(4, -(-(5 * (lc + d * (m * (m - 1) // 2))) // (5 * m + 6)))
-        lo = (n + 1) // 2 if n // 2 > 4 else 4
-        if n - (m - 1) * d >= lo:
-            break
-    return 64 * (-(-(6 * n) // 5)), 64 * n, 64 * d
-
-
 def test_tensor_core_segment_counts(kda):
     """Sequences with exactly 1, 2, 3 and many segments in one call: segment 0 alone,
     S_1 used directly by segment 1 (no combine step), one combine step, a long chain."""
     lengths = [320, 321, 576, 577, 0, 3000]
-    first, seg, dec = _segment_plan(len(lengths), 2, max(lengths))
+    first, seg, dec = segment_plan(len(lengths), 2, max(lengths))
     assert (first, seg, dec) == (320, 256, 0)
     nseg = [1 if n <= first else 1 + -(-(n - first) // seg) for n in lengths]
     assert nseg == [1, 2, 2, 3, 1, 12]
@@ -210,7 +195,7 @@ def test_tensor_core_shrinking_segments(kda):
     first segment of 11): the offsets of the combine chain's segments, a sequence ending in
     the short last segment, one in segment 1 and one inside segment 0."""
     lengths = [1792, 1000, 1]
-    plan = _segment_plan(len(lengths), 13, max(lengths))
+    plan = segment_plan(len(lengths), 13, max(lengths))
     assert plan == (11 * 64, 9 * 64, 2 * 64), plan
     x = make_inputs(None, H=13, dk=128, dv=128, dtype=torch.bfloat16, seed=23,
                     lengths=lengths, state_std=0.02)
