@@ -97,8 +97,11 @@ def test_batched_without_cu_seqlens(kda):
     assert_close(fin, rs, torch.bfloat16, "batched final_state")
 
 
-def test_zero_initial_state_and_no_final(kda):
-    x = make_inputs(130, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=11, state_std=None)
+@pytest.mark.parametrize("T", [130, 3000])
+def test_zero_initial_state_and_no_final(kda, T):
+    """No initial state and no final state: one segment (130 tokens) and twelve segments per
+    head (3000 tokens: the later segments start from combined states, the last writes none)."""
+    x = make_inputs(T, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=11, state_std=None)
     out, fin = kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV),
                              x.beta.to(DEV), output_final_state=False)
     torch.cuda.synchronize()
