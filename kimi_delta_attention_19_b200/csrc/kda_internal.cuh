@@ -147,6 +147,8 @@ struct TcPlan {
   int max_segs;      // segments of the longest sequence
   int64_t pairs;     // (sequence, head) pairs
   int64_t n_slots;   // chunk slots: ceil(T_total / chunk) + n_seqs
+  bool streamed;      // walk beside the intra-chunk kernel, one CTA per (sequence, head)
+  size_t ready_off;   // workspace offset of the per-tile ready flags (streamed schedule)
   size_t tiles_off;  // workspace offset of the per-chunk tiles
   size_t ws_bytes;   // workspace it needs, header included
 };

@@ -136,6 +136,9 @@ struct IntraArgs {
   float* gl;
   int* flags;  // the walk kernel's hand-off flags, zeroed here (block 0)
   int n_flags;
+  int* queue;      // tile counter (zero at the call's start): CTAs take tiles gridDim.x + *queue++
+  int64_t n_tiles; // chunk slots x heads
+  int* tile_ready; // streamed schedule: per tile, set to 1 once its workspace tiles are written; else null
   int H;
   float lb;
 };
@@ -150,6 +153,7 @@ struct WalkArgs {
   float* sT;
   float* sstart;  // [pairs, max_segs, D, D]  start state of segment j >= 2 (and of 1 when j = 2 exists)
   int* flags;     // [pairs, max_segs]  sstart of segment j written (1) or never coming (2); zeroed per call
+  const int* tile_ready;  // streamed schedule: per tile, 1 once the intra-chunk kernel wrote it; else null
   float* snap;    // [floor(T_total / (snap_every C)), H, D, D] or null: prefix-cache snapshots
   int snap_every; // chunks between snapshots
   int H;
@@ -256,13 +260,44 @@ __device__ __forceinline__ bool cta_wait_failed(uint64_t* bar, uint32_t parity,
 }
 
 
+// gpu-scope acquire load and release store of a flag another CTA (or kernel) reads
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait, bounded, for a flag another CTA sets (a state hand-off, a tile): true when it says published, false when
+// it says the state is not coming or the wait ran out.
+__device__ __forceinline__ bool flag_wait(const int* p, long long limit_cycles = 4000000000LL) {
+  const long long t0 = clock64();
+  int f;
+  while ((f = ld_acquire_gpu(p)) == 0)  // one thread per CTA polls: a load per L2 round trip
+    if (clock64() - t0 > limit_cycles) return false;
+  return f == 1;
+}
+
+// Orders this thread's bulk-copy (async proxy) memory accesses with its plain ones, in
+// every state space: a completed bulk store before a release, an acquire before a bulk load.
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ intra-chunk kernel
-// One CTA of 8 warps per (chunk slot, head); two CTAs per SM. Everything of a chunk
+// Persistent CTAs of 8 warps, two per SM, each taking (chunk slot, head) tiles from a
+// queue: its first tile is blockIdx.x, every next one gridDim.x + an atomic counter, drawn
+// while the current tile is worked (so tiles start in about launch order, and no CTA is
+// left with a long static share). Tensor memory and barriers are set up once per CTA,
+// which also removes the gap between one CTA's end and the next one's start on an SM
+// slot. Everything of a chunk
 // that does not depend on the state: decay tiles, the Gram products on the tensor
 // cores, the two 32x32 diagonal blocks of (I + A)^{-1} on the CUDA cores, and the WY
 // factors W = T K~, U0 = T V on the tensor cores, blocked on the two token halves so
 // that the off-diagonal block of the inverse is never formed.
 constexpr int kIntraThreads = 256;
+constexpr size_t kIntraQueueOffset = 128;  // the tile queue's counter, in the workspace header
 constexpr int kPStoreThread = 192;  // warp 6, lane 0: issues (and waits for) the P store
 struct IntraSm {
   // Raw inputs as loaded by TMA; each region is reused once its contents are read.
@@ -303,20 +338,11 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   unsigned char* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t u = static_cast<int64_t>(blockIdx.x / static_cast<unsigned>(a.H));
-  const int h = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.H));
+  // The next kernel of the stream may be scheduled once every CTA of this grid has started
+  // (it waits for this grid's completion itself before reading its results).
+  griddep_launch_dependents();
   if (blockIdx.x == 0)  // the walk kernel's hand-off flags start cleared on every call
     for (int i = tid; i < a.n_flags; i += kIntraThreads) a.flags[i] = 0;
-
-  // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
-  const int s = owner_seq(a.seq, u);
-  int64_t t0, t1;
-  if (!seq_bounds_tc(a.seq, s, t0, t1)) return;
-  const int64_t c = u - slot_base(t0, s);
-  if (c < 0 || c * C >= t1 - t0) return;  // a slot between two sequences
-  const int64_t r0 = t0 + c * C;
-  const int L = (t1 - r0) < C ? static_cast<int>(t1 - r0) : C;
-  const int64_t tile = u * a.H + h;
 
   float* tot = reinterpret_cast<float*>(sm + L_::TOT);
   float* bet = reinterpret_cast<float*>(sm + L_::BET);
@@ -326,17 +352,47 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
   uint64_t* bar_mma = bar_in + 2;
   uint64_t* bar_none = bar_in + 3;  // nothing arrives (the test-only stuck first wait)
   uint32_t* tptr = reinterpret_cast<uint32_t*>(sm + L_::TPTR);
+  int64_t* next_tile = reinterpret_cast<int64_t*>(sm + L_::TPTR + 8);
 
   if (warp == 0) {
     tmem_alloc(tptr, L_::COLS);
     tmem_relinquish();
   } else if (tid == 32) {
-    // barriers and input loads from warp 1, while warp 0 allocates tensor memory
     mbar_init(bar_in, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
     mbar_init(bar_none, 1);
     fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = *tptr;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  // phases: bar_in and bar_v complete once per live tile, bar_mma three times
+  int tiles_done = 0, mma_issued = 0, mma_done = 0;
+  bool in_done = true, v_done = true, failed = false;
+
+  int64_t tile = blockIdx.x;
+  while (tile < a.n_tiles) {
+  const int64_t u = tile / a.H;
+  const int h = static_cast<int>(tile % a.H);
+  // ---- the (sequence, chunk) that owns slot u: the last sequence whose base is <= u
+  const int s = owner_seq(a.seq, u);
+  int64_t t0 = 0, t1 = 0, c = -1;
+  if (seq_bounds_tc(a.seq, s, t0, t1)) c = u - slot_base(t0, s);
+  if (c < 0 || c * C >= t1 - t0) {  // a slot between two sequences (or a malformed table)
+    if (tid == 0) *next_tile = gridDim.x + static_cast<int64_t>(atomicAdd(a.queue, 1));
+    __syncthreads();
+    tile = *next_tile;
+    __syncthreads();
+    continue;
+  }
+  const int64_t r0 = t0 + c * C;
+  const int L = (t1 - r0) < C ? static_cast<int>(t1 - r0) : C;
+  const uint32_t par = tiles_done & 1;  // this tile's phase of bar_in and bar_v
+
+  if (tid == 32) {
     // v is needed last (by the WY products): its own barrier
     mbar_arrive_expect_tx(bar_in, 3 * K16);
     mbar_arrive_expect_tx(bar_v, K16);
@@ -348,20 +404,16 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     for (int bx = 0; bx < 2; ++bx)
       tma_load_2d(sm + L_::SV + bx * K8, &a.tm_v, bar_v, h * D + 64 * bx, static_cast<int>(r0));
   }
+  in_done = v_done = false;
+  // the CTA's next tile, drawn now and used once this one is done
+  int64_t nxt = 0;
+  if (tid == 0) nxt = gridDim.x + static_cast<int64_t>(atomicAdd(a.queue, 1));
   // beta of this thread's row, kept in a register until phase 1 is done (its load then
   // overlaps the TMA wait and phase 1 instead of delaying them)
   const float beta_r = tid < L ? __bfloat162float(a.beta[(r0 + tid) * a.H + h]) : 0.f;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = *tptr;
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  int mma_issued = 0, mma_done = 0;
-  bool in_done = false, v_done = false, failed = false;
-
 
   do {
-    if (cta_wait_failed(KDA_FIRST_WAIT_STUCK ? bar_none : bar_in, 0, KDA_FIRST_WAIT_LIMIT)) {
+    if (cta_wait_failed(KDA_FIRST_WAIT_STUCK ? bar_none : bar_in, par, KDA_FIRST_WAIT_LIMIT)) {
       failed = true;
       break;
     }
@@ -555,10 +607,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       umma_commit(bar_mma);
     }
-    mma_issued = 1;
+    ++mma_issued;
     if (tid == 32) bulk_wait_read();  // the staging tiles are rewritten from phase 4 on
-    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
-    mma_done = 1;
+    if (cta_wait_failed(bar_mma, mma_done & 1)) { failed = true; break; }
+    ++mma_done;
     tc_fence_after();
     // ---- 4-6. T = (I + A)^{-1} Diag(beta), blocked on the two 32-token halves:
     //   (I + A)^{-1} = [[N_lo, 0], [N_21, N_hi]], N_bb = (I + A_bb)^{-1},
@@ -700,7 +752,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     }
     fence_async_smem();
     tc_fence_before();
-    if (cta_wait_failed(bar_v, 0)) { failed = true; break; }  // also the barrier for T, P, +-G
+    if (cta_wait_failed(bar_v, par)) { failed = true; break; }  // also the barrier for T, P, +-G
     v_done = true;
     // ---- 7. W^T = K~^T T^T and U0^T = V^T T^T with the block-diagonal T: the lower token
     //         half is final, the upper one still lacks -G X_lo. K~ (in the Gram operand)
@@ -717,9 +769,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       umma_commit(bar_mma);
     }
-    mma_issued = 2;
-    if (cta_wait_failed(bar_mma, 1)) { failed = true; break; }
-    mma_done = 2;
+    ++mma_issued;
+    if (cta_wait_failed(bar_mma, mma_done & 1)) { failed = true; break; }
+    ++mma_done;
     tc_fence_after();
     // ---- 8. token columns 0..31 of -W^T (warps 0..3) and U0^T (warps 4..7) to the staging
     //         tiles: tensor-memory lane i holds row i
@@ -755,9 +807,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       }
       umma_commit(bar_mma);
     }
-    mma_issued = 3;
-    if (cta_wait_failed(bar_mma, 0)) { failed = true; break; }
-    mma_done = 3;
+    ++mma_issued;
+    if (cta_wait_failed(bar_mma, mma_done & 1)) { failed = true; break; }
+    ++mma_done;
     tc_fence_after();
     {
       uint32_t v[32];
@@ -778,14 +830,36 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       bulk_commit();
     }
   } while (0);
-  // the workspace stores have read their staging tiles before the CTA's shared memory is
-  // released (their writes are visible to the next kernel once this grid completes)
-  if (tid == 32 || tid == kPStoreThread) bulk_wait_read();
+  // the workspace stores have read their staging tiles before the next tile's loads (or
+  // the CTA's exit) reuse that shared memory (their writes are visible to the next kernel
+  // once this grid completes)
+  if (tid == 32 || tid == kPStoreThread) {
+    if (a.tile_ready) {
+      // streamed schedule: this tile's stores complete and ordered before the release below
+      bulk_wait_all();
+      fence_proxy_async_all();
+    } else {
+      bulk_wait_read();
+    }
+  }
+  if (failed) break;
+  ++tiles_done;
+  if (tid == 0) *next_tile = nxt;
+  fence_async_smem();  // this tile's shared-memory writes before the next tile's TMA loads
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // streamed schedule: the tile (stores, and gl by plain stores) is published to the walk,
+  // a gpu-scope release after the CTA barrier
+  if (a.tile_ready && tid == 0) st_release_gpu(a.tile_ready + tile, 1);
+  tile = *next_tile;
+  }  // tiles
   if (failed && tid == 0) {
     atomicExch(a.seq.status, kDevWaitTimeout);
     // copies and products in flight finish before the CTA releases its memory
-    if (!in_done) mbar_wait(bar_in, 0, 400000000LL);
-    if (!v_done) mbar_wait(bar_v, 0, 400000000LL);
+    const uint32_t par = tiles_done & 1;
+    if (!in_done) mbar_wait(bar_in, par, 400000000LL);
+    if (!v_done) mbar_wait(bar_v, par, 400000000LL);
     for (int m = mma_done; m < mma_issued; ++m) mbar_wait(bar_mma, m & 1, 400000000LL);
   }
   tc_fence_before();
@@ -794,7 +868,9 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     tc_fence_after();
     tmem_dealloc(tb, L_::COLS);
   }
-  griddep_launch_dependents();
+  // streamed schedule: this grid runs as the walk kernel's dependent; it completes only
+  // after the walk does, so later work on the stream still sees both finished
+  if (a.tile_ready) griddep_wait();
 }
 
 // ------------------------------------------------------------------ walk over chunks
@@ -964,6 +1040,12 @@ __device__ __forceinline__ bool walk_segment(const WalkArgs& a, unsigned char* s
       for (int n = pre; n < n_chunks; ++n) {
         const int sg = n % NS;
         if (n >= NS && !(ok = mbar_wait(bar_empty + sg, ((n - NS) / NS) & 1))) break;
+        if (a.tile_ready) {
+          // streamed schedule: the intra-chunk kernel, running beside this one, publishes
+          // each tile once its stores are complete
+          if (!(ok = flag_wait(a.tile_ready + tile0 + static_cast<int64_t>(n) * a.H))) break;
+          fence_proxy_async_all();
+        }
         issue_chunk<PC>(a, sm, bars, tile0, n);
         ++issued;
       }
@@ -1328,24 +1410,6 @@ __device__ __forceinline__ bool walk_segment(const WalkArgs& a, unsigned char* s
 struct CombTm {
   static constexpr uint32_t D = 128, AH = 256, AL = 320;
 };
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Wait, bounded, for another CTA's hand-off flag: true when it says published, false when
-// it says the state is not coming or the wait ran out.
-__device__ __forceinline__ bool flag_wait(const int* p, long long limit_cycles = 4000000000LL) {
-  const long long t0 = clock64();
-  int f;
-  while ((f = ld_acquire_gpu(p)) == 0)  // one thread per CTA polls: a load per L2 round trip
-    if (clock64() - t0 > limit_cycles) return false;
-  return f == 1;
-}
-
 // The whole CTA calls it; `publish`: segment r + 2 has a summary walk, whose CTA waits for
 // S_{r+1}. `prefetch()`, called by the load warp's thread, issues the next walk's first
 // loads: before the wait when S_r is at least a hop away (r >= 2, flag not yet set), else
@@ -1473,7 +1537,13 @@ __global__ void __launch_bounds__(kWalkThreads, 1) kda_tc_walk(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = *tptr;
-  griddep_wait();  // the workspace tiles and the cleared flags come from the intra-chunk kernel
+  if (a.tile_ready) {
+    // streamed schedule: the intra-chunk kernel runs as this grid's dependent, beside it;
+    // let it be scheduled now (the tiles are waited for one by one)
+    griddep_launch_dependents();
+  } else {
+    griddep_wait();  // the workspace tiles and the cleared flags come from the intra-chunk kernel
+  }
 
   int64_t t0 = 0, t1 = 0;
   int nseg = 0;
@@ -1588,7 +1658,23 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   const int64_t Lc = (max_len + C - 1) / C;
   const int64_t m = p.pairs > 0 ? 148 / p.pairs : 1;
   p.seg_dec = 0;
-  if (m < 2 || Lc < 16) {
+  // Streamed schedule: one output walk per (sequence, head) from the start, beside the
+  // intra-chunk kernel on the other SMs, each tile taken as soon as it is written (from L2).
+  // Chosen when a model of the two schedules (per-tile and per-chunk costs measured on the
+  // 8K x 32-head workload) favours it: the streamed time is the longer of one walk over the
+  // longest sequence (~1.9 us a chunk) and the tiles on 2 x (SMs - pairs) CTA slots; the
+  // segmented time is the tiles on all 296 slots, then the segmented walks.
+  const double tiles_us = 12.6 * static_cast<double>(p.n_slots * H);
+  const double walk_seg = (m >= 2 && Lc >= 16) ? 5.1 * static_cast<double>(Lc) / (static_cast<double>(m) + 1.26)
+                                               : 1.9 * static_cast<double>(Lc);
+  const double t_seg = tiles_us / 296.0 + walk_seg;
+  double t_str = 1e300;
+  if (p.pairs >= 1 && p.pairs <= 100) {
+    const double intra = tiles_us / (2.0 * static_cast<double>(148 - p.pairs));
+    t_str = (1.9 * static_cast<double>(Lc) > intra ? 1.9 * static_cast<double>(Lc) : intra) + 10.0;
+  }
+  p.streamed = t_str < 0.97 * t_seg;
+  if (p.streamed || m < 2 || Lc < 16) {
     p.first_tokens = p.seg_tokens = 1 << 30;  // one segment per sequence
     p.max_segs = 1;
   } else {
@@ -1609,6 +1695,8 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
   }
   const size_t state = sizeof(float) * D * D;
   size_t off = kWorkspaceHeader;
+  p.ready_off = off;  // per-tile ready flags of the streamed schedule
+  off += align_to(sizeof(int) * static_cast<size_t>(p.n_slots) * static_cast<size_t>(H), 256);
   if (p.max_segs > 2)  // the start state of every segment and its hand-off flag
     off += (state + sizeof(int)) * static_cast<size_t>(p.pairs) * static_cast<size_t>(p.max_segs);
   p.tiles_off = align_to(off, 1024);
@@ -1656,6 +1744,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   ia.seq = seq;
   ia.beta = static_cast<const __nv_bfloat16*>(pa.beta);
   ia.gl = gl;
+  ia.queue = reinterpret_cast<int*>(pa.ws + kIntraQueueOffset);
+  if (plan.streamed) {
+    ia.tile_ready = reinterpret_cast<int*>(pa.ws + plan.ready_off);
+    wa.tile_ready = ia.tile_ready;
+  }
+  ia.n_tiles = tiles;
   ia.H = pa.H;
   ia.lb = pa.lb;
 
@@ -1668,7 +1762,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
   wa.snap_every = pa.snap_every;
   if (plan.max_segs > 2) {
     const size_t units = static_cast<size_t>(plan.pairs) * plan.max_segs;
-    wa.sstart = reinterpret_cast<float*>(pa.ws + kWorkspaceHeader);
+    wa.sstart = reinterpret_cast<float*>(pa.ws + plan.ready_off +
+                                         align_to(sizeof(int) * static_cast<size_t>(tiles), 256));
     wa.flags = reinterpret_cast<int*>(wa.sstart + units * D * D);
     ia.flags = wa.flags;
     ia.n_flags = static_cast<int>(units);
@@ -1694,24 +1789,50 @@ cudaError_t launch_prefill_tc(const PrefillArgs& pa, cudaStream_t st) {
     e = cudaFuncSetAttribute(walk, cudaFuncAttributeMaxDynamicSharedMemorySize, WalkKSm::BYTES + 1024);
   if (e != cudaSuccess) return e;
 
-  intra<<<static_cast<unsigned>(tiles), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
-  // The walk kernel is launched with programmatic serialization: its CTAs may be scheduled
-  // while the intra-chunk kernel's last CTAs finish; they set up (tensor memory, barriers)
-  // and then wait for it (griddepcontrol.wait) before touching its results.
-  {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // a launch with programmatic stream serialization: it may be scheduled once every CTA of
+  // the kernel before it on the stream has triggered (griddepcontrol.launch_dependents)
+  auto launch_dep = [&](const void* fn, int64_t grid, int threads, uint32_t smem, void* arg) {
     cudaLaunchConfig_t cfg = {};
-    const int64_t per = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
-    cfg.gridDim = dim3(static_cast<unsigned>(plan.pairs * per));
-    cfg.blockDim = dim3(kWalkThreads);
-    cfg.dynamicSmemBytes = WalkKSm::BYTES + 1024;
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void* args[] = {&wa};
-    e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(walk), args);
+    void* args[] = {arg};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  };
+  if (plan.streamed) {
+    // The walk first, one CTA per (sequence, head) (pairs < SMs), then the intra-chunk
+    // kernel as its dependent on the remaining SMs, two persistent CTAs per SM: the walk's
+    // CTAs are all resident before it starts, so the two share the GPU; the walk waits for
+    // each tile's ready flag (cleared here), the intra-chunk kernel never waits for the walk
+    // until its own end.
+    e = cudaMemsetAsync(ia.tile_ready, 0, sizeof(int) * static_cast<size_t>(tiles), st);
+    if (e == cudaSuccess) {
+      walk<<<static_cast<unsigned>(plan.pairs), kWalkThreads, WalkKSm::BYTES + 1024, st>>>(wa);
+      e = cudaGetLastError();
+    }
+    const int64_t slots = 2 * (static_cast<int64_t>(sms) - plan.pairs);
+    if (e == cudaSuccess)
+      e = launch_dep(reinterpret_cast<const void*>(intra), tiles < slots ? tiles : slots,
+                     kIntraThreads, IntraSm::BYTES + 1024, &ia);
+  } else {
+    // two resident CTAs per SM, taking tiles from the queue; then the walk kernel, whose
+    // CTAs set up while the intra-chunk kernel drains and then wait for it
+    const int64_t intra_grid = tiles < 2 * static_cast<int64_t>(sms) ? tiles : 2 * static_cast<int64_t>(sms);
+    intra<<<static_cast<unsigned>(intra_grid), kIntraThreads, IntraSm::BYTES + 1024, st>>>(ia);
+    e = cudaGetLastError();
+    const int64_t per = plan.max_segs > 2 ? plan.max_segs - 1 : 1;
+    if (e == cudaSuccess)
+      e = launch_dep(reinterpret_cast<const void*>(walk), plan.pairs * per, kWalkThreads,
+                     WalkKSm::BYTES + 1024, &wa);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

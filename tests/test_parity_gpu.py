@@ -181,7 +181,7 @@ def test_tensor_core_segment_counts(kda):
     """Sequences with exactly 1, 2, 3 and many segments in one call: segment 0 alone,
     S_1 used directly by segment 1 (no combine step), one combine step, a long chain."""
     lengths = [320, 321, 576, 577, 0, 3000]
-    first, seg, dec = segment_plan(len(lengths), 2, max(lengths))
+    first, seg, dec = segment_plan(len(lengths), 2, max(lengths), sum(lengths))
     assert (first, seg, dec) == (320, 256, 0)
     nseg = [1 if n <= first else 1 + -(-(n - first) // seg) for n in lengths]
     assert nseg == [1, 2, 2, 3, 1, 12]
@@ -198,7 +198,7 @@ def test_tensor_core_shrinking_segments(kda):
     first segment of 11): the offsets of the combine chain's segments, a sequence ending in
     the short last segment, one in segment 1 and one inside segment 0."""
     lengths = [1792, 1000, 1]
-    plan = segment_plan(len(lengths), 13, max(lengths))
+    plan = segment_plan(len(lengths), 13, max(lengths), sum(lengths))
     assert plan == (11 * 64, 9 * 64, 2 * 64), plan
     x = make_inputs(None, H=13, dk=128, dv=128, dtype=torch.bfloat16, seed=23,
                     lengths=lengths, state_std=0.02)

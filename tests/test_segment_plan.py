@@ -1,4 +1,4 @@
-"""Host-side checks of the tensor-core prefill's segment plan (CPU: no kernel runs).
+"""Host-side checks of the tensor-core prefill's schedule and segment plan (CPU: no kernel runs).
 
 The walk kernel runs, per (sequence, head), one CTA per later segment, and its CTAs wait for
 one another's state hand-offs, so the plan must never ask for more CTAs than there are SMs:
@@ -33,10 +33,11 @@ def planned_max_segs(kda, n_seqs, H, max_len, T_total):
     assert ws > 0
     n_slots = -(-T_total // CHUNK) + n_seqs
     tiles_off = ws - TILE_BYTES * n_slots * H
-    if tiles_off == 1024:
+    ready = -(-(4 * n_slots * H) // 256) * 256  # per-tile ready flags
+    if tiles_off == -(-(HEADER + ready) // 1024) * 1024:
         return 0
-    segs = (tiles_off - HEADER) // (UNIT_BYTES * n_seqs * H)
-    assert -(-(HEADER + UNIT_BYTES * n_seqs * H * segs) // 1024) * 1024 == tiles_off
+    segs = (tiles_off - HEADER - ready) // (UNIT_BYTES * n_seqs * H)
+    assert -(-(HEADER + ready + UNIT_BYTES * n_seqs * H * segs) // 1024) * 1024 == tiles_off
     return segs
 
 
@@ -48,7 +49,7 @@ CASES = [(1, 32, 8192), (1, 16, 1 << 20), (8, 32, 32768), (6, 2, 3000), (3, 13, 
 @pytest.mark.parametrize("n_seqs,H,max_len", CASES)
 def test_plan_matches_library_and_fits_the_sms(kda, n_seqs, H, max_len):
     pairs = n_seqs * H
-    plan = segment_plan(n_seqs, H, max_len)
+    plan = segment_plan(n_seqs, H, max_len)  # T_total = n_seqs * max_len, as below
     want = segment_count(max_len, plan)
     got = planned_max_segs(kda, n_seqs, H, max_len, T_total=max_len * n_seqs)
     assert got == (want if want > 2 else 0), (got, want, plan)
@@ -68,7 +69,17 @@ def test_plan_matches_library_and_fits_the_sms(kda, n_seqs, H, max_len):
 
 def test_shrinking_plan_offsets():
     """Segment 0 of 11 chunks, then 9, 7, 5 chunks: a sequence ending inside each segment."""
-    plan = segment_plan(3, 13, 1792)
+    plan = segment_plan(3, 13, 1792, T_total=1792 + 1000 + 1)
     assert plan == (11 * 64, 9 * 64, 2 * 64)
     assert [segment_count(n, plan) for n in (1, 704, 705, 1280, 1281, 1728, 1729, 1792)] == \
         [1, 1, 2, 2, 3, 3, 4, 4]
+
+
+def test_streamed_schedule_choice():
+    """The 8K x 32-head workload walks each (sequence, head) in one CTA beside the intra-chunk
+    kernel; a million tokens of 16 heads, and varlen batches of 256 (sequence, head) pairs,
+    keep the segmented schedule."""
+    from tests.plan import streamed
+    assert streamed(1, 32, 8192, 8192)
+    assert not streamed(1, 16, 1 << 20, 1 << 20)
+    assert not streamed(8, 32, 32768, 147651)

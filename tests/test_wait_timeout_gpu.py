@@ -38,10 +38,11 @@ def kda():
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("T,H", [(64, 1), (3000, 2)])
+@pytest.mark.parametrize("T,H", [(64, 1), (3000, 2), (2048, 37)])
 def test_first_wait_running_out_is_reported_and_context_stays_usable(kda, T, H):
     """(64, 1): one chunk of one head (intra-chunk kernel and one output walk);
-    (3000, 2): twelve segments per head (summary walks, combine steps, later output walks)."""
+    (3000, 2): twelve segments per head (summary walks, combine steps, later output walks);
+    (2048, 37): the streamed schedule (the walks wait for tiles that never come)."""
     from kimi_delta_attention_19_b200 import build as kbuild
     assert os.path.exists(kbuild.SHORTWAIT_LIB), "build() makes the short-wait variant"
     short = kda.load_library(kbuild.SHORTWAIT_LIB)
