@@ -242,8 +242,15 @@ def bench_ours(args, world, rank, local):
     roofline = {"bound": "tensor", "achieved": round(tc_tflops, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
-                "traffic": measured_traffic("prefill_bf16_h32_t8192_d128"),
+                # the library picks the streamed schedule for this workload: its walk waits for
+                # tiles that the intra-chunk kernel, running beside it, publishes, so it cannot
+                # run under ncu (which runs kernels one at a time) and has no DRAM capture; the
+                # same call under the segmented schedule has one
+                "traffic": (measured_traffic("prefill_bf16_h32_t8192_d128_segmented")
+                            if os.environ.get("KDA_PREFILL_SCHEDULE") == "segmented" else None),
+                "traffic_segmented_schedule": measured_traffic("prefill_bf16_h32_t8192_d128_segmented"),
                 "traffic_scope": "one kda_chunk_fwd call (intra-chunk kernel + walk kernel)",
+                "schedule": os.environ.get("KDA_PREFILL_SCHEDULE") or "library model (streamed here)",
                 "peak_source": peaks["source"],
                 "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": algo_bytes},

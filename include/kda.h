@@ -113,6 +113,16 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape *shape);
  *  workspace    device scratch of >= kda_chunk_fwd_workspace_size(shape) bytes,
  *               256-byte aligned, used only for the duration of the enqueued work.
  *               Calls that share a workspace must be ordered on one stream.
+ *
+ * Schedule (bf16 with dk = dv = 128): an intra-chunk kernel and a walk kernel. Where a
+ * built-in model of the two schedules favours it, the walk runs first, one CTA per
+ * (sequence, head), and the intra-chunk kernel runs beside it as its programmatic
+ * dependent on the other SMs; the walk takes each chunk's tiles as soon as they are
+ * written (a bounded wait on a per-tile flag). Otherwise the walk runs after it, long
+ * sequences split into segments walked in parallel. KDA_PREFILL_SCHEDULE=segmented or
+ * =streamed in the environment overrides the model; a tool that runs kernels one at a time
+ * (a profiler) needs `segmented`. The workspace size depends on the schedule: keep the
+ * variable unchanged between kda_chunk_fwd_workspace_size and the call.
  */
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
                          const void *beta, const float *initial_state,

@@ -32,6 +32,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "kda_internal.cuh"
@@ -1674,6 +1676,13 @@ TcPlan tc_plan(int64_t T_total, int n_seqs, int H, int64_t max_len) {
     t_str = (1.9 * static_cast<double>(Lc) > intra ? 1.9 * static_cast<double>(Lc) : intra) + 10.0;
   }
   p.streamed = t_str < 0.97 * t_seg;
+  // KDA_PREFILL_SCHEDULE=segmented|streamed overrides the model (a tool that runs kernels one
+  // at a time, a profiler say, needs the segmented one: the streamed walk waits for tiles a
+  // kernel launched after it writes)
+  if (const char* env = std::getenv("KDA_PREFILL_SCHEDULE")) {
+    if (std::strcmp(env, "segmented") == 0) p.streamed = false;
+    else if (std::strcmp(env, "streamed") == 0) p.streamed = p.pairs >= 1 && p.pairs <= 100;
+  }
   if (p.streamed || m < 2 || Lc < 16) {
     p.first_tokens = p.seg_tokens = 1 << 30;  // one segment per sequence
     p.max_segs = 1;
