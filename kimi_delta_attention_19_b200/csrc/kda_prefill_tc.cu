@@ -598,6 +598,25 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
       bulk_commit();
     }
     if (tid == 0) {
+      // the CTA's next tile (drawn at this tile's start): its inputs into L2 now, so that its
+      // loads find them there
+      if (nxt < a.n_tiles) {
+        const int64_t un = nxt / a.H;
+        const int hn = static_cast<int>(nxt % a.H);
+        const int sn = owner_seq(a.seq, un);
+        const int64_t tn0 = seq_start(a.seq, sn);
+        const int64_t cn = un - slot_base(tn0, sn);
+        if (cn >= 0) {
+          const int yn = static_cast<int>(tn0 + cn * C);
+          if (yn < a.seq.T_total) {
+            tma_prefetch_2d(&a.tm_g, hn * D, yn);
+            tma_prefetch_2d(&a.tm_k, hn * D, yn);
+            tma_prefetch_2d(&a.tm_q, hn * D, yn);
+            tma_prefetch_2d(&a.tm_v, hn * D, yn);
+            tma_prefetch_2d(&a.tm_v, hn * D + 64, yn);
+          }
+        }
+      }
       tc_fence_after();
       const uint32_t ig = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
