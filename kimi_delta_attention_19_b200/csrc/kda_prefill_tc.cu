@@ -300,7 +300,7 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 // that the off-diagonal block of the inverse is never formed.
 constexpr int kIntraThreads = 256;
 constexpr size_t kIntraQueueOffset = 128;  // the tile queue's counter, in the workspace header
-constexpr int kPStoreThread = 192;  // warp 6, lane 0: issues (and waits for) the P store
+constexpr int kPStoreThread = 64;   // warp 2, lane 0: issues (and waits for) the P store
 struct IntraSm {
   // Raw inputs as loaded by TMA; each region is reused once its contents are read.
   static constexpr uint32_t SV = 0;        // V, swizzled: [64 s][64 j] boxes (U0's A operand)
@@ -642,7 +642,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     //   Rows r < 64 of the Gram accumulator (tensor-memory lanes 0..63) hold K~_r K^^T:
     //   warps 0, 1, 4, 5 take one row each and a half hh of its 64 columns, so the
     //   diagonal block of rows 0..31 is in the half of warp 0, that of rows 32..63 in the
-    //   half of warp 5, and A_21 in warp 1's. Warps 2, 3, 6, 7 write P from lanes 64..127.
+    //   half of warp 5, and A_21 in warp 1's. Warps 2 and 3 write P from lanes 64..127.
     //   Forward substitution on the CUDA cores, a right-hand-side column per lane, columns
     //   of the block broadcast from shared memory: warp 0 solves (I + A_11) N_lo = I,
     //   warp 5 (I + A_22) N_hi = I and, beside it, warp 6 (I + A_22) G = A_21 (so G costs
@@ -690,8 +690,10 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
     };
     {
       uint32_t v[32];
-      tmem_ld32(tb + lane_base + L_::G + 32 * hh, v);
-      tmem_ld_wait(v);
+      if (rowt || hh == 0) {  // warps 6 and 7 read no Gram row (P is warps 2 and 3's)
+        tmem_ld32(tb + lane_base + L_::G + 32 * hh, v);
+        tmem_ld_wait(v);
+      }
       if (rowt) {
         // A = Diag(beta) strict_lower(K~ K^^T), row rr, columns 32 hh ..
         const float br = bet[rr];
@@ -742,32 +744,41 @@ __global__ void __launch_bounds__(kIntraThreads, 2) kda_tc_intra(const __grid_co
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           *reinterpret_cast<uint4*>(sm + L_::T + sw128_chunk(rr, 4 * hh + q, K8)) = pack8(f + 8 * q);
-      } else {
-        // P = lower_incl(Q~ K^^T): row r, columns 32 hh .. 32 hh + 31
+      } else if (hh == 0) {
+        // P = lower_incl(Q~ K^^T): row r, both column halves (warps 2 and 3, so that warp 6
+        // goes straight to G)
         const int r = (warp & 3) * 32 + lane - 64;
-        float f[32];
+        auto stage_p = [&](const uint32_t (&pv)[32], int half) {
+          float f[32];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) f[t] = 32 * hh + t <= r ? __uint_as_float(v[t]) : 0.f;
+          for (int t = 0; t < 32; ++t) f[t] = 32 * half + t <= r ? __uint_as_float(pv[t]) : 0.f;
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          *reinterpret_cast<uint4*>(sm + L_::PS + sw128_chunk(r, 4 * hh + q8, 0)) = pack8(f + 8 * q8);
+          for (int q8 = 0; q8 < 4; ++q8)
+            *reinterpret_cast<uint4*>(sm + L_::PS + sw128_chunk(r, 4 * half + q8, 0)) = pack8(f + 8 * q8);
+        };
+        stage_p(v, 0);
+        tmem_ld32(tb + lane_base + L_::G + 32, v);
+        tmem_ld_wait(v);
+        stage_p(v, 1);
         fence_async_smem();
-        group_sync(2, 128);  // warps 2, 3, 6, 7: P is staged
+        group_sync(2, 64);  // warps 2, 3: P is staged
         if (tid == kPStoreThread) {  // P to the workspace
           tma_store_2d(&a.tm_p, sm + L_::PS, 0, static_cast<int>(tile * C));
           bulk_commit();
         }
-        if (warp == 6) {
-          // G = N_hi A_21, column `lane`, as +G and -G rows (bf16, K-major B operands)
-          group_sync(1, 96);
-          float y[32];
-          fsub(a22, [&](int r) { return a21[r * 32 + lane]; }, y);
+      } else if (warp == 6) {
+        // G = N_hi A_21, column `lane`, as +G and -G rows (bf16, K-major B operands): lane
+        // pairs trade values, even lanes write a +G pair of columns and odd lanes the -G pair
+        group_sync(1, 96);
+        float y[32];
+        fsub(a22, [&](int r) { return a21[r * 32 + lane]; }, y);
+        const int odd = lane & 1;
 #pragma unroll
-          for (int r = 0; r < 32; ++r) {
-            const uint32_t off = sw128_chunk(r, lane >> 3, 0) + (lane & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16*>(sm + L_::GP + off) = __float2bfloat16_rn(y[r]);
-            *reinterpret_cast<__nv_bfloat16*>(sm + L_::GN + off) = __float2bfloat16_rn(-y[r]);
-          }
+        for (int r = 0; r < 32; ++r) {
+          const float other = __shfl_xor_sync(0xffffffffu, y[r], 1);
+          const uint32_t off = sw128_chunk(r, lane >> 3, 0) + (lane & 6) * 2;
+          const uint32_t pr = odd ? pack_bf16(-other, -y[r]) : pack_bf16(y[r], other);
+          *reinterpret_cast<uint32_t*>(sm + (odd ? L_::GN : L_::GP) + off) = pr;
         }
       }
     }
