@@ -222,6 +222,28 @@ def test_tensor_core_segments_resume_in_place(kda):
     assert_close(state, rs, torch.bfloat16, "alias final_state")
 
 
+def test_streamed_schedule_varlen_resume_in_place(kda):
+    """Two sequences of 16 heads (4096 and 3000 tokens, the second ragged): the library walks
+    each (sequence, head) in one CTA beside the intra-chunk kernel, taking tiles as they are
+    published; final_state aliases initial_state."""
+    from tests.plan import streamed
+    lengths = [4096, 3000]
+    assert streamed(len(lengths), 16, max(lengths), sum(lengths))
+    x = make_inputs(None, H=16, dk=128, dv=128, dtype=torch.bfloat16, seed=29,
+                    lengths=lengths, state_std=0.02)
+    ro, rs = _run_oracle(x)
+    state = x.initial_state.to(DEV).clone()
+    ws = kda.alloc_workspace(kda.make_shape(sum(lengths), 16, 128, 128, torch.bfloat16,
+                                            n_seqs=2, max_seqlen=max(lengths)), DEV)
+    out, _ = kda.chunk_fwd(x.q.to(DEV), x.k.to(DEV), x.v.to(DEV), x.g.to(DEV), x.beta.to(DEV),
+                           initial_state=state, final_state=state,
+                           cu_seqlens=x.cu_seqlens.to(DEV), max_seqlen=max(lengths), workspace=ws)
+    torch.cuda.synchronize()
+    assert kda.workspace_status(ws) == (kda.KDA_OK, 0)
+    assert_close(out, ro, torch.bfloat16, "streamed out")
+    assert_close(state, rs, torch.bfloat16, "streamed final_state")
+
+
 def test_max_seqlen_too_small_reports_without_trap(kda):
     x = make_inputs(None, H=2, dk=128, dv=128, dtype=torch.bfloat16, seed=18,
                     lengths=[4000, 100], state_std=None)
