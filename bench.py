@@ -242,12 +242,13 @@ def bench_ours(args, world, rank, local):
     roofline = {"bound": "tensor", "achieved": round(tc_tflops, 2),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(tc_tflops / peaks["bf16_tflops"], 4),
-                # the library picks the streamed schedule for this workload: its walk waits for
-                # tiles that the intra-chunk kernel, running beside it, publishes, so it cannot
-                # run under ncu (which runs kernels one at a time) and has no DRAM capture; the
-                # same call under the segmented schedule has one
+                # the library picks the streamed schedule for this workload (its two kernels run
+                # together): its DRAM bytes come from an ncu capture of one whole call inside a
+                # profiler range (application-range replay, nothing serialized); the segmented
+                # schedule's from a per-kernel capture
                 "traffic": (measured_traffic("prefill_bf16_h32_t8192_d128_segmented")
-                            if os.environ.get("KDA_PREFILL_SCHEDULE") == "segmented" else None),
+                            if os.environ.get("KDA_PREFILL_SCHEDULE") == "segmented"
+                            else measured_traffic("prefill_bf16_h32_t8192_d128")),
                 "traffic_segmented_schedule": measured_traffic("prefill_bf16_h32_t8192_d128_segmented"),
                 "traffic_scope": "one kda_chunk_fwd call (intra-chunk kernel + walk kernel)",
                 "schedule": os.environ.get("KDA_PREFILL_SCHEDULE") or "library model (streamed here)",
@@ -510,9 +511,18 @@ def kernels_only(args):
         x = workload_inputs(w, device=dev)
         shape = kda.make_shape(w.T, w.H, w.dk, w.dv, w.dtype)
         ws = kda.alloc_workspace(shape, dev)
-        for _ in range(n):
+        for i in range(n):
+            # --profile-range: the last call inside a profiler range (cudaProfilerStart/Stop),
+            # for a range-replay capture that keeps the call's two kernels running together
+            last = args.profile_range and i == n - 1
+            if last:
+                torch.cuda.synchronize()
+                torch.cuda.cudart().cudaProfilerStart()
             kda.chunk_fwd(x.q, x.k, x.v, x.g, x.beta, initial_state=x.initial_state,
                           workspace=ws)
+            if last:
+                torch.cuda.synchronize()
+                torch.cuda.cudart().cudaProfilerStop()
     else:
         wd = WORKLOADS[DECODE]
         state = decode_state(wd.B, wd.H, wd.dk, wd.dv, device=dev)
@@ -533,6 +543,8 @@ def main():
                     help="tokens per reference-arm step (bounded oracle sample)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum timed oracle work for the cpu_baseline object")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="with --kernels-only prefill: put the last call inside a profiler range")
     ap.add_argument("--kernels-only", choices=["prefill", "backward", "decode"], default=None,
                     help="profiler driver: run warmup + steps calls of one path, print no "
                          "measurement (for ncu -s/-c captures)")
